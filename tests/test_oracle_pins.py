@@ -1,0 +1,331 @@
+"""Pins for the oracle: each test ties it to something other than itself --
+hand-worked fixtures, closed forms, invariants of the method, brute force on
+tiny inputs, or a library routine that the case reduces to."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.conftest import golden
+
+
+def _hex(vals):
+    return np.array([int(v, 16) for v in vals], dtype=np.uint32)
+
+
+# ------------------------------------------------------------- packing -----
+
+def test_pack_bits_fixture():
+    fx = golden("pack_bits_64.txt")
+    y = -np.ones((1, 64))
+    for j in fx["positive"]:
+        y[0, int(j)] = 1.0
+    np.testing.assert_array_equal(oracle.pack_bits(y)[0], _hex(fx["words"]))
+
+
+def test_pack_bits_zero_is_zero_bit():
+    y = np.zeros((1, 32))
+    y[0, 3] = 1e-300
+    assert oracle.pack_bits(y)[0, 0] == 8
+
+
+# ------------------------------------------------------------- encoders ----
+
+def test_lsh_fixture_nonsquare():
+    fx = golden("lsh_signed_selector.txt")
+    R = np.zeros((32, 4))
+    for j in range(32):
+        R[j, j % 4] = 1.0 if (j // 4) % 2 == 0 else -1.0
+    x = np.array([[float(v) for v in fx["x"]]])
+    np.testing.assert_array_equal(oracle.encode("lsh", x, R)[0], _hex(fx["words"]))
+
+
+def test_lsh_identity_projection_is_sign_code():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((50, 128))
+    lsh = oracle.encode("lsh", x, np.eye(128))
+    sign, _ = oracle.encode("sign", x)
+    np.testing.assert_array_equal(lsh, sign)
+
+
+def test_lsh_charikar_angle_law():
+    """Random-hyperplane LSH: P[bit differs] = angle / pi (Charikar)."""
+    rng = np.random.default_rng(11)
+    d, bits, pairs = 64, 128, 400
+    theta = 1.1
+    u = rng.standard_normal((pairs, d))
+    u /= np.linalg.norm(u, axis=1, keepdims=True)
+    w = rng.standard_normal((pairs, d))
+    w -= (w * u).sum(1, keepdims=True) * u
+    w /= np.linalg.norm(w, axis=1, keepdims=True)
+    v = math.cos(theta) * u + math.sin(theta) * w
+    total = 0
+    for i in range(pairs):
+        R = rng.standard_normal((bits, d))
+        cu = oracle.encode("lsh", u[i:i + 1], R)
+        cv = oracle.encode("lsh", v[i:i + 1], R)
+        total += int(oracle.hamming(cu, cv)[0])
+    n = pairs * bits
+    p = theta / math.pi
+    assert abs(total / n - p) < 5 * math.sqrt(p * (1 - p) / n)
+
+
+@pytest.mark.parametrize("kind", ["lsh", "sign"])
+def test_negated_input_flips_every_bit(kind):
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((20, 128))
+    R = rng.standard_normal((64, 128))
+    params = R if kind == "lsh" else None
+    c1 = oracle.encode(kind, x, params)
+    c2 = oracle.encode(kind, -x, params)
+    if kind == "sign":
+        c1, c2 = c1[0], c2[0]
+    bits = c1.shape[1] * 32
+    for i in range(20):
+        assert oracle.hamming(c1[i:i + 1], c2[i:i + 1])[0] == bits
+
+
+def _mlp_fixture_params():
+    W1 = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, -1.0]])
+    b1 = np.array([0.0, -1.0, 0.0])
+    W2 = np.zeros((32, 3))
+    b2 = -np.ones(32)
+    W2[0, 0], b2[0] = 1.0, -0.8
+    W2[1, 0], b2[1] = 1.0, -0.85
+    W2[2, 1], b2[2] = 1.0, 0.01
+    W2[3, 1], b2[3] = -1.0, 0.01
+    W2[4, 2], b2[4] = 1.0, -0.05
+    W2[5, 2], b2[5] = 1.0, -0.052
+    b2[6] = 0.5
+    b2[7] = -0.5
+    W2[8, 0], W2[8, 2], b2[8] = 1.0, -1.0, -0.77
+    return W1, b1, W2, b2
+
+
+def test_mlp_fixture():
+    fx = golden("mlp_hash_worked.txt")
+    x = np.array([[math.log(3.0), 1.0]])
+    params = _mlp_fixture_params()
+    y = oracle.presign_mlp(x, *params)
+    h0 = 0.75 * math.log(3.0)
+    h2 = (math.log(3.0) - 1.0) / (1.0 + math.e / 3.0)
+    assert abs(h0 - float(fx["h0"][0])) < 1e-13
+    assert abs(h2 - float(fx["h2"][0])) < 1e-7
+    assert abs(y[0, 0] - (h0 - 0.8)) < 1e-13
+    assert abs(y[0, 4] - (h2 - 0.05)) < 1e-13
+    assert abs(y[0, 8] - (h0 - h2 - 0.77)) < 1e-13
+    np.testing.assert_array_equal(oracle.encode("mlp", x, params)[0], _hex(fx["words"]))
+
+
+def test_mlp_zero_first_layer_gives_constant_code():
+    rng = np.random.default_rng(8)
+    d, hidden, bits = 16, 24, 64
+    W1 = np.zeros((hidden, d))
+    b1 = rng.uniform(-1, 1, hidden)
+    W2 = rng.uniform(-1, 1, (bits, hidden))
+    b2 = rng.uniform(-1, 1, bits)
+    x = rng.standard_normal((30, d))
+    y = oracle.presign_mlp(x, W1, b1, W2, b2)
+    expect = W2 @ (b1 / (1 + np.exp(-b1))) + b2
+    np.testing.assert_allclose(y, np.broadcast_to(expect, y.shape), rtol=0, atol=1e-14)
+
+
+def test_mlp_matches_torch_library_layers():
+    rng = np.random.default_rng(9)
+    d, hidden, bits = 128, 512, 128
+    W1 = rng.uniform(-0.09, 0.09, (hidden, d))
+    b1 = rng.uniform(-0.09, 0.09, hidden)
+    W2 = rng.uniform(-0.04, 0.04, (bits, hidden))
+    b2 = rng.uniform(-0.04, 0.04, bits)
+    x = rng.standard_normal((64, d))
+    T = lambda a: torch.from_numpy(a)
+    ref = torch.nn.functional.linear(torch.nn.functional.silu(torch.nn.functional.linear(T(x), T(W1), T(b1))), T(W2), T(b2))
+    np.testing.assert_allclose(oracle.presign_mlp(x, W1, b1, W2, b2), ref.numpy(), rtol=0, atol=1e-13)
+
+
+def test_sign_norms_fp16():
+    x = np.zeros((3, 128))
+    x[0, :2] = [3.0, 4.0]
+    x[1, :] = 1.0
+    x[2, 7] = -2.5
+    n = oracle.sign_norms(x)
+    assert n.dtype == np.float16
+    assert float(n[0]) == 5.0
+    assert float(n[1]) == 11.3125  # sqrt(128) = 11.3137 -> nearest fp16 (spacing 2^-7)
+    assert float(n[2]) == 2.5
+
+
+# ------------------------------------------------------------- hamming -----
+
+def test_hamming_fixture():
+    fx = golden("hamming_group.txt")
+    q = np.stack([_hex(fx["cq0"]), _hex(fx["cq1"])])
+    k = _hex(fx["ck"])[None, :]
+    assert oracle.hamming(q, k)[0] == int(fx["D"][0])
+
+
+def test_hamming_counts_differing_signs():
+    """Brute force from the pre-sign values, with no packing involved."""
+    rng = np.random.default_rng(1)
+    g, n, bits = 3, 40, 64
+    yq = rng.standard_normal((g, bits))
+    yk = rng.standard_normal((n, bits))
+    D = oracle.hamming(oracle.pack_bits(yq), oracle.pack_bits(yk))
+    for t in range(n):
+        brute = sum(int((yq[h, j] > 0) != (yk[t, j] > 0)) for h in range(g) for j in range(bits))
+        assert D[t] == brute
+
+
+# ------------------------------------------------------------- top-k -------
+
+def test_topk_fixture():
+    fx = golden("topk_ties.txt")
+    D = np.array([int(v) for v in fx["D"]])
+    lo, hi = oracle.candidate_range(len(D), int(fx["sink"][0]), int(fx["local"][0]))
+    got = oracle.select_topk(D, lo, hi, int(fx["k"][0]))
+    np.testing.assert_array_equal(got, [int(v) for v in fx["idx"]])
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_brute_force_rank(seed):
+    """Selected iff fewer than k candidates precede it in (D, t) order."""
+    rng = np.random.default_rng(seed)
+    N = int(rng.integers(1, 90))
+    s, l = int(rng.integers(0, 6)), int(rng.integers(0, 6))
+    k = int(rng.integers(0, 100))
+    D = rng.integers(0, 6, N)
+    lo, hi = oracle.candidate_range(N, s, l)
+    got = oracle.select_topk(D, lo, hi, k)
+    want = [t for t in range(lo, hi)
+            if sum(1 for u in range(lo, hi) if (D[u], u) < (D[t], t)) < k]
+    np.testing.assert_array_equal(got, want)
+
+
+def test_topk_degenerate_cases():
+    D = np.full(50, 7)
+    np.testing.assert_array_equal(oracle.select_topk(D, 4, 40, 5), [4, 5, 6, 7, 8])
+    np.testing.assert_array_equal(oracle.select_topk(D, 4, 40, 1000), np.arange(4, 40))
+    assert oracle.select_topk(D, 4, 40, 0).size == 0
+    assert oracle.select_topk(D, 10, 10, 5).size == 0
+
+
+def test_candidate_range_short_sequence():
+    assert oracle.candidate_range(100, 4, 64) == (4, 36)
+    assert oracle.candidate_range(50, 4, 64) == (4, 4)
+    assert oracle.candidate_range(3, 4, 64) == (3, 3)
+    assert oracle.candidate_range(0, 0, 0) == (0, 0)
+
+
+# ------------------------------------------------------------- attention ---
+
+def test_attention_fixture_and_merge():
+    fx = golden("attention_worked.txt")
+    q = np.array([[math.log(3.0), 0.0]])
+    K = np.array([[0.0, 5.0], [1.0, 7.0], [2.0, 0.0]])
+    V = np.array([[4.0, 0.0], [0.0, 8.0], [9.0, 9.0]])
+    o, lse = oracle.attend(q, K, V, [0, 1], 1.0)
+    np.testing.assert_allclose(o[0], [float(v) for v in fx["out"]], atol=1e-14)
+    assert abs(lse[0] - math.log(float(fx["lse_is_ln"][0]))) < 1e-14
+    o0, l0 = oracle.attend(q, K, V, [0], 1.0)
+    o1, l1 = oracle.attend(q, K, V, [1], 1.0)
+    om, lm = oracle.lse_merge(o0, l0, o1, l1)
+    np.testing.assert_allclose(om, o, atol=1e-14)
+    np.testing.assert_allclose(lm, lse, atol=1e-14)
+
+
+def test_attention_all_rows_is_library_sdpa():
+    rng = np.random.default_rng(4)
+    g, N, d = 4, 300, 128
+    q = rng.standard_normal((g, d))
+    K = rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    o, lse = oracle.attend(q, K, V, np.arange(N), 1 / math.sqrt(d))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None], torch.from_numpy(K)[None], torch.from_numpy(V)[None])[0]
+    np.testing.assert_allclose(o, ref.numpy(), atol=1e-12)
+    z = (q @ K.T) / math.sqrt(d)
+    np.testing.assert_allclose(lse, np.log(np.exp(z).sum(1)), atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(6)
+    K = rng.standard_normal((20, 8))
+    V = rng.standard_normal((20, 8))
+    q = rng.standard_normal((2, 8))
+    o, _ = oracle.attend(q, K, V, [13], 0.3)
+    np.testing.assert_allclose(o, np.stack([V[13], V[13]]), atol=1e-15)
+    o, lse = oracle.attend(np.zeros((1, 8)), K, V, [1, 4, 9], 0.3)
+    np.testing.assert_allclose(o[0], V[[1, 4, 9]].mean(0), atol=1e-15)
+    assert abs(lse[0] - math.log(3)) < 1e-15
+    o, lse = oracle.attend(q, K, V, [], 0.3)
+    assert np.all(o == 0) and np.all(np.isneginf(lse))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_lse_merge_any_partition(seed):
+    rng = np.random.default_rng(seed)
+    g, N, d = 3, 64, 16
+    q = rng.standard_normal((g, d)) * 2
+    K = rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    rows = rng.permutation(N)[:40]
+    o, lse = oracle.attend(q, K, V, rows, 0.5)
+    parts = np.array_split(rng.permutation(rows), int(rng.integers(2, 6)))
+    parts.insert(int(rng.integers(0, len(parts))), np.array([], dtype=np.int64))
+    acc_o, acc_l = oracle.attend(q, K, V, parts[0], 0.5)
+    for p in parts[1:]:
+        po, pl = oracle.attend(q, K, V, p, 0.5)
+        acc_o, acc_l = oracle.lse_merge(acc_o, acc_l, po, pl)
+    np.testing.assert_allclose(acc_o, o, atol=1e-12)
+    np.testing.assert_allclose(acc_l, lse, atol=1e-12)
+
+
+def test_lse_merge_two_empty_parts():
+    o, lse = oracle.lse_merge(np.zeros((2, 4)), np.full(2, -np.inf), np.zeros((2, 4)), np.full(2, -np.inf))
+    assert np.all(o == 0) and np.all(np.isneginf(lse))
+
+
+# ------------------------------------------------------------- composite ---
+
+def test_decode_step_full_budget_is_dense_attention():
+    """k >= candidates: the step attends every token, i.e. dense attention."""
+    rng = np.random.default_rng(12)
+    B, Hq, Hkv, N, d = 2, 4, 2, 50, 128
+    q = rng.standard_normal((B, Hq, d))
+    K = rng.standard_normal((B, Hkv, N, d))
+    V = rng.standard_normal((B, Hkv, N, d))
+    R = rng.standard_normal((64, d))
+    codes = oracle.encode("lsh", K, R)
+    res = oracle.decode_step(q, K, V, codes, N, 3, 5, 1000, "lsh", R)
+    g = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[b, h])[None, None], torch.from_numpy(K[b, h // g])[None],
+                torch.from_numpy(V[b, h // g])[None])[0, 0]
+            np.testing.assert_allclose(res["out"][b, h], ref.numpy(), atol=1e-12)
+
+
+def test_decode_step_uses_group_sum():
+    """KV head j's selection depends only on query heads j*g .. j*g+g-1, and
+    equals the brute-force top-k of their summed distances."""
+    rng = np.random.default_rng(13)
+    B, Hq, Hkv, N, d = 1, 6, 3, 200, 128
+    g = Hq // Hkv
+    q = rng.standard_normal((B, Hq, d))
+    K = rng.standard_normal((B, Hkv, N, d))
+    V = rng.standard_normal((B, Hkv, N, d))
+    codes, _ = oracle.encode("sign", K)
+    r1 = oracle.decode_step(q, K, V, codes, N, 0, 0, 10, "sign")
+    q2 = q.copy()
+    q2[0, 2 * g:] = rng.standard_normal((g, d))
+    r2 = oracle.decode_step(q2, K, V, codes, N, 0, 0, 10, "sign")
+    np.testing.assert_array_equal(r1["idx"][0, :2], r2["idx"][0, :2])
+    qc, _ = oracle.encode("sign", q)
+    for j in range(Hkv):
+        D = [sum(int(np.bitwise_count(qc[0, h] ^ codes[0, j, t]).sum()) for h in range(j * g, (j + 1) * g))
+             for t in range(N)]
+        want = sorted(sorted(range(N), key=lambda t: (D[t], t))[:10])
+        np.testing.assert_array_equal(r1["idx"][0, j], want)
