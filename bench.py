@@ -1,0 +1,439 @@
+"""Benchmark of the decode step: query encode + Hamming scan + top-k + sparse
+attention + LSE merge, through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the whole decode path over every layer of the
+workload (28 sequential layers for the default Qwen2.5-7B-shaped 512K-token
+case), captured in one CUDA graph.  Inputs are synthetic, drawn on the device
+(same distributions as the parity tests), and larger than L2: every layer has
+its own codes and K/V buffers.  Timing uses CUDA events on the launching
+stream after W warm-up steps; the value is the max over ranks.  With N > 1
+(torchrun) each rank runs its own replica of the workload (independent
+sequences: weak scaling, no collective on the data path).
+
+--impl reference times the oracle (CPU) on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch
+
+import synth
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="qwen7b_512k", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="hkv", choices=["hkv", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, local, backend="nccl"):
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm --
+
+class Layer:
+    """Device buffers of one layer: inputs, key codes, outputs."""
+
+    def __init__(self, w: synth.Workload, layer: int, dev, hkv):
+        inp = synth.device_layer_inputs(w, layer, dev)
+        self.q, self.K, self.V = inp["q"], inp["K"], inp["V"]
+        code = hkv.HKV_BF16 if w.dtype == "bf16" else hkv.HKV_F32
+        if w.hash == "lsh":
+            self.R = inp["R"]
+            self.kh = self.qh = hkv.HashParams.lsh(self.R)
+        elif w.hash == "mlp":
+            self.kmlp, self.qmlp = inp["k_mlp"], inp["q_mlp"]
+            self.kh = hkv.HashParams.mlp(*self.kmlp, dtype=code)
+            self.qh = hkv.HashParams.mlp(*self.qmlp, dtype=code)
+        else:
+            self.kh = self.qh = hkv.HashParams.sign(code)
+        self.codes = torch.empty(w.B, w.Hkv, w.N, w.words, dtype=torch.int32, device=dev)
+        self.norms = torch.empty(w.B, w.Hkv, w.N, dtype=torch.float16, device=dev) if w.hash == "sign" else None
+        self.q_codes = torch.empty(w.B, w.Hq, w.words, dtype=torch.int32, device=dev)
+        self.idx = torch.empty(w.B, w.Hkv, w.top_k, dtype=torch.int32, device=dev)
+        self.out = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
+
+    def encode_keys(self, hkv):
+        hkv.hkv_encode_keys(self.kh, self.K.view(-1, self.K.shape[-1]), self.codes.view(-1, self.codes.shape[-1]),
+                            None if self.norms is None else self.norms.view(-1))
+
+
+def graph_of(fn, warm=1):
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(warm):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def time_graph(g, steps, warmup, world):
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream()
+    start.record(stream)
+    for _ in range(steps):
+        g.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / steps  # ms per replay
+
+
+def source_digest(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_record(kernel_file: str, workload: str):
+    """DRAM traffic per launch from the committed ncu summary, if it was taken
+    on the current source of the kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(workload, {}).get(os.path.basename(kernel_file))
+    if not rec or rec.get("source_sha256_16") != source_digest(kernel_file):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+def run_gpu(args, rank, world, local):
+    import hash_sparse_kv_b200 as hkv
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    hkv.lib()
+    w = synth.WORKLOADS[args.workload]
+    per_layer_bytes = w.algorithmic_bytes()
+    n_layers = max(w.layers, math.ceil(3 * L2_BYTES / per_layer_bytes))
+    layers = [Layer(w, l % w.layers if w.layers > 1 else 0, dev, hkv) for l in range(n_layers)]
+    # prefill: encode the keys of every layer (timed separately, reported as encode)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for L in layers:
+        L.encode_keys(hkv)
+    e1.record()
+    torch.cuda.synchronize()
+    encode_ms = e0.elapsed_time(e1)
+    ws = hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
+    status = hkv.status_word(dev)
+
+    def step():
+        for L in layers:
+            hkv.hkv_decode_step(L.qh, L.q, L.codes, L.K, L.V, w.N, w.n_sink, w.n_local, w.top_k, L.out,
+                                q_codes=L.q_codes, idx=L.idx, ws=ws, status=status)
+
+    def scan_only():
+        for L in layers:
+            hkv.hkv_retrieve_topk(L.q_codes, L.codes, w.N, w.n_sink, w.n_local, w.top_k, L.idx, ws=ws, status=status)
+
+    g_step = graph_of(step)
+    rc = hkv.hkv_check(status)
+    if rc != hkv.HKV_OK:
+        raise RuntimeError(f"decode step reported status {rc}")
+    with ClockSampler(local) as clk:
+        ms = time_graph(g_step, args.steps, args.warmup, world)
+    rc = hkv.hkv_check(status)
+    if rc != hkv.HKV_OK:
+        raise RuntimeError(f"decode step reported status {rc}")
+    ms = max_over_ranks(ms, world, dev)
+    # dominant kernel alone: the scan/select launch of every layer
+    g_scan = graph_of(scan_only)
+    scan_ms = max_over_ranks(time_graph(g_scan, args.steps, args.warmup, world), world, dev)
+    # end to end: host q in, host out back, every step
+    q_host = [torch.empty_like(L.q, device="cpu").pin_memory() for L in layers]
+    o_host = [torch.empty_like(L.out, device="cpu").pin_memory() for L in layers]
+    for qh, L in zip(q_host, layers):
+        qh.copy_(L.q.cpu())
+
+    def e2e_step():
+        for qh, L in zip(q_host, layers):
+            L.q.copy_(qh, non_blocking=True)
+        step()
+        for oh, L in zip(o_host, layers):
+            oh.copy_(L.out, non_blocking=True)
+
+    g_e2e = graph_of(e2e_step)
+    e2e_ms = max_over_ranks(time_graph(g_e2e, args.steps, args.warmup, world), world, dev)
+    h2d = sum(t.numel() * t.element_size() for t in q_host)
+    d2h = sum(t.numel() * t.element_size() for t in o_host)
+    rc = hkv.hkv_check(status)
+    if rc != hkv.HKV_OK:
+        raise RuntimeError(f"e2e step reported status {rc}")
+
+    keys_per_layer = w.B * w.Hkv * w.candidates()
+    keys_step = keys_per_layer * len(layers) * world
+    value = keys_step / (ms * 1e-3)
+    peak, peak_kind = measured_peaks()
+    code_bytes = w.B * w.Hkv * w.candidates() * w.bits // 8
+    scan_launch_ms = scan_ms / len(layers)
+    achieved = code_bytes / (scan_launch_ms * 1e-3) / 1e9
+    traffic = traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "retrieve.cu"), w.name)
+    step_gbs = per_layer_bytes * len(layers) / (ms * 1e-3) / 1e9
+    out = {
+        "metric": "decode retrieval+sparse-attn keys scanned/s (also us/layer and % HBM roofline)",
+        "value": value,
+        "unit": "keys/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "us_per_layer": ms * 1e3 / len(layers),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u32 codes + " + ("bf16" if w.dtype == "bf16" else "f32") + " K/V, f32 accumulate",
+        "data": "synthetic (two-cone Gaussian keys/queries, drawn on device)",
+        "config": {
+            "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.d, "n_tokens": w.N,
+            "hash": w.hash, "code_bits": w.bits, "top_k": w.top_k, "n_sink": w.n_sink, "n_local": w.n_local,
+            "layers_per_step": len(layers), "parallelism": f"replica x{world}",
+            "l2": f"inputs larger than L2: {len(layers)} distinct layer buffers, "
+                  f"{per_layer_bytes * len(layers) / 1e9:.2f} GB algorithmic per step",
+        },
+        "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
+                     "bytes_per_layer": per_layer_bytes, "peak_kind": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": "scan_select_kernel (hkv_retrieve_topk)", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": code_bytes, "launch_us": scan_launch_ms * 1e3,
+                     "peak_kind": peak_kind},
+        "e2e": {"value": keys_step / (e2e_ms * 1e-3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "encode": {"keys_per_s": w.B * w.Hkv * w.N * len(layers) / (encode_ms * 1e-3),
+                   "ms_all_layers": encode_ms, "gbs": (w.B * w.Hkv * w.N * w.d * (2 if w.dtype == "bf16" else 4)
+                                                        * len(layers)) / (encode_ms * 1e-3) / 1e9},
+        "gpu_launches": 3 * len(layers) * args.steps,
+        "clocks": clk.summary(),
+    }
+    del g_step, g_scan, g_e2e
+    return out, layers, w
+
+
+# ------------------------------------------------------------------ oracle arm --
+
+def oracle_inputs_from_device(w: synth.Workload, L):
+    """One layer's host copies, from the bench's device buffers."""
+    q, K, V = L.q.cpu(), L.K.cpu(), L.V.cpu()
+    if w.hash == "lsh":
+        return q, K, V, L.R.cpu(), L.R.cpu()
+    if w.hash == "mlp":
+        return q, K, V, tuple(t.cpu() for t in L.qmlp), tuple(t.cpu() for t in L.kmlp)
+    return q, K, V, None, None
+
+
+def oracle_inputs_host(w: synth.Workload):
+    inp = synth.layer_inputs(w, 0, pad_junk=False)
+    if w.hash == "lsh":
+        return inp["q"], inp["K"], inp["V"], inp["R"], inp["R"]
+    if w.hash == "mlp":
+        return inp["q"], inp["K"], inp["V"], inp["q_mlp"], inp["k_mlp"]
+    return inp["q"], inp["K"], inp["V"], None, None
+
+
+class OracleLayer:
+    """The oracle's decode step on one layer of the workload.  The cache's key
+    codes are computed once by the oracle itself (setup, not timed)."""
+
+    def __init__(self, w: synth.Workload, q, K, V, qparams, kparams):
+        import oracle
+        self.w, self.q, self.K, self.V, self.qparams = w, q, K, V, qparams
+        kc = oracle.encode(w.hash, K, kparams)
+        self.kc = kc[0] if w.hash == "sign" else kc
+
+    def run(self) -> float:
+        """Seconds for one decode step of this layer (single thread)."""
+        import oracle
+        from threadpoolctl import threadpool_limits
+        w = self.w
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            oracle.decode_step(self.q, self.K, self.V, self.kc, w.N, w.n_sink, w.n_local, w.top_k, w.hash,
+                               self.qparams)
+            return time.perf_counter() - t0
+
+
+def oracle_sample(w: synth.Workload, budget_s: float, layer_inputs):
+    """Time the oracle's decode step on one whole layer, repeated until the
+    budget is spent (at most 5 times).  Returns (keys/s, sample, threads)."""
+    ol = OracleLayer(w, *layer_inputs)
+    elapsed, n = 0.0, 0
+    while n < 1 or (elapsed < budget_s and n < 5):
+        elapsed += ol.run()
+        n += 1
+    keys = n * w.B * w.Hkv * w.candidates()
+    return keys / elapsed, f"{n} decode step(s) of one {w.name} layer ({w.B * w.Hkv * w.candidates()} keys each), " \
+                           f"{elapsed:.1f} s", 1
+
+
+def run_reference(args, rank, world):
+    w = synth.WORKLOADS[args.workload]
+    if rank != 0:
+        return None
+    ol = OracleLayer(w, *oracle_inputs_host(w))
+    keys_per_step = w.B * w.Hkv * w.candidates()
+    for _ in range(args.warmup):
+        ol.run()
+    per_step_s = [ol.run() for _ in range(args.steps)]
+    value = keys_per_step / statistics.mean(per_step_s)
+    sample = f"each step: one decode step of one {w.name} layer ({keys_per_step} keys), single thread"
+    return {
+        "impl": "reference",
+        "metric": "decode retrieval+sparse-attn keys scanned/s (also us/layer and % HBM roofline)",
+        "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.mean(per_step_s) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (two-cone Gaussian, host generator)",
+        "config": {"workload": w.name, "layers_per_step": 1},
+        "cpu_baseline": {"value": value, "unit": "keys/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    init_dist(world, local)
+    res, layers, w = run_gpu(args, rank, world, local)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            v, sample, cores = oracle_sample(w, args.cpu_budget_s, oracle_inputs_from_device(w, layers[0]))
+            res["cpu_baseline"] = {"value": v, "unit": "keys/s", "cores": cores, "kind": "oracle", "sample": sample}
+        else:
+            res["cpu_baseline"] = None
+        print(json.dumps(res), flush=True)
+    del layers
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

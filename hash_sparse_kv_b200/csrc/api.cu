@@ -1,0 +1,266 @@
+// C ABI entry points: argument checks on the host, then launches on the
+// caller's stream.  Nothing here allocates device memory or synchronizes,
+// except hkv_check.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "internal.h"
+
+namespace hkv {
+
+static thread_local std::string g_last_error;
+static std::atomic<int> g_debug_flags{0};
+static std::atomic<long long> g_wait_ns{0};
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_check(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return HKV_OK;
+  return fail(HKV_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+int debug_flags() { return g_debug_flags.load(); }
+
+uint64_t wait_limit_ns() {
+  const long long v = g_wait_ns.load();
+  return v > 0 ? (uint64_t)v : kDefaultWaitNs;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return 1;
+  return n;
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static int check_hash(const hkv_hash* h) {
+  if (h == nullptr) return fail(HKV_ERR_INVALID_ARG, "hash is NULL");
+  if (h->head_dim != kHeadDim) return fail(HKV_ERR_UNSUPPORTED, "head_dim %d (only 128)", h->head_dim);
+  if (h->dtype != HKV_F32 && h->dtype != HKV_BF16) return fail(HKV_ERR_INVALID_ARG, "dtype %d", h->dtype);
+  switch (h->kind) {
+    case HKV_HASH_LSH:
+      if (h->code_bits != 64 && h->code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "LSH code_bits %d (64 or 128)", h->code_bits);
+      if (h->R == nullptr) return fail(HKV_ERR_INVALID_ARG, "LSH projection R is NULL");
+      break;
+    case HKV_HASH_MLP:
+      if (h->code_bits != 64 && h->code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "MLP code_bits %d (64 or 128)", h->code_bits);
+      if (h->hidden < 1 || h->hidden > 1024) return fail(HKV_ERR_UNSUPPORTED, "MLP hidden %d (1..1024)", h->hidden);
+      if (!h->W1 || !h->b1 || !h->W2 || !h->b2) return fail(HKV_ERR_INVALID_ARG, "MLP weight pointer is NULL");
+      break;
+    case HKV_HASH_SIGN:
+      if (h->code_bits != h->head_dim) return fail(HKV_ERR_INVALID_ARG, "SIGN code_bits %d != head_dim", h->code_bits);
+      break;
+    default:
+      return fail(HKV_ERR_INVALID_ARG, "hash kind %d", h->kind);
+  }
+  return HKV_OK;
+}
+
+static int check_heads(int B, int Hq, int Hkv) {
+  if (B < 0 || Hq < 1 || Hkv < 1) return fail(HKV_ERR_INVALID_ARG, "B %d Hq %d Hkv %d", B, Hq, Hkv);
+  if (Hq % Hkv != 0) return fail(HKV_ERR_INVALID_ARG, "Hq %d not a multiple of Hkv %d", Hq, Hkv);
+  if (Hq / Hkv > 16) return fail(HKV_ERR_UNSUPPORTED, "group size %d > 16", Hq / Hkv);
+  return HKV_OK;
+}
+
+static int check_window(int64_t cap, int64_t N, int n_sink, int n_local, int top_k) {
+  if (N < 0 || cap < N) return fail(HKV_ERR_INVALID_ARG, "n_tokens %lld, cap %lld", (long long)N, (long long)cap);
+  if (N > INT32_MAX) return fail(HKV_ERR_UNSUPPORTED, "n_tokens %lld > 2^31-1", (long long)N);
+  if (n_sink < 0 || n_local < 0 || top_k < 0) return fail(HKV_ERR_INVALID_ARG, "negative sink/local/top_k");
+  return HKV_OK;
+}
+
+// Workspace of one decode step: [retrieval scratch][attention scratch]
+// [query codes][selected indices].  The two scratch areas are separate so
+// each keeps its own zero-on-exit invariant.
+struct DecodeLayout {
+  size_t retrieve, attend, qcodes, idx, total;
+};
+
+static int decode_layout(int B, int Hq, int Hkv, int64_t N, int code_bits, int top_k, int n_sink,
+                         int n_local, DecodeLayout& L) {
+  RetrieveShape rs{B, Hq, Hkv, code_bits / 32, N, N, n_sink, n_local, top_k};
+  AttendShape as{B, Hq, Hkv, HKV_BF16, N, N, top_k, n_sink, n_local};
+  L.retrieve = align_up(retrieve_ws_bytes(rs), 256);
+  if (L.retrieve == 0 && (int64_t)B * Hkv * top_k > 0) return HKV_ERR_UNSUPPORTED;
+  L.attend = align_up(attend_ws_bytes(as), 256);
+  L.qcodes = align_up(sizeof(uint32_t) * (size_t)B * Hq * (code_bits / 32), 256);
+  L.idx = align_up(sizeof(int32_t) * (size_t)B * Hkv * top_k, 256);
+  L.total = L.retrieve + L.attend + L.qcodes + L.idx;
+  return HKV_OK;
+}
+
+}  // namespace hkv
+
+using namespace hkv;
+
+extern "C" {
+
+const char* hkv_last_error(void) { return g_last_error.c_str(); }
+
+const char* hkv_version(void) { return "hkv 0.1 sm_100a"; }
+
+int hkv_debug_set(int flags, int64_t wait_limit_ns) {
+  g_debug_flags.store(flags);
+  g_wait_ns.store(wait_limit_ns);
+  return HKV_OK;
+}
+
+int hkv_check(int32_t* status, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = cuda_check(cudaStreamSynchronize(st), "hkv_check stream sync");
+  if (rc != HKV_OK) return rc;
+  if (status == nullptr) return HKV_OK;
+  int32_t v = 0;
+  rc = cuda_check(cudaMemcpyAsync(&v, status, sizeof(v), cudaMemcpyDeviceToHost, st), "hkv_check read");
+  if (rc == HKV_OK) rc = cuda_check(cudaMemsetAsync(status, 0, sizeof(int32_t), st), "hkv_check reset");
+  if (rc == HKV_OK) rc = cuda_check(cudaStreamSynchronize(st), "hkv_check sync");
+  if (rc != HKV_OK) return rc;
+  if (v != HKV_OK) fail(v, "device reported status %d", v);
+  return v;
+}
+
+int hkv_workspace_reset(void* ws, size_t ws_bytes, void* stream) {
+  if (ws_bytes == 0) return HKV_OK;
+  if (ws == nullptr) return fail(HKV_ERR_INVALID_ARG, "workspace is NULL");
+  return cuda_check(cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)), "workspace reset");
+}
+
+size_t hkv_workspace_bytes(int B, int Hq, int Hkv, int64_t n_tokens, int code_bits, int top_k,
+                           int n_sink, int n_local) {
+  if (check_heads(B, Hq, Hkv) != HKV_OK || check_window(n_tokens, n_tokens, n_sink, n_local, top_k) != HKV_OK)
+    return 0;
+  if (code_bits != 64 && code_bits != 128) return 0;
+  DecodeLayout L;
+  if (decode_layout(B, Hq, Hkv, n_tokens, code_bits, top_k, n_sink, n_local, L) != HKV_OK) return 0;
+  return L.total;
+}
+
+int hkv_encode_keys(const hkv_hash* hash, const void* x, int64_t rows, int64_t x_stride,
+                    uint32_t* codes, int64_t code_stride, uint16_t* norms, int32_t* status,
+                    void* stream) {
+  (void)status;
+  int rc = check_hash(hash);
+  if (rc != HKV_OK) return rc;
+  if (rows < 0) return fail(HKV_ERR_INVALID_ARG, "rows %lld", (long long)rows);
+  if (rows == 0) return HKV_OK;
+  const int W = hash->code_bits / 32;
+  if (!x || !codes) return fail(HKV_ERR_INVALID_ARG, "x or codes is NULL");
+  if (x_stride < hash->head_dim || code_stride < W) return fail(HKV_ERR_INVALID_ARG, "stride too small");
+  const size_t elt = hash->dtype == HKV_BF16 ? 2 : 4;
+  if (!aligned(x, 16) || (x_stride * elt) % 16 != 0) return fail(HKV_ERR_INVALID_ARG, "x rows must be 16-byte aligned");
+  if (hash->kind == HKV_HASH_LSH && !aligned(hash->R, 16)) return fail(HKV_ERR_INVALID_ARG, "R must be 16-byte aligned");
+  RowMap m{rows, rows, 0, x_stride, 0, code_stride, 0, 1};
+  return launch_encode(*hash, x, m, codes, hash->kind == HKV_HASH_SIGN ? norms : nullptr,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int hkv_append(const hkv_hash* hash, int B, int Hkv, int T, const void* k_new, const void* v_new,
+               void* K, void* V, uint32_t* codes, uint16_t* norms, int64_t capacity, int64_t pos,
+               int32_t* status, void* stream) {
+  (void)status;
+  int rc = check_hash(hash);
+  if (rc != HKV_OK) return rc;
+  if (B < 0 || Hkv < 1 || T < 0) return fail(HKV_ERR_INVALID_ARG, "B %d Hkv %d T %d", B, Hkv, T);
+  if (pos < 0 || pos + T > capacity) return fail(HKV_ERR_CAPACITY, "pos %lld + T %d > capacity %lld", (long long)pos, T, (long long)capacity);
+  if (B == 0 || T == 0) return HKV_OK;
+  if (!k_new || !v_new || !K || !V || !codes) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(K, 16) || !aligned(V, 16))
+    return fail(HKV_ERR_INVALID_ARG, "K/V buffers must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t groups = (int64_t)B * Hkv;
+  rc = launch_copy_rows(hash->dtype, groups, T, k_new, K, capacity, pos, st);
+  if (rc == HKV_OK) rc = launch_copy_rows(hash->dtype, groups, T, v_new, V, capacity, pos, st);
+  if (rc != HKV_OK) return rc;
+  const int W = hash->code_bits / 32;
+  RowMap m{groups * T, T, (int64_t)T * hash->head_dim, hash->head_dim, capacity * W, W, capacity, 1};
+  uint16_t* nrm = (hash->kind == HKV_HASH_SIGN && norms) ? norms + pos : nullptr;
+  return launch_encode(*hash, k_new, m, codes + pos * W, nrm, st);
+}
+
+int hkv_retrieve_topk(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                      const uint32_t* k_codes, int64_t cap, int64_t n_tokens, int n_sink,
+                      int n_local, int top_k, int32_t* idx, int32_t* dist, void* ws,
+                      size_t ws_bytes, int32_t* status, void* stream) {
+  int rc = check_heads(B, Hq, Hkv);
+  if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
+  if (rc != HKV_OK) return rc;
+  if (code_bits != 64 && code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "code_bits %d (64 or 128)", code_bits);
+  if (B == 0 || top_k == 0) return HKV_OK;
+  if (!q_codes || !k_codes || !idx) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_codes, code_bits / 8)) return fail(HKV_ERR_INVALID_ARG, "k_codes must be %d-byte aligned", code_bits / 8);
+  RetrieveShape s{B, Hq, Hkv, code_bits / 32, cap, n_tokens, n_sink, n_local, top_k};
+  return launch_retrieve(s, q_codes, k_codes, idx, dist, ws, ws_bytes, status, static_cast<cudaStream_t>(stream));
+}
+
+int hkv_sparse_attend(int B, int Hq, int Hkv, int dtype, const void* q, const void* K,
+                      const void* V, int64_t cap, int64_t n_tokens, const int32_t* idx,
+                      int top_k, int n_sink, int n_local, float scale, float* out, float* lse,
+                      void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  int rc = check_heads(B, Hq, Hkv);
+  if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
+  if (rc != HKV_OK) return rc;
+  if (dtype != HKV_F32 && dtype != HKV_BF16) return fail(HKV_ERR_INVALID_ARG, "dtype %d", dtype);
+  if (!std::isfinite(scale)) return fail(HKV_ERR_INVALID_ARG, "scale is not finite");
+  if (B == 0) return HKV_OK;
+  if (!q || !K || !V || !out || (top_k > 0 && !idx)) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16))
+    return fail(HKV_ERR_INVALID_ARG, "q, K, V and out must be 16-byte aligned");
+  AttendShape s{B, Hq, Hkv, dtype, cap, n_tokens, top_k, n_sink, n_local};
+  return launch_attend(s, q, K, V, idx, scale, out, lse, ws, ws_bytes, status, static_cast<cudaStream_t>(stream));
+}
+
+int hkv_lse_merge(int rows, int d, const float* o1, const float* lse1, const float* o2,
+                  const float* lse2, float* out, float* lse_out, void* stream) {
+  if (rows < 0 || d < 1) return fail(HKV_ERR_INVALID_ARG, "rows %d d %d", rows, d);
+  if (rows == 0) return HKV_OK;
+  if (!o1 || !lse1 || !o2 || !lse2 || !out) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  return launch_lse_merge(rows, d, o1, lse1, o2, lse2, out, lse_out, static_cast<cudaStream_t>(stream));
+}
+
+int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
+                    const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
+                    int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
+                    uint32_t* q_codes, int32_t* idx, float* out, float* lse, void* ws,
+                    size_t ws_bytes, int32_t* status, void* stream) {
+  int rc = check_hash(q_hash);
+  if (rc == HKV_OK) rc = check_heads(B, Hq, Hkv);
+  if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
+  if (rc != HKV_OK) return rc;
+  if (B == 0) return HKV_OK;
+  if (!q || !k_codes || !K || !V || !out) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  DecodeLayout L;
+  rc = decode_layout(B, Hq, Hkv, n_tokens, q_hash->code_bits, top_k, n_sink, n_local, L);
+  if (rc != HKV_OK) return fail(rc, "unsupported decode shape");
+  if (ws == nullptr || ws_bytes < L.total) return fail(HKV_ERR_CAPACITY, "workspace of %zu bytes, %zu needed", ws_bytes, L.total);
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  void* ws_r = base;
+  void* ws_a = base + L.retrieve;
+  uint32_t* qc = q_codes ? q_codes : reinterpret_cast<uint32_t*>(base + L.retrieve + L.attend);
+  int32_t* ix = idx ? idx : reinterpret_cast<int32_t*>(base + L.retrieve + L.attend + L.qcodes);
+  const int W = q_hash->code_bits / 32;
+  rc = hkv_encode_keys(q_hash, q, (int64_t)B * Hq, q_hash->head_dim, qc, W, nullptr, status, stream);
+  if (rc == HKV_OK)
+    rc = hkv_retrieve_topk(B, Hq, Hkv, q_hash->code_bits, qc, k_codes, cap, n_tokens, n_sink, n_local, top_k, ix,
+                           nullptr, ws_r, L.retrieve, status, stream);
+  if (rc == HKV_OK)
+    rc = hkv_sparse_attend(B, Hq, Hkv, q_hash->dtype, q, K, V, cap, n_tokens, ix, top_k, n_sink, n_local, scale,
+                           out, lse, ws_a, L.attend, status, stream);
+  return rc;
+}
+
+}  // extern "C"

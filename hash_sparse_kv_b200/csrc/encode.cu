@@ -1,0 +1,299 @@
+// Hash encoders: vectors -> packed sign codes.
+//
+//   LSH  (HashEvict, "Abstract"): bit j = [ (R x)_j > 0 ], R Gaussian [bits, d]
+//   MLP  (Spotlight Attention, "Approach"): bit j = [ (W2 SiLU(W1 x + b1) + b2)_j > 0 ]
+//   SIGN (Self-Indexing KVCache, "Abstract"): bit i = [ x_i > 0 ], plus ||x||_2 as fp16
+//
+// Bits are packed least-significant first: bit j -> word j / 32, position j % 32.
+// In the projection kernels lane l of a warp owns bits {l + 32 i}, so word i of
+// a row is exactly the warp ballot of (y_{l + 32 i} > 0).
+#include <cstdio>
+
+#include "internal.h"
+
+namespace hkv {
+namespace {
+
+constexpr int kThreads = 256;
+
+// ---------------------------------------------------------------- LSH -----
+// Tile of 64 rows per pass; warp w owns rows [8w, 8w + 8); lane l owns bits
+// {l + 32 i : i < BITS / 32}.  R^T and the x tile (transposed) sit in shared
+// memory as fp32; products and sums are fp32.
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreads, 2)
+lsh_encode_kernel(const T* __restrict__ x, const T* __restrict__ R, RowMap m,
+                  uint32_t* __restrict__ codes) {
+  constexpr int D = kHeadDim, ROWS = 64, TB = BITS / 32, XP = ROWS + 4;
+  extern __shared__ __align__(16) float smem[];
+  float* RT = smem;          // [D][BITS]
+  float* xT = RT + D * BITS;  // [D][XP]
+  for (int i = threadIdx.x; i < BITS * D; i += kThreads) {
+    const int j = i % BITS, k = i / BITS;
+    RT[k * BITS + j] = to_f32(R[(int64_t)j * D + k]);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ntiles = (m.rows + ROWS - 1) / ROWS;
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int64_t r0 = tile * ROWS;
+    __syncthreads();
+    for (int i = threadIdx.x; i < ROWS * (D / 4); i += kThreads) {
+      const int r = i / (D / 4), k4 = (i % (D / 4)) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r0 + r < m.rows) v = load4_f32(x + m.x_off(r0 + r) + k4);
+      xT[(k4 + 0) * XP + r] = v.x;
+      xT[(k4 + 1) * XP + r] = v.y;
+      xT[(k4 + 2) * XP + r] = v.z;
+      xT[(k4 + 3) * XP + r] = v.w;
+    }
+    __syncthreads();
+    float acc[8][TB];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int i = 0; i < TB; ++i) acc[r][i] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < D; ++k) {
+      const float4 xa = *reinterpret_cast<const float4*>(&xT[k * XP + warp * 8]);
+      const float4 xb = *reinterpret_cast<const float4*>(&xT[k * XP + warp * 8 + 4]);
+      const float xr[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+      for (int i = 0; i < TB; ++i) {
+        const float rv = RT[k * BITS + lane + 32 * i];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[r][i] = fmaf(xr[r], rv, acc[r][i]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int64_t row = r0 + warp * 8 + r;
+#pragma unroll
+      for (int i = 0; i < TB; ++i) {
+        const uint32_t word = __ballot_sync(0xffffffffu, acc[r][i] > 0.f);
+        if (lane == i && row < m.rows) codes[m.c_off(row) + i] = word;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- MLP -----
+// Tile of 32 rows; warp w owns rows [4w, 4w + 4).  The hidden layer is
+// processed in chunks of 64 units: z = W1 x + b1 (lane l: units l, l + 32),
+// h = SiLU(z), then y += W2[:, chunk] h (lane l: bits l + 32 i).  fp32 throughout.
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreads, 1)
+mlp_encode_kernel(const T* __restrict__ x, const float* __restrict__ W1,
+                  const float* __restrict__ b1, const float* __restrict__ W2,
+                  const float* __restrict__ b2, int hidden, RowMap m,
+                  uint32_t* __restrict__ codes) {
+  constexpr int D = kHeadDim, ROWS = 32, HC = 64, TB = BITS / 32;
+  constexpr int XP = ROWS + 4, W1P = HC + 1, HP = HC + 1, W2P = BITS + 1;
+  extern __shared__ __align__(16) float smem[];
+  float* xT = smem;               // [D][XP]
+  float* W1T = xT + D * XP;       // [D][W1P]
+  float* hs = W1T + D * W1P;      // [ROWS][HP]
+  float* W2T = hs + ROWS * HP;    // [HC][W2P]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ntiles = (m.rows + ROWS - 1) / ROWS;
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int64_t r0 = tile * ROWS;
+    __syncthreads();
+    for (int i = threadIdx.x; i < ROWS * (D / 4); i += kThreads) {
+      const int r = i / (D / 4), k4 = (i % (D / 4)) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r0 + r < m.rows) v = load4_f32(x + m.x_off(r0 + r) + k4);
+      xT[(k4 + 0) * XP + r] = v.x;
+      xT[(k4 + 1) * XP + r] = v.y;
+      xT[(k4 + 2) * XP + r] = v.z;
+      xT[(k4 + 3) * XP + r] = v.w;
+    }
+    float y[4][TB];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int i = 0; i < TB; ++i) y[r][i] = 0.f;
+    for (int u0 = 0; u0 < hidden; u0 += HC) {
+      const int hc = min(HC, hidden - u0);
+      __syncthreads();
+      for (int i = threadIdx.x; i < HC * D; i += kThreads) {
+        const int u = i / D, k = i % D;
+        W1T[k * W1P + u] = u < hc ? W1[(int64_t)(u0 + u) * D + k] : 0.f;
+      }
+      for (int i = threadIdx.x; i < BITS * HC; i += kThreads) {
+        const int j = i / HC, u = i % HC;
+        W2T[u * W2P + j] = u < hc ? W2[(int64_t)j * hidden + u0 + u] : 0.f;
+      }
+      __syncthreads();
+      float z[4][2];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) z[r][0] = z[r][1] = 0.f;
+#pragma unroll 4
+      for (int k = 0; k < D; ++k) {
+        const float4 xv = *reinterpret_cast<const float4*>(&xT[k * XP + warp * 4]);
+        const float wa = W1T[k * W1P + lane], wb = W1T[k * W1P + lane + 32];
+        z[0][0] = fmaf(xv.x, wa, z[0][0]); z[0][1] = fmaf(xv.x, wb, z[0][1]);
+        z[1][0] = fmaf(xv.y, wa, z[1][0]); z[1][1] = fmaf(xv.y, wb, z[1][1]);
+        z[2][0] = fmaf(xv.z, wa, z[2][0]); z[2][1] = fmaf(xv.z, wb, z[2][1]);
+        z[3][0] = fmaf(xv.w, wa, z[3][0]); z[3][1] = fmaf(xv.w, wb, z[3][1]);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int u = lane + 32 * c;
+          float h = 0.f;
+          if (u < hc) {
+            const float zz = z[r][c] + b1[u0 + u];
+            h = zz / (1.f + expf(-zz));
+          }
+          hs[(warp * 4 + r) * HP + u] = h;
+        }
+      __syncthreads();
+#pragma unroll 4
+      for (int u = 0; u < HC; ++u) {
+        const float h0 = hs[(warp * 4 + 0) * HP + u], h1 = hs[(warp * 4 + 1) * HP + u];
+        const float h2 = hs[(warp * 4 + 2) * HP + u], h3 = hs[(warp * 4 + 3) * HP + u];
+#pragma unroll
+        for (int i = 0; i < TB; ++i) {
+          const float w = W2T[u * W2P + lane + 32 * i];
+          y[0][i] = fmaf(h0, w, y[0][i]);
+          y[1][i] = fmaf(h1, w, y[1][i]);
+          y[2][i] = fmaf(h2, w, y[2][i]);
+          y[3][i] = fmaf(h3, w, y[3][i]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int64_t row = r0 + warp * 4 + r;
+#pragma unroll
+      for (int i = 0; i < TB; ++i) {
+        const uint32_t word = __ballot_sync(0xffffffffu, y[r][i] + b2[lane + 32 * i] > 0.f);
+        if (lane == i && row < m.rows) codes[m.c_off(row) + i] = word;
+      }
+    }
+  }
+}
+
+// --------------------------------------------------------------- SIGN -----
+// One warp per row: lane l reads elements l + 32 i, so word i is the ballot
+// of (x_{l + 32 i} > 0).  The norm is summed in fp64 (bf16 and fp32 squares
+// are exact there), square-rooted in fp64 and rounded once to fp16.
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+sign_encode_kernel(const T* __restrict__ x, RowMap m, uint32_t* __restrict__ codes,
+                   uint16_t* __restrict__ norms) {
+  constexpr int D = kHeadDim, TB = D / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+  for (int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); row < m.rows;
+       row += warps) {
+    const T* px = x + m.x_off(row);
+    double ss = 0.0;
+#pragma unroll
+    for (int i = 0; i < TB; ++i) {
+      const float v = to_f32(px[lane + 32 * i]);
+      ss += (double)v * (double)v;
+      const uint32_t word = __ballot_sync(0xffffffffu, v > 0.f);
+      if (lane == i) codes[m.c_off(row) + i] = word;
+    }
+    if (norms != nullptr) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if (lane == 0) norms[m.n_off(row)] = __half_as_ushort(__double2half(sqrt(ss)));
+    }
+  }
+}
+
+// ------------------------------------------------------------ row copy -----
+// dst[(g * dst_group_rows + dst_row0 + t) * D + c] = src[(g * T + t) * D + c]
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+copy_rows_kernel(const T* __restrict__ src, T* __restrict__ dst, int64_t groups, int64_t Trows,
+                 int64_t dst_group_rows, int64_t dst_row0) {
+  constexpr int D = kHeadDim, V = 16 / sizeof(T);
+  const int64_t total = groups * Trows * (D / V);
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * kThreads) {
+    const int64_t row = i / (D / V), c = (i % (D / V)) * V;
+    const int64_t g = row / Trows, t = row % Trows;
+    const uint4 v = *reinterpret_cast<const uint4*>(src + row * D + c);
+    *reinterpret_cast<uint4*>(dst + ((g * dst_group_rows + dst_row0 + t) * D + c)) = v;
+  }
+}
+
+template <typename K>
+int grid_for(K kernel, size_t smem, int64_t work_items) {
+  int per_sm = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
+  if (per_sm < 1) per_sm = 1;
+  int64_t g = (int64_t)sm_count() * per_sm;
+  if (work_items < g) g = work_items;
+  return (int)(g < 1 ? 1 : g);
+}
+
+template <typename T, int BITS>
+int run_lsh(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, cudaStream_t st) {
+  auto kernel = lsh_encode_kernel<T, BITS>;
+  const size_t smem = sizeof(float) * (kHeadDim * BITS + kHeadDim * 68);
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_check(e, "lsh encode smem attribute");
+  const int grid = grid_for(kernel, smem, (m.rows + 63) / 64);
+  kernel<<<grid, kThreads, smem, st>>>(static_cast<const T*>(x), static_cast<const T*>(h.R), m, codes);
+  return cuda_check(cudaGetLastError(), "lsh encode launch");
+}
+
+template <typename T, int BITS>
+int run_mlp(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, cudaStream_t st) {
+  auto kernel = mlp_encode_kernel<T, BITS>;
+  const size_t smem = sizeof(float) * (kHeadDim * 36 + kHeadDim * 65 + 32 * 65 + 64 * (BITS + 1));
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_check(e, "mlp encode smem attribute");
+  const int grid = grid_for(kernel, smem, (m.rows + 31) / 32);
+  kernel<<<grid, kThreads, smem, st>>>(static_cast<const T*>(x), h.W1, h.b1, h.W2, h.b2, h.hidden, m, codes);
+  return cuda_check(cudaGetLastError(), "mlp encode launch");
+}
+
+template <typename T>
+int run_sign(const void* x, const RowMap& m, uint32_t* codes, uint16_t* norms, cudaStream_t st) {
+  auto kernel = sign_encode_kernel<T>;
+  const int grid = grid_for(kernel, 0, (m.rows + 7) / 8);
+  kernel<<<grid, kThreads, 0, st>>>(static_cast<const T*>(x), m, codes, norms);
+  return cuda_check(cudaGetLastError(), "sign encode launch");
+}
+
+}  // namespace
+
+int launch_encode(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes,
+                  uint16_t* norms, cudaStream_t st) {
+  if (m.rows == 0) return HKV_OK;
+  const bool bf = h.dtype == HKV_BF16;
+  switch (h.kind) {
+    case HKV_HASH_LSH:
+      if (h.code_bits == 128) return bf ? run_lsh<__nv_bfloat16, 128>(h, x, m, codes, st) : run_lsh<float, 128>(h, x, m, codes, st);
+      return bf ? run_lsh<__nv_bfloat16, 64>(h, x, m, codes, st) : run_lsh<float, 64>(h, x, m, codes, st);
+    case HKV_HASH_MLP:
+      if (h.code_bits == 128) return bf ? run_mlp<__nv_bfloat16, 128>(h, x, m, codes, st) : run_mlp<float, 128>(h, x, m, codes, st);
+      return bf ? run_mlp<__nv_bfloat16, 64>(h, x, m, codes, st) : run_mlp<float, 64>(h, x, m, codes, st);
+    case HKV_HASH_SIGN:
+      return bf ? run_sign<__nv_bfloat16>(x, m, codes, norms, st) : run_sign<float>(x, m, codes, norms, st);
+  }
+  return fail(HKV_ERR_INVALID_ARG, "unknown hash kind %d", h.kind);
+}
+
+int launch_copy_rows(int dtype, int64_t groups, int64_t T, const void* src, void* dst,
+                     int64_t dst_group_rows, int64_t dst_row0, cudaStream_t st) {
+  const int64_t items = groups * T * (dtype == HKV_BF16 ? 16 : 32);
+  if (items == 0) return HKV_OK;
+  int64_t grid = (items + kThreads - 1) / kThreads;
+  if (grid > 4L * sm_count()) grid = 4L * sm_count();
+  if (dtype == HKV_BF16)
+    copy_rows_kernel<__nv_bfloat16><<<(int)grid, kThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst), groups, T, dst_group_rows, dst_row0);
+  else
+    copy_rows_kernel<float><<<(int)grid, kThreads, 0, st>>>(
+        static_cast<const float*>(src), static_cast<float*>(dst), groups, T, dst_group_rows, dst_row0);
+  return cuda_check(cudaGetLastError(), "append copy launch");
+}
+
+}  // namespace hkv

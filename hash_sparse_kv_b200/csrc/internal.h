@@ -1,0 +1,70 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "hkv.h"
+
+namespace hkv {
+
+// Records a printf-style message for hkv_last_error() and returns `code`.
+int fail(int code, const char* fmt, ...);
+// HKV_ERR_CUDA with the CUDA error string, or HKV_OK for cudaSuccess.
+int cuda_check(cudaError_t e, const char* where);
+
+int debug_flags();
+uint64_t wait_limit_ns();
+int sm_count();
+
+constexpr int kDebugSkipArrive = 1;
+
+// ---- encoders (encode.cu) ----
+int launch_encode(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes,
+                  uint16_t* norms, cudaStream_t st);
+int launch_copy_rows(int dtype, int64_t groups, int64_t T, const void* src, void* dst,
+                     int64_t dst_group_rows, int64_t dst_row0, cudaStream_t st);
+
+// ---- retrieval (retrieve.cu) ----
+struct RetrieveShape {
+  int B, Hq, Hkv, words;
+  int64_t cap, N;
+  int n_sink, n_local, top_k;
+};
+size_t retrieve_ws_bytes(const RetrieveShape& s);
+int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,
+                    int32_t* idx, int32_t* dist, void* ws, size_t ws_bytes, int32_t* status,
+                    cudaStream_t st);
+
+// ---- attention (attend.cu) ----
+struct AttendShape {
+  int B, Hq, Hkv, dtype;
+  int64_t cap, N;
+  int top_k, n_sink, n_local;
+};
+size_t attend_ws_bytes(const AttendShape& s);
+int launch_attend(const AttendShape& s, const void* q, const void* K, const void* V,
+                  const int32_t* idx, float scale, float* out, float* lse, void* ws,
+                  size_t ws_bytes, int32_t* status, cudaStream_t st);
+int launch_lse_merge(int rows, int d, const float* o1, const float* lse1, const float* o2,
+                     const float* lse2, float* out, float* lse_out, cudaStream_t st);
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+// Candidate window shared by retrieval and attention.
+struct Window {
+  int64_t sink_end, local_start, C;
+};
+inline Window window(int64_t N, int64_t n_sink, int64_t n_local) {
+  Window w;
+  w.sink_end = n_sink < N ? n_sink : N;
+  int64_t ls = N - n_local;
+  w.local_start = ls > w.sink_end ? ls : w.sink_end;
+  w.C = w.local_start - w.sink_end;
+  return w;
+}
+
+}  // namespace hkv

@@ -1,0 +1,218 @@
+/*
+ * hkv.h -- C ABI of the B200 hash-code KV retrieval library.
+ *
+ * The library implements the decode-time path shared by these pages:
+ *   - Spotlight Attention: Towards Efficient LLM Generation via Non-linear
+ *     Hashing-based KV Cache Retrieval ("Approach", "Key results"): keys and
+ *     queries hashed to short binary codes (sign of a two-layer MLP), top-k
+ *     keys retrieved per decode step, exact attention over only those keys,
+ *     sink and local-window tokens kept.
+ *   - HashEvict: A Pre-Attention KV Cache Eviction Strategy using
+ *     Locality-Sensitive Hashing ("Abstract"): codes are signs of Gaussian
+ *     projections, scored by Hamming distance against a binary structure
+ *     kept in GPU memory, updated at every decoding step.
+ *   - Self-Indexing KVCache: Predicting Sparse Attention from Compressed Keys
+ *     ("Abstract"): sign(k) as a 1-bit code that is both storage and index.
+ *   - RetrievalAttention: Accelerating Long-Context LLM Inference via Vector
+ *     Retrieval ("Summary", "Approach"): a resident sink/window partial and
+ *     the retrieved partial merged by exact log-sum-exp rescaling.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer is a DEVICE pointer owned by the caller, unless stated.
+ *     The library keeps no pointer after a call returns and allocates no
+ *     device memory; scratch comes from the caller's workspace `ws`.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and never synchronizes, except hkv_check.
+ *   - Return value: HKV_OK or a negative hkv_status.  Argument errors are
+ *     caught on the host before any launch; hkv_last_error() then describes
+ *     the failure (thread-local string, valid until the next call on the
+ *     same thread).
+ *   - Errors found on the device (an index out of range, a wait that ran out
+ *     of time) are written to the caller's int32 status word `status`
+ *     (device memory, start at 0): the first error wins, later ones are
+ *     dropped.  Read it with hkv_check.
+ *   - Layouts are dense row-major with the strides stated.  Codes are uint32
+ *     words; bit j of a code is 1 iff the j-th pre-sign value is > 0, stored
+ *     in word j / 32 at bit position j % 32.
+ *   - Sequences in a batch share n_tokens (N).  Candidates for retrieval are
+ *     the tokens [sink_end, local_start) with sink_end = min(n_sink, N) and
+ *     local_start = max(sink_end, N - n_local); sink tokens [0, sink_end) and
+ *     local tokens [local_start, N) are always attended.
+ */
+#ifndef HKV_H
+#define HKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HKV_OK = 0,
+  HKV_ERR_INVALID_ARG = -1,  /* bad pointer, size, stride or alignment */
+  HKV_ERR_UNSUPPORTED = -2,  /* valid but not implemented (e.g. head_dim != 128) */
+  HKV_ERR_CAPACITY = -3,     /* pos + T > capacity, or workspace too small */
+  HKV_ERR_CUDA = -4,         /* a CUDA runtime call failed */
+  HKV_ERR_TIMEOUT = -5,      /* device: a cross-block wait ran out of time */
+  HKV_ERR_DEVICE_RANGE = -6  /* device: an index outside [0, n_tokens) was skipped */
+} hkv_status;
+
+typedef enum { HKV_F32 = 0, HKV_BF16 = 1 } hkv_dtype;
+
+typedef enum {
+  HKV_HASH_LSH = 0,  /* code = sign(R x), R [code_bits, head_dim] Gaussian (HashEvict) */
+  HKV_HASH_MLP = 1,  /* code = sign(W2 SiLU(W1 x + b1) + b2) (Spotlight Attention) */
+  HKV_HASH_SIGN = 2  /* code = sign(x), code_bits == head_dim (Self-Indexing KVCache) */
+} hkv_hash_kind;
+
+/* One hash function.  Queries and keys may use different ones (the MLP hash
+ * has separate query and key networks).  All pointers are device pointers.
+ *   kind       hkv_hash_kind
+ *   head_dim   d; 128 is the supported value
+ *   code_bits  64 or 128 for LSH and MLP; equal to head_dim for SIGN
+ *   hidden     MLP hidden width (1..1024; 512 in the Spotlight setting), 0 otherwise
+ *   dtype      hkv_dtype of the hashed vectors x (and of R)
+ *   R          LSH: [code_bits, head_dim] in `dtype`, row-major
+ *   W1, b1     MLP: [hidden, head_dim], [hidden] fp32
+ *   W2, b2     MLP: [code_bits, hidden], [code_bits] fp32
+ * For bit-exact agreement with an fp64 reference, R (bf16 inputs) and the MLP
+ * weights should hold bf16-representable values and no pre-sign value should
+ * lie within 1e-3 of zero. */
+typedef struct {
+  int32_t kind;
+  int32_t head_dim;
+  int32_t code_bits;
+  int32_t hidden;
+  int32_t dtype;
+  int32_t reserved;
+  const void* R;
+  const float* W1;
+  const float* b1;
+  const float* W2;
+  const float* b2;
+} hkv_hash;
+
+/* Description of the last host-side error on this thread ("" if none). */
+const char* hkv_last_error(void);
+
+/* Library version string, e.g. "hkv 0.1 sm_100a". */
+const char* hkv_version(void);
+
+/* Synchronizes `stream`, reads the device status word, resets it to 0 and
+ * returns the value read (HKV_OK, HKV_ERR_TIMEOUT or HKV_ERR_DEVICE_RANGE),
+ * or HKV_ERR_CUDA if the stream reported a CUDA error. */
+int hkv_check(int32_t* status, void* stream);
+
+/* Bytes of workspace that hkv_retrieve_topk, hkv_sparse_attend and
+ * hkv_decode_step need for this shape on the current device (0 if the shape
+ * is invalid or unsupported).  The workspace
+ * must be zero-filled once before first use (hkv_workspace_reset); every call
+ * leaves it zero-filled again, including calls that end in a device error.
+ * Calls that share one workspace must not overlap on the GPU. */
+size_t hkv_workspace_bytes(int B, int Hq, int Hkv, int64_t n_tokens, int code_bits, int top_k,
+                           int n_sink, int n_local);
+
+/* cudaMemsetAsync(ws, 0, ws_bytes, stream). */
+int hkv_workspace_reset(void* ws, size_t ws_bytes, void* stream);
+
+/* Encode `rows` vectors into codes (S1 for keys at prefill, S2 for queries).
+ * Spotlight Attention "Approach"; HashEvict "Abstract"; Self-Indexing KVCache
+ * "Abstract".
+ *   x          rows x head_dim in hash->dtype; row r starts at x + r * x_stride
+ *              elements (x_stride >= head_dim; 16-byte aligned rows)
+ *   codes      row r written at codes + r * code_stride (uint32 words;
+ *              code_stride >= code_bits / 32)
+ *   norms      SIGN only, nullable: fp16 bit patterns of ||x_r||_2, row r at
+ *              norms[r] (computed in fp64, rounded to nearest even)
+ * rows == 0 is a no-op. */
+int hkv_encode_keys(const hkv_hash* hash, const void* x, int64_t rows, int64_t x_stride,
+                    uint32_t* codes, int64_t code_stride, uint16_t* norms,
+                    int32_t* status, void* stream);
+
+/* Decode-time append (S3; HashEvict "Abstract": the binary structure is
+ * updated at every decoding step): copy T new key/value rows per (batch, KV
+ * head) into the cache at token positions [pos, pos + T) and encode the new
+ * keys into `codes` (and `norms` for SIGN).
+ *   k_new, v_new  [B, Hkv, T, head_dim] in hash->dtype
+ *   K, V          [B, Hkv, capacity, head_dim] in hash->dtype
+ *   codes         [B, Hkv, capacity, code_bits / 32]
+ *   norms         SIGN only, nullable: [B, Hkv, capacity] fp16 bits
+ * Returns HKV_ERR_CAPACITY if pos < 0 or pos + T > capacity. */
+int hkv_append(const hkv_hash* hash, int B, int Hkv, int T, const void* k_new, const void* v_new,
+               void* K, void* V, uint32_t* codes, uint16_t* norms, int64_t capacity, int64_t pos,
+               int32_t* status, void* stream);
+
+/* Hamming scan + top-k (S4, S5).  HashEvict "Abstract" (Hamming distance of
+ * binarized projections); Spotlight Attention "Approach" (top-k retrieval).
+ * For KV head j of batch b the score of token t is
+ *   D(t) = sum over the g = Hq / Hkv query heads h of that KV head of
+ *          popcount(q_code[b, h] XOR k_code[b, j, t]),
+ * and the k_eff = min(top_k, candidates) candidates with the smallest D are
+ * selected, ties to the lowest t.
+ *   q_codes  [B, Hq, code_bits / 32]
+ *   k_codes  [B, Hkv, cap, code_bits / 32]; only rows < n_tokens are read
+ *   idx      [B, Hkv, top_k] int32: selected tokens in ascending order, then -1
+ *   dist     nullable [B, Hkv, top_k] int32: D of each selected token, then -1
+ * code_bits is 64 or 128; Hq % Hkv == 0, Hq / Hkv <= 16.  Cross-block waits
+ * are bounded; on expiry the status word gets HKV_ERR_TIMEOUT. */
+int hkv_retrieve_topk(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                      const uint32_t* k_codes, int64_t cap, int64_t n_tokens, int n_sink,
+                      int n_local, int top_k, int32_t* idx, int32_t* dist, void* ws,
+                      size_t ws_bytes, int32_t* status, void* stream);
+
+/* Sparse attention over sink + selected + local rows, with the log-sum-exp
+ * merge of the partials (S6, S7, S8).  Spotlight Attention "Approach" (exact
+ * attention over the retrieved tokens); RetrievalAttention "Approach" (exact
+ * log-sum-exp rescaling of partial attention).
+ * For query head h (KV head j = h / g):
+ *   out[b, h] = sum_t softmax_t(scale * q[b, h] . K[b, j, t]) V[b, j, t]
+ *   lse[b, h] = log sum_t exp(scale * q[b, h] . K[b, j, t])
+ * over t in [0, sink_end) + {idx[b, j, i] >= 0} + [local_start, n_tokens).
+ *   q       [B, Hq, 128] in dtype;  K, V  [B, Hkv, cap, 128] in dtype
+ *   idx     [B, Hkv, top_k] int32 (-1 entries are skipped; entries outside
+ *           [0, n_tokens) are skipped and reported as HKV_ERR_DEVICE_RANGE)
+ *   out     [B, Hq, 128] fp32;  lse  nullable [B, Hq] fp32
+ * The selected indices must not repeat a sink or local token. */
+int hkv_sparse_attend(int B, int Hq, int Hkv, int dtype, const void* q, const void* K,
+                      const void* V, int64_t cap, int64_t n_tokens, const int32_t* idx,
+                      int top_k, int n_sink, int n_local, float scale, float* out, float* lse,
+                      void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
+/* Elementwise log-sum-exp merge of two partial attention results (S8 alone).
+ * RetrievalAttention "Approach".  For each of `rows` rows:
+ *   m = max(lse1, lse2), w_i = exp(lse_i - m)
+ *   out = (w1 o1 + w2 o2) / (w1 + w2), lse_out = m + log(w1 + w2)
+ * A part with lse = -inf is empty; two empty parts give out = 0, lse = -inf.
+ *   o1, o2, out  [rows, d] fp32;  lse1, lse2, lse_out  [rows] fp32 */
+int hkv_lse_merge(int rows, int d, const float* o1, const float* lse1, const float* o2,
+                  const float* lse2, float* out, float* lse_out, void* stream);
+
+/* One whole decode step in one launch: encode the query heads with q_hash,
+ * scan + select, attend + merge (S2, S4-S8).  Results equal hkv_encode_keys
+ * on q, then hkv_retrieve_topk, then hkv_sparse_attend: q_codes and idx
+ * bit-identical, out and lse within floating-point rounding.
+ *   q_hash   hash for the queries (q_hash->dtype is the dtype of q, K, V)
+ *   q        [B, Hq, 128];  k_codes [B, Hkv, cap, code_bits / 32]
+ *   K, V     [B, Hkv, cap, 128]
+ *   q_codes  nullable [B, Hq, code_bits / 32] out
+ *   idx      nullable [B, Hkv, top_k] out
+ *   out      [B, Hq, 128] fp32;  lse nullable [B, Hq] fp32 */
+int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
+                    const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
+                    int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
+                    uint32_t* q_codes, int32_t* idx, float* out, float* lse, void* ws,
+                    size_t ws_bytes, int32_t* status, void* stream);
+
+/* Testing aid (process-wide).  flags bit 0: in the next retrieval launches,
+ * block 0 does not signal its arrival at the cross-block wait, so the wait
+ * runs out and reports HKV_ERR_TIMEOUT.  wait_limit_ns: limit of every
+ * cross-block wait (0 restores the default of 2 s). */
+int hkv_debug_set(int flags, int64_t wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HKV_H */

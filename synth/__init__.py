@@ -148,12 +148,14 @@ def cone_rows(seed: int, layer: int, tensor: int, mu: np.ndarray, n_rows: int, d
     t = _store(x, dtype)
     if bad_rows is None:
         return t
+    bad = np.flatnonzero(bad_rows(t))
     for attempt in range(1, max_attempts + 1):
-        bad = np.flatnonzero(bad_rows(t))
         if bad.size == 0:
             return t
         z = _rng(seed, layer, tensor, _REDRAW_BASE + attempt, 0).standard_normal((bad.size, d), dtype=np.float32)
-        t[torch.from_numpy(bad)] = _store(mu.astype(np.float32) + np.float32(0.3) * z, dtype)
+        rows = torch.from_numpy(bad)
+        t[rows] = _store(mu.astype(np.float32) + np.float32(0.3) * z, dtype)
+        bad = bad[np.asarray(bad_rows(t[rows]), dtype=bool)]
     raise RuntimeError(f"margin redraw did not converge for tensor {tensor}")
 
 

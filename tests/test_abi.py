@@ -1,0 +1,69 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol that
+include/hkv.h declares, and rejects bad arguments on the host."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hash_sparse_kv_b200 as hkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "hkv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hkv_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(hkv.lib_path):
+        from hash_sparse_kv_b200 import build
+        build.build()
+    return hkv.lib()
+
+
+def test_header_declares_the_bound_api():
+    assert _declared() == sorted(hkv.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_version(lib):
+    assert "sm_100a" in hkv.hkv_version()
+
+
+def test_host_side_argument_errors(lib):
+    h = hkv.hkv_hash(hkv.HKV_HASH_LSH, 64, 128, 0, hkv.HKV_BF16, 0, None, None, None, None, None)
+    rc = lib.hkv_encode_keys(ctypes.byref(h), None, 10, 128, None, 4, None, None, None)
+    assert rc == hkv.HKV_ERR_UNSUPPORTED and "head_dim" in hkv.hkv_last_error()
+    h.head_dim = 128
+    rc = lib.hkv_encode_keys(ctypes.byref(h), None, 10, 128, None, 4, None, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG  # R is NULL
+    rc = lib.hkv_encode_keys(None, None, 10, 128, None, 4, None, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG
+    rc = lib.hkv_retrieve_topk(1, 6, 4, 128, None, None, 10, 10, 0, 0, 4, None, None, None, 0, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG and "multiple" in hkv.hkv_last_error()
+    rc = lib.hkv_retrieve_topk(1, 4, 4, 96, None, None, 10, 10, 0, 0, 4, None, None, None, 0, None, None)
+    assert rc == hkv.HKV_ERR_UNSUPPORTED
+    rc = lib.hkv_retrieve_topk(1, 4, 4, 128, None, None, 5, 10, 0, 0, 4, None, None, None, 0, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG  # cap < n_tokens
+    hs = hkv.hkv_hash(hkv.HKV_HASH_SIGN, 128, 128, 0, hkv.HKV_BF16, 0, None, None, None, None, None)
+    rc = lib.hkv_append(ctypes.byref(hs), 1, 1, 4, None, None, None, None, None, None, 10, 8, None, None)
+    assert rc == hkv.HKV_ERR_CAPACITY
+    rc = lib.hkv_lse_merge(-1, 128, None, None, None, None, None, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG
+    rc = lib.hkv_sparse_attend(1, 4, 4, 7, None, None, None, 10, 10, None, 0, 0, 0, 0.1, None, None, None, 0, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG
+
+
+def test_zero_sized_calls_are_noops(lib):
+    h = hkv.hkv_hash(hkv.HKV_HASH_SIGN, 128, 128, 0, hkv.HKV_BF16, 0, None, None, None, None, None)
+    assert lib.hkv_encode_keys(ctypes.byref(h), None, 0, 128, None, 4, None, None, None) == hkv.HKV_OK
+    assert lib.hkv_retrieve_topk(0, 4, 4, 128, None, None, 10, 10, 0, 0, 4, None, None, None, 0, None, None) == hkv.HKV_OK
+    assert lib.hkv_lse_merge(0, 128, None, None, None, None, None, None, None) == hkv.HKV_OK
