@@ -323,8 +323,12 @@ __global__ void __launch_bounds__(kThreads, kMaxBlocksPerSM) scan_select_kernel(
         const uint32_t msel = __ballot_sync(0xffffffffu, sel);
         if (sel) {
           const uint32_t pos = run_sel + __popc(msel & below_lane);
-          idx_out[pos] = (int32_t)(a.lo + s0 + i);
-          if (dist_out) dist_out[pos] = Dv;
+          if (sel_base + pos < k_eff) {
+            idx_out[pos] = (int32_t)(a.lo + s0 + i);
+            if (dist_out) dist_out[pos] = Dv;
+          } else {
+            report(a.status, HKV_ERR_DEVICE_RANGE);  // unreachable when the counts agree
+          }
         }
         run_eq += __popc(meq);
         run_sel += __popc(msel);
