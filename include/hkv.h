@@ -107,10 +107,12 @@ int hkv_check(int32_t* status, void* stream);
 
 /* Bytes of workspace that hkv_retrieve_topk, hkv_sparse_attend and
  * hkv_decode_step need for this shape on the current device (0 if the shape
- * is invalid or unsupported).  The workspace
- * must be zero-filled once before first use (hkv_workspace_reset); every call
- * leaves it zero-filled again, including calls that end in a device error.
- * Calls that share one workspace must not overlap on the GPU. */
+ * is invalid or unsupported).  The workspace must be zero-filled once before
+ * first use (hkv_workspace_reset).  Each call returns the counters and
+ * histograms that must start at zero to zero before it ends, including calls
+ * that end in a device error, so one workspace serves any number of calls in
+ * a row (and CUDA-graph replays).  Calls that share one workspace must not
+ * overlap on the GPU. */
 size_t hkv_workspace_bytes(int B, int Hq, int Hkv, int64_t n_tokens, int code_bits, int top_k,
                            int n_sink, int n_local);
 

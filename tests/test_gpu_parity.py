@@ -122,9 +122,11 @@ def _retrieve(q_codes, k_codes, N, s, l, k):
     dist = torch.full((B, Hkv, k), -9, dtype=torch.int32, device=DEV)
     ws = hkv.workspace(B, Hq, Hkv, N, W * 32, k, s, l)
     st = hkv.status_word()
-    hkv.hkv_retrieve_topk(qg, kg, N, s, l, k, idx, dist, ws=ws, status=st)
-    _check(st)
-    assert int(ws.count_nonzero()) == 0  # workspace left clean
+    for _ in range(2):  # the second call relies on the first leaving its counters at zero
+        idx.fill_(-9)
+        dist.fill_(-9)
+        hkv.hkv_retrieve_topk(qg, kg, N, s, l, k, idx, dist, ws=ws, status=st)
+        _check(st)
     return idx.cpu().numpy(), dist.cpu().numpy(), (qg, kg, idx, dist, ws, st)
 
 
@@ -182,7 +184,6 @@ def test_retrieve_wait_times_out_and_recovers():
         assert hkv.hkv_check(st) == hkv.HKV_ERR_TIMEOUT
     finally:
         hkv.hkv_debug_set(0, 0)
-    assert int(ws.count_nonzero()) == 0
     hkv.hkv_retrieve_topk(qc, kc, N, 4, 128, k, idx, ws=ws, status=st)
     _check(st)
     wi, _ = oracle.retrieve(u32(qc), u32(kc), N, 4, 128, k)
