@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--impl", default="hkv", choices=["hkv", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="number of layer buffers (default: the workload's layers, at least 3x L2 of data); "
+                         "a small value makes a small case for profiling")
     return ap.parse_args()
 
 
@@ -227,7 +230,7 @@ def run_gpu(args, rank, world, local):
     hkv.lib()
     w = synth.WORKLOADS[args.workload]
     per_layer_bytes = w.algorithmic_bytes()
-    n_layers = max(w.layers, math.ceil(3 * L2_BYTES / per_layer_bytes))
+    n_layers = args.layers or max(w.layers, math.ceil(3 * L2_BYTES / per_layer_bytes))
     layers = [Layer(w, l % w.layers if w.layers > 1 else 0, dev, hkv) for l in range(n_layers)]
     # prefill: encode the keys of every layer (timed separately, reported as encode)
     torch.cuda.synchronize()
@@ -246,9 +249,22 @@ def run_gpu(args, rank, world, local):
             hkv.hkv_decode_step(L.qh, L.q, L.codes, L.K, L.V, w.N, w.n_sink, w.n_local, w.top_k, L.out,
                                 q_codes=L.q_codes, idx=L.idx, ws=ws, status=status)
 
+    # standalone calls get their own workspaces (each entry point has its own layout)
+    ws_r = hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
+    ws_a = hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
+    ws_f = hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
+
+    given = hkv.HashParams.given(hkv.HKV_BF16 if w.dtype == "bf16" else hkv.HKV_F32, w.bits)
+
+    def fused_only():
+        for L in layers:
+            hkv.hkv_decode_step(given, L.q, L.codes, L.K, L.V, w.N, w.n_sink, w.n_local, w.top_k, L.out,
+                                q_codes=L.q_codes, idx=L.idx, ws=ws_f, status=status)
+
     def scan_only():
         for L in layers:
-            hkv.hkv_retrieve_topk(L.q_codes, L.codes, w.N, w.n_sink, w.n_local, w.top_k, L.idx, ws=ws, status=status)
+            hkv.hkv_retrieve_topk(L.q_codes, L.codes, w.N, w.n_sink, w.n_local, w.top_k, L.idx, ws=ws_r,
+                                  status=status)
 
     g_step = graph_of(step)
     rc = hkv.hkv_check(status)
@@ -260,9 +276,25 @@ def run_gpu(args, rank, world, local):
     if rc != hkv.HKV_OK:
         raise RuntimeError(f"decode step reported status {rc}")
     ms = max_over_ranks(ms, world, dev)
-    # dominant kernel alone: the scan/select launch of every layer
+    # each kernel alone, one launch per layer
+    def qenc_only():
+        for L in layers:
+            hkv.hkv_encode_keys(L.qh, L.q.view(-1, w.d), L.q_codes.view(-1, w.words))
+
+    def attend_only():
+        for L in layers:
+            hkv.hkv_sparse_attend(L.q, L.K, L.V, w.N, L.idx, w.n_sink, w.n_local, L.out, ws=ws_a, status=status)
+
+    g_fused = graph_of(fused_only)
+    fused_ms = max_over_ranks(time_graph(g_fused, args.steps, args.warmup, world), world, dev)
+    del g_fused
     g_scan = graph_of(scan_only)
     scan_ms = max_over_ranks(time_graph(g_scan, args.steps, args.warmup, world), world, dev)
+    g_qenc = graph_of(qenc_only)
+    qenc_ms = max_over_ranks(time_graph(g_qenc, args.steps, args.warmup, world), world, dev)
+    g_att = graph_of(attend_only)
+    att_ms = max_over_ranks(time_graph(g_att, args.steps, args.warmup, world), world, dev)
+    del g_qenc, g_att
     # end to end: host q in, host out back, every step
     q_host = [torch.empty_like(L.q, device="cpu").pin_memory() for L in layers]
     o_host = [torch.empty_like(L.out, device="cpu").pin_memory() for L in layers]
@@ -288,10 +320,10 @@ def run_gpu(args, rank, world, local):
     keys_step = keys_per_layer * len(layers) * world
     value = keys_step / (ms * 1e-3)
     peak, peak_kind = measured_peaks()
-    code_bytes = w.B * w.Hkv * w.candidates() * w.bits // 8
-    scan_launch_ms = scan_ms / len(layers)
-    achieved = code_bytes / (scan_launch_ms * 1e-3) / 1e9
+    fused_launch_ms = fused_ms / len(layers)
+    achieved = per_layer_bytes / (fused_launch_ms * 1e-3) / 1e9
     traffic = traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "retrieve.cu"), w.name)
+    code_bytes = w.B * w.Hkv * w.candidates() * w.bits // 8
     step_gbs = per_layer_bytes * len(layers) / (ms * 1e-3) / 1e9
     out = {
         "metric": "decode retrieval+sparse-attn keys scanned/s (also us/layer and % HBM roofline)",
@@ -316,16 +348,20 @@ def run_gpu(args, rank, world, local):
         },
         "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
                      "bytes_per_layer": per_layer_bytes, "peak_kind": peak_kind},
-        "roofline": {"bound": "hbm", "kernel": "scan_select_kernel (hkv_retrieve_topk)", "achieved": achieved,
-                     "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": code_bytes, "launch_us": scan_launch_ms * 1e3,
-                     "peak_kind": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": "fused_kernel (scan + select + attend + merge, one layer)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": per_layer_bytes,
+                     "launch_us": fused_launch_ms * 1e3, "peak_kind": peak_kind},
         "e2e": {"value": keys_step / (e2e_ms * 1e-3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "encode": {"keys_per_s": w.B * w.Hkv * w.N * len(layers) / (encode_ms * 1e-3),
                    "ms_all_layers": encode_ms, "gbs": (w.B * w.Hkv * w.N * w.d * (2 if w.dtype == "bf16" else 4)
                                                         * len(layers)) / (encode_ms * 1e-3) / 1e9},
-        "gpu_launches": 3 * len(layers) * args.steps,
+        "kernels_us_per_launch": {"encode_q": qenc_ms * 1e3 / len(layers),
+                                  "fused_decode": fused_launch_ms * 1e3,
+                                  "retrieve_only": scan_ms * 1e3 / len(layers),
+                                  "sparse_attend_only": att_ms * 1e3 / len(layers)},
+        "gpu_launches": 2 * len(layers) * args.steps,
         "clocks": clk.summary(),
     }
     del g_step, g_scan, g_e2e

@@ -25,7 +25,7 @@ import torch
 __all__ = [
     "HKV_OK", "HKV_ERR_INVALID_ARG", "HKV_ERR_UNSUPPORTED", "HKV_ERR_CAPACITY", "HKV_ERR_CUDA",
     "HKV_ERR_TIMEOUT", "HKV_ERR_DEVICE_RANGE", "HKV_F32", "HKV_BF16", "HKV_HASH_LSH", "HKV_HASH_MLP",
-    "HKV_HASH_SIGN", "HkvError", "HashParams", "lib", "lib_path", "workspace", "status_word",
+    "HKV_HASH_SIGN", "HKV_HASH_NONE", "HkvError", "HashParams", "lib", "lib_path", "workspace", "status_word",
     "hkv_version", "hkv_last_error", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
     "hkv_encode_keys", "hkv_append", "hkv_retrieve_topk", "hkv_sparse_attend", "hkv_lse_merge",
     "hkv_decode_step", "hkv_debug_set", "EXPORTS",
@@ -34,7 +34,7 @@ __all__ = [
 HKV_OK, HKV_ERR_INVALID_ARG, HKV_ERR_UNSUPPORTED, HKV_ERR_CAPACITY = 0, -1, -2, -3
 HKV_ERR_CUDA, HKV_ERR_TIMEOUT, HKV_ERR_DEVICE_RANGE = -4, -5, -6
 HKV_F32, HKV_BF16 = 0, 1
-HKV_HASH_LSH, HKV_HASH_MLP, HKV_HASH_SIGN = 0, 1, 2
+HKV_HASH_LSH, HKV_HASH_MLP, HKV_HASH_SIGN, HKV_HASH_NONE = 0, 1, 2, 3
 
 # Every symbol include/hkv.h declares.
 EXPORTS = (
@@ -162,6 +162,11 @@ class HashParams:
     @classmethod
     def sign(cls, dtype: int, head_dim: int = 128) -> "HashParams":
         return cls(HKV_HASH_SIGN, dtype, head_dim)
+
+    @classmethod
+    def given(cls, dtype: int, code_bits: int) -> "HashParams":
+        """For hkv_decode_step: the query codes are supplied in q_codes."""
+        return cls(HKV_HASH_NONE, dtype, code_bits)
 
 
 def status_word(device=None) -> torch.Tensor:

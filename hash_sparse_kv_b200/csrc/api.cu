@@ -47,8 +47,14 @@ int sm_count() {
 
 static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-static int check_hash(const hkv_hash* h) {
+static int check_hash(const hkv_hash* h, bool allow_none = false) {
   if (h == nullptr) return fail(HKV_ERR_INVALID_ARG, "hash is NULL");
+  if (allow_none && h->kind == HKV_HASH_NONE) {
+    if (h->head_dim != kHeadDim) return fail(HKV_ERR_UNSUPPORTED, "head_dim %d (only 128)", h->head_dim);
+    if (h->dtype != HKV_F32 && h->dtype != HKV_BF16) return fail(HKV_ERR_INVALID_ARG, "dtype %d", h->dtype);
+    if (h->code_bits != 64 && h->code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "code_bits %d", h->code_bits);
+    return HKV_OK;
+  }
   if (h->head_dim != kHeadDim) return fail(HKV_ERR_UNSUPPORTED, "head_dim %d (only 128)", h->head_dim);
   if (h->dtype != HKV_F32 && h->dtype != HKV_BF16) return fail(HKV_ERR_INVALID_ARG, "dtype %d", h->dtype);
   switch (h->kind) {
@@ -84,23 +90,24 @@ static int check_window(int64_t cap, int64_t N, int n_sink, int n_local, int top
   return HKV_OK;
 }
 
-// Workspace of one decode step: [retrieval scratch][attention scratch]
-// [query codes][selected indices].  The two scratch areas are separate so
-// each keeps its own zero-on-exit invariant.
+// Workspace of one decode step: [fused scan/select/attend scratch]
+// [attention scratch, used when there are no candidates][query codes]
+// [selected indices].  Each scratch area keeps its own zero-on-exit invariant.
 struct DecodeLayout {
-  size_t retrieve, attend, qcodes, idx, total;
+  size_t fused, attend, qcodes, idx, total;
 };
 
 static int decode_layout(int B, int Hq, int Hkv, int64_t N, int code_bits, int top_k, int n_sink,
                          int n_local, DecodeLayout& L) {
   RetrieveShape rs{B, Hq, Hkv, code_bits / 32, N, N, n_sink, n_local, top_k};
   AttendShape as{B, Hq, Hkv, HKV_BF16, N, N, top_k, n_sink, n_local};
-  L.retrieve = align_up(retrieve_ws_bytes(rs), 256);
-  if (L.retrieve == 0 && (int64_t)B * Hkv * top_k > 0) return HKV_ERR_UNSUPPORTED;
+  const size_t r = retrieve_ws_bytes(rs), d = decode_ws_bytes(rs);
+  if ((r == 0 || d == 0) && (int64_t)B * Hkv * top_k > 0) return HKV_ERR_UNSUPPORTED;
+  L.fused = align_up(r > d ? r : d, 256);
   L.attend = align_up(attend_ws_bytes(as), 256);
   L.qcodes = align_up(sizeof(uint32_t) * (size_t)B * Hq * (code_bits / 32), 256);
   L.idx = align_up(sizeof(int32_t) * (size_t)B * Hkv * top_k, 256);
-  L.total = L.retrieve + L.attend + L.qcodes + L.idx;
+  L.total = L.fused + L.attend + L.qcodes + L.idx;
   return HKV_OK;
 }
 
@@ -237,30 +244,52 @@ int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* 
                     int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
                     uint32_t* q_codes, int32_t* idx, float* out, float* lse, void* ws,
                     size_t ws_bytes, int32_t* status, void* stream) {
-  int rc = check_hash(q_hash);
+  int rc = check_hash(q_hash, true);
   if (rc == HKV_OK) rc = check_heads(B, Hq, Hkv);
   if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
   if (rc != HKV_OK) return rc;
+  if (!std::isfinite(scale)) return fail(HKV_ERR_INVALID_ARG, "scale is not finite");
+  const bool given_codes = q_hash->kind == HKV_HASH_NONE;
+  if (given_codes && q_codes == nullptr) return fail(HKV_ERR_INVALID_ARG, "HKV_HASH_NONE needs q_codes");
   if (B == 0) return HKV_OK;
   if (!q || !k_codes || !K || !V || !out) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) ||
+      !aligned(k_codes, q_hash->code_bits / 8))
+    return fail(HKV_ERR_INVALID_ARG, "q, K, V, out and k_codes must be aligned");
   DecodeLayout L;
   rc = decode_layout(B, Hq, Hkv, n_tokens, q_hash->code_bits, top_k, n_sink, n_local, L);
   if (rc != HKV_OK) return fail(rc, "unsupported decode shape");
   if (ws == nullptr || ws_bytes < L.total) return fail(HKV_ERR_CAPACITY, "workspace of %zu bytes, %zu needed", ws_bytes, L.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   unsigned char* base = static_cast<unsigned char*>(ws);
-  void* ws_r = base;
-  void* ws_a = base + L.retrieve;
-  uint32_t* qc = q_codes ? q_codes : reinterpret_cast<uint32_t*>(base + L.retrieve + L.attend);
-  int32_t* ix = idx ? idx : reinterpret_cast<int32_t*>(base + L.retrieve + L.attend + L.qcodes);
+  void* ws_f = base;
+  void* ws_a = base + L.fused;
+  uint32_t* qc = q_codes ? q_codes : reinterpret_cast<uint32_t*>(base + L.fused + L.attend);
+  int32_t* ix = idx ? idx : reinterpret_cast<int32_t*>(base + L.fused + L.attend + L.qcodes);
   const int W = q_hash->code_bits / 32;
-  rc = hkv_encode_keys(q_hash, q, (int64_t)B * Hq, q_hash->head_dim, qc, W, nullptr, status, stream);
-  if (rc == HKV_OK)
-    rc = hkv_retrieve_topk(B, Hq, Hkv, q_hash->code_bits, qc, k_codes, cap, n_tokens, n_sink, n_local, top_k, ix,
-                           nullptr, ws_r, L.retrieve, status, stream);
-  if (rc == HKV_OK)
-    rc = hkv_sparse_attend(B, Hq, Hkv, q_hash->dtype, q, K, V, cap, n_tokens, ix, top_k, n_sink, n_local, scale,
-                           out, lse, ws_a, L.attend, status, stream);
-  return rc;
+  const Window w = window(n_tokens, n_sink, n_local);
+  RetrieveShape rs{B, Hq, Hkv, W, cap, n_tokens, n_sink, n_local, top_k};
+  const bool fused_encode = !given_codes && w.C > 0 && top_k > 0 &&
+                            decode_encodes_queries(rs, q_hash->kind, q_hash->dtype);
+  if (!given_codes && !fused_encode) {
+    RowMap m{(int64_t)B * Hq, (int64_t)B * Hq, 0, q_hash->head_dim, 0, W, 0, 1};
+    rc = launch_encode(*q_hash, q, m, qc, nullptr, st);
+    if (rc != HKV_OK) return rc;
+  }
+  if (w.C == 0 || top_k == 0) {
+    // nothing to retrieve: attend the resident rows only
+    if (top_k > 0) {
+      rc = cuda_check(cudaMemsetAsync(ix, 0xff, sizeof(int32_t) * (size_t)B * Hkv * top_k, st), "idx fill");
+      if (rc != HKV_OK) return rc;
+    }
+    AttendShape as{B, Hq, Hkv, q_hash->dtype, cap, n_tokens, top_k, n_sink, n_local};
+    return launch_attend(as, q, K, V, ix, scale, out, lse, ws_a, L.attend, status, st);
+  }
+  if (fused_encode)
+    return launch_decode(rs, q_hash->dtype, q_hash->kind, q_hash->R, nullptr, qc, k_codes, ix, q, K, V, scale, out,
+                         lse, ws_f, L.fused, status, st);
+  return launch_decode(rs, q_hash->dtype, HKV_HASH_NONE, nullptr, qc, nullptr, k_codes, ix, q, K, V, scale, out, lse,
+                       ws_f, L.fused, status, st);
 }
 
 }  // extern "C"

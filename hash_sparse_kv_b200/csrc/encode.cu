@@ -15,6 +15,7 @@ namespace hkv {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int64_t kFewRows = 2048;  // up to this many rows use the per-16-row projection kernel
 
 // ---------------------------------------------------------------- LSH -----
 // Tile of 64 rows per pass; warp w owns rows [8w, 8w + 8); lane l owns bits
@@ -73,6 +74,55 @@ lsh_encode_kernel(const T* __restrict__ x, const T* __restrict__ R, RowMap m,
         if (lane == i && row < m.rows) codes[m.c_off(row) + i] = word;
       }
     }
+  }
+}
+
+// Few rows (query heads of a decode step, short appends): 16 rows per block,
+// R staged once per block with padded rows (odd word stride, so the lanes of
+// a warp -- consecutive bits j -- read distinct banks).  Thread t owns bit
+// j = t % BITS of rows {t / BITS + SLOTS * i}.
+template <typename T, int BITS>
+__global__ void __launch_bounds__(kThreads)
+lsh_rows_kernel(const T* __restrict__ x, const T* __restrict__ R, RowMap m, uint32_t* __restrict__ codes) {
+  constexpr int D = kHeadDim, ROWS = 16, SLOTS = kThreads / BITS, RPT = ROWS / SLOTS;
+  constexpr int RP = D + (sizeof(T) == 2 ? 2 : 1);
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* x_s = reinterpret_cast<float*>(smem_raw);            // [ROWS][D]
+  T* R_s = reinterpret_cast<T*>(x_s + ROWS * D);               // [BITS][RP]
+  constexpr int V = 16 / sizeof(T);
+  for (int i = threadIdx.x; i < BITS * (D / V); i += kThreads) {
+    const int j = i / (D / V), c = (i % (D / V)) * V;
+    const uint4 raw = *reinterpret_cast<const uint4*>(R + (int64_t)j * D + c);
+    const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+    for (int u = 0; u < V; ++u) R_s[j * RP + c + u] = e[u];
+  }
+  const int64_t r0 = (int64_t)blockIdx.x * ROWS;
+  for (int i = threadIdx.x; i < ROWS * (D / 4); i += kThreads) {
+    const int r = i / (D / 4), c = (i % (D / 4)) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r0 + r < m.rows) v = load4_f32(x + m.x_off(r0 + r) + c);
+    *reinterpret_cast<float4*>(&x_s[r * D + c]) = v;
+  }
+  __syncthreads();
+  const int j = threadIdx.x % BITS, slot = threadIdx.x / BITS, lane = threadIdx.x & 31;
+  float acc[RPT];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) acc[i] = 0.f;
+#pragma unroll 4
+  for (int k = 0; k < D; k += 2) {
+    const float r_a = to_f32(R_s[j * RP + k]), r_b = to_f32(R_s[j * RP + k + 1]);
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+      const float2 xv = *reinterpret_cast<const float2*>(&x_s[(slot + SLOTS * i) * D + k]);
+      acc[i] = fmaf(xv.x, r_a, fmaf(xv.y, r_b, acc[i]));
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const int64_t row = r0 + slot + SLOTS * i;
+    const uint32_t word = __ballot_sync(0xffffffffu, acc[i] > 0.f);
+    if (lane == 0 && row < m.rows) codes[m.c_off(row) + j / 32] = word;
   }
 }
 
@@ -234,6 +284,15 @@ int grid_for(K kernel, size_t smem, int64_t work_items) {
 
 template <typename T, int BITS>
 int run_lsh(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, cudaStream_t st) {
+  if (m.rows <= kFewRows) {
+    auto kernel = lsh_rows_kernel<T, BITS>;
+    const size_t smem = sizeof(float) * 16 * kHeadDim + sizeof(T) * BITS * (kHeadDim + (sizeof(T) == 2 ? 2 : 1));
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_check(e, "lsh rows smem attribute");
+    kernel<<<(unsigned)((m.rows + 15) / 16), kThreads, smem, st>>>(static_cast<const T*>(x),
+                                                                      static_cast<const T*>(h.R), m, codes);
+    return cuda_check(cudaGetLastError(), "lsh rows launch");
+  }
   auto kernel = lsh_encode_kernel<T, BITS>;
   const size_t smem = sizeof(float) * (kHeadDim * BITS + kHeadDim * 68);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

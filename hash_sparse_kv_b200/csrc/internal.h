@@ -37,6 +37,16 @@ size_t retrieve_ws_bytes(const RetrieveShape& s);
 int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,
                     int32_t* idx, int32_t* dist, void* ws, size_t ws_bytes, int32_t* status,
                     cudaStream_t st);
+// Scan + select + attention + merge in one launch (candidates must be
+// non-empty).  q_kind HKV_HASH_LSH / HKV_HASH_SIGN: the kernel encodes the
+// query heads itself (when decode_encodes_queries says it can) and writes
+// them to q_codes_out if non-null; otherwise q_codes_in holds them.
+size_t decode_ws_bytes(const RetrieveShape& s);
+bool decode_encodes_queries(const RetrieveShape& s, int kind, int dtype);
+int launch_decode(const RetrieveShape& s, int dtype, int q_kind, const void* R, const uint32_t* q_codes_in,
+                  uint32_t* q_codes_out, const uint32_t* k_codes, int32_t* idx, const void* q, const void* K,
+                  const void* V, float scale, float* out, float* lse, void* ws, size_t ws_bytes,
+                  int32_t* status, cudaStream_t st);
 
 // ---- attention (attend.cu) ----
 struct AttendShape {

@@ -1,63 +1,103 @@
-// Hamming scan + top-k selection (S4, S5).
+// Hamming scan + top-k selection (S4, S5), optionally fused with the query
+// encoding (S2), the sparse attention over the selected and resident rows and
+// the log-sum-exp merge (S6-S8): one decode step in one launch.
 //
 // HashEvict ("Abstract") scores cached keys by the Hamming distance between
 // binarized projections of the query and of each key; Spotlight Attention
-// ("Approach", "Key results") keeps the top-k keys per decode step.  With
-// grouped-query attention a KV head's score of token t is the sum over its g
-// query heads:  D(t) = sum_h popcount(cq_h XOR ck_t)  in [0, g * bits].
+// ("Approach", "Key results") keeps the top-k keys per decode step and
+// attends over them exactly, with sink and local-window tokens kept;
+// RetrievalAttention ("Approach") merges partial attention results by exact
+// log-sum-exp rescaling.  With grouped-query attention a KV head's score of
+// token t is the sum over its g query heads:
+//     D(t) = sum_h popcount(cq_h XOR ck_t)  in [0, g * bits].
 //
-// Design (one cooperative launch):
+// One cooperative launch, one block of 512 threads per SM:
 //  * The candidate tokens of all (batch, KV head) pairs are laid end to end
-//    and cut into equal contiguous ranges, one per block, so every SM gets the
-//    same number of code bytes whatever the batch shape.  A block's range
-//    covers one or more "segments" (its part of one pair).
-//  * Phase A, per segment: stream the codes once (16-byte loads that skip
-//    L1), compute D for each token, keep D in shared memory (uint16), and
-//    build the segment's histogram of D in shared memory.  Publish the
-//    segment's cumulative histogram and add its counts into the pair's global
-//    histogram.  Then arrive at the pair's barrier.
-//  * Phase B, per segment: wait (bounded) until every segment of the pair has
-//    arrived; read the pair's histogram and find the threshold T: the
-//    smallest D whose cumulative count reaches k_eff.  Tokens with D < T are
-//    all selected; tokens with D == T are admitted in ascending token order
-//    until k_eff is reached.  From the lower segments' cumulative histograms a
-//    block knows how many selected tokens precede its segment, so it writes
-//    its selected tokens straight to their final, ascending positions.
-//  * The last block to leave a pair zeroes the pair's global scratch, so the
-//    workspace is clean for the next call.
+//    and cut into equal contiguous ranges, one per block, so every SM streams
+//    the same number of code bytes.  A block's range covers one or more
+//    "segments" (its part of one pair).
+//  * Phase A.  Each thread streams its tokens through a private ring of
+//    cp.async slots (no block-wide synchronisation) while the block encodes
+//    the query heads it needs.  Per token it computes D, keeps it in shared
+//    memory (uint16) and counts it in its segment's histogram.
+//  * Publication.  A segment publishes its cumulative histogram only up to
+//    hi = its own k-th smallest D (all bins if it holds fewer than k_eff
+//    tokens).  The global threshold T (smallest D whose global cumulative
+//    count reaches k_eff) is at most min over segments of hi, because that
+//    segment alone already has k_eff tokens at or below its hi; so the
+//    published windows hold every count needed to find T.
+//  * Phase B, per segment.  Wait (bounded) for all segments of the pair, read
+//    the windows of all segments in one parallel pass, find T and the counts
+//    of the lower segments, then write this segment's selected tokens
+//    straight to their final, ascending positions in idx: tokens with D < T,
+//    and tokens with D == T in ascending order until k_eff is reached.
+//  * Attention.  While waiting, a block attends its share of the pair's
+//    resident sink/local rows; afterwards it adds its own selected rows
+//    (online softmax over tiles of 64 gathered K/V rows, all g query heads at
+//    once) and writes one partial (m, l, acc).  The last g blocks of the pair
+//    to finish merge one head each: M = max m_s, L = sum l_s e^{m_s - M},
+//    out = sum acc_s e^{m_s - M} / L, lse = M + log L.
+//  * The last block out of a pair returns the pair's counters to zero, so the
+//    workspace is ready for the next call.
 //
-// The group-summed distance is computed with bit-sliced arithmetic instead of
-// g * W popcounts.  For bit position j let c_j = #{h : bit j of cq_h is 1}.
-// The contribution of position j is (ck_j ? g - c_j : c_j).  The NP bit planes
-// of c_j (C planes) and of g - c_j (U planes) are built once per segment; per
-// token each word gives NP planes V_b = (ck & U_b) | (~ck & C_b), the words'
-// planes are added with carry-save adders, and D = sum_b 2^b popcount(S_b).
+// The group-summed distance uses bit-sliced arithmetic instead of g * W
+// popcounts.  For bit position j let c_j = #{h : bit j of cq_h is 1}; the
+// contribution of j is (ck_j ? g - c_j : c_j).  The NP bit planes of c_j (C
+// planes) and of g - c_j (U planes) are built once per segment; per token each
+// word gives NP planes V_b = (ck & U_b) | (~ck & C_b), words are added with
+// carry-save adders, and D = sum_b 2^b popcount(S_b).
+#include <math.h>
+
+#include <algorithm>
+
 #include "internal.h"
 
 namespace hkv {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 4;
-constexpr int kMaxTokensPerBlock = 24576;  // uint16 distances kept in shared memory
-constexpr int kMinTokensPerBlock = 1024;
-constexpr int kMaxBlocksPerSM = 3;
+constexpr int kGroups = 4;                  // cp.async groups in flight per thread
+constexpr int kSlots = 2 * kGroups;         // two tokens per group
+constexpr int kMaxTokensPerBlock = 32768;   // uint16 distances in shared memory
+constexpr int kMinTokensPerBlock = 2048;
+constexpr int kMaxSegsPerPair = 160;        // blocks per pair (shared header buffer)
+constexpr int kMaxGroup = 16;
+constexpr int kQRows = 32;                  // query rows one block may encode
+constexpr int kRows = 64;                   // attention tile
+constexpr int kKP = kHeadDim + 4;     // K tile pitch: float4-aligned rows
+constexpr int kPart = kHeadDim + 2;         // m, l, acc[128]
+constexpr int kSync = 4;                    // per pair: arrivals, departures, merge ticket, merges done
+constexpr int kSelCap = 2048;               // selected rows kept in shared memory
+constexpr int kOut = (kMaxGroup * kHeadDim + kThreads - 1) / kThreads;
 
-struct RetrieveArgs {
-  const uint32_t* q_codes;
+enum QEnc { kQGiven = 0, kQLsh = 1, kQSign = 2 };
+
+struct FusedArgs {
+  const uint32_t* q_codes_in;  // kQGiven: [B, Hq, W]
+  uint32_t* q_codes_out;       // nullable: written by each pair's first segment
+  const void* R;               // kQLsh: [bits, 128] in the dtype of q
+  int qenc;
   const uint32_t* k_codes;
   int32_t* idx;
   int32_t* dist;
+  const void* q;
+  const void* K;
+  const void* V;
+  float* out;
+  float* lse;
+  float scale;
   int Hq, Hkv, g;
-  int64_t cap, lo, C;
-  int k_eff, top_k;
-  int p0, P;
-  int64_t per_block;
-  int nbins, max_seg;
-  uint32_t* sync;  // [pairs][2]: arrivals, departures
-  uint32_t* hist;  // [pairs][nbins]
-  uint32_t* cum;   // [pairs][max_seg][nbins]
+  int64_t cap, lo;
+  int C, k_eff, top_k;
+  int sink_n, local_start, local_n;
+  int p0, nseg, per_block;
+  int nbins, nbins_pad;
+  uint32_t off_q, off_aq, off_sel, off_hist, off_dist;  // shared memory carve-up (bytes)
+  uint32_t* sync;  // [pairs][kSync]
+  uint32_t* hdr;   // [pairs][nseg][2]: window lo, hi
+  uint32_t* cum;   // [pairs][nseg][nbins]: cumulative counts, window only
+  float* part;     // [pairs][nseg][g][kPart]
   int32_t* status;
   uint64_t wait_ns;
   int skip_arrive;
@@ -71,7 +111,7 @@ struct Planes {
 
 // Bit-sliced counters: C planes count the query codes' ones, U planes their zeros.
 template <int W, int NP>
-__device__ __forceinline__ void build_planes(const uint32_t* __restrict__ qc, int g, Planes<W, NP>& p) {
+__device__ __forceinline__ void build_planes(const uint32_t* qc, int g, Planes<W, NP>& p) {
 #pragma unroll
   for (int b = 0; b < NP; ++b)
 #pragma unroll
@@ -79,7 +119,7 @@ __device__ __forceinline__ void build_planes(const uint32_t* __restrict__ qc, in
   for (int h = 0; h < g; ++h) {
 #pragma unroll
     for (int w = 0; w < W; ++w) {
-      const uint32_t q = __ldg(qc + h * W + w);
+      const uint32_t q = qc[h * W + w];
       uint32_t carry = q;
 #pragma unroll
       for (int b = 0; b < NP; ++b) {
@@ -140,6 +180,34 @@ __device__ __forceinline__ int token_distance(const uint32_t (&ck)[W], const Pla
   }
 }
 
+// ---- cp.async helpers (per-thread ring; each thread reads only its own slots)
+template <int W>
+__device__ __forceinline__ void cp_async_code(uint32_t* dst, const uint32_t* src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  if constexpr (W == 4)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int W>
+__device__ __forceinline__ void load_slot(const uint32_t* sl, uint32_t (&ck)[W]) {
+  if constexpr (W == 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(sl);
+    ck[0] = v.x;
+    ck[1] = v.y;
+    ck[2] = v.z;
+    ck[3] = v.w;
+  } else {
+    const uint2 v = *reinterpret_cast<const uint2*>(sl);
+    ck[0] = v.x;
+    ck[1] = v.y;
+  }
+}
+
 // In-place inclusive prefix sum over a[0, n) in shared memory.
 __device__ void block_inclusive_scan(uint32_t* a, int n, uint32_t* warp_tmp) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -164,212 +232,689 @@ __device__ void block_inclusive_scan(uint32_t* a, int n, uint32_t* warp_tmp) {
   __syncthreads();
 }
 
-__device__ __forceinline__ uint32_t block_sum(uint32_t v, uint32_t* warp_tmp) {
+// Exclusive prefix of v over the block's threads; *total receives the sum.
+__device__ __forceinline__ uint32_t block_exclusive(uint32_t v, uint32_t* warp_tmp, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
   __syncthreads();
-  if ((threadIdx.x & 31) == 0) warp_tmp[threadIdx.x >> 5] = v;
+  if (lane == 31) warp_tmp[warp] = x;
   __syncthreads();
-  uint32_t s = 0;
+  uint32_t base = 0, tot = 0;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) s += warp_tmp[w];
-  return s;
+  for (int w = 0; w < kWarps; ++w) {
+    const uint32_t t = warp_tmp[w];
+    base += w < warp ? t : 0u;
+    tot += t;
+  }
+  *total = tot;
+  return base + x - v;
 }
 
-template <int W, int NP>
-__global__ void __launch_bounds__(kThreads, kMaxBlocksPerSM) scan_select_kernel(RetrieveArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem_raw);
-  uint16_t* dist_s = reinterpret_cast<uint16_t*>(hist_s + ((a.nbins + 3) & ~3));
-  __shared__ uint32_t warp_tmp[kWarps];
-  __shared__ uint32_t warp_lt[kWarps], warp_eq[kWarps];
-  __shared__ int s_flag, s_T;
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t C = a.C;
-  const int64_t U = (int64_t)a.P * C;
-  const int64_t f0 = (int64_t)blockIdx.x * a.per_block;
-  const int64_t f1 = min(f0 + a.per_block, U);
-  if (f0 >= f1) return;
-  const int pa = (int)(f0 / C), pb = (int)((f1 - 1) / C);
-
-  // ---------------- phase A: distances, histograms ----------------
-  int64_t soff = 0;
-  for (int pl = pa; pl <= pb; ++pl) {
-    const int p = a.p0 + pl;
-    const int64_t s0 = max(f0, pl * C) - pl * C, s1 = min(f1, (pl + 1) * C) - pl * C;
-    const int seg = (int)(blockIdx.x - (pl * C) / a.per_block);
-    for (int i = tid; i < a.nbins; i += kThreads) hist_s[i] = 0u;
-    const int b = p / a.Hkv, kvh = p % a.Hkv;
-    Planes<W, NP> planes;
-    build_planes<W, NP>(a.q_codes + ((int64_t)b * a.Hq + (int64_t)kvh * a.g) * W, a.g, planes);
-    __syncthreads();
-    const uint32_t* kc = a.k_codes + ((int64_t)p * a.cap + a.lo) * W;
-    uint16_t* dseg = dist_s + soff;
-    for (int64_t base = s0; base < s1; base += kThreads * kUnroll) {
-      uint32_t ck[kUnroll][W];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t i = base + u * kThreads + tid;
-        if (i < s1) ld_stream(kc + i * W, ck[u]);
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t i = base + u * kThreads + tid;
-        if (i < s1) {
-          const int Dv = token_distance<W, NP>(ck[u], planes);
-          dseg[i - s0] = (uint16_t)Dv;
-          atomicAdd(&hist_s[Dv], 1u);
-        }
-      }
-    }
-    __syncthreads();
-    block_inclusive_scan(hist_s, a.nbins, warp_tmp);
-    uint32_t* cum_out = a.cum + ((int64_t)p * a.max_seg + seg) * a.nbins;
-    uint32_t* hist_out = a.hist + (int64_t)p * a.nbins;
-    for (int v = tid; v < a.nbins; v += kThreads) {
-      const uint32_t c = hist_s[v];
-      const uint32_t n = c - (v > 0 ? hist_s[v - 1] : 0u);
-      cum_out[v] = c;
-      if (n) atomicAdd(&hist_out[v], n);
-    }
-    soff += s1 - s0;
-    __syncthreads();
+// Bounded wait until *ctr >= target.  Returns false on expiry.
+__device__ bool wait_count(const uint32_t* ctr, uint32_t target, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0; ld_acquire_gpu(ctr) < target; ++it) {
+    if (globaltimer_ns() - t0 > limit_ns || it > (1u << 28)) return false;
+    __nanosleep(32);
   }
-  if (tid == 0) {
-    __threadfence();
-    if (!(a.skip_arrive && blockIdx.x == 0))
-      for (int pl = pa; pl <= pb; ++pl) atomicAdd(&a.sync[2 * (a.p0 + pl)], 1u);
-  }
+  return true;
+}
 
-  // ---------------- phase B: threshold, ordered compaction ----------------
-  soff = 0;
-  for (int pl = pa; pl <= pb; ++pl) {
-    const int p = a.p0 + pl;
-    const int64_t s0 = max(f0, pl * C) - pl * C, s1 = min(f1, (pl + 1) * C) - pl * C;
-    const int first = (int)((pl * C) / a.per_block);
-    const int last = (int)(((pl + 1) * C - 1) / a.per_block);
-    const int nseg = last - first + 1, seg = (int)blockIdx.x - first;
-    if (tid == 0) {
-      const uint64_t t0 = globaltimer_ns();
-      int ok = 1;
-      for (uint32_t it = 0; ld_acquire_gpu(&a.sync[2 * p]) < (uint32_t)nseg; ++it) {
-        if (globaltimer_ns() - t0 > a.wait_ns || it > (1u << 28)) {
-          ok = 0;
-          break;
-        }
-        __nanosleep(64);
-      }
-      __threadfence();
-      s_flag = ok;
-    }
+template <typename T>
+__device__ __forceinline__ const T* tptr(const void* p) { return static_cast<const T*>(p); }
+
+// Bring one K row and one V row (element row index `row`) into L2.
+template <typename T>
+__device__ __forceinline__ void prefetch_row_l2(const void* K, const void* V, int64_t row) {
+  constexpr uint32_t kBytes = kHeadDim * sizeof(T);
+  const T* k = tptr<T>(K) + row * kHeadDim;
+  const T* v = tptr<T>(V) + row * kHeadDim;
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(k), "r"(kBytes) : "memory");
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(v), "r"(kBytes) : "memory");
+}
+
+// Counter increments that publish the block's earlier writes (after a
+// __syncthreads, a release by one thread covers the whole block's writes).
+__device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// ---------------------------------------------------------------- attention
+struct AttnSmem {
+  float* q;  // [kMaxGroup][128]
+  float* K;  // [kRows][kKP]
+  float* V;  // [kRows][128]
+  float* z;  // [kMaxGroup][kRows]
+  int* tok;  // [kRows]
+  float* m;
+  float* l;
+  float* alpha;
+};
+
+__device__ void attn_begin(int g, const AttnSmem& sm, float (&acc)[kOut]) {
+#pragma unroll
+  for (int j = 0; j < kOut; ++j) acc[j] = 0.f;
+  if (threadIdx.x < g) {
+    sm.m[threadIdx.x] = -INFINITY;
+    sm.l[threadIdx.x] = 0.f;
+  }
+}
+
+// Adds `nrows` rows (token row_at(i), or -1 to skip) to the online softmax.
+template <typename T, typename RowAt>
+__device__ void attn_rows(const FusedArgs& a, int p, int nrows, RowAt row_at, const AttnSmem& sm,
+                          float (&acc)[kOut]) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
+  const T* Kp = tptr<T>(a.K) + (int64_t)p * a.cap * kHeadDim;
+  const T* Vp = tptr<T>(a.V) + (int64_t)p * a.cap * kHeadDim;
+  for (int r0 = 0; r0 < nrows; r0 += kRows) {
+    const int nr = min(kRows, nrows - r0);
     __syncthreads();
-    if (s_flag) {
-      const uint32_t* hist_in = a.hist + (int64_t)p * a.nbins;
-      for (int v = tid; v < a.nbins; v += kThreads) hist_s[v] = __ldcg(hist_in + v);
-      if (tid == 0) s_T = a.nbins - 1;
-      __syncthreads();
-      block_inclusive_scan(hist_s, a.nbins, warp_tmp);
-      const uint32_t k_eff = (uint32_t)a.k_eff;
-      for (int v = tid; v < a.nbins; v += kThreads)
-        if (hist_s[v] >= k_eff && (v == 0 || hist_s[v - 1] < k_eff)) s_T = v;
-      __syncthreads();
-      const int T = s_T;
-      const uint32_t below = T > 0 ? hist_s[T - 1] : 0u;
-      const uint32_t ties_needed = k_eff - below;
-      // selected-before counts from the lower segments of this pair
-      uint32_t lt = 0, le = 0;
-      for (int s = tid; s < seg; s += kThreads) {
-        const uint32_t* cs = a.cum + ((int64_t)p * a.max_seg + s) * a.nbins;
-        lt += T > 0 ? __ldcg(cs + T - 1) : 0u;
-        le += __ldcg(cs + T);
-      }
-      const uint32_t lower_lt = block_sum(lt, warp_tmp);
-      const uint32_t lower_eq = block_sum(le, warp_tmp) - lower_lt;
-      const uint32_t quota = ties_needed > lower_eq ? ties_needed - lower_eq : 0u;
-      const uint32_t sel_base = lower_lt + min(lower_eq, ties_needed);
-      // ordered compaction of this segment
-      const int64_t len = s1 - s0;
-      const int64_t per_w = ((len + kWarps * 32 - 1) / (kWarps * 32)) * 32;
-      const int64_t w0 = min((int64_t)warp * per_w, len), w1 = min(w0 + per_w, len);
-      const uint16_t* dseg = dist_s + soff;
-      uint32_t clt = 0, ceq = 0;
-      for (int64_t c = w0; c < w1; c += 32) {
-        const int64_t i = c + lane;
-        const int Dv = i < w1 ? (int)dseg[i] : 0x7fffffff;
-        clt += __popc(__ballot_sync(0xffffffffu, Dv < T));
-        ceq += __popc(__ballot_sync(0xffffffffu, Dv == T));
-      }
-      if (lane == 0) {
-        warp_lt[warp] = clt;
-        warp_eq[warp] = ceq;
-      }
-      __syncthreads();
-      uint32_t ex_lt = 0, ex_eq = 0;
-      for (int w = 0; w < warp; ++w) {
-        ex_lt += warp_lt[w];
-        ex_eq += warp_eq[w];
-      }
-      uint32_t run_eq = ex_eq, run_sel = ex_lt + min(ex_eq, quota);
-      int32_t* idx_out = a.idx + (int64_t)p * a.top_k + sel_base;
-      int32_t* dist_out = a.dist ? a.dist + (int64_t)p * a.top_k + sel_base : nullptr;
-      const uint32_t below_lane = lanemask_lt();
-      for (int64_t c = w0; c < w1; c += 32) {
-        const int64_t i = c + lane;
-        const int Dv = i < w1 ? (int)dseg[i] : 0x7fffffff;
-        const uint32_t meq = __ballot_sync(0xffffffffu, Dv == T);
-        const bool take_eq = Dv == T && run_eq + __popc(meq & below_lane) < quota;
-        const bool sel = Dv < T || take_eq;
-        const uint32_t msel = __ballot_sync(0xffffffffu, sel);
-        if (sel) {
-          const uint32_t pos = run_sel + __popc(msel & below_lane);
-          if (sel_base + pos < k_eff) {
-            idx_out[pos] = (int32_t)(a.lo + s0 + i);
-            if (dist_out) dist_out[pos] = Dv;
-          } else {
-            report(a.status, HKV_ERR_DEVICE_RANGE);  // unreachable when the counts agree
+    for (int i = tid; i < nr; i += kThreads) sm.tok[i] = row_at(r0 + i);
+    __syncthreads();
+    {
+      // all of this thread's K/V loads are issued before any shared store
+      constexpr int kPer = kRows * (kHeadDim / 4) / kThreads;
+      float4 kv[kPer], vv[kPer];
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int i = tid + u * kThreads, r = i / (kHeadDim / 4), c = (i % (kHeadDim / 4)) * 4;
+        kv[u] = vv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < nr) {
+          const int t = sm.tok[r];
+          if (t >= 0) {
+            kv[u] = load4_f32(Kp + (int64_t)t * kHeadDim + c);
+            vv[u] = load4_f32(Vp + (int64_t)t * kHeadDim + c);
           }
         }
-        run_eq += __popc(meq);
-        run_sel += __popc(msel);
       }
-    } else if (tid == 0) {
-      report(a.status, HKV_ERR_TIMEOUT);
-    }
-    soff += s1 - s0;
-    // depart; the last block out of this pair cleans its scratch
-    __syncthreads();
-    if (tid == 0) {
-      __threadfence();
-      s_flag = atomicAdd(&a.sync[2 * p + 1], 1u) == (uint32_t)(nseg - 1);
-    }
-    __syncthreads();
-    if (s_flag) {
-      __threadfence();
-      uint32_t* hist_out = a.hist + (int64_t)p * a.nbins;
-      for (int v = tid; v < a.nbins; v += kThreads) hist_out[v] = 0u;
-      for (int i = a.k_eff + tid; i < a.top_k; i += kThreads) {
-        a.idx[(int64_t)p * a.top_k + i] = -1;
-        if (a.dist) a.dist[(int64_t)p * a.top_k + i] = -1;
-      }
-      if (tid == 0) {
-        a.sync[2 * p] = 0u;
-        a.sync[2 * p + 1] = 0u;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        const int i = tid + u * kThreads, r = i / (kHeadDim / 4), c = (i % (kHeadDim / 4)) * 4;
+        if (r < nr) {
+          *reinterpret_cast<float4*>(&sm.K[r * kKP + c]) = kv[u];
+          *reinterpret_cast<float4*>(&sm.V[r * kHeadDim + c]) = vv[u];
+        }
       }
     }
     __syncthreads();
+    // logits: four lanes per (head, row), each over interleaved float4 columns
+    for (int t0 = 0; t0 < g * nr * 4; t0 += kThreads) {
+      const int t = t0 + tid, pr = t >> 2, qd = t & 3;
+      const bool live = pr < g * nr;
+      const int h = live ? pr / nr : 0, r = live ? pr % nr : 0;
+      float s = 0.f;
+      if (live && sm.tok[r] >= 0) {
+        const float* qh = sm.q + h * kHeadDim + 4 * qd;
+        const float* kr = sm.K + r * kKP + 4 * qd;
+#pragma unroll
+        for (int i = 0; i < kHeadDim / 16; ++i) {
+          const float4 x = *reinterpret_cast<const float4*>(qh + 16 * i);
+          const float4 y = *reinterpret_cast<const float4*>(kr + 16 * i);
+          s = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, s))));
+        }
+      }
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (live && qd == 0) sm.z[h * kRows + r] = sm.tok[r] >= 0 ? s * a.scale : -INFINITY;
+    }
+    __syncthreads();
+    for (int h = warp; h < g; h += kWarps) {
+      float mt = -INFINITY;
+      for (int r = lane; r < nr; r += 32) mt = fmaxf(mt, sm.z[h * kRows + r]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+      const float m_old = sm.m[h];
+      const float m_new = fmaxf(m_old, mt);
+      float ls = 0.f;
+      for (int r = lane; r < nr; r += 32) {
+        const float z = sm.z[h * kRows + r];
+        const float e = z == -INFINITY ? 0.f : expf(z - m_new);
+        sm.z[h * kRows + r] = e;
+        ls += e;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
+      if (lane == 0) {
+        const float alpha = m_new == -INFINITY ? 1.f : expf(m_old - m_new);
+        sm.alpha[h] = alpha;
+        sm.m[h] = m_new;
+        sm.l[h] = sm.l[h] * alpha + ls;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kOut; ++j) {
+      const int o = tid + j * kThreads;
+      if (o < g * kHeadDim) {
+        const int h = o / kHeadDim, c = o % kHeadDim;
+        float s = acc[j] * sm.alpha[h];
+        for (int r = 0; r < nr; ++r) s = fmaf(sm.z[h * kRows + r], sm.V[r * kHeadDim + c], s);
+        acc[j] = s;
+      }
+    }
   }
 }
 
-using KernelFn = void (*)(RetrieveArgs);
+__device__ void attn_end(int g, const AttnSmem& sm, const float (&acc)[kOut], float* dst) {
+  const int tid = threadIdx.x;
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kOut; ++j) {
+    const int o = tid + j * kThreads;
+    if (o < g * kHeadDim) {
+      const int h = o / kHeadDim, c = o % kHeadDim;
+      dst[h * kPart + 2 + c] = acc[j];
+      if (c == 0) {
+        dst[h * kPart + 0] = sm.m[h];
+        dst[h * kPart + 1] = sm.l[h];
+      }
+    }
+  }
+}
 
-KernelFn pick_kernel(int words, int np) {
-#define HKV_PICK(W, NPV) \
-  if (words == W && np == NPV) return scan_select_kernel<W, NPV>;
+// Merge head h of pair p over its nseg partials into out / lse.  Every load
+// of a thread is issued before its results are combined.
+__device__ void merge_head(const FusedArgs& a, int p, int nseg, int h, float* w_s, float* red_s, float* ml_s) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
+  const float* parts = a.part + (int64_t)p * nseg * g * kPart;
+  if (warp == 0) {
+    constexpr int kPerLane = (kMaxSegsPerPair + 31) / 32;
+    float2 ml[kPerLane];
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) {
+      const int s = lane + 32 * u;
+      ml[u] = s < nseg ? __ldcg(reinterpret_cast<const float2*>(parts + ((int64_t)s * g + h) * kPart))
+                       : make_float2(-INFINITY, 0.f);
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) M = fmaxf(M, ml[u].x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+#pragma unroll
+    for (int u = 0; u < kPerLane; ++u) {
+      const int s = lane + 32 * u;
+      const float w = ml[u].x == -INFINITY ? 0.f : expf(ml[u].x - M);
+      if (s < nseg) w_s[s] = w;
+      L = fmaf(ml[u].y, w, L);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (lane == 0) {
+      ml_s[0] = M;
+      ml_s[1] = L;
+    }
+  }
+  __syncthreads();
+  constexpr int kQuarters = kThreads / kHeadDim;
+  constexpr int kBatch = 8;
+  const int c = tid % kHeadDim, qtr = tid / kHeadDim;
+  float o = 0.f;
+  if (ml_s[1] > 0.f) {
+    for (int s0 = qtr; s0 < nseg; s0 += kBatch * kQuarters) {
+      float x[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int s = s0 + u * kQuarters;
+        x[u] = s < nseg ? __ldcg(parts + ((int64_t)s * g + h) * kPart + 2 + c) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int s = s0 + u * kQuarters;
+        if (s < nseg) o = fmaf(w_s[s], x[u], o);
+      }
+    }
+  }
+  red_s[qtr * kHeadDim + c] = o;
+  __syncthreads();
+  if (tid < kHeadDim) {
+    const float L = ml_s[1];
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < kQuarters; ++q) sum += red_s[q * kHeadDim + tid];
+    const int b = p / a.Hkv, kvh = p % a.Hkv;
+    const int64_t orow = (int64_t)b * a.Hq + (int64_t)kvh * g + h;
+    a.out[orow * kHeadDim + tid] = L > 0.f ? sum / L : 0.f;
+    if (tid == 0 && a.lse != nullptr) a.lse[orow] = L > 0.f ? ml_s[0] + logf(L) : -INFINITY;
+  }
+  __syncthreads();
+}
+
+// ------------------------------------------------- query encoding (in kernel)
+// The block's g query heads are encoded into qc_s[h * W + w] (h < g).
+// bf16 LSH: one m16n8k16 tensor-core tile per (16 rows, 8 bits, 16 dims):
+// products of bf16 values are exact and accumulate in fp32.  Warp w owns bits
+// [8w, 8w + 8); each lane packs its two sign bits and a 4-lane OR builds one
+// byte of a row's code (bit n of the code = bit n % 8 of byte n / 8).
+template <int W>
+struct ProjLoads {
+  static constexpr int kRV = W * 32 * (kHeadDim / 8) / kThreads;
+  static constexpr int kXV = kQRows * (kHeadDim / 8) / kThreads;
+  uint4 rv[kRV], xv[kXV];
+};
+
+// Global loads of R and the query rows into registers (issued early).
+template <int W>
+__device__ __forceinline__ void project_bf16_issue(const __nv_bfloat16* x0, int64_t x_stride, int rows,
+                                                   const __nv_bfloat16* R, ProjLoads<W>& L) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int u = 0; u < ProjLoads<W>::kRV; ++u) {
+    const int i = tid + u * kThreads, n = i / (kHeadDim / 8), c = (i % (kHeadDim / 8)) * 8;
+    L.rv[u] = *reinterpret_cast<const uint4*>(R + (int64_t)n * kHeadDim + c);
+  }
+#pragma unroll
+  for (int u = 0; u < ProjLoads<W>::kXV; ++u) {
+    const int i = tid + u * kThreads, r = i / (kHeadDim / 8), c = (i % (kHeadDim / 8)) * 8;
+    L.xv[u] = r < rows ? *reinterpret_cast<const uint4*>(x0 + (int64_t)r * x_stride + c) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+template <int W>
+__device__ void project_bf16_mma(const ProjLoads<W>& L, int rows, unsigned char* qbuf, uint32_t* qc_s) {
+  constexpr int BITS = W * 32, XP = kHeadDim + 8;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __nv_bfloat16* xq = reinterpret_cast<__nv_bfloat16*>(qbuf);  // [kQRows][XP]
+  __nv_bfloat16* Rq = xq + kQRows * XP;                         // [BITS][XP]
+  unsigned char* qbytes = reinterpret_cast<unsigned char*>(Rq + BITS * XP);  // [kQRows][BITS / 8]
+#pragma unroll
+  for (int u = 0; u < ProjLoads<W>::kRV; ++u) {
+    const int i = tid + u * kThreads, n = i / (kHeadDim / 8), c = (i % (kHeadDim / 8)) * 8;
+    *reinterpret_cast<uint4*>(Rq + n * XP + c) = L.rv[u];
+  }
+#pragma unroll
+  for (int u = 0; u < ProjLoads<W>::kXV; ++u) {
+    const int i = tid + u * kThreads, r = i / (kHeadDim / 8), c = (i % (kHeadDim / 8)) * 8;
+    *reinterpret_cast<uint4*>(xq + r * XP + c) = L.xv[u];
+  }
+  __syncthreads();
+  const int gid = lane >> 2, tq = lane & 3;
+  if (warp < BITS / 8) {
+    const int n0 = warp * 8;
+    for (int m0 = 0; m0 < rows; m0 += 16) {
+      float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+#pragma unroll
+      for (int k0 = 0; k0 < kHeadDim; k0 += 16) {
+        const uint32_t* xa = reinterpret_cast<const uint32_t*>(xq + (m0 + gid) * XP + k0 + 2 * tq);
+        const uint32_t* xb = reinterpret_cast<const uint32_t*>(xq + (m0 + gid + 8) * XP + k0 + 2 * tq);
+        const uint32_t* rb = reinterpret_cast<const uint32_t*>(Rq + (n0 + gid) * XP + k0 + 2 * tq);
+        const uint32_t a0 = xa[0], a1 = xb[0], a2 = xa[4], a3 = xb[4], b0 = rb[0], b1 = rb[4];
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(c0), "+f"(c1), "+f"(c2), "+f"(c3)
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+      }
+      uint32_t lo = ((c0 > 0.f ? 1u : 0u) | (c1 > 0.f ? 2u : 0u)) << (2 * tq);
+      uint32_t hi = ((c2 > 0.f ? 1u : 0u) | (c3 > 0.f ? 2u : 0u)) << (2 * tq);
+      lo |= __shfl_xor_sync(0xffffffffu, lo, 1);
+      lo |= __shfl_xor_sync(0xffffffffu, lo, 2);
+      hi |= __shfl_xor_sync(0xffffffffu, hi, 1);
+      hi |= __shfl_xor_sync(0xffffffffu, hi, 2);
+      if (tq == 0) {
+        if (m0 + gid < rows) qbytes[(m0 + gid) * (BITS / 8) + warp] = (unsigned char)lo;
+        if (m0 + gid + 8 < rows) qbytes[(m0 + gid + 8) * (BITS / 8) + warp] = (unsigned char)hi;
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < rows * W; i += kThreads) qc_s[i] = reinterpret_cast<const uint32_t*>(qbytes)[i];
+}
+
+// fp32 LSH (exact fp32 FMA, no tensor cores): thread t owns bit t % BITS of
+// rows t / BITS, t / BITS + kThreads / BITS, ...
+template <int W>
+__device__ void project_f32_simt(const float* x0, int64_t x_stride, int rows, const float* R, unsigned char* qbuf,
+                                 uint32_t* qc_s) {
+  constexpr int BITS = W * 32, RP = kHeadDim + 1, SL = kThreads / BITS;
+  const int tid = threadIdx.x, lane = tid & 31;
+  float* xs = reinterpret_cast<float*>(qbuf);  // [kQRows][128]
+  float* Rs = xs + kQRows * kHeadDim;          // [BITS][RP]
+  for (int i = tid; i < BITS * kHeadDim; i += kThreads) Rs[(i / kHeadDim) * RP + i % kHeadDim] = R[i];
+  for (int i = tid; i < rows * kHeadDim; i += kThreads) xs[i] = x0[(int64_t)(i / kHeadDim) * x_stride + i % kHeadDim];
+  __syncthreads();
+  const int j = tid % BITS, slot = tid / BITS;
+  for (int r0 = 0; r0 < rows; r0 += SL) {  // a warp shares one slot, so the ballot is converged
+    const int r = r0 + slot;
+    float acc = 0.f;
+    if (r < rows)
+      for (int k = 0; k < kHeadDim; ++k) acc = fmaf(xs[r * kHeadDim + k], Rs[j * RP + k], acc);
+    const uint32_t word = __ballot_sync(0xffffffffu, acc > 0.f);
+    if (lane == 0 && r < rows) qc_s[r * W + j / 32] = word;
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+// Block b serves pair p0 + b / nseg and its candidate range
+// [s0, s1) = [(b % nseg) * per_block, ...): no block straddles two pairs.
+template <int W, int NP, bool ATTEND, typename T>
+__global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* ring = reinterpret_cast<uint32_t*>(smem);
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + a.off_hist);
+  uint16_t* dist_s = reinterpret_cast<uint16_t*>(smem + a.off_dist);
+  int32_t* sel_s = reinterpret_cast<int32_t*>(smem + a.off_sel);
+  float* aq_s = reinterpret_cast<float*>(smem + a.off_aq);  // [g][128] attention queries (fp32)
+  __shared__ uint32_t qc_s[kMaxGroup * W];
+  __shared__ uint32_t warp_tmp[kWarps];
+  __shared__ uint32_t hdr_s[2 * kMaxSegsPerPair];
+  __shared__ int sh[8];
+  __shared__ float m_s[kMaxGroup], l_s[kMaxGroup], alpha_s[kMaxGroup], ml_s[2];
+  __shared__ int tok_s[kRows];
+
+  const int tid = threadIdx.x;
+  const int C = a.C, nseg = a.nseg;
+  const int p = a.p0 + (int)blockIdx.x / nseg, seg = (int)blockIdx.x % nseg;
+  const int s0 = seg * a.per_block, s1 = min(s0 + a.per_block, C);
+  const int len = s1 - s0;
+  const int nt = tid < len ? (len - tid + kThreads - 1) / kThreads : 0;
+  uint32_t* sync = a.sync + kSync * p;
+  (void)aq_s;
+
+  // ---------------- phase A: small loads first, then the code stream ------
+  // Loads issued before the code prefetch are ahead of it in the memory queues.
+  const int gw = a.g * W;
+  const int b = p / a.Hkv, kvh = p % a.Hkv;
+  const int64_t qrow0 = (int64_t)b * a.Hq + (int64_t)kvh * a.g;  // first query head of the pair
+  uint32_t qcode_reg = 0u;
+  ProjLoads<W> pj;
+  if (a.qenc == kQGiven) {
+    if (tid < gw) qcode_reg = __ldg(a.q_codes_in + qrow0 * W + tid);
+  } else if (a.qenc == kQLsh) {
+    if constexpr (sizeof(T) == 2)
+      project_bf16_issue<W>(tptr<__nv_bfloat16>(a.q) + qrow0 * kHeadDim, kHeadDim, a.g, tptr<__nv_bfloat16>(a.R), pj);
+  }
+  float4 aq = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (ATTEND && tid < a.g * (kHeadDim / 4))
+    aq = load4_f32(tptr<T>(a.q) + qrow0 * kHeadDim + (tid / (kHeadDim / 4)) * kHeadDim + (tid % (kHeadDim / 4)) * 4);
+  const uint32_t* pf_ptr = a.k_codes + ((int64_t)p * a.cap + a.lo + s0 + tid) * W;
+  constexpr int64_t kStep = (int64_t)kThreads * W;
+  auto slot = [&](int k) { return ring + ((size_t)(k % kSlots) * kThreads + tid) * 4; };
+#pragma unroll
+  for (int k = 0; k < kSlots; ++k) {
+    if (k < nt) cp_async_code<W>(slot(k), pf_ptr + k * kStep);
+    if (k & 1) cp_async_commit();
+  }
+  const int R_res = a.sink_n + a.local_n;
+  const int n_res = seg < R_res ? (R_res - seg + nseg - 1) / nseg : 0;
+  if (ATTEND && tid < n_res) {
+    // the block's resident rows go to L2 now; they are attended after the scan
+    const int v = seg + tid * nseg;
+    const int t = v < a.sink_n ? v : a.local_start + (v - a.sink_n);
+    prefetch_row_l2<T>(a.K, a.V, (int64_t)p * a.cap + t);
+  }
+  // ---------------- phase A: query codes, histogram reset -------------------
+  if (ATTEND && tid < a.g * (kHeadDim / 4)) *reinterpret_cast<float4*>(&aq_s[tid * 4]) = aq;
+  if (a.qenc == kQGiven) {
+    if (tid < gw) qc_s[tid] = qcode_reg;
+  } else if (a.qenc == kQSign) {
+    const T* x0 = tptr<T>(a.q) + qrow0 * kHeadDim;
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int r = warp; r < a.g; r += kWarps) {
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        const uint32_t word = __ballot_sync(0xffffffffu, to_f32(x0[(int64_t)r * kHeadDim + lane + 32 * w]) > 0.f);
+        if (lane == 0) qc_s[r * W + w] = word;
+      }
+    }
+  } else if constexpr (sizeof(T) == 2) {
+    project_bf16_mma<W>(pj, a.g, smem + a.off_q, qc_s);
+  } else {
+    project_f32_simt<W>(tptr<float>(a.q) + qrow0 * kHeadDim, kHeadDim, a.g, tptr<float>(a.R), smem + a.off_q, qc_s);
+  }
+  for (int i = tid; i < a.nbins_pad; i += kThreads) hist_s[i] = 0u;
+  __syncthreads();
+  if (a.q_codes_out != nullptr && seg == 0)
+    for (int i = tid; i < gw; i += kThreads) a.q_codes_out[qrow0 * W + i] = qc_s[i];
+
+  // ---------------- phase A: distances and histogram -------------------------
+  {
+    Planes<W, NP> planes;
+    build_planes<W, NP>(qc_s, a.g, planes);
+    for (int k = 0; k < nt; k += 2) {
+      cp_async_wait<kGroups - 1>();
+      uint32_t ck0[W], ck1[W];
+      load_slot<W>(slot(k), ck0);
+      const bool two = k + 1 < nt;
+      if (two) load_slot<W>(slot(k + 1), ck1);
+      const int D0 = token_distance<W, NP>(ck0, planes);
+      const int D1 = two ? token_distance<W, NP>(ck1, planes) : 0;
+      const int j0 = tid + k * kThreads;
+      dist_s[j0] = (uint16_t)D0;
+      atomicAdd(&hist_s[D0], 1u);
+      if (two) {
+        dist_s[j0 + kThreads] = (uint16_t)D1;
+        atomicAdd(&hist_s[D1], 1u);
+      }
+      if (k + kSlots < nt) cp_async_code<W>(slot(k), pf_ptr + (k + kSlots) * kStep);
+      if (k + 1 + kSlots < nt) cp_async_code<W>(slot(k + 1), pf_ptr + (k + 1 + kSlots) * kStep);
+      cp_async_commit();
+    }
+    cp_async_wait<0>();
+  }
+  if (tid == 0) {
+    sh[0] = a.nbins;  // lo
+    sh[1] = a.nbins;  // hi
+  }
+  __syncthreads();
+
+  // ---------------- publication: windowed cumulative histogram ---------------
+  const uint32_t k_eff = (uint32_t)a.k_eff;
+  {
+    block_inclusive_scan(hist_s, a.nbins, warp_tmp);
+    const bool enough = hist_s[a.nbins - 1] >= k_eff;
+    for (int v = tid; v < a.nbins; v += kThreads) {
+      const uint32_t prev = v > 0 ? hist_s[v - 1] : 0u;
+      if (hist_s[v] > 0u && prev == 0u) sh[0] = v;
+      if (enough && hist_s[v] >= k_eff && prev < k_eff) sh[1] = v;
+    }
+    __syncthreads();
+    const int lo = sh[0], hi = enough ? sh[1] : a.nbins - 1;
+    uint32_t* cum_out = a.cum + ((int64_t)p * nseg + seg) * a.nbins;
+    for (int v = lo + tid; v <= hi; v += kThreads) cum_out[v] = hist_s[v];
+    if (tid == 0) {
+      a.hdr[((int64_t)p * nseg + seg) * 2 + 0] = (uint32_t)lo;
+      a.hdr[((int64_t)p * nseg + seg) * 2 + 1] = (uint32_t)hi;
+    }
+    __syncthreads();
+    if (tid == 0 && !(a.skip_arrive && blockIdx.x == 0)) red_release_add(&sync[0], 1u);
+  }
+
+  // ---------------- phase B: threshold and ordered compaction ---------------
+  uint32_t n_sel = 0, sel_base = 0;
+  if (tid == 0) sh[2] = wait_count(&sync[0], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
+  __syncthreads();
+  if (sh[2]) {
+    for (int i = tid; i < 2 * nseg; i += kThreads) hdr_s[i] = __ldcg(a.hdr + (int64_t)p * nseg * 2 + i);
+    if (tid == 0) {
+      sh[3] = a.nbins;
+      sh[4] = a.nbins;
+    }
+    __syncthreads();
+    for (int i = tid; i < nseg; i += kThreads) {
+      atomicMin(&sh[3], (int)hdr_s[2 * i]);
+      atomicMin(&sh[4], (int)hdr_s[2 * i + 1]);
+    }
+    __syncthreads();
+    const int wlo = sh[3], whi = sh[4], width = whi - wlo + 1;
+    uint32_t* G = hist_s;           // [width]: all segments of the pair
+    uint32_t* GL = hist_s + width;  // [width]: segments before this one
+    for (int i = tid; i < 2 * width; i += kThreads) hist_s[i] = 0u;
+    if (tid == 0) sh[5] = width - 1;
+    __syncthreads();
+    const uint32_t* cum_p = a.cum + (int64_t)p * nseg * a.nbins;
+    constexpr int kWL = 8;  // window loads in flight per thread
+    const int total = nseg * width;
+    for (int base = 0; base < total; base += kWL * kThreads) {
+      uint32_t val[kWL];
+      int at[kWL];
+#pragma unroll
+      for (int u = 0; u < kWL; ++u) {
+        const int i = base + tid + u * kThreads;
+        val[u] = 0u;
+        at[u] = -1;
+        if (i < total) {
+          const int ss = i / width, v = wlo + i % width;
+          at[u] = (i % width) | (ss < seg ? 0x40000000 : 0);
+          if (v >= (int)hdr_s[2 * ss]) val[u] = __ldcg(cum_p + (int64_t)ss * a.nbins + v);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kWL; ++u) {
+        if (at[u] >= 0 && val[u]) {
+          atomicAdd(&G[at[u] & 0xffff], val[u]);
+          if (at[u] & 0x40000000) atomicAdd(&GL[at[u] & 0xffff], val[u]);
+        }
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < width; i += kThreads)
+      if (G[i] >= k_eff && (i == 0 || G[i - 1] < k_eff)) sh[5] = i;
+    __syncthreads();
+    const int ti = sh[5], thr = wlo + ti;
+    const uint32_t below = ti > 0 ? G[ti - 1] : 0u;
+    const uint32_t lower_lt = ti > 0 ? GL[ti - 1] : 0u;
+    const uint32_t lower_eq = GL[ti] - lower_lt;
+    const uint32_t ties_needed = k_eff - below;
+    const uint32_t quota = ties_needed > lower_eq ? ties_needed - lower_eq : 0u;
+    sel_base = lower_lt + min(lower_eq, ties_needed);
+    // thread tid owns a contiguous run of this block's distances, read 8 at a time
+    const int per8 = (((len + kThreads - 1) / kThreads) + 7) & ~7;
+    const int r0 = min(tid * per8, len), r1 = min(r0 + per8, len);
+    const int nch = (r1 - r0 + 7) >> 3;
+    uint32_t lt = 0, eq = 0;
+    for (int c = 0; c < nch; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(dist_s + r0 + 8 * c);
+      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int Dv = (int)((wd[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+        if (r0 + 8 * c + e < r1) {
+          lt += Dv < thr;
+          eq += Dv == thr;
+        }
+      }
+    }
+    uint32_t tot;
+    const uint32_t ex = block_exclusive(lt | (eq << 16), warp_tmp, &tot);
+    const uint32_t ex_lt = ex & 0xffffu, ex_eq = ex >> 16;
+    n_sel = (tot & 0xffffu) + min(tot >> 16, quota);
+    uint32_t run_eq = ex_eq, pos = ex_lt + min(ex_eq, quota);
+    int32_t* idx_out = a.idx + (int64_t)p * a.top_k + sel_base;
+    int32_t* dist_out = a.dist ? a.dist + (int64_t)p * a.top_k + sel_base : nullptr;
+    if (lt | eq) {
+      for (int c = 0; c < nch; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(dist_s + r0 + 8 * c);
+        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int Dv = (int)((wd[e >> 1] >> (16 * (e & 1))) & 0xffffu);
+          const int i = r0 + 8 * c + e;
+          if (i >= r1) continue;
+          bool take = Dv < thr;
+          if (Dv == thr) take = run_eq++ < quota;
+          if (take) {
+            const int tok = (int)a.lo + s0 + i;
+            if (sel_base + pos < k_eff) {
+              idx_out[pos] = tok;
+              if (dist_out) dist_out[pos] = Dv;
+              if constexpr (ATTEND) {
+                if (pos < (uint32_t)kSelCap) sel_s[pos] = tok;
+                prefetch_row_l2<T>(a.K, a.V, (int64_t)p * a.cap + tok);
+              }
+            } else {
+              report(a.status, HKV_ERR_DEVICE_RANGE);  // unreachable when the counts agree
+            }
+            ++pos;
+          }
+        }
+      }
+    }
+    if (sel_base + n_sel > k_eff) n_sel = k_eff > sel_base ? k_eff - sel_base : 0u;
+  } else if (tid == 0) {
+    report(a.status, HKV_ERR_TIMEOUT);
+  }
+  __syncthreads();
+
+  if constexpr (ATTEND) {
+    // ---------------- attention over selected + resident rows, partial -----
+    float* attn = reinterpret_cast<float*>(smem);
+    const AttnSmem sm{aq_s, attn, attn + kRows * kKP, attn + kRows * kKP + kRows * kHeadDim, tok_s, m_s, l_s, alpha_s};
+    float acc[kOut];
+    const int ns = (int)n_sel;
+    const int32_t* sel_g = a.idx + (int64_t)p * a.top_k + sel_base;
+    attn_begin(a.g, sm, acc);
+    attn_rows<T>(a, p, ns + n_res, [&](int i) -> int {
+      if (i < ns) return i < kSelCap ? sel_s[i] : sel_g[i];
+      const int v = seg + (i - ns) * nseg;
+      return v < a.sink_n ? v : a.local_start + (v - a.sink_n);
+    }, sm, acc);
+    attn_end(a.g, sm, acc, a.part + ((int64_t)p * nseg + seg) * a.g * kPart);
+    __syncthreads();
+    if (tid == 0) sh[6] = (int)atom_acq_rel_add(&sync[2], 1u);
+    __syncthreads();
+    // ---------------- the last g blocks of the pair merge one head each -----
+    const int nm = min(a.g, nseg);
+    const int mi = sh[6] - (nseg - nm);
+    if (mi >= 0) {
+      if (tid == 0) sh[7] = wait_count(&sync[2], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
+      __syncthreads();
+      if (sh[7]) {
+        for (int h = mi; h < a.g; h += nm) merge_head(a, p, nseg, h, sm.K, sm.V, ml_s);
+      } else if (tid == 0) {
+        report(a.status, HKV_ERR_TIMEOUT);
+      }
+      __syncthreads();
+      if (tid == 0 && atomicAdd(&sync[3], 1u) == (uint32_t)(nm - 1)) {
+        sync[2] = 0u;
+        sync[3] = 0u;
+      }
+    }
+  }
+
+  // ---------------- departure; the last block out resets the counters -------
+  __syncthreads();
+  if (tid == 0) sh[2] = atom_acq_rel_add(&sync[1], 1u) == (uint32_t)(nseg - 1);
+  __syncthreads();
+  if (sh[2]) {
+    for (int i = a.k_eff + tid; i < a.top_k; i += kThreads) {
+      a.idx[(int64_t)p * a.top_k + i] = -1;
+      if (a.dist) a.dist[(int64_t)p * a.top_k + i] = -1;
+    }
+    if (tid == 0) {
+      sync[0] = 0u;
+      sync[1] = 0u;
+    }
+  }
+}
+
+using KernelFn = void (*)(FusedArgs);
+
+template <bool ATTEND, typename T>
+KernelFn pick(int words, int np) {
+#define HKV_PICK(WV, NPV) \
+  if (words == WV && np == NPV) return fused_kernel<WV, NPV, ATTEND, T>;
   HKV_PICK(2, 1) HKV_PICK(2, 2) HKV_PICK(2, 3) HKV_PICK(2, 4) HKV_PICK(2, 5)
   HKV_PICK(4, 1) HKV_PICK(4, 2) HKV_PICK(4, 3) HKV_PICK(4, 4) HKV_PICK(4, 5)
 #undef HKV_PICK
   return nullptr;
+}
+
+KernelFn pick_kernel(bool attend, int dtype, int words, int np) {
+  if (!attend) return pick<false, float>(words, np);
+  return dtype == HKV_BF16 ? pick<true, __nv_bfloat16>(words, np) : pick<true, float>(words, np);
 }
 
 int bit_length(int v) {
@@ -382,115 +927,129 @@ int bit_length(int v) {
 }
 
 struct Plan {
-  int nbins, np;
+  int g, nbins, nbins_pad, np;
   int64_t C, lo;
   int k_eff;
-  int pairs_per_launch;
-  int64_t per_block;  // for a full batch of pairs_per_launch pairs
-  int max_seg;
-  int blocks_per_sm;
+  int nseg, per_block, pairs_per_launch;
+  bool cooperative;
+  uint32_t off_q, off_aq, off_sel, off_hist, off_dist;
   size_t smem;
-  size_t ws_sync, ws_hist, ws_cum, ws_total;
+  size_t ws_sync, ws_hdr, ws_cum, ws_part, ws_total;
 };
 
-int make_plan(const RetrieveShape& s, Plan& pl) {
-  const int g = s.Hq / s.Hkv;
+// q_elt: 0 when the query codes are given or are signs; else the element size
+// of q (the kernel stages R and the query rows in shared memory).
+int make_plan(const RetrieveShape& s, bool attend, int q_elt, Plan& pl) {
+  pl.g = s.Hq / s.Hkv;
   const int bits = s.words * 32;
   const Window w = window(s.N, s.n_sink, s.n_local);
   pl.C = w.C;
   pl.lo = w.sink_end;
   pl.k_eff = (int)(s.top_k < w.C ? s.top_k : w.C);
-  pl.nbins = g * bits + 1;
-  pl.np = bit_length(g);
-  pl.smem = align_up(sizeof(uint32_t) * ((pl.nbins + 3) & ~3), 16) + sizeof(uint16_t) * kMaxTokensPerBlock;
-  KernelFn k = pick_kernel(s.words, pl.np);
-  if (k == nullptr) return fail(HKV_ERR_UNSUPPORTED, "no scan kernel for %d-bit codes and group size %d", bits, g);
-  int per_sm = 0;
-  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, pl.smem);
-  if (e != cudaSuccess) return cuda_check(e, "scan occupancy");
-  if (per_sm > kMaxBlocksPerSM) per_sm = kMaxBlocksPerSM;
-  if (per_sm < 1) return fail(HKV_ERR_UNSUPPORTED, "scan kernel does not fit on an SM");
-  pl.blocks_per_sm = per_sm;
-  const int64_t gmax = (int64_t)sm_count() * per_sm;
+  pl.nbins = pl.g * bits + 1;
+  pl.nbins_pad = (pl.nbins + 3) & ~3;
+  pl.np = bit_length(pl.g);
+  if (pick_kernel(attend, HKV_BF16, s.words, pl.np) == nullptr)
+    return fail(HKV_ERR_UNSUPPORTED, "no scan kernel for %d-bit codes and group size %d", bits, pl.g);
+  const int64_t G = sm_count();
   const int P = s.B * s.Hkv;
   const int64_t C = pl.C > 0 ? pl.C : 1;
-  if (C > gmax * kMaxTokensPerBlock)
-    return fail(HKV_ERR_UNSUPPORTED, "%lld candidates exceed one launch (%lld)", (long long)C,
-                (long long)(gmax * kMaxTokensPerBlock));
-  int64_t ppl = P;
-  if ((int64_t)P * C > gmax * kMaxTokensPerBlock) ppl = (gmax * kMaxTokensPerBlock) / C;
-  if (ppl < 1) ppl = 1;
-  pl.pairs_per_launch = (int)ppl;
-  const int64_t Uf = ppl * C;
-  int64_t per = ceil_div(Uf, gmax);
-  if (per < kMinTokensPerBlock) per = kMinTokensPerBlock;
-  per = ceil_div(per, 32) * 32;
-  if (per > kMaxTokensPerBlock) per = kMaxTokensPerBlock;
-  pl.per_block = per;
-  // Smaller (last) batches use the same per_block, so this bounds them too.
-  pl.max_seg = (int)(ceil_div(C, per) + 1);
-  pl.ws_sync = align_up(sizeof(uint32_t) * 2 * P, 256);
-  pl.ws_hist = align_up(sizeof(uint32_t) * (size_t)P * pl.nbins, 256);
-  pl.ws_cum = align_up(sizeof(uint32_t) * (size_t)P * pl.max_seg * pl.nbins, 256);
-  pl.ws_total = pl.ws_sync + pl.ws_hist + pl.ws_cum;
+  // blocks per pair: fill the SMs, keep blocks between kMinTokensPerBlock and
+  // kMaxTokensPerBlock candidates
+  int64_t bpp = std::max<int64_t>(1, G / std::max(P, 1));
+  bpp = std::min<int64_t>(bpp, ceil_div(C, kMinTokensPerBlock));
+  bpp = std::max<int64_t>(bpp, ceil_div(C, kMaxTokensPerBlock));
+  if (bpp > G || bpp + 1 > kMaxSegsPerPair)
+    return fail(HKV_ERR_UNSUPPORTED, "%lld candidates per sequence is too many for one launch", (long long)C);
+  pl.per_block = (int)(ceil_div(ceil_div(C, bpp), 32) * 32);
+  pl.nseg = (int)ceil_div(C, pl.per_block);
+  pl.cooperative = pl.nseg > 1;
+  pl.pairs_per_launch = pl.cooperative ? (int)std::max<int64_t>(1, G / pl.nseg) : std::max(P, 1);
+  const size_t ring = (size_t)kSlots * kThreads * 16;
+  const size_t attn = sizeof(float) * (kRows * kKP + kRows * kHeadDim + kMaxGroup * kRows);
+  size_t off = attend ? std::max(ring, attn) : ring;
+  pl.off_aq = (uint32_t)off;
+  if (attend) off += sizeof(float) * kMaxGroup * kHeadDim;
+  pl.off_q = (uint32_t)off;
+  if (q_elt == 2) off += align_up(sizeof(uint16_t) * (kQRows + bits) * (kHeadDim + 8) + kQRows * bits / 8, 16);
+  if (q_elt == 4) off += align_up(sizeof(float) * (kQRows * kHeadDim + bits * (kHeadDim + 1)), 16);
+  pl.off_sel = (uint32_t)off;
+  if (attend) off += sizeof(int32_t) * kSelCap;
+  pl.off_hist = (uint32_t)off;
+  off += sizeof(uint32_t) * 2 * (size_t)pl.nbins_pad;
+  pl.off_dist = (uint32_t)off;
+  off += sizeof(uint16_t) * ((size_t)pl.per_block + 16);  // vector reads may run 7 past the end
+  pl.smem = align_up(off, 16);
+  pl.ws_sync = align_up(sizeof(uint32_t) * kSync * P, 256);
+  pl.ws_hdr = align_up(sizeof(uint32_t) * 2 * (size_t)P * pl.nseg, 256);
+  pl.ws_cum = align_up(sizeof(uint32_t) * (size_t)P * pl.nseg * pl.nbins, 256);
+  pl.ws_part = attend ? align_up(sizeof(float) * (size_t)P * pl.nseg * pl.g * kPart, 256) : 0;
+  pl.ws_total = pl.ws_sync + pl.ws_hdr + pl.ws_cum + pl.ws_part;
   return HKV_OK;
 }
 
-}  // namespace
-
-size_t retrieve_ws_bytes(const RetrieveShape& s) {
-  Plan pl;
-  if (make_plan(s, pl) != HKV_OK) return 0;
-  return pl.ws_total;
-}
-
-int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,
-                    int32_t* idx, int32_t* dist, void* ws, size_t ws_bytes, int32_t* status,
-                    cudaStream_t st) {
+int launch_fused(const RetrieveShape& s, bool attend, int dtype, int qenc, const void* R,
+                 const uint32_t* q_codes_in, uint32_t* q_codes_out, const uint32_t* k_codes, int32_t* idx,
+                 int32_t* dist, const void* q, const void* K, const void* V, float scale, float* out,
+                 float* lse, void* ws, size_t ws_bytes, int32_t* status, cudaStream_t st) {
   const int P = s.B * s.Hkv;
-  if (P == 0 || s.top_k == 0) return HKV_OK;
+  const int q_elt = (qenc == kQLsh) ? (dtype == HKV_BF16 ? 2 : 4) : 0;
   Plan pl;
-  int rc = make_plan(s, pl);
+  int rc = make_plan(s, attend, q_elt, pl);
   if (rc != HKV_OK) return rc;
-  if (pl.k_eff == 0) {
-    rc = cuda_check(cudaMemsetAsync(idx, 0xff, sizeof(int32_t) * (size_t)P * s.top_k, st), "idx fill");
-    if (rc == HKV_OK && dist)
-      rc = cuda_check(cudaMemsetAsync(dist, 0xff, sizeof(int32_t) * (size_t)P * s.top_k, st), "dist fill");
-    return rc;
-  }
   if (ws_bytes < pl.ws_total || ws == nullptr)
     return fail(HKV_ERR_CAPACITY, "workspace of %zu bytes, %zu needed", ws_bytes, pl.ws_total);
   unsigned char* base = static_cast<unsigned char*>(ws);
-  RetrieveArgs a;
-  a.q_codes = q_codes;
+  const Window w = window(s.N, s.n_sink, s.n_local);
+  FusedArgs a{};
+  a.q_codes_in = q_codes_in;
+  a.q_codes_out = q_codes_out;
+  a.R = R;
+  a.qenc = qenc;
   a.k_codes = k_codes;
   a.idx = idx;
   a.dist = dist;
+  a.q = q;
+  a.K = K;
+  a.V = V;
+  a.out = out;
+  a.lse = lse;
+  a.scale = scale;
   a.Hq = s.Hq;
   a.Hkv = s.Hkv;
-  a.g = s.Hq / s.Hkv;
+  a.g = pl.g;
   a.cap = s.cap;
   a.lo = pl.lo;
-  a.C = pl.C;
+  a.C = (int)pl.C;
   a.k_eff = pl.k_eff;
   a.top_k = s.top_k;
+  a.sink_n = (int)w.sink_end;
+  a.local_start = (int)w.local_start;
+  a.local_n = (int)(s.N - w.local_start);
+  a.nseg = pl.nseg;
   a.per_block = pl.per_block;
   a.nbins = pl.nbins;
-  a.max_seg = pl.max_seg;
+  a.nbins_pad = pl.nbins_pad;
+  a.off_q = pl.off_q;
+  a.off_aq = pl.off_aq;
+  a.off_sel = pl.off_sel;
+  a.off_hist = pl.off_hist;
+  a.off_dist = pl.off_dist;
   a.sync = reinterpret_cast<uint32_t*>(base);
-  a.hist = reinterpret_cast<uint32_t*>(base + pl.ws_sync);
-  a.cum = reinterpret_cast<uint32_t*>(base + pl.ws_sync + pl.ws_hist);
+  a.hdr = reinterpret_cast<uint32_t*>(base + pl.ws_sync);
+  a.cum = reinterpret_cast<uint32_t*>(base + pl.ws_sync + pl.ws_hdr);
+  a.part = reinterpret_cast<float*>(base + pl.ws_sync + pl.ws_hdr + pl.ws_cum);
   a.status = status;
   a.wait_ns = wait_limit_ns();
   a.skip_arrive = (debug_flags() & kDebugSkipArrive) ? 1 : 0;
-  KernelFn k = pick_kernel(s.words, pl.np);
+  KernelFn k = pick_kernel(attend, dtype, s.words, pl.np);
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+  if (e != cudaSuccess) return cuda_check(e, "fused kernel shared memory");
   for (int p0 = 0; p0 < P; p0 += pl.pairs_per_launch) {
     a.p0 = p0;
-    a.P = P - p0 < pl.pairs_per_launch ? P - p0 : pl.pairs_per_launch;
-    const int64_t grid = ceil_div((int64_t)a.P * pl.C, pl.per_block);
+    const int np = P - p0 < pl.pairs_per_launch ? P - p0 : pl.pairs_per_launch;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
+    cfg.gridDim = dim3((unsigned)(np * pl.nseg));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = st;
@@ -498,11 +1057,57 @@ int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint3
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = grid > 1 ? 1 : 0;
+    cfg.numAttrs = pl.cooperative ? 1 : 0;
     rc = cuda_check(cudaLaunchKernelEx(&cfg, k, a), "scan/select launch");
     if (rc != HKV_OK) return rc;
   }
   return HKV_OK;
+}
+
+}  // namespace
+
+size_t retrieve_ws_bytes(const RetrieveShape& s) {
+  Plan pl;
+  if (make_plan(s, false, 0, pl) != HKV_OK) return 0;
+  return pl.ws_total;
+}
+
+size_t decode_ws_bytes(const RetrieveShape& s) {
+  Plan pl;
+  if (make_plan(s, true, 0, pl) != HKV_OK) return 0;
+  return pl.ws_total;
+}
+
+bool decode_encodes_queries(const RetrieveShape& s, int kind, int dtype) {
+  if (kind != HKV_HASH_LSH && kind != HKV_HASH_SIGN) return false;
+  Plan pl;
+  const int q_elt = kind == HKV_HASH_LSH ? (dtype == HKV_BF16 ? 2 : 4) : 0;
+  return make_plan(s, true, q_elt, pl) == HKV_OK && pl.g <= kQRows;
+}
+
+int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,
+                    int32_t* idx, int32_t* dist, void* ws, size_t ws_bytes, int32_t* status,
+                    cudaStream_t st) {
+  const int P = s.B * s.Hkv;
+  if (P == 0 || s.top_k == 0) return HKV_OK;
+  const Window w = window(s.N, s.n_sink, s.n_local);
+  if (w.C == 0) {
+    int rc = cuda_check(cudaMemsetAsync(idx, 0xff, sizeof(int32_t) * (size_t)P * s.top_k, st), "idx fill");
+    if (rc == HKV_OK && dist)
+      rc = cuda_check(cudaMemsetAsync(dist, 0xff, sizeof(int32_t) * (size_t)P * s.top_k, st), "dist fill");
+    return rc;
+  }
+  return launch_fused(s, false, HKV_F32, kQGiven, nullptr, q_codes, nullptr, k_codes, idx, dist, nullptr,
+                      nullptr, nullptr, 0.f, nullptr, nullptr, ws, ws_bytes, status, st);
+}
+
+int launch_decode(const RetrieveShape& s, int dtype, int q_kind, const void* R, const uint32_t* q_codes_in,
+                  uint32_t* q_codes_out, const uint32_t* k_codes, int32_t* idx, const void* q, const void* K,
+                  const void* V, float scale, float* out, float* lse, void* ws, size_t ws_bytes,
+                  int32_t* status, cudaStream_t st) {
+  const int qenc = q_kind == HKV_HASH_LSH ? kQLsh : q_kind == HKV_HASH_SIGN ? kQSign : kQGiven;
+  return launch_fused(s, true, dtype, qenc, R, q_codes_in, q_codes_out, k_codes, idx, nullptr, q, K, V, scale,
+                      out, lse, ws, ws_bytes, status, st);
 }
 
 }  // namespace hkv

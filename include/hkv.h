@@ -64,7 +64,8 @@ typedef enum { HKV_F32 = 0, HKV_BF16 = 1 } hkv_dtype;
 typedef enum {
   HKV_HASH_LSH = 0,  /* code = sign(R x), R [code_bits, head_dim] Gaussian (HashEvict) */
   HKV_HASH_MLP = 1,  /* code = sign(W2 SiLU(W1 x + b1) + b2) (Spotlight Attention) */
-  HKV_HASH_SIGN = 2  /* code = sign(x), code_bits == head_dim (Self-Indexing KVCache) */
+  HKV_HASH_SIGN = 2, /* code = sign(x), code_bits == head_dim (Self-Indexing KVCache) */
+  HKV_HASH_NONE = 3  /* hkv_decode_step only: q_codes already holds the query codes */
 } hkv_hash_kind;
 
 /* One hash function.  Queries and keys may use different ones (the MLP hash
@@ -191,14 +192,17 @@ int hkv_sparse_attend(int B, int Hq, int Hkv, int dtype, const void* q, const vo
 int hkv_lse_merge(int rows, int d, const float* o1, const float* lse1, const float* o2,
                   const float* lse2, float* out, float* lse_out, void* stream);
 
-/* One whole decode step in one launch: encode the query heads with q_hash,
- * scan + select, attend + merge (S2, S4-S8).  Results equal hkv_encode_keys
- * on q, then hkv_retrieve_topk, then hkv_sparse_attend: q_codes and idx
- * bit-identical, out and lse within floating-point rounding.
- *   q_hash   hash for the queries (q_hash->dtype is the dtype of q, K, V)
+/* One whole decode step (S2, S4-S8) in two launches: the query encoder, then
+ * one kernel that scans, selects, attends and merges.  Results equal
+ * hkv_encode_keys on q, then hkv_retrieve_topk, then hkv_sparse_attend:
+ * q_codes and idx bit-identical, out and lse within floating-point rounding.
+ *   q_hash   hash for the queries (q_hash->dtype is the dtype of q, K, V).  With
+ *            kind HKV_HASH_NONE nothing is encoded: q_codes is an input that
+ *            already holds the query codes (one launch)
  *   q        [B, Hq, 128];  k_codes [B, Hkv, cap, code_bits / 32]
  *   K, V     [B, Hkv, cap, 128]
- *   q_codes  nullable [B, Hq, code_bits / 32] out
+ *   q_codes  [B, Hq, code_bits / 32]: output (nullable) or, for HKV_HASH_NONE,
+ *            input (required)
  *   idx      nullable [B, Hkv, top_k] out
  *   out      [B, Hq, 128] fp32;  lse nullable [B, Hq] fp32 */
 int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,

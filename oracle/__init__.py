@@ -98,21 +98,33 @@ def sign_norms(x) -> np.ndarray:
 def encode(kind: str, x, params=None):
     """Codes of the rows of x (any leading shape, last dim d).
     kind "lsh": params = R; "mlp": params = (W1, b1, W2, b2); "sign": none.
-    Returns uint32 codes [..., bits // 32] (and fp16 norms for "sign")."""
-    xs = as_f64(x)
-    lead = xs.shape[:-1]
-    flat = xs.reshape(-1, xs.shape[-1])
-    if kind == "lsh":
-        y = presign_lsh(flat, params)
-    elif kind == "mlp":
-        y = presign_mlp(flat, *params)
-    elif kind == "sign":
-        y = presign_sign(flat)
-    else:
-        raise ValueError(kind)
-    codes = pack_bits(y).reshape(*lead, -1)
+    Returns uint32 codes [..., bits // 32] (and fp16 norms for "sign").
+    Rows are processed in chunks of ROW_CHUNK to bound memory."""
+    lead = tuple(x.shape[:-1])
+    d = x.shape[-1]
+    flat = x.reshape(-1, d)
+    n = flat.shape[0]
+    codes, norms = None, None
+    for r0 in range(0, max(n, 1), ROW_CHUNK):
+        xs = as_f64(flat[r0:r0 + ROW_CHUNK])
+        if kind == "lsh":
+            y = presign_lsh(xs, params)
+        elif kind == "mlp":
+            y = presign_mlp(xs, *params)
+        elif kind == "sign":
+            y = presign_sign(xs)
+        else:
+            raise ValueError(kind)
+        c = pack_bits(y)
+        if codes is None:
+            codes = np.empty((n, c.shape[1]), dtype=np.uint32)
+            norms = np.empty(n, dtype=np.float16) if kind == "sign" else None
+        codes[r0:r0 + ROW_CHUNK] = c
+        if kind == "sign":
+            norms[r0:r0 + ROW_CHUNK] = sign_norms(xs)
+    codes = codes.reshape(*lead, -1)
     if kind == "sign":
-        return codes, sign_norms(flat).reshape(lead)
+        return codes, norms.reshape(lead)
     return codes
 
 
