@@ -27,8 +27,8 @@ __all__ = [
     "HKV_ERR_TIMEOUT", "HKV_ERR_DEVICE_RANGE", "HKV_F32", "HKV_BF16", "HKV_HASH_LSH", "HKV_HASH_MLP",
     "HKV_HASH_SIGN", "HKV_HASH_NONE", "HkvError", "HashParams", "lib", "lib_path", "workspace", "status_word",
     "hkv_version", "hkv_last_error", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
-    "hkv_encode_keys", "hkv_append", "hkv_retrieve_topk", "hkv_sparse_attend", "hkv_lse_merge",
-    "hkv_decode_step", "hkv_debug_set", "EXPORTS",
+    "hkv_encode_keys", "hkv_append", "hkv_retrieve_topk", "hkv_retrieve_topk_static", "hkv_sparse_attend",
+    "hkv_lse_merge", "hkv_decode_step", "hkv_debug_set", "EXPORTS",
 ]
 
 HKV_OK, HKV_ERR_INVALID_ARG, HKV_ERR_UNSUPPORTED, HKV_ERR_CAPACITY = 0, -1, -2, -3
@@ -39,8 +39,8 @@ HKV_HASH_LSH, HKV_HASH_MLP, HKV_HASH_SIGN, HKV_HASH_NONE = 0, 1, 2, 3
 # Every symbol include/hkv.h declares.
 EXPORTS = (
     "hkv_last_error", "hkv_version", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
-    "hkv_encode_keys", "hkv_append", "hkv_retrieve_topk", "hkv_sparse_attend", "hkv_lse_merge",
-    "hkv_decode_step", "hkv_debug_set",
+    "hkv_encode_keys", "hkv_append", "hkv_retrieve_topk", "hkv_retrieve_topk_static", "hkv_sparse_attend",
+    "hkv_lse_merge", "hkv_decode_step", "hkv_debug_set",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -72,6 +72,7 @@ _SIGS = {
     "hkv_encode_keys": (_I, [ctypes.POINTER(hkv_hash), _P, _I64, _I64, _P, _I64, _P, _P, _P]),
     "hkv_append": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P]),
     "hkv_retrieve_topk": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _SZ, _P, _P]),
+    "hkv_retrieve_topk_static": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P]),
     "hkv_sparse_attend": (_I, [_I, _I, _I, _I, _P, _P, _P, _I64, _I64, _P, _I, _I, _I, _F, _P, _P, _P, _SZ, _P, _P]),
     "hkv_lse_merge": (_I, [_I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "hkv_decode_step": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _F,
@@ -252,6 +253,22 @@ def hkv_retrieve_topk(q_codes, k_codes, n_tokens: int, n_sink: int, n_local: int
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _ok(lib().hkv_retrieve_topk(B, Hq, Hkv, W * 32, _ptr(q_codes), _ptr(k_codes), cap, n_tokens, n_sink, n_local,
                                 top_k, _ptr(idx), _ptr(dist), _ptr(ws), nbytes, _ptr(status), _stream(stream)))
+
+
+def hkv_retrieve_topk_static(q_codes, k_codes, n_tokens: int, n_sink: int, n_local: int, top_k: int, idx,
+                             dist=None, status=None, stream=None) -> None:
+    """hkv_retrieve_topk with the library's fixed scratch (no workspace): for
+    callers that cannot allocate device memory.  Make the first call on a
+    device before any stream capture; calls must not overlap on the GPU."""
+    B, Hq, W = q_codes.shape
+    _, Hkv, cap, W2 = k_codes.shape
+    _need(q_codes, "q_codes", _U32)
+    _need(k_codes, "k_codes", _U32, shape=(B, Hkv, cap, W))
+    _need(idx, "idx", torch.int32, shape=(B, Hkv, top_k))
+    if dist is not None:
+        _need(dist, "dist", torch.int32, shape=(B, Hkv, top_k))
+    _ok(lib().hkv_retrieve_topk_static(B, Hq, Hkv, W * 32, _ptr(q_codes), _ptr(k_codes), cap, n_tokens, n_sink,
+                                       n_local, top_k, _ptr(idx), _ptr(dist), _ptr(status), _stream(stream)))
 
 
 def hkv_sparse_attend(q, K, V, n_tokens: int, idx, n_sink: int, n_local: int, out, lse=None,

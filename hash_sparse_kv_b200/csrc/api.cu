@@ -214,6 +214,24 @@ int hkv_retrieve_topk(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_c
   return launch_retrieve(s, q_codes, k_codes, idx, dist, ws, ws_bytes, status, static_cast<cudaStream_t>(stream));
 }
 
+int hkv_retrieve_topk_static(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                             const uint32_t* k_codes, int64_t cap, int64_t n_tokens, int n_sink,
+                             int n_local, int top_k, int32_t* idx, int32_t* dist, int32_t* status,
+                             void* stream) {
+  int rc = check_heads(B, Hq, Hkv);
+  if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
+  if (rc != HKV_OK) return rc;
+  if (code_bits != 64 && code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "code_bits %d (64 or 128)", code_bits);
+  if (B == 0 || top_k == 0) return HKV_OK;
+  if (!q_codes || !k_codes || !idx) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_codes, code_bits / 8)) return fail(HKV_ERR_INVALID_ARG, "k_codes must be %d-byte aligned", code_bits / 8);
+  RetrieveShape s{B, Hq, Hkv, code_bits / 32, cap, n_tokens, n_sink, n_local, top_k};
+  const Window w = window(n_tokens, n_sink, n_local);
+  if (w.C == 0)  // nothing to scan: the workspace path only fills idx/dist with -1
+    return launch_retrieve(s, q_codes, k_codes, idx, dist, nullptr, 0, status, static_cast<cudaStream_t>(stream));
+  return launch_retrieve_static(s, q_codes, k_codes, idx, dist, status, static_cast<cudaStream_t>(stream));
+}
+
 int hkv_sparse_attend(int B, int Hq, int Hkv, int dtype, const void* q, const void* K,
                       const void* V, int64_t cap, int64_t n_tokens, const int32_t* idx,
                       int top_k, int n_sink, int n_local, float scale, float* out, float* lse,

@@ -37,6 +37,10 @@ size_t retrieve_ws_bytes(const RetrieveShape& s);
 int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,
                     int32_t* idx, int32_t* dist, void* ws, size_t ws_bytes, int32_t* status,
                     cudaStream_t st);
+// hkv_retrieve_topk with the library's fixed scratch instead of a workspace.
+constexpr size_t kStaticScratchBytes = (size_t)8 << 20;
+int launch_retrieve_static(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,
+                           int32_t* idx, int32_t* dist, int32_t* status, cudaStream_t st);
 // Scan + select + attention + merge in one launch (candidates must be
 // non-empty).  q_kind HKV_HASH_LSH / HKV_HASH_SIGN: the kernel encodes the
 // query heads itself (when decode_encodes_queries says it can) and writes

@@ -49,6 +49,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "internal.h"
 
@@ -1099,6 +1100,61 @@ int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint3
   }
   return launch_fused(s, false, HKV_F32, kQGiven, nullptr, q_codes, nullptr, k_codes, idx, dist, nullptr,
                       nullptr, nullptr, 0.f, nullptr, nullptr, ws, ws_bytes, status, st);
+}
+
+// ---------------------------------------------------------------------------
+// Retrieval with a fixed, library-owned scratch area instead of a caller
+// workspace, for callers that cannot allocate device memory.  The area is a
+// file-scope device array: every GPU that loads the library holds it until
+// the process exits.  Host code must not pass the array's name to a kernel
+// (on the host it is only a stand-in); its device address is looked up once
+// per device with cudaGetSymbolAddress and cached.
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device.  The first
+// call on a device looks it up and zero-fills it (synchronously).
+int static_scratch(void** out) {
+  int dev = 0;
+  int rc = cuda_check(cudaGetDevice(&dev), "current device");
+  if (rc != HKV_OK) return rc;
+  if (dev < 0 || dev >= kMaxDevices) return fail(HKV_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    rc = cuda_check(cudaGetSymbolAddress(&p, g_static_scratch), "static scratch address");
+    if (rc != HKV_OK) return rc;
+    rc = cuda_check(cudaMemset(p, 0, kStaticScratchBytes), "static scratch zero fill");
+    if (rc != HKV_OK) return rc;
+    g_static_ptr[dev] = p;
+  }
+  *out = g_static_ptr[dev];
+  return HKV_OK;
+}
+}  // namespace
+
+int launch_retrieve_static(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,
+                           int32_t* idx, int32_t* dist, int32_t* status, cudaStream_t st) {
+  const int P = s.B * s.Hkv;
+  if (P == 0 || s.top_k == 0) return HKV_OK;
+  Plan pl;
+  int rc = make_plan(s, false, 0, pl);
+  if (rc != HKV_OK) return rc;
+  if (pl.ws_total > kStaticScratchBytes)
+    return fail(HKV_ERR_CAPACITY, "this shape needs %zu bytes of scratch; the static scratch holds %zu bytes",
+                pl.ws_total, kStaticScratchBytes);
+  void* ws = nullptr;
+  rc = static_scratch(&ws);
+  if (rc != HKV_OK) return rc;
+  // The counters must start at zero; the previous call normally leaves them
+  // so, but clear them anyway (the area keeps the last call's contents).
+  rc = cuda_check(cudaMemsetAsync(ws, 0, pl.ws_sync, st), "static scratch counters");
+  if (rc != HKV_OK) return rc;
+  return launch_retrieve(s, q_codes, k_codes, idx, dist, ws, kStaticScratchBytes, status, st);
 }
 
 int launch_decode(const RetrieveShape& s, int dtype, int q_kind, const void* R, const uint32_t* q_codes_in,

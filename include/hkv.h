@@ -165,6 +165,32 @@ int hkv_retrieve_topk(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_c
                       int n_local, int top_k, int32_t* idx, int32_t* dist, void* ws,
                       size_t ws_bytes, int32_t* status, void* stream);
 
+/* hkv_retrieve_topk without a workspace argument: the same computation and
+ * results, with its scratch taken from a fixed area inside the library.
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory -- for example code running inside a
+ * serving runtime whose allocator owns every byte of the GPU, or a plugin
+ * that is handed buffers but may not call cudaMalloc itself -- and so cannot
+ * provide `ws`.
+ *   - The scratch is one static device array of 8 MiB, present on every GPU
+ *     that loads the library until the process exits.  Shapes whose
+ *     hkv_workspace_bytes-style scratch need exceeds 8 MiB are rejected with
+ *     HKV_ERR_CAPACITY (the message states the bytes needed).  The retrieval
+ *     scratch is about nbins * 4 bytes per block plus 16 bytes per
+ *     (batch, KV head): e.g. 0.5 MiB for 4 KV heads x 512K tokens.
+ *   - The first call on a device looks up the array's device address and
+ *     zero-fills it, synchronously; make that first call before any stream
+ *     capture.  Later calls only enqueue work on `stream`.
+ *   - Every call uses the same array and clears the counters that must
+ *     start at zero before it runs.  Calls that overlap on the GPU (other
+ *     streams, other host threads) race on the array and must not be issued.
+ *   - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ * Arguments are those of hkv_retrieve_topk, without ws and ws_bytes. */
+int hkv_retrieve_topk_static(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                             const uint32_t* k_codes, int64_t cap, int64_t n_tokens, int n_sink,
+                             int n_local, int top_k, int32_t* idx, int32_t* dist, int32_t* status,
+                             void* stream);
+
 /* Sparse attention over sink + selected + local rows, with the log-sum-exp
  * merge of the partials (S6, S7, S8).  Spotlight Attention "Approach" (exact
  * attention over the retrieved tokens); RetrievalAttention "Approach" (exact
