@@ -79,6 +79,13 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def job_throughput(units_per_rank_step: float, ms_local: float, world: int, device):
+    """Whole-job throughput: every rank processes units_per_rank_step per step;
+    the step time is the slowest rank's.  Returns (units/s, max ms)."""
+    ms = max_over_ranks(ms_local, world, device)
+    return units_per_rank_step * world / (ms * 1e-3), ms
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -275,7 +282,8 @@ def run_gpu(args, rank, world, local):
     rc = hkv.hkv_check(status)
     if rc != hkv.HKV_OK:
         raise RuntimeError(f"decode step reported status {rc}")
-    ms = max_over_ranks(ms, world, dev)
+    keys_per_layer = w.B * w.Hkv * w.candidates()
+    value, ms = job_throughput(keys_per_layer * len(layers), ms, world, dev)
     # each kernel alone, one launch per layer
     def qenc_only():
         for L in layers:
@@ -316,9 +324,7 @@ def run_gpu(args, rank, world, local):
     if rc != hkv.HKV_OK:
         raise RuntimeError(f"e2e step reported status {rc}")
 
-    keys_per_layer = w.B * w.Hkv * w.candidates()
     keys_step = keys_per_layer * len(layers) * world
-    value = keys_step / (ms * 1e-3)
     peak, peak_kind = measured_peaks()
     fused_launch_ms = fused_ms / len(layers)
     achieved = per_layer_bytes / (fused_launch_ms * 1e-3) / 1e9
@@ -361,7 +367,9 @@ def run_gpu(args, rank, world, local):
                                   "fused_decode": fused_launch_ms * 1e3,
                                   "retrieve_only": scan_ms * 1e3 / len(layers),
                                   "sparse_attend_only": att_ms * 1e3 / len(layers)},
-        "gpu_launches": 2 * len(layers) * args.steps,
+        # decode with an LSH or sign query hash (query heads per KV head <= 32) is one
+        # fused launch a layer; an MLP query hash adds the separate query encode launch
+        "gpu_launches": (1 if w.hash in ("lsh", "sign") and w.g <= 32 else 2) * len(layers) * args.steps,
         "clocks": clk.summary(),
     }
     del g_step, g_scan, g_e2e
