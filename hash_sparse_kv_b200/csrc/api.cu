@@ -160,7 +160,6 @@ size_t hkv_workspace_bytes(int B, int Hq, int Hkv, int64_t n_tokens, int code_bi
 int hkv_encode_keys(const hkv_hash* hash, const void* x, int64_t rows, int64_t x_stride,
                     uint32_t* codes, int64_t code_stride, uint16_t* norms, int32_t* status,
                     void* stream) {
-  (void)status;
   int rc = check_hash(hash);
   if (rc != HKV_OK) return rc;
   if (rows < 0) return fail(HKV_ERR_INVALID_ARG, "rows %lld", (long long)rows);
@@ -173,13 +172,12 @@ int hkv_encode_keys(const hkv_hash* hash, const void* x, int64_t rows, int64_t x
   if (hash->kind == HKV_HASH_LSH && !aligned(hash->R, 16)) return fail(HKV_ERR_INVALID_ARG, "R must be 16-byte aligned");
   RowMap m{rows, rows, 0, x_stride, 0, code_stride, 0, 1};
   return launch_encode(*hash, x, m, codes, hash->kind == HKV_HASH_SIGN ? norms : nullptr,
-                       static_cast<cudaStream_t>(stream));
+                       static_cast<cudaStream_t>(stream), status);
 }
 
 int hkv_append(const hkv_hash* hash, int B, int Hkv, int T, const void* k_new, const void* v_new,
                void* K, void* V, uint32_t* codes, uint16_t* norms, int64_t capacity, int64_t pos,
                int32_t* status, void* stream) {
-  (void)status;
   int rc = check_hash(hash);
   if (rc != HKV_OK) return rc;
   if (B < 0 || Hkv < 1 || T < 0) return fail(HKV_ERR_INVALID_ARG, "B %d Hkv %d T %d", B, Hkv, T);
@@ -196,7 +194,7 @@ int hkv_append(const hkv_hash* hash, int B, int Hkv, int T, const void* k_new, c
   const int W = hash->code_bits / 32;
   RowMap m{groups * T, T, (int64_t)T * hash->head_dim, hash->head_dim, capacity * W, W, capacity, 1};
   uint16_t* nrm = (hash->kind == HKV_HASH_SIGN && norms) ? norms + pos : nullptr;
-  return launch_encode(*hash, k_new, m, codes + pos * W, nrm, st);
+  return launch_encode(*hash, k_new, m, codes + pos * W, nrm, st, status);
 }
 
 int hkv_retrieve_topk(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
@@ -291,7 +289,7 @@ int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* 
                             decode_encodes_queries(rs, q_hash->kind, q_hash->dtype);
   if (!given_codes && !fused_encode) {
     RowMap m{(int64_t)B * Hq, (int64_t)B * Hq, 0, q_hash->head_dim, 0, W, 0, 1};
-    rc = launch_encode(*q_hash, q, m, qc, nullptr, st);
+    rc = launch_encode(*q_hash, q, m, qc, nullptr, st, status);
     if (rc != HKV_OK) return rc;
   }
   if (w.C == 0 || top_k == 0) {

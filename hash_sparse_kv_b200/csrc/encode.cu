@@ -324,8 +324,9 @@ int run_sign(const void* x, const RowMap& m, uint32_t* codes, uint16_t* norms, c
 }  // namespace
 
 int launch_encode(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes,
-                  uint16_t* norms, cudaStream_t st) {
+                  uint16_t* norms, cudaStream_t st, int32_t* status) {
   if (m.rows == 0) return HKV_OK;
+  if (lsh_tc_eligible(h, x, m, codes)) return launch_lsh_tc(h, x, m, codes, status, st);
   const bool bf = h.dtype == HKV_BF16;
   switch (h.kind) {
     case HKV_HASH_LSH:

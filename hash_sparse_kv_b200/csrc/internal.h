@@ -23,7 +23,11 @@ constexpr int kDebugSkipArrive = 1;
 
 // ---- encoders (encode.cu) ----
 int launch_encode(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes,
-                  uint16_t* norms, cudaStream_t st);
+                  uint16_t* norms, cudaStream_t st, int32_t* status = nullptr);
+// Tensor-core LSH encoder (encode_tc.cu) for large bf16 batches in one group.
+bool lsh_tc_eligible(const hkv_hash& h, const void* x, const RowMap& m, const uint32_t* codes);
+int launch_lsh_tc(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, int32_t* status,
+                  cudaStream_t st);
 int launch_copy_rows(int dtype, int64_t groups, int64_t T, const void* src, void* dst,
                      int64_t dst_group_rows, int64_t dst_row0, cudaStream_t st);
 

@@ -69,6 +69,31 @@ def test_encode_lsh(dtype, bits):
     assert (codes[:, bits // 32:] == -7).all()
 
 
+@pytest.mark.parametrize("bits,rows,x_pitch,code_pitch", [
+    (128, 70001, 192, 8),    # tensor-core path, ragged last tile, padded rows and codes
+    (128, 4096, 128, 4),     # tensor-core path, whole tiles only
+    (64, 4097, 136, 2),      # tensor-core path, 64-bit codes
+    (128, 5000, 128, 7),     # code pitch not a multiple of the code width: SIMT path
+])
+def test_encode_lsh_large_batches(bits, rows, x_pitch, code_pitch):
+    """Large bf16 batches (the prefill of a cache) against the fp64 oracle, bit-exact."""
+    R = synth.gaussian_projection(24, 1, bits, 128, "bf16")
+    from tests.helpers import lsh_bad
+    x = _rows(24, rows, 128, "bf16", lsh_bad(R))
+    wide = torch.zeros(rows, x_pitch, dtype=torch.bfloat16)
+    wide[:, :128] = x
+    xg = wide.to(DEV)[:, :128]
+    W = bits // 32
+    codes = torch.full((rows, code_pitch), -7, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    h = hkv.HashParams.lsh(R.to(DEV))
+    for _ in range(2):
+        hkv.hkv_encode_keys(h, xg, codes[:, :W], status=status)
+    assert hkv.hkv_check(status) == hkv.HKV_OK
+    np.testing.assert_array_equal(u32(codes[:, :W]), oracle.encode("lsh", x, R))
+    assert (codes[:, W:] == -7).all()
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("bits,hidden", [(128, 512), (64, 200)])
 def test_encode_mlp(dtype, bits, hidden):
