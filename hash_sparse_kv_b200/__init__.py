@@ -27,7 +27,8 @@ __all__ = [
     "HKV_ERR_TIMEOUT", "HKV_ERR_DEVICE_RANGE", "HKV_F32", "HKV_BF16", "HKV_HASH_LSH", "HKV_HASH_MLP",
     "HKV_HASH_SIGN", "HKV_HASH_NONE", "HkvError", "HashParams", "lib", "lib_path", "workspace", "status_word",
     "hkv_version", "hkv_last_error", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
-    "hkv_encode_keys", "hkv_append", "hkv_retrieve_topk", "hkv_retrieve_topk_static", "hkv_sparse_attend",
+    "hkv_encode_keys", "hkv_mlp_pack_bytes", "hkv_mlp_pack", "hkv_append", "hkv_retrieve_topk",
+    "hkv_retrieve_topk_static", "hkv_sparse_attend",
     "hkv_lse_merge", "hkv_decode_step", "hkv_debug_set", "EXPORTS",
 ]
 
@@ -39,7 +40,8 @@ HKV_HASH_LSH, HKV_HASH_MLP, HKV_HASH_SIGN, HKV_HASH_NONE = 0, 1, 2, 3
 # Every symbol include/hkv.h declares.
 EXPORTS = (
     "hkv_last_error", "hkv_version", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
-    "hkv_encode_keys", "hkv_append", "hkv_retrieve_topk", "hkv_retrieve_topk_static", "hkv_sparse_attend",
+    "hkv_encode_keys", "hkv_mlp_pack_bytes", "hkv_mlp_pack", "hkv_append", "hkv_retrieve_topk",
+    "hkv_retrieve_topk_static", "hkv_sparse_attend",
     "hkv_lse_merge", "hkv_decode_step", "hkv_debug_set",
 )
 
@@ -58,7 +60,7 @@ class hkv_hash(ctypes.Structure):
         ("kind", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("code_bits", ctypes.c_int32),
         ("hidden", ctypes.c_int32), ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
         ("R", ctypes.c_void_p), ("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p),
-        ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p),
+        ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p), ("packed", ctypes.c_void_p),
     ]
 
 
@@ -70,6 +72,8 @@ _SIGS = {
     "hkv_workspace_bytes": (_SZ, [_I, _I, _I, _I64, _I, _I, _I, _I]),
     "hkv_workspace_reset": (_I, [_P, _SZ, _P]),
     "hkv_encode_keys": (_I, [ctypes.POINTER(hkv_hash), _P, _I64, _I64, _P, _I64, _P, _P, _P]),
+    "hkv_mlp_pack_bytes": (_SZ, [_I, _I]),
+    "hkv_mlp_pack": (_I, [ctypes.POINTER(hkv_hash), _P, _SZ, _P]),
     "hkv_append": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P]),
     "hkv_retrieve_topk": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _SZ, _P, _P]),
     "hkv_retrieve_topk_static": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P]),
@@ -155,10 +159,24 @@ class HashParams:
         return cls(HKV_HASH_LSH, _dtype_code(R), R.shape[0], R=R)
 
     @classmethod
-    def mlp(cls, W1, b1, W2, b2, dtype: int) -> "HashParams":
+    def mlp(cls, W1, b1, W2, b2, dtype: int, pack: bool = True) -> "HashParams":
+        """With pack (bf16 inputs only), the 16-bit weight copy that the
+        tensor-core encoder reads is written by hkv_mlp_pack on the current stream."""
         for t in (W1, b1, W2, b2):
             _need(t, "MLP weight", torch.float32)
-        return cls(HKV_HASH_MLP, dtype, W2.shape[0], W1=W1, b1=b1, W2=W2, b2=b2)
+        hp = cls(HKV_HASH_MLP, dtype, W2.shape[0], W1=W1, b1=b1, W2=W2, b2=b2)
+        if pack and dtype == HKV_BF16:
+            hp.pack()
+        return hp
+
+    def pack(self, stream=None) -> None:
+        n = lib().hkv_mlp_pack_bytes(self.c.hidden, self.code_bits)
+        if n == 0:
+            raise ValueError(f"no packed layout for hidden {self.c.hidden}, code_bits {self.code_bits}")
+        buf = torch.empty(n, dtype=torch.uint8, device=self.tensors[0].device)
+        _ok(lib().hkv_mlp_pack(ctypes.byref(self.c), _ptr(buf), n, _stream(stream)))
+        self.packed = buf
+        self.c.packed = buf.data_ptr()
 
     @classmethod
     def sign(cls, dtype: int, head_dim: int = 128) -> "HashParams":
@@ -223,6 +241,16 @@ def hkv_encode_keys(h: HashParams, x: torch.Tensor, codes: torch.Tensor, norms: 
         _need(norms, "norms", (torch.float16, torch.int16), shape=(x.shape[0],))
     _ok(lib().hkv_encode_keys(ctypes.byref(h.c), _ptr(x), x.shape[0], x.stride(0), _ptr(codes), codes.stride(0),
                               _ptr(norms), _ptr(status), _stream(stream)))
+
+
+def hkv_mlp_pack_bytes(hidden: int, code_bits: int) -> int:
+    return int(lib().hkv_mlp_pack_bytes(hidden, code_bits))
+
+
+def hkv_mlp_pack(h: HashParams, packed: torch.Tensor, stream=None) -> None:
+    """Writes the 16-bit weight copy of an MLP hash into `packed` (uint8, on the device)."""
+    _need(packed, "packed", torch.uint8)
+    _ok(lib().hkv_mlp_pack(ctypes.byref(h.c), _ptr(packed), packed.numel(), _stream(stream)))
 
 
 def hkv_append(h: HashParams, k_new, v_new, K, V, codes, pos: int, norms=None, status=None, stream=None) -> None:

@@ -175,6 +175,18 @@ int hkv_encode_keys(const hkv_hash* hash, const void* x, int64_t rows, int64_t x
                        static_cast<cudaStream_t>(stream), status);
 }
 
+size_t hkv_mlp_pack_bytes(int hidden, int code_bits) { return mlp_pack_bytes(hidden, code_bits); }
+
+int hkv_mlp_pack(const hkv_hash* hash, void* packed, size_t packed_bytes, void* stream) {
+  int rc = check_hash(hash);
+  if (rc != HKV_OK) return rc;
+  if (hash->kind != HKV_HASH_MLP) return fail(HKV_ERR_INVALID_ARG, "hkv_mlp_pack needs an MLP hash");
+  const size_t need = mlp_pack_bytes(hash->hidden, hash->code_bits);
+  if (packed == nullptr || !aligned(packed, 16)) return fail(HKV_ERR_INVALID_ARG, "packed must be 16-byte aligned");
+  if (packed_bytes < need) return fail(HKV_ERR_CAPACITY, "packed holds %zu bytes, %zu needed", packed_bytes, need);
+  return launch_mlp_pack(*hash, packed, static_cast<cudaStream_t>(stream));
+}
+
 int hkv_append(const hkv_hash* hash, int B, int Hkv, int T, const void* k_new, const void* v_new,
                void* K, void* V, uint32_t* codes, uint16_t* norms, int64_t capacity, int64_t pos,
                int32_t* status, void* stream) {

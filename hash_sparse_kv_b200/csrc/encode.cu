@@ -327,6 +327,7 @@ int launch_encode(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* c
                   uint16_t* norms, cudaStream_t st, int32_t* status) {
   if (m.rows == 0) return HKV_OK;
   if (lsh_tc_eligible(h, x, m, codes)) return launch_lsh_tc(h, x, m, codes, status, st);
+  if (mlp_tc_eligible(h, x, m, codes)) return launch_mlp_tc(h, x, m, codes, status, st);
   const bool bf = h.dtype == HKV_BF16;
   switch (h.kind) {
     case HKV_HASH_LSH:

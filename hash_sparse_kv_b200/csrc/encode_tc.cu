@@ -236,6 +236,361 @@ int run_lsh_tc(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* code
   return cuda_check(cudaGetLastError(), "lsh tc launch");
 }
 
+
+// ====================================================================== MLP
+// MLP key encoder on the tensor cores (Spotlight Attention, "Approach": the
+// code is the sign pattern of W2 SiLU(W1 k + b1) + b2).  Per 128-row tile and
+// per 64-unit slice c of the hidden layer:
+//   GEMM1  H_c = X W1_c^T        bf16 x bf16 -> fp32 in TMEM (M 128, N 64, K 128)
+//   epilogue  h = SiLU(H_c + b1_c), rounded to fp16, written to shared memory
+//             in the swizzled K-major layout the next MMA reads
+//   GEMM2  Y += h W2_c^T          fp16 x fp16 -> fp32 in TMEM (M 128, N bits, K 64)
+// and finally bit j = [Y_j + b2_j > 0].  GEMM1 of slice c+1 is issued before
+// GEMM2 of slice c, so the SiLU epilogue of one slice overlaps the MMAs of
+// the next.  SiLU(z) = z sigmoid(z) with sigmoid(z) = (1 + tanh(z / 2)) / 2
+// from the hardware tanh approximation (one special-function op per unit).
+// Error budget against the fp64 definition: fp16 rounding of h (relative
+// 2^-11) and the tanh approximation give |dy| of order 1e-5 here, well inside
+// the 1e-3 margin of the sign test.
+//
+// Warps: 0 TMA (key tiles, weight slices), 1 TMEM + MMA issue, 2..9 epilogue
+// (two warps per TMEM lane quarter, each owning half of the columns).
+constexpr int kMlpThreads = 320;
+constexpr int kMlpEpi = 256;        // epilogue threads
+constexpr int kSlice = 64;          // hidden units per slice
+constexpr int kWStages = 3;
+
+struct MlpTcArgs {
+  uint32_t* codes;
+  int64_t code_stride;
+  int64_t rows;
+  int64_t n_tiles;
+  int n_slices;
+  const float* b1;  // [hidden]
+  const float* b2;  // [bits]
+  int hidden;
+  int32_t* status;
+  uint64_t wait_ns;
+};
+
+template <int BITS>
+struct MlpLayout {
+  static constexpr uint32_t kX = 0;                                   // [2][32 KB] key tiles
+  static constexpr uint32_t kW1Bytes = kSlice * 256;                  // 64 rows x 128 bf16 (2 boxes)
+  static constexpr uint32_t kW2Bytes = BITS * 128;                    // BITS rows x 64 fp16
+  static constexpr uint32_t kWStage = kW1Bytes + kW2Bytes;
+  static constexpr uint32_t kW = kX + 2 * kTileBytes;                 // [kWStages][kWStage]
+  static constexpr uint32_t kA2 = kW + kWStages * kWStage;            // [2][128 rows x 128 B]
+  static constexpr uint32_t kB1 = kA2 + 2 * kTileRows * 128;          // [1024] fp32
+  static constexpr uint32_t kB2 = kB1 + 1024 * 4;                     // [BITS] fp32
+  static constexpr uint32_t kBars = kB2 + BITS * 4;
+  static constexpr uint32_t kEnd = kBars + 256;
+  static constexpr uint32_t kTmemCols = 2 * kSlice + 2 * BITS <= 256 ? 256 : 512;
+  static constexpr uint32_t kTmemY = 2 * kSlice;                      // Y accumulators after the two H buffers
+};
+
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kMlpThreads, 1)
+mlp_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap w1map,
+              const __grid_constant__ CUtensorMap w2map, MlpTcArgs a) {
+  using L = MlpLayout<BITS>;
+  constexpr int W = BITS / 32;
+  constexpr uint32_t kIdesc1 = tc::idesc_bf16_f32(kTileRows, kSlice);
+  // fp16 A and B: the A/B format fields stay 0
+  constexpr uint32_t kIdesc2 = (1u << 4) | ((uint32_t)(BITS >> 3) << 17) | ((uint32_t)(kTileRows >> 4) << 24);
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const uint32_t raw = tc::smem_u32(smem_raw);
+  unsigned char* smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
+  float* b1_s = reinterpret_cast<float*>(smem + L::kB1);
+  float* b2_s = reinterpret_cast<float*>(smem + L::kB2);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint64_t* xfull = bars;            // [2]
+  uint64_t* xempty = bars + 2;       // [2]
+  uint64_t* wfull = bars + 4;        // [kWStages]
+  uint64_t* wempty = wfull + kWStages;
+  uint64_t* hfull = wempty + kWStages;  // [2]
+  uint64_t* hempty = hfull + 2;         // [2] count kMlpEpi
+  uint64_t* afull = hempty + 2;         // [2] count kMlpEpi
+  uint64_t* aempty = afull + 2;         // [2]
+  uint64_t* yfull = aempty + 2;         // [2]
+  uint64_t* yempty = yfull + 2;         // [2] count kMlpEpi
+  uint64_t* done = yempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ns = a.n_slices;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&xfull[i], 1);
+      tc::mbar_init(&xempty[i], 1);
+      tc::mbar_init(&hfull[i], 1);
+      tc::mbar_init(&hempty[i], kMlpEpi);
+      tc::mbar_init(&afull[i], kMlpEpi);
+      tc::mbar_init(&aempty[i], 1);
+      tc::mbar_init(&yfull[i], 1);
+      tc::mbar_init(&yempty[i], kMlpEpi);
+    }
+    for (int s = 0; s < kWStages; ++s) {
+      tc::mbar_init(&wfull[s], 1);
+      tc::mbar_init(&wempty[s], 1);
+    }
+    tc::mbar_init(done, 1);
+    *abort = 0;
+    tc::mbar_init_fence();
+  }
+  for (int i = threadIdx.x; i < ns * kSlice; i += kMlpThreads) b1_s[i] = i < a.hidden ? a.b1[i] : 0.f;
+  for (int i = threadIdx.x; i < BITS; i += kMlpThreads) b2_s[i] = a.b2[i];
+  if (warp == 1) tc::tmem_alloc(tmem_slot, L::kTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer ----------------
+    tc::tma_prefetch_map(&xmap);
+    uint32_t x_armed = 0, x_phase = 0, w_armed = 0, w_phase = 0;
+    auto load_x = [&](int64_t t, int64_t i) -> bool {
+      const int b = (int)(i & 1);
+      if (!tc::mbar_wait(&xempty[b], (uint32_t)((i >> 1) & 1) ^ 1u, abort, a.wait_ns)) return false;
+      tc::mbar_expect_tx(&xfull[b], kTileBytes);
+      unsigned char* dst = smem + L::kX + b * kTileBytes;
+      tc::tma_load_2d(dst, &xmap, 0, (int)(t * kTileRows), &xfull[b]);
+      tc::tma_load_2d(dst + kBoxBytes, &xmap, 64, (int)(t * kTileRows), &xfull[b]);
+      x_armed |= 1u << b;
+      x_phase = (x_phase & ~(1u << b)) | ((uint32_t)((i >> 1) & 1) << b);
+      return true;
+    };
+    int ws = 0;
+    uint32_t wph = 0;
+    bool ok = blockIdx.x < a.n_tiles ? load_x(blockIdx.x, 0) : true;
+    int64_t i = 0;
+    for (int64_t t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x, ++i) {
+      if (t + gridDim.x < a.n_tiles && !load_x(t + gridDim.x, i + 1)) break;
+      for (int c = 0; c < ns; ++c) {
+        if (!tc::mbar_wait(&wempty[ws], wph ^ 1u, abort, a.wait_ns)) {
+          ok = false;
+          break;
+        }
+        unsigned char* dst = smem + L::kW + ws * L::kWStage;
+        tc::mbar_expect_tx(&wfull[ws], L::kWStage);
+        tc::tma_load_2d(dst, &w1map, 0, c * kSlice, &wfull[ws]);
+        tc::tma_load_2d(dst + kSlice * 128, &w1map, 64, c * kSlice, &wfull[ws]);
+        tc::tma_load_2d(dst + L::kW1Bytes, &w2map, c * kSlice, 0, &wfull[ws]);
+        w_armed |= 1u << ws;
+        w_phase = (w_phase & ~(1u << ws)) | (wph << ws);
+        if (++ws == kWStages) {
+          ws = 0;
+          wph ^= 1u;
+        }
+      }
+    }
+    if (*abort) {
+      for (int b = 0; b < 2; ++b)
+        if (x_armed >> b & 1u) tc::mbar_drain(&xfull[b], x_phase >> b & 1u, a.wait_ns);
+      for (int s = 0; s < kWStages; ++s)
+        if (w_armed >> s & 1u) tc::mbar_drain(&wfull[s], w_phase >> s & 1u, a.wait_ns);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    const uint32_t tmem_h = tmem, tmem_y = tmem + L::kTmemY;
+    int ws = 0, ws_prev = 0;
+    uint32_t wph = 0;
+    int64_t hc = 0, ac = 0, i = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x, ++i) {
+      const int xb = (int)(i & 1), yb = (int)(i & 1);
+      if (!(ok = tc::mbar_wait(&xfull[xb], (uint32_t)((i >> 1) & 1), abort, a.wait_ns))) break;
+      const uint32_t x_addr = tc::smem_u32(smem + L::kX + xb * kTileBytes);
+      for (int c = 0; c <= ns && ok; ++c) {
+        if (c < ns) {
+          const int hb = (int)(hc & 1);
+          if (!(ok = tc::mbar_wait(&wfull[ws], wph, abort, a.wait_ns))) break;
+          if (!(ok = tc::mbar_wait(&hempty[hb], (uint32_t)((hc >> 1) & 1) ^ 1u, abort, a.wait_ns))) break;
+          tc::fence_after_sync();
+          const uint32_t w1_addr = tc::smem_u32(smem + L::kW + ws * L::kWStage);
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tc::mma_bf16(tmem_h + hb * kSlice, tc::sw128_desc(x_addr + kb * kBoxBytes + kk * 32),
+                           tc::sw128_desc(w1_addr + kb * (kSlice * 128) + kk * 32), kIdesc1, (kb | kk) != 0);
+          tc::mma_commit(&hfull[hb]);
+          if (c == ns - 1) tc::mma_commit(&xempty[xb]);
+          ++hc;
+        }
+        if (c > 0) {
+          const int cc = c - 1, ab = (int)(ac & 1);
+          if (!(ok = tc::mbar_wait(&afull[ab], (uint32_t)((ac >> 1) & 1), abort, a.wait_ns))) break;
+          if (cc == 0 && !(ok = tc::mbar_wait(&yempty[yb], (uint32_t)((i >> 1) & 1) ^ 1u, abort, a.wait_ns))) break;
+          tc::fence_after_sync();
+          const uint32_t a2_addr = tc::smem_u32(smem + L::kA2 + ab * (kTileRows * 128));
+          const uint32_t w2_addr = tc::smem_u32(smem + L::kW + ws_prev * L::kWStage + L::kW1Bytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc::mma_bf16(tmem_y + yb * BITS, tc::sw128_desc(a2_addr + kk * 32), tc::sw128_desc(w2_addr + kk * 32),
+                         kIdesc2, (cc | kk) != 0);
+          tc::mma_commit(&aempty[ab]);
+          tc::mma_commit(&wempty[ws_prev]);
+          if (cc == ns - 1) tc::mma_commit(&yfull[yb]);
+          ++ac;
+        }
+        if (c < ns) {
+          ws_prev = ws;
+          if (++ws == kWStages) {
+            ws = 0;
+            wph ^= 1u;
+          }
+        }
+      }
+    }
+    tc::mma_commit(done);
+    tc::mbar_drain(done, 0, a.wait_ns);
+  } else if (warp >= 2) {
+    // ---------------- epilogue ----------------
+    const int e = warp - 2;
+    const int quarter = warp & 3, half = e >> 2;  // TMEM lane quarter; which half of the columns
+    const int r = quarter * 32 + lane;            // row within the tile
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    int64_t hc = 0, ac = 0, i = 0;
+    for (int64_t t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++i) {
+      bool ok = true;
+      for (int c = 0; c < ns; ++c) {
+        const int hb = (int)(hc & 1);
+        ok = tc::mbar_wait(&hfull[hb], (uint32_t)((hc >> 1) & 1), abort, a.wait_ns);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        uint32_t v[32];
+        tc::tmem_ld32(tmem + lane_base + hb * kSlice + half * 32, v);
+        tc::tmem_wait_ld();
+        tc::fence_before_sync();
+        tc::mbar_arrive(&hempty[hb]);
+        ++hc;
+        uint32_t hp[16];
+        const float* bb = b1_s + c * kSlice + half * 32;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float z0 = __uint_as_float(v[2 * j]) + bb[2 * j];
+          const float z1 = __uint_as_float(v[2 * j + 1]) + bb[2 * j + 1];
+          const float h0 = z0 * fmaf(0.5f, tanh_approx(0.5f * z0), 0.5f);
+          const float h1 = z1 * fmaf(0.5f, tanh_approx(0.5f * z1), 0.5f);
+          const __half2 p = __floats2half2_rn(h0, h1);
+          hp[j] = *reinterpret_cast<const uint32_t*>(&p);
+        }
+        const int ab = (int)(ac & 1);
+        ok = tc::mbar_wait(&aempty[ab], (uint32_t)((ac >> 1) & 1) ^ 1u, abort, a.wait_ns);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        unsigned char* row = smem + L::kA2 + ab * (kTileRows * 128) + r * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = half * 4 + q;  // 16-byte chunk (8 hidden units) within the 128-byte row
+          *reinterpret_cast<uint4*>(row + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(hp[4 * q], hp[4 * q + 1], hp[4 * q + 2], hp[4 * q + 3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc::mbar_arrive(&afull[ab]);
+        ++ac;
+      }
+      if (!ok) break;
+      const int yb = (int)(i & 1);
+      ok = tc::mbar_wait(&yfull[yb], (uint32_t)((i >> 1) & 1), abort, a.wait_ns);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc::fence_after_sync();
+      constexpr int WH = W / 2;  // words per thread: this warp's half of the code
+      uint32_t words[WH];
+#pragma unroll
+      for (int w = 0; w < WH; ++w) {
+        uint32_t v[32];
+        const int col = (half * WH + w) * 32;
+        tc::tmem_ld32(tmem + L::kTmemY + lane_base + yb * BITS + col, v);
+        tc::tmem_wait_ld();
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) word |= (uint32_t)(__uint_as_float(v[j]) + b2_s[col + j] > 0.f) << j;
+        words[w] = word;
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(&yempty[yb]);
+      const int64_t row = t * kTileRows + r;
+      if (row < a.rows) {
+        uint32_t* dst = a.codes + row * a.code_stride + half * WH;
+        if constexpr (WH == 2)
+          *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
+        else
+          *dst = words[0];
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort) report(a.status, HKV_ERR_TIMEOUT);
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_free(tmem, L::kTmemCols);
+  }
+}
+
+__global__ void mlp_pack_kernel(const float* __restrict__ W1, const float* __restrict__ W2, int hidden, int hp,
+                                int bits, __nv_bfloat16* __restrict__ w1p, __half* __restrict__ w2p) {
+  const int64_t n1 = (int64_t)hp * kHeadDim, n2 = (int64_t)bits * hp;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n1 + n2; i += (int64_t)gridDim.x * blockDim.x) {
+    if (i < n1) {
+      const int64_t row = i / kHeadDim;
+      w1p[i] = __float2bfloat16_rn(row < hidden ? W1[i] : 0.f);
+    } else {
+      const int64_t k = i - n1, j = k / hp, h = k % hp;
+      w2p[k] = __float2half_rn(h < hidden ? W2[j * hidden + h] : 0.f);
+    }
+  }
+}
+
+template <int BITS>
+int run_mlp_tc(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, int32_t* status,
+               cudaStream_t st) {
+  using L = MlpLayout<BITS>;
+  const int hp = (h.hidden + kSlice - 1) / kSlice * kSlice;
+  alignas(64) CUtensorMap xmap, w1map, w2map;
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return fail(HKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  int rc = bf16_rows_map(&xmap, x, m.rows, m.x_row * 2, kTileRows);
+  if (rc == HKV_OK) rc = bf16_rows_map(&w1map, h.packed, hp, kHeadDim * 2, kSlice);
+  if (rc != HKV_OK) return rc;
+  {
+    const void* w2 = static_cast<const unsigned char*>(h.packed) + (size_t)hp * kHeadDim * 2;
+    const cuuint64_t dims[2] = {(cuuint64_t)hp, (cuuint64_t)BITS};
+    const cuuint64_t strides[1] = {(cuuint64_t)hp * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kSlice, (cuuint32_t)BITS};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(&w2map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(w2), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(HKV_ERR_CUDA, "cuTensorMapEncodeTiled (W2) failed (%d)", (int)r);
+  }
+  auto kernel = mlp_tc_kernel<BITS>;
+  constexpr size_t smem = 1024 + L::kEnd;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_check(e, "mlp tc smem attribute");
+  MlpTcArgs args{codes, m.c_row, m.rows, (m.rows + kTileRows - 1) / kTileRows, hp / kSlice, h.b1, h.b2,
+                 h.hidden, status, wait_limit_ns()};
+  const int64_t grid = args.n_tiles < sm_count() ? args.n_tiles : sm_count();
+  kernel<<<(unsigned)grid, kMlpThreads, smem, st>>>(xmap, w1map, w2map, args);
+  return cuda_check(cudaGetLastError(), "mlp tc launch");
+}
+
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 }  // namespace
@@ -251,6 +606,33 @@ bool lsh_tc_eligible(const hkv_hash& h, const void* x, const RowMap& m, const ui
 int launch_lsh_tc(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, int32_t* status,
                   cudaStream_t st) {
   return h.code_bits == 128 ? run_lsh_tc<128>(h, x, m, codes, status, st) : run_lsh_tc<64>(h, x, m, codes, status, st);
+}
+
+bool mlp_tc_eligible(const hkv_hash& h, const void* x, const RowMap& m, const uint32_t* codes) {
+  const int W = h.code_bits / 32;
+  return h.kind == HKV_HASH_MLP && h.packed != nullptr && h.dtype == HKV_BF16 && h.head_dim == kHeadDim &&
+         (h.code_bits == 64 || h.code_bits == 128) && h.hidden >= 1 && h.hidden <= 1024 && m.rows >= kTcMinRows &&
+         m.per_group == m.rows && m.rows < ((int64_t)1 << 31) && aligned_to(x, 16) && (m.x_row * 2) % 16 == 0 &&
+         aligned_to(h.packed, 16) && aligned_to(codes, 2 * W) && m.c_row % (W / 2) == 0;
+}
+
+int launch_mlp_tc(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, int32_t* status,
+                  cudaStream_t st) {
+  return h.code_bits == 128 ? run_mlp_tc<128>(h, x, m, codes, status, st) : run_mlp_tc<64>(h, x, m, codes, status, st);
+}
+
+size_t mlp_pack_bytes(int hidden, int bits) {
+  if (hidden < 1 || hidden > 1024 || (bits != 64 && bits != 128)) return 0;
+  const size_t hp = (size_t)(hidden + kSlice - 1) / kSlice * kSlice;
+  return hp * kHeadDim * 2 + (size_t)bits * hp * 2;
+}
+
+int launch_mlp_pack(const hkv_hash& h, void* packed, cudaStream_t st) {
+  const int hp = (h.hidden + kSlice - 1) / kSlice * kSlice;
+  auto* w1p = static_cast<__nv_bfloat16*>(packed);
+  auto* w2p = reinterpret_cast<__half*>(static_cast<unsigned char*>(packed) + (size_t)hp * kHeadDim * 2);
+  mlp_pack_kernel<<<2 * sm_count(), 256, 0, st>>>(h.W1, h.W2, h.hidden, hp, h.code_bits, w1p, w2p);
+  return cuda_check(cudaGetLastError(), "mlp pack launch");
 }
 
 }  // namespace hkv

@@ -28,6 +28,12 @@ int launch_encode(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* c
 bool lsh_tc_eligible(const hkv_hash& h, const void* x, const RowMap& m, const uint32_t* codes);
 int launch_lsh_tc(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, int32_t* status,
                   cudaStream_t st);
+// Tensor-core MLP encoder (encode_tc.cu); needs the packed 16-bit weights.
+bool mlp_tc_eligible(const hkv_hash& h, const void* x, const RowMap& m, const uint32_t* codes);
+int launch_mlp_tc(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, int32_t* status,
+                  cudaStream_t st);
+size_t mlp_pack_bytes(int hidden, int bits);
+int launch_mlp_pack(const hkv_hash& h, void* packed, cudaStream_t st);
 int launch_copy_rows(int dtype, int64_t groups, int64_t T, const void* src, void* dst,
                      int64_t dst_group_rows, int64_t dst_row0, cudaStream_t st);
 

@@ -78,6 +78,9 @@ typedef enum {
  *   R          LSH: [code_bits, head_dim] in `dtype`, row-major
  *   W1, b1     MLP: [hidden, head_dim], [hidden] fp32
  *   W2, b2     MLP: [code_bits, hidden], [code_bits] fp32
+ *   packed     MLP, nullable: the 16-bit copy of W1 and W2 that hkv_mlp_pack
+ *              wrote.  With it, large bf16 batches are encoded on the tensor
+ *              cores; without it, by the fp32 kernels.
  * For bit-exact agreement with an fp64 reference, R (bf16 inputs) and the MLP
  * weights should hold bf16-representable values and no pre-sign value should
  * lie within 1e-3 of zero. */
@@ -93,6 +96,7 @@ typedef struct {
   const float* b1;
   const float* W2;
   const float* b2;
+  const void* packed;
 } hkv_hash;
 
 /* Description of the last host-side error on this thread ("" if none). */
@@ -133,6 +137,21 @@ int hkv_workspace_reset(void* ws, size_t ws_bytes, void* stream);
 int hkv_encode_keys(const hkv_hash* hash, const void* x, int64_t rows, int64_t x_stride,
                     uint32_t* codes, int64_t code_stride, uint16_t* norms,
                     int32_t* status, void* stream);
+
+/* Bytes of the packed MLP weights for this hidden width and code width:
+ * W1 as bf16 [hidden_pad, head_dim] then W2 as fp16 [code_bits, hidden_pad],
+ * hidden_pad = hidden rounded up to a multiple of 64 (padding is zero).
+ * 0 for an invalid shape. */
+size_t hkv_mlp_pack_bytes(int hidden, int code_bits);
+
+/* Writes the packed copy of hash->W1 and hash->W2 (the MLP hash's weights,
+ * Spotlight Attention "Approach") into `packed` (device, 16-byte aligned,
+ * hkv_mlp_pack_bytes bytes, owned by the caller).  W1 becomes bf16 (exact for
+ * bf16-representable weights), W2 fp16 (exact for such weights above 2^-14 in
+ * magnitude; smaller ones round to the fp16 subnormal grid, an absolute error
+ * below 2^-25).  Set hash->packed to `packed` afterwards; the copy must be
+ * redone whenever W1 or W2 change.  Asynchronous on `stream`. */
+int hkv_mlp_pack(const hkv_hash* hash, void* packed, size_t packed_bytes, void* stream);
 
 /* Decode-time append (S3; HashEvict "Abstract": the binary structure is
  * updated at every decoding step): copy T new key/value rows per (batch, KV

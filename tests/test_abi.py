@@ -67,3 +67,12 @@ def test_zero_sized_calls_are_noops(lib):
     assert lib.hkv_encode_keys(ctypes.byref(h), None, 0, 128, None, 4, None, None, None) == hkv.HKV_OK
     assert lib.hkv_retrieve_topk(0, 4, 4, 128, None, None, 10, 10, 0, 0, 4, None, None, None, 0, None, None) == hkv.HKV_OK
     assert lib.hkv_lse_merge(0, 128, None, None, None, None, None, None, None) == hkv.HKV_OK
+
+
+def test_mlp_pack_sizes(lib):
+    """Packed MLP weights: bf16 W1 [hidden_pad, 128] then fp16 W2 [bits, hidden_pad]."""
+    assert lib.hkv_mlp_pack_bytes(512, 128) == 512 * 128 * 2 + 128 * 512 * 2
+    assert lib.hkv_mlp_pack_bytes(200, 64) == 256 * 128 * 2 + 64 * 256 * 2
+    assert lib.hkv_mlp_pack_bytes(0, 128) == 0
+    assert lib.hkv_mlp_pack_bytes(2048, 128) == 0
+    assert lib.hkv_mlp_pack_bytes(512, 96) == 0

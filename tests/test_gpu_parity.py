@@ -94,6 +94,32 @@ def test_encode_lsh_large_batches(bits, rows, x_pitch, code_pitch):
     assert (codes[:, W:] == -7).all()
 
 
+@pytest.mark.parametrize("bits,hidden,rows,x_pitch,code_pitch", [
+    (128, 512, 40000, 128, 4),   # tensor-core path; 313 tiles, so some CTAs run three
+    (64, 200, 4097, 136, 2),     # hidden width padded to 256 inside the packed weights
+])
+def test_encode_mlp_large_batches(bits, hidden, rows, x_pitch, code_pitch):
+    """Large bf16 batches through the packed-weight tensor-core MLP encoder,
+    bit-exact against the fp64 oracle; the unpacked hash gives the same codes."""
+    params = synth.mlp_params(25, 0, "k", 128, hidden, bits)
+    from tests.helpers import mlp_bad
+    x = _rows(25, rows, 128, "bf16", mlp_bad(params))
+    wide = torch.zeros(rows, x_pitch, dtype=torch.bfloat16)
+    wide[:, :128] = x
+    xg = wide.to(DEV)[:, :128]
+    W = bits // 32
+    want = oracle.encode("mlp", x, params)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    for pack in (True, False):
+        h = hkv.HashParams.mlp(*(t.to(DEV) for t in params), dtype=hkv.HKV_BF16, pack=pack)
+        codes = torch.full((rows, code_pitch), -7, dtype=torch.int32, device=DEV)
+        for _ in range(2):
+            hkv.hkv_encode_keys(h, xg, codes[:, :W], status=status)
+        assert hkv.hkv_check(status) == hkv.HKV_OK
+        np.testing.assert_array_equal(u32(codes[:, :W]), want)
+        assert (codes[:, W:] == -7).all()
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("bits,hidden", [(128, 512), (64, 200)])
 def test_encode_mlp(dtype, bits, hidden):
