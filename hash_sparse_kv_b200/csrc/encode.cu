@@ -7,6 +7,7 @@
 // Bits are packed least-significant first: bit j -> word j / 32, position j % 32.
 // In the projection kernels lane l of a warp owns bits {l + 32 i}, so word i of
 // a row is exactly the warp ballot of (y_{l + 32 i} > 0).
+#include <cooperative_groups.h>
 #include <cstdio>
 
 #include "internal.h"
@@ -130,6 +131,152 @@ lsh_rows_kernel(const T* __restrict__ x, const T* __restrict__ R, RowMap m, uint
 // Tile of 32 rows; warp w owns rows [4w, 4w + 4).  The hidden layer is
 // processed in chunks of 64 units: z = W1 x + b1 (lane l: units l, l + 32),
 // h = SiLU(z), then y += W2[:, chunk] h (lane l: bits l + 32 i).  fp32 throughout.
+// Small batches (queries at decode time): a cluster of 8 CTAs per 16 rows.
+// CTA c computes hidden units [c hs, (c + 1) hs) of all 16 rows into its
+// shared memory; after a cluster barrier every CTA copies the full hidden
+// vectors out of the 8 CTAs' shared memory (distributed shared memory) and
+// computes output bits [c BITS / 8, (c + 1) BITS / 8).  fp32 arithmetic as in
+// the batch kernel; no global scratch and one launch.
+constexpr int kMlpCluster = 8;
+constexpr int kMlpClusterRows = 16;
+// hidden units per CTA: a multiple of 4 so the hidden vectors move as float4
+__host__ __device__ inline int mlp_rows_slice(int hidden) {
+  return ((hidden + kMlpCluster - 1) / kMlpCluster + 3) & ~3;
+}
+
+// Copies n floats (n % 4 == 0, 16-byte aligned) from global memory into
+// shared rows of `cols` floats at pitch `pitch`; every load of a thread is
+// issued before its first shared store.
+template <int U>
+__device__ __forceinline__ void stage_rows(float* dst, int pitch, const float* __restrict__ src, int rows, int cols) {
+  const int per_row = cols / 4, n4 = rows * per_row;
+  for (int base = 0; base < n4; base += U * kThreads) {
+    float4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + threadIdx.x + u * kThreads;
+      if (i < n4) v[u] = __ldg(reinterpret_cast<const float4*>(src) + i);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + threadIdx.x + u * kThreads;
+      if (i < n4) *reinterpret_cast<float4*>(dst + (i / per_row) * pitch + (i % per_row) * 4) = v[u];
+    }
+  }
+}
+
+template <typename T, int BITS>
+__global__ void __cluster_dims__(kMlpCluster, 1, 1) __launch_bounds__(kThreads)
+mlp_rows_kernel(const T* __restrict__ x, const float* __restrict__ W1, const float* __restrict__ b1,
+                const float* __restrict__ W2, const float* __restrict__ b2, int hidden, RowMap m,
+                uint32_t* __restrict__ codes) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  constexpr int D = kHeadDim, R = kMlpClusterRows, NB = BITS / kMlpCluster, DP = D + 4;
+  const int rank = (int)cluster.block_rank(), tid = threadIdx.x;
+  const int64_t row0 = (int64_t)(blockIdx.x / kMlpCluster) * R;
+  const int hs = mlp_rows_slice(hidden), hid_pad = hs * kMlpCluster, HP = ((hidden + 3) & ~3) + 4;
+  const int u0 = rank * hs, un = max(0, min(hs, hidden - u0));
+  extern __shared__ __align__(16) float msm[];
+  float* W1_s = msm;                  // [hs][DP]
+  float* x_s = W1_s + hs * DP;        // [R][D]
+  float* h_s = x_s + R * D;           // [R][hs], read by the whole cluster
+  float* h_all = h_s + R * hs;        // [R][hid_pad]
+  float* W2_s = h_all + R * hid_pad;  // [NB][HP]
+  {
+    // x rows: one 16-byte load per thread (bf16) or two (fp32), issued first
+    constexpr int EPL = 16 / sizeof(T), PER_ROW = D / EPL, N = R * PER_ROW;
+    uint4 raw[(N + kThreads - 1) / kThreads];
+#pragma unroll
+    for (int u = 0; u < (N + kThreads - 1) / kThreads; ++u) {
+      const int i = tid + u * kThreads;
+      const int64_t row = row0 + i / PER_ROW;
+      raw[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < N && row < m.rows) raw[u] = __ldg(reinterpret_cast<const uint4*>(x + m.x_off(row)) + i % PER_ROW);
+    }
+    stage_rows<8>(W1_s, DP, W1 + (int64_t)u0 * D, un, D);
+    if (hidden % 4 == 0) {
+      stage_rows<8>(W2_s, HP, W2 + (int64_t)(rank * NB) * hidden, NB, hidden);
+    } else {
+      for (int i = tid; i < NB * hidden; i += kThreads)
+        W2_s[(i / hidden) * HP + i % hidden] = W2[(int64_t)(rank * NB) * hidden + i];
+    }
+#pragma unroll
+    for (int u = 0; u < (N + kThreads - 1) / kThreads; ++u) {
+      const int i = tid + u * kThreads;
+      if (i >= N) continue;
+      float* dst = x_s + (i / PER_ROW) * D + (i % PER_ROW) * EPL;
+      if constexpr (sizeof(T) == 2) {
+        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(b[e]);
+          dst[2 * e] = f.x;
+          dst[2 * e + 1] = f.y;
+        }
+      } else {
+        *reinterpret_cast<uint4*>(dst) = raw[u];
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < R * hs; i += kThreads) {
+    const int r = i / hs, u = i % hs;
+    float h = 0.f;
+    if (u < un) {
+      float z = b1[u0 + u];
+      const float4* w = reinterpret_cast<const float4*>(W1_s + u * DP);
+      const float4* xv = reinterpret_cast<const float4*>(x_s + r * D);
+#pragma unroll 8
+      for (int k = 0; k < D / 4; ++k) {
+        const float4 a = w[k], c = xv[k];
+        z = fmaf(a.x, c.x, fmaf(a.y, c.y, fmaf(a.z, c.z, fmaf(a.w, c.w, z))));
+      }
+      h = z / (1.f + expf(-z));
+    }
+    h_s[i] = h;
+  }
+  cluster.sync();
+  {
+    // hidden vectors of all 16 rows from the 8 CTAs (hs % 4 == 0: float4 moves)
+    const int n4 = R * hs / 4;
+    for (int base = 0; base < n4; base += kThreads) {
+      float4 v[kMlpCluster];
+      const int i = base + tid;
+#pragma unroll
+      for (int c = 0; c < kMlpCluster; ++c)
+        if (i < n4) v[c] = reinterpret_cast<const float4*>(cluster.map_shared_rank(h_s, c))[i];
+#pragma unroll
+      for (int c = 0; c < kMlpCluster; ++c)
+        if (i < n4) *reinterpret_cast<float4*>(h_all + ((4 * i) / hs) * hid_pad + c * hs + (4 * i) % hs) = v[c];
+    }
+  }
+  cluster.sync();  // no CTA leaves while another still reads its h_s
+  bool bit = false;
+  const int r = tid / NB, j = tid % NB;
+  if (tid < R * NB) {
+    float y = b2[rank * NB + j];
+    const float* w = W2_s + j * HP;
+    const float* h = h_all + r * hid_pad;
+    const int h4 = hidden & ~3;
+    for (int k = 0; k < h4; k += 4) {
+      const float4 a = *reinterpret_cast<const float4*>(w + k), c = *reinterpret_cast<const float4*>(h + k);
+      y = fmaf(a.x, c.x, fmaf(a.y, c.y, fmaf(a.z, c.z, fmaf(a.w, c.w, y))));
+    }
+    for (int k = h4; k < hidden; ++k) y = fmaf(w[k], h[k], y);
+    bit = y > 0.f;
+  }
+  const uint32_t bal = __ballot_sync(0xffffffffu, bit);
+  const int64_t row = row0 + r;
+  if (tid < R * NB && j == 0 && row < m.rows) {
+    const int lane = tid & 31;
+    if constexpr (NB == 16)
+      reinterpret_cast<uint16_t*>(codes)[m.c_off(row) * 2 + rank] = (uint16_t)(bal >> lane);
+    else
+      reinterpret_cast<uint8_t*>(codes)[m.c_off(row) * 4 + rank] = (uint8_t)(bal >> lane);
+  }
+}
+
 template <typename T, int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
 mlp_encode_kernel(const T* __restrict__ x, const float* __restrict__ W1,
@@ -304,6 +451,19 @@ int run_lsh(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, 
 
 template <typename T, int BITS>
 int run_mlp(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, cudaStream_t st) {
+  if (m.rows <= kFewRows) {
+    auto kernel = mlp_rows_kernel<T, BITS>;
+    const int hs = mlp_rows_slice(h.hidden);
+    const size_t smem = sizeof(float) * ((size_t)hs * (kHeadDim + 4) + kMlpClusterRows * kHeadDim +
+                                         (size_t)kMlpClusterRows * hs + (size_t)kMlpClusterRows * hs * kMlpCluster +
+                                         (size_t)(BITS / kMlpCluster) * (((h.hidden + 3) & ~3) + 4));
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_check(e, "mlp rows smem attribute");
+    const int64_t clusters = (m.rows + kMlpClusterRows - 1) / kMlpClusterRows;
+    kernel<<<(unsigned)(clusters * kMlpCluster), kThreads, smem, st>>>(static_cast<const T*>(x), h.W1, h.b1, h.W2,
+                                                                        h.b2, h.hidden, m, codes);
+    return cuda_check(cudaGetLastError(), "mlp rows launch");
+  }
   auto kernel = mlp_encode_kernel<T, BITS>;
   const size_t smem = sizeof(float) * (kHeadDim * 36 + kHeadDim * 65 + 32 * 65 + 64 * (BITS + 1));
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -275,8 +275,11 @@ __device__ __forceinline__ void prefetch_row_l2(const void* K, const void* V, in
   constexpr uint32_t kBytes = kHeadDim * sizeof(T);
   const T* k = tptr<T>(K) + row * kHeadDim;
   const T* v = tptr<T>(V) + row * kHeadDim;
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(k), "r"(kBytes) : "memory");
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(v), "r"(kBytes) : "memory");
+#pragma unroll
+  for (uint32_t o = 0; o < kBytes; o += 128) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(k) + o));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char*>(v) + o));
+  }
 }
 
 // Counter increments that publish the block's earlier writes (after a
@@ -311,60 +314,77 @@ __device__ void attn_begin(int g, const AttnSmem& sm, float (&acc)[kOut]) {
   }
 }
 
-// Adds `nrows` rows (token row_at(i), or -1 to skip) to the online softmax.
+// 16-byte chunk of a K or V row: bf16 rows hold 8 elements per chunk, fp32 rows 4.
+__device__ __forceinline__ void chunk_to_f32(const uint4& raw, float* dst, __nv_bfloat16) {
+  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  const float2 f0 = __bfloat1622float2(b[0]), f1 = __bfloat1622float2(b[1]);
+  const float2 f2 = __bfloat1622float2(b[2]), f3 = __bfloat1622float2(b[3]);
+  *reinterpret_cast<float4*>(dst) = make_float4(f0.x, f0.y, f1.x, f1.y);
+  *reinterpret_cast<float4*>(dst + 4) = make_float4(f2.x, f2.y, f3.x, f3.y);
+}
+__device__ __forceinline__ void chunk_to_f32(const uint4& raw, float* dst, float) {
+  *reinterpret_cast<uint4*>(dst) = raw;
+}
+
+// Adds `nrows` rows (token row_at(i), or -1 to skip) to the online softmax,
+// 64 rows per tile.  The K/V rows of tile i + 1 are loaded into registers
+// while tile i is computed, so the gather latency overlaps the arithmetic.
 template <typename T, typename RowAt>
 __device__ void attn_rows(const FusedArgs& a, int p, int nrows, RowAt row_at, const AttnSmem& sm,
                           float (&acc)[kOut]) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
   const T* Kp = tptr<T>(a.K) + (int64_t)p * a.cap * kHeadDim;
   const T* Vp = tptr<T>(a.V) + (int64_t)p * a.cap * kHeadDim;
-  for (int r0 = 0; r0 < nrows; r0 += kRows) {
-    const int nr = min(kRows, nrows - r0);
-    __syncthreads();
-    for (int i = tid; i < nr; i += kThreads) sm.tok[i] = row_at(r0 + i);
-    __syncthreads();
-    {
-      // all of this thread's K/V loads are issued before any shared store
-      constexpr int kPer = kRows * (kHeadDim / 4) / kThreads;
-      float4 kv[kPer], vv[kPer];
+  constexpr int EPC = 16 / sizeof(T);           // elements per 16-byte chunk
+  constexpr int CPR = kHeadDim / EPC;           // chunks per row
+  constexpr int kPer = kRows * CPR / kThreads;  // chunks of each matrix per thread and tile
+  uint4 kr[kPer], vr[kPer];
+  int tk[kPer];
+  auto issue = [&](int r0) {
 #pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int i = tid + u * kThreads, r = i / (kHeadDim / 4), c = (i % (kHeadDim / 4)) * 4;
-        kv[u] = vv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < nr) {
-          const int t = sm.tok[r];
-          if (t >= 0) {
-            kv[u] = load4_f32(Kp + (int64_t)t * kHeadDim + c);
-            vv[u] = load4_f32(Vp + (int64_t)t * kHeadDim + c);
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        const int i = tid + u * kThreads, r = i / (kHeadDim / 4), c = (i % (kHeadDim / 4)) * 4;
-        if (r < nr) {
-          *reinterpret_cast<float4*>(&sm.K[r * kKP + c]) = kv[u];
-          *reinterpret_cast<float4*>(&sm.V[r * kHeadDim + c]) = vv[u];
-        }
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kThreads, r = i / CPR, c = i % CPR;
+      tk[u] = r0 + r < nrows ? row_at(r0 + r) : -1;
+      kr[u] = vr[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (tk[u] >= 0) {
+        kr[u] = __ldg(reinterpret_cast<const uint4*>(Kp + (int64_t)tk[u] * kHeadDim) + c);
+        vr[u] = __ldg(reinterpret_cast<const uint4*>(Vp + (int64_t)tk[u] * kHeadDim) + c);
       }
     }
+  };
+  if (nrows > 0) issue(0);
+  for (int r0 = 0; r0 < nrows; r0 += kRows) {
+    const int nr = min(kRows, nrows - r0);
+    __syncthreads();  // the previous tile is no longer read
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kThreads, r = i / CPR, c = i % CPR;
+      chunk_to_f32(kr[u], &sm.K[r * kKP + c * EPC], T());
+      chunk_to_f32(vr[u], &sm.V[r * kHeadDim + c * EPC], T());
+      if (c == 0) sm.tok[r] = tk[u];
+    }
     __syncthreads();
+    if (r0 + kRows < nrows) issue(r0 + kRows);  // in flight during this tile's arithmetic
     // logits: four lanes per (head, row), each over interleaved float4 columns
     for (int t0 = 0; t0 < g * nr * 4; t0 += kThreads) {
       const int t = t0 + tid, pr = t >> 2, qd = t & 3;
       const bool live = pr < g * nr;
       const int h = live ? pr / nr : 0, r = live ? pr % nr : 0;
-      float s = 0.f;
+      float s0 = 0.f, s1 = 0.f;
       if (live && sm.tok[r] >= 0) {
         const float* qh = sm.q + h * kHeadDim + 4 * qd;
-        const float* kr = sm.K + r * kKP + 4 * qd;
+        const float* kq = sm.K + r * kKP + 4 * qd;
 #pragma unroll
-        for (int i = 0; i < kHeadDim / 16; ++i) {
-          const float4 x = *reinterpret_cast<const float4*>(qh + 16 * i);
-          const float4 y = *reinterpret_cast<const float4*>(kr + 16 * i);
-          s = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, s))));
+        for (int i = 0; i < kHeadDim / 16; i += 2) {
+          const float4 x0 = *reinterpret_cast<const float4*>(qh + 16 * i);
+          const float4 y0 = *reinterpret_cast<const float4*>(kq + 16 * i);
+          const float4 x1 = *reinterpret_cast<const float4*>(qh + 16 * i + 16);
+          const float4 y1 = *reinterpret_cast<const float4*>(kq + 16 * i + 16);
+          s0 = fmaf(x0.x, y0.x, fmaf(x0.y, y0.y, fmaf(x0.z, y0.z, fmaf(x0.w, y0.w, s0))));
+          s1 = fmaf(x1.x, y1.x, fmaf(x1.y, y1.y, fmaf(x1.z, y1.z, fmaf(x1.w, y1.w, s1))));
         }
       }
+      float s = s0 + s1;
       s += __shfl_xor_sync(0xffffffffu, s, 1);
       s += __shfl_xor_sync(0xffffffffu, s, 2);
       if (live && qd == 0) sm.z[h * kRows + r] = sm.tok[r] >= 0 ? s * a.scale : -INFINITY;
@@ -399,11 +419,206 @@ __device__ void attn_rows(const FusedArgs& a, int p, int nrows, RowAt row_at, co
       const int o = tid + j * kThreads;
       if (o < g * kHeadDim) {
         const int h = o / kHeadDim, c = o % kHeadDim;
-        float s = acc[j] * sm.alpha[h];
-        for (int r = 0; r < nr; ++r) s = fmaf(sm.z[h * kRows + r], sm.V[r * kHeadDim + c], s);
-        acc[j] = s;
+        const float* zh = sm.z + h * kRows;
+        float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+        int r = 0;
+        for (; r + 4 <= nr; r += 4) {
+          p0 = fmaf(zh[r], sm.V[r * kHeadDim + c], p0);
+          p1 = fmaf(zh[r + 1], sm.V[(r + 1) * kHeadDim + c], p1);
+          p2 = fmaf(zh[r + 2], sm.V[(r + 2) * kHeadDim + c], p2);
+          p3 = fmaf(zh[r + 3], sm.V[(r + 3) * kHeadDim + c], p3);
+        }
+        for (; r < nr; ++r) p0 = fmaf(zh[r], sm.V[r * kHeadDim + c], p0);
+        acc[j] = fmaf(acc[j], sm.alpha[h], (p0 + p1) + (p2 + p3));
       }
     }
+  }
+}
+
+// ---- bf16 attention on the tensor cores (mma.sync m16n8k16) ------------------
+// Heads are the M dimension (g <= 16, rows >= g are zero), a 64-row tile of
+// selected tokens is N for the logits and K for P V.  K/V tiles stay bf16 in
+// shared memory (row pitch 272 bytes: conflict-free fragment loads) and are
+// fetched with cp.async, two tiles in flight.  Logits: bf16 q and K, exact
+// products, fp32 accumulation.  P V: the fp32 probabilities are split into
+// bf16 hi + lo parts (two MMAs), so P keeps 16 significant bits.
+constexpr int kKVPitch = kHeadDim + 8;           // bf16 elements per shared row
+constexpr int kKVTile = kRows * kKVPitch * 2;    // bytes per K or V tile
+constexpr int kZP = kRows + 8;                   // probability row pitch (floats)
+constexpr size_t kAttnMmaBytes = 4 * (size_t)kKVTile + sizeof(float) * kMaxGroup * kZP;
+
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(valid ? 16 : 0) : "memory");
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
+  return (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+}
+
+// Splits two fp32 values into bf16 hi and lo pairs (x ~= hi + lo).
+__device__ __forceinline__ void split2(float2 x, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(x.x), h1 = __float2bfloat16_rn(x.y);
+  hi = pack_bf16(h0, h1);
+  lo = pack_bf16(__float2bfloat16_rn(x.x - __bfloat162float(h0)), __float2bfloat16_rn(x.y - __bfloat162float(h1)));
+}
+
+// Online-softmax attention of the pair's query heads over `nrows` rows
+// (token row_at(i), or -1 to skip); writes the partial (m, l, acc) of every
+// head to dst[h * kPart ...].  Uses smem_attn (kAttnMmaBytes) and tok[2 * kRows].
+template <typename RowAt>
+__device__ void attn_mma(const FusedArgs& a, int p, int64_t qrow0, int nrows, RowAt row_at, unsigned char* smem_attn,
+                         int* tok, float* m_s, float* l_s, float* alpha_s, float* dst) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
+  const int gid = lane >> 2, tq = lane & 3;
+  const __nv_bfloat16* Kp = tptr<__nv_bfloat16>(a.K) + (int64_t)p * a.cap * kHeadDim;
+  const __nv_bfloat16* Vp = tptr<__nv_bfloat16>(a.V) + (int64_t)p * a.cap * kHeadDim;
+  float* z = reinterpret_cast<float*>(smem_attn + 4 * kKVTile);  // [kMaxGroup][kZP]
+  auto kbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem_attn + (2 * b) * kKVTile); };
+  auto vbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem_attn + (2 * b + 1) * kKVTile); };
+  constexpr int CPR = kHeadDim / 8;                 // 16-byte chunks per row
+  constexpr int kPer = kRows * CPR / kThreads;      // chunks per thread per matrix
+  auto issue = [&](int r0, int b) {
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kThreads, r = i / CPR, c = i % CPR;
+      const int t = r0 + r < nrows ? row_at(r0 + r) : -1;
+      if (c == 0) tok[b * kRows + r] = t;
+      const int64_t off = (int64_t)(t >= 0 ? t : 0) * kHeadDim + c * 8;
+      cp_async16_zfill(kbuf(b) + r * kKVPitch + c * 8, Kp + off, t >= 0);
+      cp_async16_zfill(vbuf(b) + r * kKVPitch + c * 8, Vp + off, t >= 0);
+    }
+    cp_async_commit();
+  };
+  // query fragments (rows = heads), kept in registers by the eight logit warps
+  uint32_t qa[kHeadDim / 16][4];
+  if (warp < kRows / 8) {
+    const __nv_bfloat16* q0 = tptr<__nv_bfloat16>(a.q) + qrow0 * kHeadDim;
+#pragma unroll
+    for (int ks = 0; ks < kHeadDim / 16; ++ks) {
+      const int k0 = ks * 16 + 2 * tq;
+      qa[ks][0] = gid < g ? *reinterpret_cast<const uint32_t*>(q0 + gid * kHeadDim + k0) : 0u;
+      qa[ks][1] = gid + 8 < g ? *reinterpret_cast<const uint32_t*>(q0 + (gid + 8) * kHeadDim + k0) : 0u;
+      qa[ks][2] = gid < g ? *reinterpret_cast<const uint32_t*>(q0 + gid * kHeadDim + k0 + 8) : 0u;
+      qa[ks][3] = gid + 8 < g ? *reinterpret_cast<const uint32_t*>(q0 + (gid + 8) * kHeadDim + k0 + 8) : 0u;
+    }
+  }
+  if (tid < g) {
+    m_s[tid] = -INFINITY;
+    l_s[tid] = 0.f;
+  }
+  float o[4] = {0.f, 0.f, 0.f, 0.f};  // P V accumulator: heads gid, gid + 8; dims 8 warp + 2 tq (+1)
+  if (nrows > 0) issue(0, 0);
+  for (int r0 = 0, it = 0; r0 < nrows; r0 += kRows, ++it) {
+    const int b = it & 1, nr = min(kRows, nrows - r0);
+    if (r0 + kRows < nrows) {
+      issue(r0 + kRows, b ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const __nv_bfloat16* Ks = kbuf(b);
+    const __nv_bfloat16* Vs = vbuf(b);
+    const int* tk = tok + b * kRows;
+    if (warp < kRows / 8) {
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      const __nv_bfloat16* kr = Ks + (warp * 8 + gid) * kKVPitch + 2 * tq;
+#pragma unroll
+      for (int ks = 0; ks < kHeadDim / 16; ++ks) {
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr + ks * 16);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + ks * 16 + 8);
+        mma16816(c, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+      }
+      const int r = warp * 8 + 2 * tq;
+      const bool v0 = r < nr && tk[r] >= 0, v1 = r + 1 < nr && tk[r + 1] >= 0;
+      if (gid < g) {
+        z[gid * kZP + r] = v0 ? c[0] * a.scale : -INFINITY;
+        z[gid * kZP + r + 1] = v1 ? c[1] * a.scale : -INFINITY;
+      }
+      if (gid + 8 < g) {
+        z[(gid + 8) * kZP + r] = v0 ? c[2] * a.scale : -INFINITY;
+        z[(gid + 8) * kZP + r + 1] = v1 ? c[3] * a.scale : -INFINITY;
+      }
+    }
+    __syncthreads();
+    for (int h = warp; h < g; h += kWarps) {
+      float* zh = z + h * kZP;
+      const float z0 = zh[lane], z1 = zh[lane + 32];
+      float mt = fmaxf(z0, z1);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+      const float m_old = m_s[h];
+      const float m_new = fmaxf(m_old, mt);
+      const float e0 = z0 == -INFINITY ? 0.f : expf(z0 - m_new);
+      const float e1 = z1 == -INFINITY ? 0.f : expf(z1 - m_new);
+      zh[lane] = e0;
+      zh[lane + 32] = e1;
+      float ls = e0 + e1;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
+      if (lane == 0) {
+        const float alpha = m_new == -INFINITY ? 1.f : expf(m_old - m_new);
+        alpha_s[h] = alpha;
+        m_s[h] = m_new;
+        l_s[h] = l_s[h] * alpha + ls;
+      }
+    }
+    __syncthreads();
+    {
+      // warp w: output dims [8w, 8w + 8)
+      const float al0 = gid < g ? alpha_s[gid] : 1.f, al1 = gid + 8 < g ? alpha_s[gid + 8] : 1.f;
+      o[0] *= al0;
+      o[1] *= al0;
+      o[2] *= al1;
+      o[3] *= al1;
+      const int col = warp * 8 + gid;
+#pragma unroll
+      for (int ks = 0; ks < kRows / 16; ++ks) {
+        const int k0 = ks * 16 + 2 * tq;
+        float2 p00 = make_float2(0.f, 0.f), p10 = p00, p01 = p00, p11 = p00;
+        if (gid < g) {
+          p00 = *reinterpret_cast<const float2*>(z + gid * kZP + k0);
+          p01 = *reinterpret_cast<const float2*>(z + gid * kZP + k0 + 8);
+        }
+        if (gid + 8 < g) {
+          p10 = *reinterpret_cast<const float2*>(z + (gid + 8) * kZP + k0);
+          p11 = *reinterpret_cast<const float2*>(z + (gid + 8) * kZP + k0 + 8);
+        }
+        uint32_t h0, l0, h1, l1, h2, l2, h3, l3;
+        split2(p00, h0, l0);
+        split2(p10, h1, l1);
+        split2(p01, h2, l2);
+        split2(p11, h3, l3);
+        const uint32_t b0 = pack_bf16(Vs[k0 * kKVPitch + col], Vs[(k0 + 1) * kKVPitch + col]);
+        const uint32_t b1 = pack_bf16(Vs[(k0 + 8) * kKVPitch + col], Vs[(k0 + 9) * kKVPitch + col]);
+        mma16816(o, h0, h1, h2, h3, b0, b1);
+        mma16816(o, l0, l1, l2, l3, b0, b1);
+      }
+    }
+    __syncthreads();  // buffer b is refilled by the next iteration's issue
+  }
+  // partial of every head: m, l, acc[128]
+  const int c0 = warp * 8 + 2 * tq;
+  if (gid < g) {
+    dst[gid * kPart + 2 + c0] = o[0];
+    dst[gid * kPart + 2 + c0 + 1] = o[1];
+  }
+  if (gid + 8 < g) {
+    dst[(gid + 8) * kPart + 2 + c0] = o[2];
+    dst[(gid + 8) * kPart + 2 + c0 + 1] = o[3];
+  }
+  if (tid < g) {
+    dst[tid * kPart + 0] = m_s[tid];
+    dst[tid * kPart + 1] = l_s[tid];
   }
 }
 
@@ -613,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   __shared__ uint32_t hdr_s[2 * kMaxSegsPerPair];
   __shared__ int sh[8];
   __shared__ float m_s[kMaxGroup], l_s[kMaxGroup], alpha_s[kMaxGroup], ml_s[2];
-  __shared__ int tok_s[kRows];
+  __shared__ int tok_s[2 * kRows];
 
   const int tid = threadIdx.x;
   const int C = a.C, nseg = a.nseg;
@@ -851,18 +1066,24 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
 
   if constexpr (ATTEND) {
     // ---------------- attention over selected + resident rows, partial -----
-    float* attn = reinterpret_cast<float*>(smem);
-    const AttnSmem sm{aq_s, attn, attn + kRows * kKP, attn + kRows * kKP + kRows * kHeadDim, tok_s, m_s, l_s, alpha_s};
-    float acc[kOut];
     const int ns = (int)n_sel;
     const int32_t* sel_g = a.idx + (int64_t)p * a.top_k + sel_base;
-    attn_begin(a.g, sm, acc);
-    attn_rows<T>(a, p, ns + n_res, [&](int i) -> int {
+    auto row_at = [&](int i) -> int {
       if (i < ns) return i < kSelCap ? sel_s[i] : sel_g[i];
       const int v = seg + (i - ns) * nseg;
       return v < a.sink_n ? v : a.local_start + (v - a.sink_n);
-    }, sm, acc);
-    attn_end(a.g, sm, acc, a.part + ((int64_t)p * nseg + seg) * a.g * kPart);
+    };
+    float* dst = a.part + ((int64_t)p * nseg + seg) * a.g * kPart;
+    if constexpr (sizeof(T) == 2) {
+      attn_mma(a, p, qrow0, ns + n_res, row_at, smem, tok_s, m_s, l_s, alpha_s, dst);
+    } else {
+      float* attn = reinterpret_cast<float*>(smem);
+      const AttnSmem sm{aq_s, attn, attn + kRows * kKP, attn + kRows * kKP + kRows * kHeadDim, tok_s, m_s, l_s, alpha_s};
+      float acc[kOut];
+      attn_begin(a.g, sm, acc);
+      attn_rows<T>(a, p, ns + n_res, row_at, sm, acc);
+      attn_end(a.g, sm, acc, dst);
+    }
     __syncthreads();
     if (tid == 0) sh[6] = (int)atom_acq_rel_add(&sync[2], 1u);
     __syncthreads();
@@ -873,7 +1094,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       if (tid == 0) sh[7] = wait_count(&sync[2], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
       __syncthreads();
       if (sh[7]) {
-        for (int h = mi; h < a.g; h += nm) merge_head(a, p, nseg, h, sm.K, sm.V, ml_s);
+        float* scratch = reinterpret_cast<float*>(smem);  // [kMaxSegsPerPair] weights, then [kThreads] sums
+        for (int h = mi; h < a.g; h += nm) merge_head(a, p, nseg, h, scratch, scratch + 256, ml_s);
       } else if (tid == 0) {
         report(a.status, HKV_ERR_TIMEOUT);
       }
@@ -967,7 +1189,7 @@ int make_plan(const RetrieveShape& s, bool attend, int q_elt, Plan& pl) {
   pl.cooperative = pl.nseg > 1;
   pl.pairs_per_launch = pl.cooperative ? (int)std::max<int64_t>(1, G / pl.nseg) : std::max(P, 1);
   const size_t ring = (size_t)kSlots * kThreads * 16;
-  const size_t attn = sizeof(float) * (kRows * kKP + kRows * kHeadDim + kMaxGroup * kRows);
+  const size_t attn = std::max(sizeof(float) * (kRows * kKP + kRows * kHeadDim + kMaxGroup * kRows), kAttnMmaBytes);
   size_t off = attend ? std::max(ring, attn) : ring;
   pl.off_aq = (uint32_t)off;
   if (attend) off += sizeof(float) * kMaxGroup * kHeadDim;
