@@ -96,7 +96,7 @@ struct FusedArgs {
   int nbins, nbins_pad;
   uint32_t off_q, off_aq, off_sel, off_hist, off_dist;  // shared memory carve-up (bytes)
   uint32_t* sync;  // [pairs][kSync]
-  uint32_t* hdr;   // [pairs][nseg][2]: window lo, hi
+  uint32_t* gh;    // [pairs][nbins]: histogram of the pair (returns to zero)
   uint32_t* cum;   // [pairs][nseg][nbins]: cumulative counts, window only
   float* part;     // [pairs][nseg][g][kPart]
   int32_t* status;
@@ -256,6 +256,30 @@ __device__ __forceinline__ uint32_t block_exclusive(uint32_t v, uint32_t* warp_t
   return base + x - v;
 }
 
+// Block-wide sums of x and y; every thread receives both totals.
+// warp_tmp needs 2 * kWarps words.
+__device__ __forceinline__ void block_sum2(uint32_t& x, uint32_t& y, uint32_t* warp_tmp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    x += __shfl_xor_sync(0xffffffffu, x, off);
+    y += __shfl_xor_sync(0xffffffffu, y, off);
+  }
+  __syncthreads();
+  if (lane == 0) {
+    warp_tmp[warp] = x;
+    warp_tmp[kWarps + warp] = y;
+  }
+  __syncthreads();
+  x = 0;
+  y = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    x += warp_tmp[w];
+    y += warp_tmp[kWarps + w];
+  }
+}
+
 // Bounded wait until *ctr >= target.  Returns false on expiry.
 __device__ bool wait_count(const uint32_t* ctr, uint32_t target, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
@@ -286,6 +310,9 @@ __device__ __forceinline__ void prefetch_row_l2(const void* K, const void* V, in
 // __syncthreads, a release by one thread covers the whole block's writes).
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
   uint32_t old;
@@ -639,71 +666,62 @@ __device__ void attn_end(int g, const AttnSmem& sm, const float (&acc)[kOut], fl
   }
 }
 
-// Merge head h of pair p over its nseg partials into out / lse.  Every load
-// of a thread is issued before its results are combined.
-__device__ void merge_head(const FusedArgs& a, int p, int nseg, int h, float* w_s, float* red_s, float* ml_s) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
+// Merge head h of pair p over its nseg partials into out / lse.  Thread t
+// takes column t % 128 of the partials s = t / 128 (mod 4) and folds them
+// into a running (M, L, O) by log-sum-exp rescaling; all loads of a batch are
+// issued before any is used.  The four column groups are then combined.
+// red_s: 3 * kThreads floats of shared scratch.
+__device__ void merge_head(const FusedArgs& a, int p, int nseg, int h, float* red_s) {
+  constexpr int kQ = kThreads / kHeadDim, kB = 16;
+  const int tid = threadIdx.x, g = a.g, c = tid % kHeadDim, q = tid / kHeadDim;
   const float* parts = a.part + (int64_t)p * nseg * g * kPart;
-  if (warp == 0) {
-    constexpr int kPerLane = (kMaxSegsPerPair + 31) / 32;
-    float2 ml[kPerLane];
+  float M = -INFINITY, L = 0.f, O = 0.f;
+  for (int s0 = q; s0 < nseg; s0 += kB * kQ) {
+    float2 ml[kB];
+    float x[kB];
 #pragma unroll
-    for (int u = 0; u < kPerLane; ++u) {
-      const int s = lane + 32 * u;
-      ml[u] = s < nseg ? __ldcg(reinterpret_cast<const float2*>(parts + ((int64_t)s * g + h) * kPart))
-                       : make_float2(-INFINITY, 0.f);
-    }
-    float M = -INFINITY;
-#pragma unroll
-    for (int u = 0; u < kPerLane; ++u) M = fmaxf(M, ml[u].x);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
-#pragma unroll
-    for (int u = 0; u < kPerLane; ++u) {
-      const int s = lane + 32 * u;
-      const float w = ml[u].x == -INFINITY ? 0.f : expf(ml[u].x - M);
-      if (s < nseg) w_s[s] = w;
-      L = fmaf(ml[u].y, w, L);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    if (lane == 0) {
-      ml_s[0] = M;
-      ml_s[1] = L;
-    }
-  }
-  __syncthreads();
-  constexpr int kQuarters = kThreads / kHeadDim;
-  constexpr int kBatch = 8;
-  const int c = tid % kHeadDim, qtr = tid / kHeadDim;
-  float o = 0.f;
-  if (ml_s[1] > 0.f) {
-    for (int s0 = qtr; s0 < nseg; s0 += kBatch * kQuarters) {
-      float x[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int s = s0 + u * kQuarters;
-        x[u] = s < nseg ? __ldcg(parts + ((int64_t)s * g + h) * kPart + 2 + c) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int s = s0 + u * kQuarters;
-        if (s < nseg) o = fmaf(w_s[s], x[u], o);
+    for (int u = 0; u < kB; ++u) {
+      const int s = s0 + u * kQ;
+      ml[u] = make_float2(-INFINITY, 0.f);
+      x[u] = 0.f;
+      if (s < nseg) {
+        const float* src = parts + ((int64_t)s * g + h) * kPart;
+        ml[u] = __ldcg(reinterpret_cast<const float2*>(src));
+        x[u] = __ldcg(src + 2 + c);
       }
     }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      if (ml[u].x == -INFINITY) continue;
+      const float mn = fmaxf(M, ml[u].x);
+      const float a1 = M == -INFINITY ? 0.f : expf(M - mn), a2 = expf(ml[u].x - mn);
+      L = fmaf(L, a1, ml[u].y * a2);
+      O = fmaf(O, a1, x[u] * a2);
+      M = mn;
+    }
   }
-  red_s[qtr * kHeadDim + c] = o;
+  red_s[tid] = M;
+  red_s[kThreads + tid] = L;
+  red_s[2 * kThreads + tid] = O;
   __syncthreads();
   if (tid < kHeadDim) {
-    const float L = ml_s[1];
-    float sum = 0.f;
+    float Mt = -INFINITY;
 #pragma unroll
-    for (int q = 0; q < kQuarters; ++q) sum += red_s[q * kHeadDim + tid];
+    for (int j = 0; j < kQ; ++j) Mt = fmaxf(Mt, red_s[j * kHeadDim + tid]);
+    float Lt = 0.f, Ot = 0.f;
+    if (Mt != -INFINITY) {
+#pragma unroll
+      for (int j = 0; j < kQ; ++j) {
+        const float mj = red_s[j * kHeadDim + tid];
+        const float w = mj == -INFINITY ? 0.f : expf(mj - Mt);
+        Lt = fmaf(red_s[kThreads + j * kHeadDim + tid], w, Lt);
+        Ot = fmaf(red_s[2 * kThreads + j * kHeadDim + tid], w, Ot);
+      }
+    }
     const int b = p / a.Hkv, kvh = p % a.Hkv;
     const int64_t orow = (int64_t)b * a.Hq + (int64_t)kvh * g + h;
-    a.out[orow * kHeadDim + tid] = L > 0.f ? sum / L : 0.f;
-    if (tid == 0 && a.lse != nullptr) a.lse[orow] = L > 0.f ? ml_s[0] + logf(L) : -INFINITY;
+    a.out[orow * kHeadDim + tid] = Lt > 0.f ? Ot / Lt : 0.f;
+    if (tid == 0 && a.lse != nullptr) a.lse[orow] = Lt > 0.f ? Mt + logf(Lt) : -INFINITY;
   }
   __syncthreads();
 }
@@ -824,10 +842,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   int32_t* sel_s = reinterpret_cast<int32_t*>(smem + a.off_sel);
   float* aq_s = reinterpret_cast<float*>(smem + a.off_aq);  // [g][128] attention queries (fp32)
   __shared__ uint32_t qc_s[kMaxGroup * W];
-  __shared__ uint32_t warp_tmp[kWarps];
-  __shared__ uint32_t hdr_s[2 * kMaxSegsPerPair];
+  __shared__ uint32_t warp_tmp[2 * kWarps];
   __shared__ int sh[8];
-  __shared__ float m_s[kMaxGroup], l_s[kMaxGroup], alpha_s[kMaxGroup], ml_s[2];
+  __shared__ float m_s[kMaxGroup], l_s[kMaxGroup], alpha_s[kMaxGroup];
   __shared__ int tok_s[2 * kRows];
 
   const int tid = threadIdx.x;
@@ -920,29 +937,32 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     }
     cp_async_wait<0>();
   }
-  if (tid == 0) {
-    sh[0] = a.nbins;  // lo
-    sh[1] = a.nbins;  // hi
-  }
+  if (tid == 0) sh[1] = a.nbins;  // hi
   __syncthreads();
 
-  // ---------------- publication: windowed cumulative histogram ---------------
+  // ---------------- publication -----------------------------------------------
+  // The segment adds its histogram counts up to hi (its own k-th smallest D,
+  // or all bins if it holds fewer than k_eff tokens) into the pair's global
+  // histogram, and stores its cumulative counts over [0, hi].  The pair's
+  // threshold T is at most min over segments of hi (that segment alone has
+  // k_eff tokens at or below its hi), so the global histogram is complete on
+  // [0, T] and every segment's cumulative counts are known at T - 1 and T.
   const uint32_t k_eff = (uint32_t)a.k_eff;
   {
     block_inclusive_scan(hist_s, a.nbins, warp_tmp);
     const bool enough = hist_s[a.nbins - 1] >= k_eff;
     for (int v = tid; v < a.nbins; v += kThreads) {
       const uint32_t prev = v > 0 ? hist_s[v - 1] : 0u;
-      if (hist_s[v] > 0u && prev == 0u) sh[0] = v;
       if (enough && hist_s[v] >= k_eff && prev < k_eff) sh[1] = v;
     }
     __syncthreads();
-    const int lo = sh[0], hi = enough ? sh[1] : a.nbins - 1;
+    const int hi = enough ? sh[1] : a.nbins - 1;
     uint32_t* cum_out = a.cum + ((int64_t)p * nseg + seg) * a.nbins;
-    for (int v = lo + tid; v <= hi; v += kThreads) cum_out[v] = hist_s[v];
-    if (tid == 0) {
-      a.hdr[((int64_t)p * nseg + seg) * 2 + 0] = (uint32_t)lo;
-      a.hdr[((int64_t)p * nseg + seg) * 2 + 1] = (uint32_t)hi;
+    uint32_t* gh = a.gh + (int64_t)p * a.nbins;
+    for (int v = tid; v <= hi; v += kThreads) {
+      const uint32_t c = hist_s[v], prev = v > 0 ? hist_s[v - 1] : 0u;
+      cum_out[v] = c;
+      if (c != prev) red_add_gpu(&gh[v], c - prev);
     }
     __syncthreads();
     if (tid == 0 && !(a.skip_arrive && blockIdx.x == 0)) red_release_add(&sync[0], 1u);
@@ -953,66 +973,57 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   if (tid == 0) sh[2] = wait_count(&sync[0], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
   __syncthreads();
   if (sh[2]) {
-    for (int i = tid; i < 2 * nseg; i += kThreads) hdr_s[i] = __ldcg(a.hdr + (int64_t)p * nseg * 2 + i);
-    if (tid == 0) {
-      sh[3] = a.nbins;
-      sh[4] = a.nbins;
-    }
-    __syncthreads();
-    for (int i = tid; i < nseg; i += kThreads) {
-      atomicMin(&sh[3], (int)hdr_s[2 * i]);
-      atomicMin(&sh[4], (int)hdr_s[2 * i + 1]);
-    }
-    __syncthreads();
-    const int wlo = sh[3], whi = sh[4], width = whi - wlo + 1;
-    uint32_t* G = hist_s;           // [width]: all segments of the pair
-    uint32_t* GL = hist_s + width;  // [width]: segments before this one
-    for (int i = tid; i < 2 * width; i += kThreads) hist_s[i] = 0u;
-    if (tid == 0) sh[5] = width - 1;
-    __syncthreads();
-    const uint32_t* cum_p = a.cum + (int64_t)p * nseg * a.nbins;
-    constexpr int kWL = 8;  // window loads in flight per thread
-    const int total = nseg * width;
-    for (int base = 0; base < total; base += kWL * kThreads) {
-      uint32_t val[kWL];
-      int at[kWL];
+    {
+      // the pair's histogram, all loads in flight at once
+      constexpr int kGL = 5;  // ceil(2049 / kThreads): up to g * bits + 1 bins
+      const uint32_t* gh = a.gh + (int64_t)p * a.nbins;
+      uint32_t gv[kGL];
 #pragma unroll
-      for (int u = 0; u < kWL; ++u) {
-        const int i = base + tid + u * kThreads;
-        val[u] = 0u;
-        at[u] = -1;
-        if (i < total) {
-          const int ss = i / width, v = wlo + i % width;
-          at[u] = (i % width) | (ss < seg ? 0x40000000 : 0);
-          if (v >= (int)hdr_s[2 * ss]) val[u] = __ldcg(cum_p + (int64_t)ss * a.nbins + v);
-        }
+      for (int u = 0; u < kGL; ++u) {
+        const int v = tid + u * kThreads;
+        gv[u] = v < a.nbins ? __ldcg(gh + v) : 0u;
       }
 #pragma unroll
-      for (int u = 0; u < kWL; ++u) {
-        if (at[u] >= 0 && val[u]) {
-          atomicAdd(&G[at[u] & 0xffff], val[u]);
-          if (at[u] & 0x40000000) atomicAdd(&GL[at[u] & 0xffff], val[u]);
-        }
+      for (int u = 0; u < kGL; ++u) {
+        const int v = tid + u * kThreads;
+        if (v < a.nbins) hist_s[v] = gv[u];
       }
     }
+    if (tid == 0) sh[5] = a.nbins - 1;
     __syncthreads();
-    for (int i = tid; i < width; i += kThreads)
-      if (G[i] >= k_eff && (i == 0 || G[i - 1] < k_eff)) sh[5] = i;
+    block_inclusive_scan(hist_s, a.nbins, warp_tmp);
+    for (int v = tid; v < a.nbins; v += kThreads)
+      if (hist_s[v] >= k_eff && (v == 0 || hist_s[v - 1] < k_eff)) sh[5] = v;
     __syncthreads();
-    const int ti = sh[5], thr = wlo + ti;
-    const uint32_t below = ti > 0 ? G[ti - 1] : 0u;
-    const uint32_t lower_lt = ti > 0 ? GL[ti - 1] : 0u;
-    const uint32_t lower_eq = GL[ti] - lower_lt;
+    const int thr = sh[5];
+    const uint32_t below = thr > 0 ? hist_s[thr - 1] : 0u;
+    // tokens of the lower segments below and at the threshold
+    uint32_t seg_lt = 0, seg_le = 0;
+    for (int ss = tid; ss < seg; ss += kThreads) {
+      const uint32_t* c = a.cum + ((int64_t)p * nseg + ss) * a.nbins;
+      seg_lt += thr > 0 ? __ldcg(c + thr - 1) : 0u;
+      seg_le += __ldcg(c + thr);
+    }
+    block_sum2(seg_lt, seg_le, warp_tmp);
+    const uint32_t lower_lt = seg_lt, lower_eq = seg_le - seg_lt;
     const uint32_t ties_needed = k_eff - below;
     const uint32_t quota = ties_needed > lower_eq ? ties_needed - lower_eq : 0u;
     sel_base = lower_lt + min(lower_eq, ties_needed);
-    // thread tid owns a contiguous run of this block's distances, read 8 at a time
+    // thread tid owns a contiguous run of this block's distances, read 8 at a
+    // time; a chunk whose smallest distance exceeds T (almost all of them,
+    // since k_eff is a small fraction of the tokens) is skipped after one
+    // SIMD minimum
     const int per8 = (((len + kThreads - 1) / kThreads) + 7) & ~7;
     const int r0 = min(tid * per8, len), r1 = min(r0 + per8, len);
     const int nch = (r1 - r0 + 7) >> 3;
+    auto chunk_min = [](const uint4& v) {
+      const uint32_t m = __vminu2(__vminu2(v.x, v.y), __vminu2(v.z, v.w));
+      return min(m & 0xffffu, m >> 16);
+    };
     uint32_t lt = 0, eq = 0;
     for (int c = 0; c < nch; ++c) {
       const uint4 v = *reinterpret_cast<const uint4*>(dist_s + r0 + 8 * c);
+      if (chunk_min(v) > (uint32_t)thr) continue;
       const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -1033,6 +1044,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     if (lt | eq) {
       for (int c = 0; c < nch; ++c) {
         const uint4 v = *reinterpret_cast<const uint4*>(dist_s + r0 + 8 * c);
+        if (chunk_min(v) > (uint32_t)thr) continue;
         const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -1094,8 +1106,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       if (tid == 0) sh[7] = wait_count(&sync[2], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
       __syncthreads();
       if (sh[7]) {
-        float* scratch = reinterpret_cast<float*>(smem);  // [kMaxSegsPerPair] weights, then [kThreads] sums
-        for (int h = mi; h < a.g; h += nm) merge_head(a, p, nseg, h, scratch, scratch + 256, ml_s);
+        for (int h = mi; h < a.g; h += nm) merge_head(a, p, nseg, h, reinterpret_cast<float*>(smem));
       } else if (tid == 0) {
         report(a.status, HKV_ERR_TIMEOUT);
       }
@@ -1116,6 +1127,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       a.idx[(int64_t)p * a.top_k + i] = -1;
       if (a.dist) a.dist[(int64_t)p * a.top_k + i] = -1;
     }
+    for (int v = tid; v < a.nbins; v += kThreads) a.gh[(int64_t)p * a.nbins + v] = 0u;
     if (tid == 0) {
       sync[0] = 0u;
       sync[1] = 0u;
@@ -1157,7 +1169,7 @@ struct Plan {
   bool cooperative;
   uint32_t off_q, off_aq, off_sel, off_hist, off_dist;
   size_t smem;
-  size_t ws_sync, ws_hdr, ws_cum, ws_part, ws_total;
+  size_t ws_sync, ws_gh, ws_cum, ws_part, ws_total;
 };
 
 // q_elt: 0 when the query codes are given or are signs; else the element size
@@ -1204,10 +1216,10 @@ int make_plan(const RetrieveShape& s, bool attend, int q_elt, Plan& pl) {
   off += sizeof(uint16_t) * ((size_t)pl.per_block + 16);  // vector reads may run 7 past the end
   pl.smem = align_up(off, 16);
   pl.ws_sync = align_up(sizeof(uint32_t) * kSync * P, 256);
-  pl.ws_hdr = align_up(sizeof(uint32_t) * 2 * (size_t)P * pl.nseg, 256);
+  pl.ws_gh = align_up(sizeof(uint32_t) * (size_t)P * pl.nbins, 256);
   pl.ws_cum = align_up(sizeof(uint32_t) * (size_t)P * pl.nseg * pl.nbins, 256);
   pl.ws_part = attend ? align_up(sizeof(float) * (size_t)P * pl.nseg * pl.g * kPart, 256) : 0;
-  pl.ws_total = pl.ws_sync + pl.ws_hdr + pl.ws_cum + pl.ws_part;
+  pl.ws_total = pl.ws_sync + pl.ws_gh + pl.ws_cum + pl.ws_part;
   return HKV_OK;
 }
 
@@ -1259,9 +1271,9 @@ int launch_fused(const RetrieveShape& s, bool attend, int dtype, int qenc, const
   a.off_hist = pl.off_hist;
   a.off_dist = pl.off_dist;
   a.sync = reinterpret_cast<uint32_t*>(base);
-  a.hdr = reinterpret_cast<uint32_t*>(base + pl.ws_sync);
-  a.cum = reinterpret_cast<uint32_t*>(base + pl.ws_sync + pl.ws_hdr);
-  a.part = reinterpret_cast<float*>(base + pl.ws_sync + pl.ws_hdr + pl.ws_cum);
+  a.gh = reinterpret_cast<uint32_t*>(base + pl.ws_sync);
+  a.cum = reinterpret_cast<uint32_t*>(base + pl.ws_sync + pl.ws_gh);
+  a.part = reinterpret_cast<float*>(base + pl.ws_sync + pl.ws_gh + pl.ws_cum);
   a.status = status;
   a.wait_ns = wait_limit_ns();
   a.skip_arrive = (debug_flags() & kDebugSkipArrive) ? 1 : 0;
@@ -1372,9 +1384,10 @@ int launch_retrieve_static(const RetrieveShape& s, const uint32_t* q_codes, cons
   void* ws = nullptr;
   rc = static_scratch(&ws);
   if (rc != HKV_OK) return rc;
-  // The counters must start at zero; the previous call normally leaves them
-  // so, but clear them anyway (the area keeps the last call's contents).
-  rc = cuda_check(cudaMemsetAsync(ws, 0, pl.ws_sync, st), "static scratch counters");
+  // The counters and the pair histograms must start at zero.  A call of the
+  // same shape leaves them so, but the previous call may have had another
+  // shape (and so another layout of the area), so clear them every time.
+  rc = cuda_check(cudaMemsetAsync(ws, 0, pl.ws_sync + pl.ws_gh, st), "static scratch counters");
   if (rc != HKV_OK) return rc;
   return launch_retrieve(s, q_codes, k_codes, idx, dist, ws, kStaticScratchBytes, status, st);
 }

@@ -116,8 +116,9 @@ int hkv_check(int32_t* status, void* stream);
  * first use (hkv_workspace_reset).  Each call returns the counters and
  * histograms that must start at zero to zero before it ends, including calls
  * that end in a device error, so one workspace serves any number of calls in
- * a row (and CUDA-graph replays).  Calls that share one workspace must not
- * overlap on the GPU. */
+ * a row (and CUDA-graph replays).  The layout depends on the shape: before
+ * a call of another shape reuses a workspace, zero it again.  Calls that
+ * share one workspace must not overlap on the GPU. */
 size_t hkv_workspace_bytes(int B, int Hq, int Hkv, int64_t n_tokens, int code_bits, int top_k,
                            int n_sink, int n_local);
 
@@ -195,13 +196,14 @@ int hkv_retrieve_topk(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_c
  *     that loads the library until the process exits.  Shapes whose
  *     hkv_workspace_bytes-style scratch need exceeds 8 MiB are rejected with
  *     HKV_ERR_CAPACITY (the message states the bytes needed).  The retrieval
- *     scratch is about nbins * 4 bytes per block plus 16 bytes per
- *     (batch, KV head): e.g. 0.5 MiB for 4 KV heads x 512K tokens.
+ *     scratch is about nbins * 4 bytes per block plus nbins * 4 + 16 bytes
+ *     per (batch, KV head), nbins = g * code_bits + 1: e.g. 0.2 MiB for
+ *     4 KV heads x 512K tokens with g = 7.
  *   - The first call on a device looks up the array's device address and
  *     zero-fills it, synchronously; make that first call before any stream
  *     capture.  Later calls only enqueue work on `stream`.
- *   - Every call uses the same array and clears the counters that must
- *     start at zero before it runs.  Calls that overlap on the GPU (other
+ *   - Every call uses the same array and clears the counters and
+ *     histograms that must start at zero before it runs.  Calls that overlap on the GPU (other
  *     streams, other host threads) race on the array and must not be issued.
  *   - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
  * Arguments are those of hkv_retrieve_topk, without ws and ws_bytes. */
