@@ -36,6 +36,7 @@ import synth
 
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse():
@@ -98,6 +99,35 @@ def measured_peaks():
             p = json.load(f)
         return float(p["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_tflops():
+    """Burst dense bf16 peak (a kernel timed alone)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def encode_roofline(w: synth.Workload, n_layers: int, encode_ms: float):
+    """Prefill key encode: LSH and sign are bound by HBM (keys in, codes out),
+    the MLP hash by the tensor cores (2 (d hidden + hidden bits) flops a key)."""
+    keys = w.B * w.Hkv * w.N * n_layers
+    elt = 2 if w.dtype == "bf16" else 4
+    sec = encode_ms * 1e-3
+    out = {"keys_per_s": keys / sec, "ms_all_layers": encode_ms,
+           "gbs": keys * (w.d * elt + w.bits // 8) / sec / 1e9}
+    if w.hash == "mlp":
+        peak, kind = measured_bf16_tflops()
+        tf = keys * 2.0 * (w.d * w.hidden + w.hidden * w.bits) / sec / 1e12
+        out.update({"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                    "peak_kind": kind})
+    else:
+        peak, kind = measured_peaks()
+        out.update({"bound": "hbm", "achieved": out["gbs"], "peak": peak, "unit": "GB/s", "frac": out["gbs"] / peak,
+                    "peak_kind": kind})
+    return out
 
 
 class ClockSampler:
@@ -375,9 +405,9 @@ def run_gpu(args, rank, world, local):
                      "launch_us": fused_launch_ms * 1e3, "peak_kind": peak_kind},
         "e2e": {"value": keys_step / (e2e_ms * 1e-3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "encode": {"keys_per_s": w.B * w.Hkv * w.N * len(layers) / (encode_ms * 1e-3),
-                   "ms_all_layers": encode_ms, "gbs": (w.B * w.Hkv * w.N * w.d * (2 if w.dtype == "bf16" else 4)
-                                                        * len(layers)) / (encode_ms * 1e-3) / 1e9},
+        "encode": dict(encode_roofline(w, len(layers), encode_ms),
+                       traffic=traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "encode_tc.cu"),
+                                              w.name) if w.hash == "lsh" else None),
         "kernels_us_per_launch": {"encode_q": qenc_ms * 1e3 / len(layers),
                                   "fused_decode": fused_launch_ms * 1e3,
                                   "retrieve_only": scan_ms * 1e3 / len(layers),
