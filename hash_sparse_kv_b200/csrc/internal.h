@@ -18,6 +18,7 @@ int cuda_check(cudaError_t e, const char* where);
 int debug_flags();
 uint64_t wait_limit_ns();
 int sm_count();
+int max_smem_optin();  // opt-in dynamic shared memory per block, bytes
 
 constexpr int kDebugSkipArrive = 1;
 

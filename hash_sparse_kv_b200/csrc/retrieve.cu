@@ -60,7 +60,9 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kGroups = 4;                  // cp.async groups in flight per thread
 constexpr int kSlots = 2 * kGroups;         // two tokens per group
-constexpr int kMaxTokensPerBlock = 32768;   // uint16 distances in shared memory
+constexpr int kMaxTokensPerBlock = 65536;   // uint16 distances in shared memory (when it fits)
+constexpr int kTokensPerBlockSmall = 32768; // the cap when the larger one does not fit
+constexpr size_t kStaticSmem = 4096;        // bound on the kernel's static shared memory
 constexpr int kMinTokensPerBlock = 2048;
 constexpr int kMaxSegsPerPair = 160;        // blocks per pair (shared header buffer)
 constexpr int kMaxGroup = 16;
@@ -234,22 +236,23 @@ __device__ void block_inclusive_scan(uint32_t* a, int n, uint32_t* warp_tmp) {
 }
 
 // Exclusive prefix of v over the block's threads; *total receives the sum.
-__device__ __forceinline__ uint32_t block_exclusive(uint32_t v, uint32_t* warp_tmp, uint32_t* total) {
+// warp_tmp: kWarps 8-byte words.
+__device__ __forceinline__ uint64_t block_exclusive(uint64_t v, uint64_t* warp_tmp, uint64_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t x = v;
+  uint64_t x = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
+    const uint64_t y = __shfl_up_sync(0xffffffffu, x, off);
     if (lane >= off) x += y;
   }
   __syncthreads();
   if (lane == 31) warp_tmp[warp] = x;
   __syncthreads();
-  uint32_t base = 0, tot = 0;
+  uint64_t base = 0, tot = 0;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
-    const uint32_t t = warp_tmp[w];
-    base += w < warp ? t : 0u;
+    const uint64_t t = warp_tmp[w];
+    base += w < warp ? t : 0ull;
     tot += t;
   }
   *total = tot;
@@ -502,8 +505,8 @@ __device__ __forceinline__ void split2(float2 x, uint32_t& hi, uint32_t& lo) {
 // (token row_at(i), or -1 to skip); writes the partial (m, l, acc) of every
 // head to dst[h * kPart ...].  Uses smem_attn (kAttnMmaBytes) and tok[2 * kRows].
 template <typename RowAt>
-__device__ void attn_mma(const FusedArgs& a, int p, int64_t qrow0, int nrows, RowAt row_at, unsigned char* smem_attn,
-                         int* tok, float* m_s, float* l_s, float* alpha_s, float* dst) {
+__device__ void attn_mma(const FusedArgs& a, int p, const float* aq_s, int nrows, RowAt row_at,
+                         unsigned char* smem_attn, int* tok, float* m_s, float* l_s, float* alpha_s, float* dst) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
   const int gid = lane >> 2, tq = lane & 3;
   const __nv_bfloat16* Kp = tptr<__nv_bfloat16>(a.K) + (int64_t)p * a.cap * kHeadDim;
@@ -525,17 +528,22 @@ __device__ void attn_mma(const FusedArgs& a, int p, int64_t qrow0, int nrows, Ro
     }
     cp_async_commit();
   };
-  // query fragments (rows = heads), kept in registers by the eight logit warps
+  // query fragments (rows = heads) from the block's fp32 copy of the bf16
+  // queries (exact), kept in registers by the eight logit warps
   uint32_t qa[kHeadDim / 16][4];
   if (warp < kRows / 8) {
-    const __nv_bfloat16* q0 = tptr<__nv_bfloat16>(a.q) + qrow0 * kHeadDim;
+    auto qpair = [&](int h, int k) -> uint32_t {
+      if (h >= g) return 0u;
+      const float2 f = *reinterpret_cast<const float2*>(aq_s + h * kHeadDim + k);
+      return pack_bf16(__float2bfloat16_rn(f.x), __float2bfloat16_rn(f.y));
+    };
 #pragma unroll
     for (int ks = 0; ks < kHeadDim / 16; ++ks) {
       const int k0 = ks * 16 + 2 * tq;
-      qa[ks][0] = gid < g ? *reinterpret_cast<const uint32_t*>(q0 + gid * kHeadDim + k0) : 0u;
-      qa[ks][1] = gid + 8 < g ? *reinterpret_cast<const uint32_t*>(q0 + (gid + 8) * kHeadDim + k0) : 0u;
-      qa[ks][2] = gid < g ? *reinterpret_cast<const uint32_t*>(q0 + gid * kHeadDim + k0 + 8) : 0u;
-      qa[ks][3] = gid + 8 < g ? *reinterpret_cast<const uint32_t*>(q0 + (gid + 8) * kHeadDim + k0 + 8) : 0u;
+      qa[ks][0] = qpair(gid, k0);
+      qa[ks][1] = qpair(gid + 8, k0);
+      qa[ks][2] = qpair(gid, k0 + 8);
+      qa[ks][3] = qpair(gid + 8, k0 + 8);
     }
   }
   if (tid < g) {
@@ -842,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   int32_t* sel_s = reinterpret_cast<int32_t*>(smem + a.off_sel);
   float* aq_s = reinterpret_cast<float*>(smem + a.off_aq);  // [g][128] attention queries (fp32)
   __shared__ uint32_t qc_s[kMaxGroup * W];
-  __shared__ uint32_t warp_tmp[2 * kWarps];
+  __shared__ __align__(8) uint32_t warp_tmp[2 * kWarps];
   __shared__ int sh[8];
   __shared__ float m_s[kMaxGroup], l_s[kMaxGroup], alpha_s[kMaxGroup];
   __shared__ int tok_s[2 * kRows];
@@ -1034,10 +1042,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
         }
       }
     }
-    uint32_t tot;
-    const uint32_t ex = block_exclusive(lt | (eq << 16), warp_tmp, &tot);
-    const uint32_t ex_lt = ex & 0xffffu, ex_eq = ex >> 16;
-    n_sel = (tot & 0xffffu) + min(tot >> 16, quota);
+    uint64_t tot;
+    const uint64_t ex = block_exclusive((uint64_t)lt | ((uint64_t)eq << 32), reinterpret_cast<uint64_t*>(warp_tmp), &tot);
+    const uint32_t ex_lt = (uint32_t)ex, ex_eq = (uint32_t)(ex >> 32);
+    n_sel = (uint32_t)tot + min((uint32_t)(tot >> 32), quota);
     uint32_t run_eq = ex_eq, pos = ex_lt + min(ex_eq, quota);
     int32_t* idx_out = a.idx + (int64_t)p * a.top_k + sel_base;
     int32_t* dist_out = a.dist ? a.dist + (int64_t)p * a.top_k + sel_base : nullptr;
@@ -1087,7 +1095,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     };
     float* dst = a.part + ((int64_t)p * nseg + seg) * a.g * kPart;
     if constexpr (sizeof(T) == 2) {
-      attn_mma(a, p, qrow0, ns + n_res, row_at, smem, tok_s, m_s, l_s, alpha_s, dst);
+      attn_mma(a, p, aq_s, ns + n_res, row_at, smem, tok_s, m_s, l_s, alpha_s, dst);
     } else {
       float* attn = reinterpret_cast<float*>(smem);
       const AttnSmem sm{aq_s, attn, attn + kRows * kKP, attn + kRows * kKP + kRows * kHeadDim, tok_s, m_s, l_s, alpha_s};
@@ -1190,10 +1198,12 @@ int make_plan(const RetrieveShape& s, bool attend, int q_elt, Plan& pl) {
   const int P = s.B * s.Hkv;
   const int64_t C = pl.C > 0 ? pl.C : 1;
   // blocks per pair: fill the SMs, keep blocks between kMinTokensPerBlock and
-  // kMaxTokensPerBlock candidates
+  // max_tok candidates; max_tok = kMaxTokensPerBlock when the shared memory
+  // of such a block fits, else kTokensPerBlockSmall
+  for (const int max_tok : {kMaxTokensPerBlock, kTokensPerBlockSmall}) {
   int64_t bpp = std::max<int64_t>(1, G / std::max(P, 1));
   bpp = std::min<int64_t>(bpp, ceil_div(C, kMinTokensPerBlock));
-  bpp = std::max<int64_t>(bpp, ceil_div(C, kMaxTokensPerBlock));
+  bpp = std::max<int64_t>(bpp, ceil_div(C, max_tok));
   if (bpp > G || bpp + 1 > kMaxSegsPerPair)
     return fail(HKV_ERR_UNSUPPORTED, "%lld candidates per sequence is too many for one launch", (long long)C);
   pl.per_block = (int)(ceil_div(ceil_div(C, bpp), 32) * 32);
@@ -1215,6 +1225,8 @@ int make_plan(const RetrieveShape& s, bool attend, int q_elt, Plan& pl) {
   pl.off_dist = (uint32_t)off;
   off += sizeof(uint16_t) * ((size_t)pl.per_block + 16);  // vector reads may run 7 past the end
   pl.smem = align_up(off, 16);
+  if (pl.smem + kStaticSmem <= (size_t)max_smem_optin() || max_tok == kTokensPerBlockSmall) break;
+  }
   pl.ws_sync = align_up(sizeof(uint32_t) * kSync * P, 256);
   pl.ws_gh = align_up(sizeof(uint32_t) * (size_t)P * pl.nbins, 256);
   pl.ws_cum = align_up(sizeof(uint32_t) * (size_t)P * pl.nseg * pl.nbins, 256);

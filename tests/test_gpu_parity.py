@@ -208,6 +208,22 @@ def test_retrieve_heavy_ties_across_blocks():
         np.testing.assert_array_equal(dist, wd)
 
 
+def test_retrieve_one_block_per_pair_over_32k_candidates():
+    """148 (batch, KV head) pairs of 40001 tokens: one block per pair holds all
+    of its distances (more than 32768) in shared memory.  Keys from three
+    codes put tens of thousands of ties on both sides of the threshold."""
+    B, Hq, Hkv, N, k = 37, 8, 4, 40001, 30000
+    base = synth.random_codes(12, 3, 2).numpy()
+    pick = np.random.default_rng(13).integers(0, 3, B * Hkv * N)
+    kc = torch.from_numpy(base[pick].copy()).view(B, Hkv, N, 2)
+    qc = synth.random_codes(14, B * Hq, 2).view(B, Hq, 2)
+    for _ in range(2):
+        idx, dist, _ = _retrieve(qc, kc, N, 4, 64, k)
+        wi, wd = oracle.retrieve(qc.numpy().view(np.uint32), kc.numpy().view(np.uint32), N, 4, 64, k)
+        np.testing.assert_array_equal(idx, wi)
+        np.testing.assert_array_equal(dist, wd)
+
+
 def test_retrieve_in_pair_batches():
     """More candidates than one launch keeps in shared memory: several launches."""
     B, Hq, Hkv, N, k = 16, 32, 8, 100000, 512
