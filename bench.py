@@ -43,6 +43,8 @@ def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--prefetch-hint", action="store_true",
+                    help="time the step with each layer passing the next layer's codes as the L2 prefetch hint")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="qwen7b_512k", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="hkv", choices=["hkv", "reference"])
@@ -296,10 +298,14 @@ def run_gpu(args, rank, world, local):
     ws = hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
     status = hkv.status_word(dev)
 
-    def step():
-        for L in layers:
+    def step(hint=args.prefetch_hint):
+        # layer i tells the library that layer i + 1 (wrapping to the next
+        # step's layer 0) scans next, so its codes stream into L2 during layer
+        # i's selection and attention
+        for i, L in enumerate(layers):
+            nxt = layers[(i + 1) % len(layers)].codes if hint and len(layers) > 1 else None
             hkv.hkv_decode_step(L.qh, L.q, L.codes, L.K, L.V, w.N, w.n_sink, w.n_local, w.top_k, L.out,
-                                q_codes=L.q_codes, idx=L.idx, ws=ws, status=status)
+                                q_codes=L.q_codes, idx=L.idx, ws=ws, status=status, next_k_codes=nxt)
 
     # standalone calls get their own workspaces (each entry point has its own layout)
     ws_r = hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
@@ -329,6 +335,9 @@ def run_gpu(args, rank, world, local):
         raise RuntimeError(f"decode step reported status {rc}")
     keys_per_layer = w.B * w.Hkv * w.candidates()
     value, ms = job_throughput(keys_per_layer * len(layers), ms, world, dev)
+    g_other = graph_of(lambda: step(hint=not args.prefetch_hint))
+    other_ms = max_over_ranks(time_graph(g_other, args.steps, args.warmup, world), world, dev)
+    del g_other
     # each kernel alone, one launch per layer
     def qenc_only():
         for L in layers:
@@ -385,6 +394,8 @@ def run_gpu(args, rank, world, local):
         "warmup": args.warmup,
         "ms_per_step": ms,
         "us_per_layer": ms * 1e3 / len(layers),
+        ("us_per_layer_without_prefetch_hint" if args.prefetch_hint else "us_per_layer_with_prefetch_hint"):
+            other_ms * 1e3 / len(layers),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -394,6 +405,7 @@ def run_gpu(args, rank, world, local):
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.d, "n_tokens": w.N,
             "hash": w.hash, "code_bits": w.bits, "top_k": w.top_k, "n_sink": w.n_sink, "n_local": w.n_local,
             "layers_per_step": len(layers), "parallelism": f"replica x{world}",
+            "next_layer_prefetch_hint": args.prefetch_hint,
             "l2": f"inputs larger than L2: {len(layers)} distinct layer buffers, "
                   f"{per_layer_bytes * len(layers) / 1e9:.2f} GB algorithmic per step",
         },

@@ -80,7 +80,7 @@ _SIGS = {
     "hkv_sparse_attend": (_I, [_I, _I, _I, _I, _P, _P, _P, _I64, _I64, _P, _I, _I, _I, _F, _P, _P, _P, _SZ, _P, _P]),
     "hkv_lse_merge": (_I, [_I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "hkv_decode_step": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _F,
-                             _P, _P, _P, _P, _P, _SZ, _P, _P]),
+                             _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "hkv_debug_set": (_I, [_I, _I64]),
 }
 _lib = None
@@ -334,8 +334,9 @@ def hkv_lse_merge(o1, lse1, o2, lse2, out, lse_out=None, stream=None) -> None:
 
 def hkv_decode_step(h: HashParams, q, k_codes, K, V, n_tokens: int, n_sink: int, n_local: int, top_k: int, out,
                     lse=None, q_codes=None, idx=None, scale: Optional[float] = None, ws=None, status=None,
-                    stream=None) -> None:
-    """One decode step (query encode, retrieval, attention) in the library's kernels."""
+                    stream=None, next_k_codes=None) -> None:
+    """One decode step (query encode, retrieval, attention) in the library's kernels.
+    next_k_codes: optional hint, the key codes (same shape) the next call will scan."""
     B, Hq, d = q.shape
     _, Hkv, cap, W = k_codes.shape
     _need(q, "q", (torch.bfloat16, torch.float32))
@@ -349,8 +350,10 @@ def hkv_decode_step(h: HashParams, q, k_codes, K, V, n_tokens: int, n_sink: int,
         _need(idx, "idx", torch.int32, shape=(B, Hkv, top_k))
     if lse is not None:
         _need(lse, "lse", torch.float32, shape=(B, Hq))
+    if next_k_codes is not None:
+        _need(next_k_codes, "next_k_codes", _U32, shape=tuple(k_codes.shape))
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _ok(lib().hkv_decode_step(ctypes.byref(h.c), B, Hq, Hkv, _ptr(q), _ptr(k_codes), _ptr(K), _ptr(V), cap, n_tokens,
-                              n_sink, n_local, top_k, scale, _ptr(q_codes), _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws),
-                              nbytes, _ptr(status), _stream(stream)))
+                              n_sink, n_local, top_k, scale, _ptr(q_codes), _ptr(idx), _ptr(out), _ptr(lse),
+                              _ptr(next_k_codes), _ptr(ws), nbytes, _ptr(status), _stream(stream)))

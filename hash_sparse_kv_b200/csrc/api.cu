@@ -278,8 +278,9 @@ int hkv_lse_merge(int rows, int d, const float* o1, const float* lse1, const flo
 int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
                     const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
                     int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
-                    uint32_t* q_codes, int32_t* idx, float* out, float* lse, void* ws,
-                    size_t ws_bytes, int32_t* status, void* stream) {
+                    uint32_t* q_codes, int32_t* idx, float* out, float* lse,
+                    const uint32_t* next_k_codes, void* ws, size_t ws_bytes, int32_t* status,
+                    void* stream) {
   int rc = check_hash(q_hash, true);
   if (rc == HKV_OK) rc = check_heads(B, Hq, Hkv);
   if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
@@ -290,7 +291,7 @@ int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* 
   if (B == 0) return HKV_OK;
   if (!q || !k_codes || !K || !V || !out) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) ||
-      !aligned(k_codes, q_hash->code_bits / 8))
+      !aligned(k_codes, q_hash->code_bits / 8) || !aligned(next_k_codes, q_hash->code_bits / 8))
     return fail(HKV_ERR_INVALID_ARG, "q, K, V, out and k_codes must be aligned");
   DecodeLayout L;
   rc = decode_layout(B, Hq, Hkv, n_tokens, q_hash->code_bits, top_k, n_sink, n_local, L);
@@ -322,10 +323,10 @@ int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* 
     return launch_attend(as, q, K, V, ix, scale, out, lse, ws_a, L.attend, status, st);
   }
   if (fused_encode)
-    return launch_decode(rs, q_hash->dtype, q_hash->kind, q_hash->R, nullptr, qc, k_codes, ix, q, K, V, scale, out,
-                         lse, ws_f, L.fused, status, st);
-  return launch_decode(rs, q_hash->dtype, HKV_HASH_NONE, nullptr, qc, nullptr, k_codes, ix, q, K, V, scale, out, lse,
-                       ws_f, L.fused, status, st);
+    return launch_decode(rs, q_hash->dtype, q_hash->kind, q_hash->R, nullptr, qc, k_codes, next_k_codes, ix, q, K, V,
+                         scale, out, lse, ws_f, L.fused, status, st);
+  return launch_decode(rs, q_hash->dtype, HKV_HASH_NONE, nullptr, qc, nullptr, k_codes, next_k_codes, ix, q, K, V,
+                       scale, out, lse, ws_f, L.fused, status, st);
 }
 
 }  // extern "C"

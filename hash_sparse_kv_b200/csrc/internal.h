@@ -59,7 +59,8 @@ int launch_retrieve_static(const RetrieveShape& s, const uint32_t* q_codes, cons
 size_t decode_ws_bytes(const RetrieveShape& s);
 bool decode_encodes_queries(const RetrieveShape& s, int kind, int dtype);
 int launch_decode(const RetrieveShape& s, int dtype, int q_kind, const void* R, const uint32_t* q_codes_in,
-                  uint32_t* q_codes_out, const uint32_t* k_codes, int32_t* idx, const void* q, const void* K,
+                  uint32_t* q_codes_out, const uint32_t* k_codes,
+                  const uint32_t* next_codes, int32_t* idx, const void* q, const void* K,
                   const void* V, float scale, float* out, float* lse, void* ws, size_t ws_bytes,
                   int32_t* status, cudaStream_t st);
 

@@ -62,7 +62,7 @@ constexpr int kGroups = 4;                  // cp.async groups in flight per thr
 constexpr int kSlots = 2 * kGroups;         // two tokens per group
 constexpr int kMaxTokensPerBlock = 65536;   // uint16 distances in shared memory (when it fits)
 constexpr int kTokensPerBlockSmall = 32768; // the cap when the larger one does not fit
-constexpr size_t kStaticSmem = 4096;        // bound on the kernel's static shared memory
+constexpr size_t kStaticSmem = 2048;        // bound on the kernel's static shared memory
 constexpr int kMinTokensPerBlock = 2048;
 constexpr int kMaxSegsPerPair = 160;        // blocks per pair (shared header buffer)
 constexpr int kMaxGroup = 16;
@@ -99,6 +99,7 @@ struct FusedArgs {
   uint32_t off_q, off_aq, off_sel, off_hist, off_dist;  // shared memory carve-up (bytes)
   uint32_t* sync;  // [pairs][kSync]
   uint32_t* gh;    // [pairs][nbins]: histogram of the pair (returns to zero)
+  const uint32_t* next_codes;  // nullable: codes of the next call, prefetched to L2 after the scan
   uint32_t* cum;   // [pairs][nseg][nbins]: cumulative counts, window only
   float* part;     // [pairs][nseg][g][kPart]
   int32_t* status;
@@ -474,8 +475,11 @@ __device__ void attn_rows(const FusedArgs& a, int p, int nrows, RowAt row_at, co
 // bf16 hi + lo parts (two MMAs), so P keeps 16 significant bits.
 constexpr int kKVPitch = kHeadDim + 8;           // bf16 elements per shared row
 constexpr int kKVTile = kRows * kKVPitch * 2;    // bytes per K or V tile
-constexpr int kZP = kRows + 8;                   // probability row pitch (floats)
-constexpr size_t kAttnMmaBytes = 4 * (size_t)kKVTile + sizeof(float) * kMaxGroup * kZP;
+constexpr int kZP = kRows + 8;                   // logit row pitch (floats)
+constexpr int kPP = kRows / 2 + 4;               // probability row pitch (bf16 pairs)
+constexpr int kQP = kHeadDim + 8;                // bf16 query row pitch (conflict-free fragment loads)
+constexpr size_t kAttnMmaBytes = 4 * (size_t)kKVTile + sizeof(float) * kMaxGroup * kZP +
+                                 2 * sizeof(uint32_t) * kMaxGroup * kPP + 2 * kMaxGroup * kQP;
 
 __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
@@ -488,6 +492,14 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Four 8x8 b16 matrices, transposed: lane l supplies the address of row l
+// (rows 8i..8i+7 form matrix i); r[i] receives the fragment of matrix i.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(__nv_bfloat16 lo, __nv_bfloat16 hi) {
@@ -511,7 +523,20 @@ __device__ void attn_mma(const FusedArgs& a, int p, const float* aq_s, int nrows
   const int gid = lane >> 2, tq = lane & 3;
   const __nv_bfloat16* Kp = tptr<__nv_bfloat16>(a.K) + (int64_t)p * a.cap * kHeadDim;
   const __nv_bfloat16* Vp = tptr<__nv_bfloat16>(a.V) + (int64_t)p * a.cap * kHeadDim;
-  float* z = reinterpret_cast<float*>(smem_attn + 4 * kKVTile);  // [kMaxGroup][kZP]
+  float* z = reinterpret_cast<float*>(smem_attn + 4 * kKVTile);  // [kMaxGroup][kZP] scratch
+  float* pmax = z;                                  // [8 warps][kMaxGroup] tile maxima
+  float* psum = z + (kRows / 8) * kMaxGroup;        // [8 warps][kMaxGroup] tile sums
+  float* m_next = z + 2 * (kRows / 8) * kMaxGroup;  // [kMaxGroup]
+  // probabilities as bf16 hi and lo parts, rows of the tile in pairs: [kMaxGroup][kPP]
+  uint32_t* ph = reinterpret_cast<uint32_t*>(z + kMaxGroup * kZP);
+  uint32_t* pl = ph + kMaxGroup * kPP;
+  for (int i = tid; i < 2 * kMaxGroup * kPP; i += kThreads) ph[i] = 0u;  // heads >= g stay zero
+  // the queries as bf16 (exact: they are bf16 inputs), rows >= g zero
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(pl + kMaxGroup * kPP);  // [kMaxGroup][kQP]
+  for (int i = tid; i < kMaxGroup * kHeadDim; i += kThreads) {
+    const int h = i / kHeadDim, k = i % kHeadDim;
+    qs[h * kQP + k] = __float2bfloat16_rn(h < g ? aq_s[h * kHeadDim + k] : 0.f);
+  }
   auto kbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem_attn + (2 * b) * kKVTile); };
   auto vbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem_attn + (2 * b + 1) * kKVTile); };
   constexpr int CPR = kHeadDim / 8;                 // 16-byte chunks per row
@@ -528,24 +553,6 @@ __device__ void attn_mma(const FusedArgs& a, int p, const float* aq_s, int nrows
     }
     cp_async_commit();
   };
-  // query fragments (rows = heads) from the block's fp32 copy of the bf16
-  // queries (exact), kept in registers by the eight logit warps
-  uint32_t qa[kHeadDim / 16][4];
-  if (warp < kRows / 8) {
-    auto qpair = [&](int h, int k) -> uint32_t {
-      if (h >= g) return 0u;
-      const float2 f = *reinterpret_cast<const float2*>(aq_s + h * kHeadDim + k);
-      return pack_bf16(__float2bfloat16_rn(f.x), __float2bfloat16_rn(f.y));
-    };
-#pragma unroll
-    for (int ks = 0; ks < kHeadDim / 16; ++ks) {
-      const int k0 = ks * 16 + 2 * tq;
-      qa[ks][0] = qpair(gid, k0);
-      qa[ks][1] = qpair(gid + 8, k0);
-      qa[ks][2] = qpair(gid, k0 + 8);
-      qa[ks][3] = qpair(gid + 8, k0 + 8);
-    }
-  }
   if (tid < g) {
     m_s[tid] = -INFINITY;
     l_s[tid] = 0.f;
@@ -564,50 +571,94 @@ __device__ void attn_mma(const FusedArgs& a, int p, const float* aq_s, int nrows
     const __nv_bfloat16* Ks = kbuf(b);
     const __nv_bfloat16* Vs = vbuf(b);
     const int* tk = tok + b * kRows;
+    // logits of rows 8 w + 2 tq (+1) for heads gid and gid + 8 (warps 0..7),
+    // then the tile maximum of each head through shared memory, and the
+    // probabilities straight from the registers: no separate softmax pass
+    float s00 = -INFINITY, s01 = -INFINITY, s10 = -INFINITY, s11 = -INFINITY;
     if (warp < kRows / 8) {
       float c[4] = {0.f, 0.f, 0.f, 0.f};
       const __nv_bfloat16* kr = Ks + (warp * 8 + gid) * kKVPitch + 2 * tq;
+      const __nv_bfloat16* q0 = qs + gid * kQP + 2 * tq;
+      const __nv_bfloat16* q1 = qs + (gid + 8) * kQP + 2 * tq;
 #pragma unroll
       for (int ks = 0; ks < kHeadDim / 16; ++ks) {
         const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr + ks * 16);
         const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + ks * 16 + 8);
-        mma16816(c, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(q0 + ks * 16);
+        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(q1 + ks * 16);
+        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(q0 + ks * 16 + 8);
+        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(q1 + ks * 16 + 8);
+        mma16816(c, a0, a1, a2, a3, b0, b1);
       }
       const int r = warp * 8 + 2 * tq;
       const bool v0 = r < nr && tk[r] >= 0, v1 = r + 1 < nr && tk[r + 1] >= 0;
       if (gid < g) {
-        z[gid * kZP + r] = v0 ? c[0] * a.scale : -INFINITY;
-        z[gid * kZP + r + 1] = v1 ? c[1] * a.scale : -INFINITY;
+        s00 = v0 ? c[0] * a.scale : -INFINITY;
+        s01 = v1 ? c[1] * a.scale : -INFINITY;
       }
       if (gid + 8 < g) {
-        z[(gid + 8) * kZP + r] = v0 ? c[2] * a.scale : -INFINITY;
-        z[(gid + 8) * kZP + r + 1] = v1 ? c[3] * a.scale : -INFINITY;
+        s10 = v0 ? c[2] * a.scale : -INFINITY;
+        s11 = v1 ? c[3] * a.scale : -INFINITY;
+      }
+      float mx0 = fmaxf(s00, s01), mx1 = fmaxf(s10, s11);
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      if (tq == 0) {
+        pmax[warp * kMaxGroup + gid] = mx0;
+        pmax[warp * kMaxGroup + gid + 8] = mx1;
       }
     }
     __syncthreads();
-    for (int h = warp; h < g; h += kWarps) {
-      float* zh = z + h * kZP;
-      const float z0 = zh[lane], z1 = zh[lane + 32];
-      float mt = fmaxf(z0, z1);
+    if (warp < kRows / 8) {
+      float t0 = -INFINITY, t1 = -INFINITY;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
-      const float m_old = m_s[h];
-      const float m_new = fmaxf(m_old, mt);
-      const float e0 = z0 == -INFINITY ? 0.f : expf(z0 - m_new);
-      const float e1 = z1 == -INFINITY ? 0.f : expf(z1 - m_new);
-      zh[lane] = e0;
-      zh[lane + 32] = e1;
-      float ls = e0 + e1;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
-      if (lane == 0) {
-        const float alpha = m_new == -INFINITY ? 1.f : expf(m_old - m_new);
-        alpha_s[h] = alpha;
-        m_s[h] = m_new;
-        l_s[h] = l_s[h] * alpha + ls;
+      for (int w = 0; w < kRows / 8; ++w) {
+        t0 = fmaxf(t0, pmax[w * kMaxGroup + gid]);
+        t1 = fmaxf(t1, pmax[w * kMaxGroup + gid + 8]);
+      }
+      const float mo0 = m_s[gid < g ? gid : 0], mo1 = m_s[gid + 8 < g ? gid + 8 : 0];
+      const float mn0 = fmaxf(mo0, t0), mn1 = fmaxf(mo1, t1);
+      const float e00 = s00 == -INFINITY ? 0.f : expf(s00 - mn0), e01 = s01 == -INFINITY ? 0.f : expf(s01 - mn0);
+      const float e10 = s10 == -INFINITY ? 0.f : expf(s10 - mn1), e11 = s11 == -INFINITY ? 0.f : expf(s11 - mn1);
+      const int pr = warp * 4 + tq;  // pair index of rows 8 w + 2 tq, + 1
+      uint32_t hi, lo;
+      if (gid < g) {
+        split2(make_float2(e00, e01), hi, lo);
+        ph[gid * kPP + pr] = hi;
+        pl[gid * kPP + pr] = lo;
+      }
+      if (gid + 8 < g) {
+        split2(make_float2(e10, e11), hi, lo);
+        ph[(gid + 8) * kPP + pr] = hi;
+        pl[(gid + 8) * kPP + pr] = lo;
+      }
+      float ps0 = e00 + e01, ps1 = e10 + e11;
+      ps0 += __shfl_xor_sync(0xffffffffu, ps0, 1);
+      ps0 += __shfl_xor_sync(0xffffffffu, ps0, 2);
+      ps1 += __shfl_xor_sync(0xffffffffu, ps1, 1);
+      ps1 += __shfl_xor_sync(0xffffffffu, ps1, 2);
+      if (tq == 0) {
+        psum[warp * kMaxGroup + gid] = ps0;
+        psum[warp * kMaxGroup + gid + 8] = ps1;
+        if (warp == 0) {
+          m_next[gid] = mn0;
+          m_next[gid + 8] = mn1;
+          alpha_s[gid] = mn0 == -INFINITY ? 1.f : expf(mo0 - mn0);
+          alpha_s[gid + 8] = mn1 == -INFINITY ? 1.f : expf(mo1 - mn1);
+        }
       }
     }
     __syncthreads();
+    if (tid < g) {
+      // running (m, l) of head tid; nothing reads them again before the next tile's second barrier
+      float ls = 0.f;
+#pragma unroll
+      for (int w = 0; w < kRows / 8; ++w) ls += psum[w * kMaxGroup + tid];
+      l_s[tid] = l_s[tid] * alpha_s[tid] + ls;
+      m_s[tid] = m_next[tid];
+    }
     {
       // warp w: output dims [8w, 8w + 8)
       const float al0 = gid < g ? alpha_s[gid] : 1.f, al1 = gid + 8 < g ? alpha_s[gid + 8] : 1.f;
@@ -615,28 +666,21 @@ __device__ void attn_mma(const FusedArgs& a, int p, const float* aq_s, int nrows
       o[1] *= al0;
       o[2] *= al1;
       o[3] *= al1;
-      const int col = warp * 8 + gid;
+      const uint32_t vrow = static_cast<uint32_t>(__cvta_generic_to_shared(Vs)) + (uint32_t)(warp * 8 * 2);
 #pragma unroll
-      for (int ks = 0; ks < kRows / 16; ++ks) {
-        const int k0 = ks * 16 + 2 * tq;
-        float2 p00 = make_float2(0.f, 0.f), p10 = p00, p01 = p00, p11 = p00;
-        if (gid < g) {
-          p00 = *reinterpret_cast<const float2*>(z + gid * kZP + k0);
-          p01 = *reinterpret_cast<const float2*>(z + gid * kZP + k0 + 8);
+      for (int kp = 0; kp < kRows / 32; ++kp) {
+        uint32_t bv[4];  // B fragments of k-steps 2 kp and 2 kp + 1 (rows 32 kp + lane)
+        ldsm_x4_trans(vrow + (uint32_t)((kp * 32 + lane) * kKVPitch * 2), bv);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int c0 = (2 * kp + half) * 8 + tq;  // pair index of rows 16 ks + 2 tq
+          const uint32_t* h0 = ph + gid * kPP + c0;
+          const uint32_t* h1 = ph + (gid + 8) * kPP + c0;
+          const uint32_t* l0 = pl + gid * kPP + c0;
+          const uint32_t* l1 = pl + (gid + 8) * kPP + c0;
+          mma16816(o, h0[0], h1[0], h0[4], h1[4], bv[2 * half], bv[2 * half + 1]);
+          mma16816(o, l0[0], l1[0], l0[4], l1[4], bv[2 * half], bv[2 * half + 1]);
         }
-        if (gid + 8 < g) {
-          p10 = *reinterpret_cast<const float2*>(z + (gid + 8) * kZP + k0);
-          p11 = *reinterpret_cast<const float2*>(z + (gid + 8) * kZP + k0 + 8);
-        }
-        uint32_t h0, l0, h1, l1, h2, l2, h3, l3;
-        split2(p00, h0, l0);
-        split2(p10, h1, l1);
-        split2(p01, h2, l2);
-        split2(p11, h3, l3);
-        const uint32_t b0 = pack_bf16(Vs[k0 * kKVPitch + col], Vs[(k0 + 1) * kKVPitch + col]);
-        const uint32_t b1 = pack_bf16(Vs[(k0 + 8) * kKVPitch + col], Vs[(k0 + 9) * kKVPitch + col]);
-        mma16816(o, h0, h1, h2, h3, b0, b1);
-        mma16816(o, l0, l1, l2, l3, b0, b1);
       }
     }
     __syncthreads();  // buffer b is refilled by the next iteration's issue
@@ -945,6 +989,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     }
     cp_async_wait<0>();
   }
+  if (a.next_codes != nullptr && tid < 32) {
+    // the next call's codes for this block's range go to L2 while this call
+    // selects and attends (16-byte aligned pieces; the hint skips ragged ends)
+    const uintptr_t beg = reinterpret_cast<uintptr_t>(a.next_codes + ((int64_t)p * a.cap + a.lo + s0) * W);
+    const uintptr_t end = (beg + (uintptr_t)len * W * 4) & ~(uintptr_t)15;
+    constexpr uintptr_t kPiece = 16384;
+    for (uintptr_t o = ((beg + 15) & ~(uintptr_t)15) + (uintptr_t)tid * kPiece; o < end; o += 32 * kPiece) {
+      const uint32_t n = (uint32_t)(end - o < kPiece ? end - o : kPiece);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(o), "r"(n) : "memory");
+    }
+  }
   if (tid == 0) sh[1] = a.nbins;  // hi
   __syncthreads();
 
@@ -1214,7 +1269,7 @@ int make_plan(const RetrieveShape& s, bool attend, int q_elt, Plan& pl) {
   const size_t attn = std::max(sizeof(float) * (kRows * kKP + kRows * kHeadDim + kMaxGroup * kRows), kAttnMmaBytes);
   size_t off = attend ? std::max(ring, attn) : ring;
   pl.off_aq = (uint32_t)off;
-  if (attend) off += sizeof(float) * kMaxGroup * kHeadDim;
+  if (attend) off += sizeof(float) * pl.g * kHeadDim;
   pl.off_q = (uint32_t)off;
   if (q_elt == 2) off += align_up(sizeof(uint16_t) * (kQRows + bits) * (kHeadDim + 8) + kQRows * bits / 8, 16);
   if (q_elt == 4) off += align_up(sizeof(float) * (kQRows * kHeadDim + bits * (kHeadDim + 1)), 16);
@@ -1238,7 +1293,8 @@ int make_plan(const RetrieveShape& s, bool attend, int q_elt, Plan& pl) {
 int launch_fused(const RetrieveShape& s, bool attend, int dtype, int qenc, const void* R,
                  const uint32_t* q_codes_in, uint32_t* q_codes_out, const uint32_t* k_codes, int32_t* idx,
                  int32_t* dist, const void* q, const void* K, const void* V, float scale, float* out,
-                 float* lse, void* ws, size_t ws_bytes, int32_t* status, cudaStream_t st) {
+                 float* lse, void* ws, size_t ws_bytes, int32_t* status, cudaStream_t st,
+                 const uint32_t* next_codes = nullptr) {
   const int P = s.B * s.Hkv;
   const int q_elt = (qenc == kQLsh) ? (dtype == HKV_BF16 ? 2 : 4) : 0;
   Plan pl;
@@ -1254,6 +1310,7 @@ int launch_fused(const RetrieveShape& s, bool attend, int dtype, int qenc, const
   a.R = R;
   a.qenc = qenc;
   a.k_codes = k_codes;
+  a.next_codes = next_codes;
   a.idx = idx;
   a.dist = dist;
   a.q = q;
@@ -1405,12 +1462,12 @@ int launch_retrieve_static(const RetrieveShape& s, const uint32_t* q_codes, cons
 }
 
 int launch_decode(const RetrieveShape& s, int dtype, int q_kind, const void* R, const uint32_t* q_codes_in,
-                  uint32_t* q_codes_out, const uint32_t* k_codes, int32_t* idx, const void* q, const void* K,
-                  const void* V, float scale, float* out, float* lse, void* ws, size_t ws_bytes,
-                  int32_t* status, cudaStream_t st) {
+                  uint32_t* q_codes_out, const uint32_t* k_codes, const uint32_t* next_codes, int32_t* idx,
+                  const void* q, const void* K, const void* V, float scale, float* out, float* lse, void* ws,
+                  size_t ws_bytes, int32_t* status, cudaStream_t st) {
   const int qenc = q_kind == HKV_HASH_LSH ? kQLsh : q_kind == HKV_HASH_SIGN ? kQSign : kQGiven;
   return launch_fused(s, true, dtype, qenc, R, q_codes_in, q_codes_out, k_codes, idx, nullptr, q, K, V, scale,
-                      out, lse, ws, ws_bytes, status, st);
+                      out, lse, ws, ws_bytes, status, st, next_codes);
 }
 
 }  // namespace hkv

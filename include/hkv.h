@@ -239,23 +239,29 @@ int hkv_sparse_attend(int B, int Hq, int Hkv, int dtype, const void* q, const vo
 int hkv_lse_merge(int rows, int d, const float* o1, const float* lse1, const float* o2,
                   const float* lse2, float* out, float* lse_out, void* stream);
 
-/* One whole decode step (S2, S4-S8) in two launches: the query encoder, then
- * one kernel that scans, selects, attends and merges.  Results equal
- * hkv_encode_keys on q, then hkv_retrieve_topk, then hkv_sparse_attend:
- * q_codes and idx bit-identical, out and lse within floating-point rounding.
+/* One whole decode step (S2, S4-S8): one kernel that encodes the query heads
+ * (LSH, sign), scans, selects, attends and merges; the MLP query hash adds one
+ * launch before it.  Results equal hkv_encode_keys on q, then
+ * hkv_retrieve_topk, then hkv_sparse_attend: q_codes and idx bit-identical,
+ * out and lse within floating-point rounding.
  *   q_hash   hash for the queries (q_hash->dtype is the dtype of q, K, V).  With
  *            kind HKV_HASH_NONE nothing is encoded: q_codes is an input that
- *            already holds the query codes (one launch)
+ *            already holds the query codes
  *   q        [B, Hq, 128];  k_codes [B, Hkv, cap, code_bits / 32]
  *   K, V     [B, Hkv, cap, 128]
  *   q_codes  [B, Hq, code_bits / 32]: output (nullable) or, for HKV_HASH_NONE,
  *            input (required)
  *   idx      nullable [B, Hkv, top_k] out
- *   out      [B, Hq, 128] fp32;  lse nullable [B, Hq] fp32 */
+ *   out      [B, Hq, 128] fp32;  lse nullable [B, Hq] fp32
+ *   next_k_codes  nullable hint: the key codes the next call on this stream
+ *            will scan (same shape, e.g. the next layer's).  After its own
+ *            scan the kernel asks L2 to prefetch them, so that stream overlaps
+ *            this call's selection and attention.  Never read otherwise; the
+ *            results do not depend on it. */
 int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
                     const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
                     int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
-                    uint32_t* q_codes, int32_t* idx, float* out, float* lse, void* ws,
+                    uint32_t* q_codes, int32_t* idx, float* out, float* lse, const uint32_t* next_k_codes, void* ws,
                     size_t ws_bytes, int32_t* status, void* stream);
 
 /* Testing aid (process-wide).  flags bit 0: in the next retrieval launches,

@@ -373,8 +373,9 @@ def test_append(kind):
 
 # --------------------------------------------------------------- decode step
 
-def run_decode(w, inp, layer_codes=None):
-    """GPU: encode keys, then one decode step; returns host results."""
+def run_decode(w, inp, layer_codes=None, next_k_codes=False):
+    """GPU: encode keys, then one decode step; returns host results.  With
+    next_k_codes, the step also gets a same-shape buffer as its L2 prefetch hint."""
     tdt, code = _dt(w.dtype)
     B, Hq, Hkv, N, cap, W = w.B, w.Hq, w.Hkv, w.N, inp["cap"], w.words
     K, V, q = inp["K"].to(DEV), inp["V"].to(DEV), inp["q"].to(DEV)
@@ -387,8 +388,9 @@ def run_decode(w, inp, layer_codes=None):
     qc = torch.zeros(B, Hq, W, dtype=torch.int32, device=DEV)
     ws = hkv.workspace(B, Hq, Hkv, N, w.bits, w.top_k, w.n_sink, w.n_local)
     st = hkv.status_word()
+    nxt = torch.randint(-2**31, 2**31 - 1, codes.shape, dtype=torch.int32, device=DEV) if next_k_codes else None
     hkv.hkv_decode_step(qh, q, codes, K, V, N, w.n_sink, w.n_local, w.top_k, out, lse, q_codes=qc, idx=idx,
-                        ws=ws, status=st)
+                        ws=ws, status=st, next_k_codes=nxt)
     _check(st)
     return {"codes": u32(codes), "q_codes": u32(qc), "idx": idx.cpu().numpy(), "out": out.cpu().numpy(),
             "lse": lse.cpu().numpy()}
@@ -417,8 +419,11 @@ SMALL = {
 }
 
 
+@pytest.mark.parametrize("hint", [False, True])
 @pytest.mark.parametrize("name", list(SMALL))
-def test_decode_step_small(name):
+def test_decode_step_small(name, hint):
+    """Every workload at a small size; with `hint` the step also prefetches
+    another code buffer (the next layer's), which must not change anything."""
     w = synth.WORKLOADS[name].with_(**SMALL[name])
     inp = margin_inputs(w, cap=w.N + 5)
-    compare_decode(w, inp, run_decode(w, inp))
+    compare_decode(w, inp, run_decode(w, inp, next_k_codes=hint))
