@@ -373,31 +373,60 @@ mlp_encode_kernel(const T* __restrict__ x, const float* __restrict__ W1,
 }
 
 // --------------------------------------------------------------- SIGN -----
-// One warp per row: lane l reads elements l + 32 i, so word i is the ballot
-// of (x_{l + 32 i} > 0).  The norm is summed in fp64 (bf16 and fp32 squares
-// are exact there), square-rooted in fp64 and rounded once to fp16.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 sign_encode_kernel(const T* __restrict__ x, RowMap m, uint32_t* __restrict__ codes,
-                   uint16_t* __restrict__ norms) {
-  constexpr int D = kHeadDim, TB = D / 32;
-  const int lane = threadIdx.x & 31;
+                   uint16_t* __restrict__ norms, bool vec_store) {
+  // eight lanes per row, 16 dimensions per lane (bf16: two 16-byte loads,
+  // fp32: four); a warp covers four rows per step and keeps kU steps of loads
+  // in flight
+  constexpr int D = kHeadDim, EPL = 16, V = 16 / sizeof(T), NV = EPL / V, kU = 4;
+  const int lane = threadIdx.x & 31, sub = lane & 7, slot = lane >> 3;
   const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
-  for (int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); row < m.rows;
-       row += warps) {
-    const T* px = x + m.x_off(row);
-    double ss = 0.0;
+  const int64_t warp_id = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+  for (int64_t row0 = warp_id * 4 * kU; row0 < m.rows; row0 += warps * 4 * kU) {
+    uint4 raw[kU][NV];
 #pragma unroll
-    for (int i = 0; i < TB; ++i) {
-      const float v = to_f32(px[lane + 32 * i]);
-      ss += (double)v * (double)v;
-      const uint32_t word = __ballot_sync(0xffffffffu, v > 0.f);
-      if (lane == i) codes[m.c_off(row) + i] = word;
+    for (int u = 0; u < kU; ++u) {
+      const int64_t row = row0 + u * 4 + slot;
+#pragma unroll
+      for (int v = 0; v < NV; ++v)
+        raw[u][v] = row < m.rows ? __ldg(reinterpret_cast<const uint4*>(x + m.x_off(row) + sub * EPL) + v)
+                                 : make_uint4(0u, 0u, 0u, 0u);
     }
-    if (norms != nullptr) {
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-      if (lane == 0) norms[m.n_off(row)] = __half_as_ushort(__double2half(sqrt(ss)));
+    for (int u = 0; u < kU; ++u) {
+      const int64_t row = row0 + u * 4 + slot;
+      const T* e = reinterpret_cast<const T*>(raw[u]);
+      uint32_t bits = 0;
+      double ss = 0.0;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const float f = to_f32(e[i]);
+        bits |= (uint32_t)(f > 0.f) << i;
+        ss = fma((double)f, (double)f, ss);
+      }
+      // word w = dims [32 w, 32 w + 32) = lanes 2 w (low half) and 2 w + 1
+      const uint32_t hi_half = __shfl_down_sync(0xffffffffu, bits, 1);
+      const uint32_t word = bits | (hi_half << 16);
+      const uint32_t w1 = __shfl_down_sync(0xffffffffu, word, 2);
+      const uint32_t w2 = __shfl_down_sync(0xffffffffu, word, 4);
+      const uint32_t w3 = __shfl_down_sync(0xffffffffu, word, 6);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+      if (sub == 0 && row < m.rows) {
+        uint32_t* dst = codes + m.c_off(row);
+        if (vec_store) {
+          *reinterpret_cast<uint4*>(dst) = make_uint4(word, w1, w2, w3);
+        } else {
+          dst[0] = word;
+          dst[1] = w1;
+          dst[2] = w2;
+          dst[3] = w3;
+        }
+        if (norms != nullptr) norms[m.n_off(row)] = __half_as_ushort(__double2half(sqrt(ss)));
+      }
     }
   }
 }
@@ -449,8 +478,156 @@ int run_lsh(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, 
   return cuda_check(cudaGetLastError(), "lsh encode launch");
 }
 
+// Small bf16 batches with the packed 16-bit weights: the same cluster layout
+// as mlp_rows_kernel with both layers on the tensor cores (mma.sync m16n8k16;
+// rows are M).  Layer 1 in bf16 with fp32 sums; h = SiLU(z) with
+// sigmoid(z) = (1 + tanh(z / 2)) / 2 (hardware tanh), rounded to fp16; layer 2
+// in fp16 with fp32 sums: the arithmetic of the tensor-core batch encoder.
+__device__ __forceinline__ void mma16816_any(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1, bool f16) {
+  if (f16)
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void cp16(void* dst, const void* src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ float silu_tanh(float z) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+  return z * fmaf(0.5f, t, 0.5f);
+}
+
+template <int BITS>
+__global__ void __cluster_dims__(kMlpCluster, 1, 1) __launch_bounds__(kThreads)
+mlp_rows_tc_kernel(const __nv_bfloat16* __restrict__ x, const void* __restrict__ packed, const float* __restrict__ b1,
+                   const float* __restrict__ b2, int hidden, RowMap m, uint32_t* __restrict__ codes) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  constexpr int D = kHeadDim, R = kMlpClusterRows, NB = BITS / kMlpCluster, XP = D + 8;
+  const int rank = (int)cluster.block_rank(), tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, tq = lane & 3;
+  const int64_t row0 = (int64_t)(blockIdx.x / kMlpCluster) * R;
+  const int hp = (hidden + 63) & ~63, uc = hp / kMlpCluster, u0 = rank * uc;  // uc: multiple of 8
+  const int HP = hp + 8, UP = uc + 8;
+  const __nv_bfloat16* W1p = static_cast<const __nv_bfloat16*>(packed);
+  const __half* W2p = reinterpret_cast<const __half*>(W1p + (size_t)hp * D);
+  extern __shared__ __align__(16) unsigned char msm_raw[];
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(msm_raw);  // [R][XP]
+  __nv_bfloat16* w1s = xs + R * XP;                                // [uc][XP]
+  __half* hs = reinterpret_cast<__half*>(w1s + uc * XP);           // [R][UP], read by the cluster
+  __half* hall = hs + R * UP;                                      // [R][HP]
+  __half* w2s = hall + R * HP;                                     // [NB][HP]
+  // stage x rows, this CTA's W1 rows and W2 rows with cp.async (16 bytes each)
+  for (int i = tid; i < R * (D / 8); i += kThreads) {
+    const int r = i / (D / 8), c = i % (D / 8);
+    const int64_t row = row0 + r;
+    if (row < m.rows)
+      cp16(xs + r * XP + c * 8, x + m.x_off(row) + c * 8);
+    else
+      *reinterpret_cast<uint4*>(xs + r * XP + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  for (int i = tid; i < uc * (D / 8); i += kThreads) {
+    const int r = i / (D / 8), c = i % (D / 8);
+    cp16(w1s + r * XP + c * 8, W1p + (size_t)(u0 + r) * D + c * 8);
+  }
+  for (int i = tid; i < NB * (hp / 8); i += kThreads) {
+    const int r = i / (hp / 8), c = i % (hp / 8);
+    cp16(w2s + r * HP + c * 8, W2p + (size_t)(rank * NB + r) * hp + c * 8);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  // layer 1: warp w takes hidden columns [8 w', 8 w' + 8) for w' = w, w + 8, ...
+  for (int nt = warp; nt < uc / 8; nt += kThreads / 32) {
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const int k0 = ks * 16 + 2 * tq;
+      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(xs + gid * XP + k0);
+      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(xs + (gid + 8) * XP + k0);
+      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(xs + gid * XP + k0 + 8);
+      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(xs + (gid + 8) * XP + k0 + 8);
+      const uint32_t bb0 = *reinterpret_cast<const uint32_t*>(w1s + (nt * 8 + gid) * XP + k0);
+      const uint32_t bb1 = *reinterpret_cast<const uint32_t*>(w1s + (nt * 8 + gid) * XP + k0 + 8);
+      mma16816_any(c, a0, a1, a2, a3, bb0, bb1, false);
+    }
+    const int u = nt * 8 + 2 * tq;  // local hidden unit of c[0] (rows gid) and c[1]
+    const float bias0 = u0 + u < hidden ? b1[u0 + u] : 0.f, bias1 = u0 + u + 1 < hidden ? b1[u0 + u + 1] : 0.f;
+    *reinterpret_cast<__half2*>(hs + gid * UP + u) =
+        __floats2half2_rn(silu_tanh(c[0] + bias0), silu_tanh(c[1] + bias1));
+    *reinterpret_cast<__half2*>(hs + (gid + 8) * UP + u) =
+        __floats2half2_rn(silu_tanh(c[2] + bias0), silu_tanh(c[3] + bias1));
+  }
+  cluster.sync();
+  {
+    // all hidden units of the 16 rows: 16-byte pieces from the 8 CTAs
+    const int per_cta = R * (uc / 8);
+    for (int i = tid; i < kMlpCluster * per_cta; i += kThreads) {
+      const int cc = i / per_cta, j = i % per_cta, r = j / (uc / 8), c8 = j % (uc / 8);
+      const __half* remote = cluster.map_shared_rank(hs, cc);
+      *reinterpret_cast<uint4*>(hall + r * HP + cc * uc + c8 * 8) =
+          *reinterpret_cast<const uint4*>(remote + r * UP + c8 * 8);
+    }
+  }
+  cluster.sync();  // no CTA leaves while another still reads its hidden units
+  // layer 2: warp w < NB / 8 takes output bits [8 w, 8 w + 8) of this CTA's NB
+  if (warp < NB / 8) {
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int ks = 0; ks < hp / 16; ++ks) {
+      const int k0 = ks * 16 + 2 * tq;
+      const uint32_t a0 = *reinterpret_cast<const uint32_t*>(hall + gid * HP + k0);
+      const uint32_t a1 = *reinterpret_cast<const uint32_t*>(hall + (gid + 8) * HP + k0);
+      const uint32_t a2 = *reinterpret_cast<const uint32_t*>(hall + gid * HP + k0 + 8);
+      const uint32_t a3 = *reinterpret_cast<const uint32_t*>(hall + (gid + 8) * HP + k0 + 8);
+      const uint32_t bb0 = *reinterpret_cast<const uint32_t*>(w2s + (warp * 8 + gid) * HP + k0);
+      const uint32_t bb1 = *reinterpret_cast<const uint32_t*>(w2s + (warp * 8 + gid) * HP + k0 + 8);
+      mma16816_any(c, a0, a1, a2, a3, bb0, bb1, true);
+    }
+    const int j = rank * NB + warp * 8 + 2 * tq;  // output bit of c[0]
+    uint32_t lo = (uint32_t)(c[0] + b2[j] > 0.f) | ((uint32_t)(c[1] + b2[j + 1] > 0.f) << 1);
+    uint32_t hi = (uint32_t)(c[2] + b2[j] > 0.f) | ((uint32_t)(c[3] + b2[j + 1] > 0.f) << 1);
+    lo <<= 2 * tq;
+    hi <<= 2 * tq;
+    lo |= __shfl_xor_sync(0xffffffffu, lo, 1);
+    lo |= __shfl_xor_sync(0xffffffffu, lo, 2);
+    hi |= __shfl_xor_sync(0xffffffffu, hi, 1);
+    hi |= __shfl_xor_sync(0xffffffffu, hi, 2);
+    if (tq == 0) {
+      // byte (rank * NB + 8 warp) / 8 of the row's code
+      const int byte = (rank * NB) / 8 + warp;
+      if (row0 + gid < m.rows) reinterpret_cast<uint8_t*>(codes)[m.c_off(row0 + gid) * 4 + byte] = (uint8_t)lo;
+      if (row0 + gid + 8 < m.rows)
+        reinterpret_cast<uint8_t*>(codes)[m.c_off(row0 + gid + 8) * 4 + byte] = (uint8_t)hi;
+    }
+  }
+}
+
 template <typename T, int BITS>
 int run_mlp(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, cudaStream_t st) {
+  if (m.rows <= kFewRows && sizeof(T) == 2 && h.packed != nullptr) {
+    auto kernel = mlp_rows_tc_kernel<BITS>;
+    const int hp = (h.hidden + 63) & ~63, uc = hp / kMlpCluster;
+    const size_t smem = 2 * ((size_t)kMlpClusterRows * (kHeadDim + 8) + (size_t)uc * (kHeadDim + 8) +
+                             (size_t)kMlpClusterRows * (uc + 8) + (size_t)kMlpClusterRows * (hp + 8) +
+                             (size_t)(BITS / kMlpCluster) * (hp + 8));
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_check(e, "mlp rows tc smem attribute");
+    const int64_t clusters = (m.rows + kMlpClusterRows - 1) / kMlpClusterRows;
+    kernel<<<(unsigned)(clusters * kMlpCluster), kThreads, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(x), h.packed, h.b1, h.b2, h.hidden, m, codes);
+    return cuda_check(cudaGetLastError(), "mlp rows tc launch");
+  }
   if (m.rows <= kFewRows) {
     auto kernel = mlp_rows_kernel<T, BITS>;
     const int hs = mlp_rows_slice(h.hidden);
@@ -476,8 +653,9 @@ int run_mlp(const hkv_hash& h, const void* x, const RowMap& m, uint32_t* codes, 
 template <typename T>
 int run_sign(const void* x, const RowMap& m, uint32_t* codes, uint16_t* norms, cudaStream_t st) {
   auto kernel = sign_encode_kernel<T>;
-  const int grid = grid_for(kernel, 0, (m.rows + 7) / 8);
-  kernel<<<grid, kThreads, 0, st>>>(static_cast<const T*>(x), m, codes, norms);
+  const int grid = grid_for(kernel, 0, (m.rows + 127) / 128);
+  const bool vec = reinterpret_cast<uintptr_t>(codes) % 16 == 0 && m.c_row % 4 == 0 && m.c_group % 4 == 0;
+  kernel<<<grid, kThreads, 0, st>>>(static_cast<const T*>(x), m, codes, norms, vec);
   return cuda_check(cudaGetLastError(), "sign encode launch");
 }
 

@@ -134,17 +134,21 @@ def test_encode_mlp(dtype, bits, hidden):
     np.testing.assert_array_equal(u32(codes), oracle.encode("mlp", x, params))
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_encode_sign_and_norms(dtype):
+@pytest.mark.parametrize("dtype,rows,code_pitch", [("f32", 2049, 4), ("bf16", 2049, 4), ("bf16", 70001, 4),
+                                                   ("bf16", 3001, 5)])
+def test_encode_sign_and_norms(dtype, rows, code_pitch):
+    """Sign codes and fp16 norms, bit-exact; a code pitch of 5 words takes
+    the scalar-store path."""
     tdt, code = _dt(dtype)
     from tests.helpers import sign_bad
-    x = _rows(23, 2049, 128, dtype, sign_bad())
-    codes = torch.zeros(2049, 4, dtype=torch.int32, device=DEV)
-    norms = torch.zeros(2049, dtype=torch.float16, device=DEV)
-    hkv.hkv_encode_keys(hkv.HashParams.sign(code), x.to(DEV), codes, norms)
+    x = _rows(23, rows, 128, dtype, sign_bad())
+    codes = torch.full((rows, code_pitch), -7, dtype=torch.int32, device=DEV)
+    norms = torch.zeros(rows, dtype=torch.float16, device=DEV)
+    hkv.hkv_encode_keys(hkv.HashParams.sign(code), x.to(DEV), codes[:, :4], norms)
     torch.cuda.synchronize()
     wc, wn = oracle.encode("sign", x)
-    np.testing.assert_array_equal(u32(codes), wc)
+    np.testing.assert_array_equal(u32(codes[:, :4]), wc)
+    assert (codes[:, 4:] == -7).all()
     np.testing.assert_array_equal(norms.cpu().numpy().view(np.uint16), wn.view(np.uint16))
 
 
