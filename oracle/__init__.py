@@ -236,6 +236,32 @@ def retrieve(q_codes, k_codes, N: int, n_sink: int, n_local: int, top_k: int):
     return idx, dist
 
 
+def evict_victim(q_codes, k_codes, N: int, n_sink: int, n_local: int):
+    """[HE] eviction: at each decoding step the token expected to receive the
+    lowest attention -- the cached key whose code is least similar to the
+    current query's, i.e. the largest D(t) -- is replaced by the new token.
+    Candidates are [sink_end, local_start) (sink and local rows stay); ties go
+    to the lowest index.  q_codes [B, Hq, W]; k_codes [B, Hkv, cap, W].
+    Returns victim [B, Hkv] int64 (-1 without candidates) and its D (-1)."""
+    q_codes = np.asarray(q_codes, dtype=np.uint32)
+    k_codes = np.asarray(k_codes, dtype=np.uint32)
+    B, Hq, _ = q_codes.shape
+    Hkv = k_codes.shape[1]
+    g = Hq // Hkv
+    lo, hi = candidate_range(N, n_sink, n_local)
+    victim = np.full((B, Hkv), -1, dtype=np.int64)
+    vdist = np.full((B, Hkv), -1, dtype=np.int64)
+    if hi <= lo:
+        return victim, vdist
+    for b in range(B):
+        for kh in range(Hkv):
+            D = hamming(q_codes[b, kh * g:(kh + 1) * g], k_codes[b, kh, lo:hi])
+            best = int(D.max())
+            victim[b, kh] = lo + int(np.flatnonzero(D == best)[0])
+            vdist[b, kh] = best
+    return victim, vdist
+
+
 def decode_step(q, K, V, k_codes, N: int, n_sink: int, n_local: int, top_k: int,
                 kind: str, q_params=None, scale: float | None = None):
     """One decode step: encode the query heads, retrieve the top-k keys of each

@@ -329,3 +329,56 @@ def test_decode_step_uses_group_sum():
              for t in range(N)]
         want = sorted(sorted(range(N), key=lambda t: (D[t], t))[:10])
         np.testing.assert_array_equal(r1["idx"][0, j], want)
+
+
+# --------------------------------------------------------------- eviction
+
+def test_evict_fixture():
+    gl = golden("evict_dissimilar.txt")
+    q = np.array([[[int(gl["q"][0], 16)]]], dtype=np.uint32)
+    keys = np.array([int(v, 16) for v in gl["keys"]], dtype=np.uint32).reshape(1, 1, -1, 1)
+    s, l = (int(v) for v in gl["sink_local"])
+    victim, vdist = oracle.evict_victim(q, keys, keys.shape[2], s, l)
+    assert victim[0, 0] == int(gl["victim"][0]) and vdist[0, 0] == int(gl["vdist"][0])
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_evict_brute_force(seed):
+    """Bit strings and a plain maximum scan, independent of the oracle's
+    vectorised popcount and argmax."""
+    rng = np.random.default_rng(seed)
+    B, Hq, Hkv, W, N, s, l = 2, 6, 2, 2, 23, 2, 3
+    # few distinct codes, so the maximum is often tied
+    pool = rng.integers(0, 2**32, size=(4, W), dtype=np.uint64).astype(np.uint32)
+    k = pool[rng.integers(0, 4, size=(B, Hkv, N))]
+    q = rng.integers(0, 2**32, size=(B, Hq, W), dtype=np.uint64).astype(np.uint32)
+    victim, vdist = oracle.evict_victim(q, k, N, s, l)
+    g = Hq // Hkv
+    for b in range(B):
+        for j in range(Hkv):
+            best, arg = -1, -1
+            for t in range(s, N - l):
+                d = sum(bin(int(q[b, j * g + h, w]) ^ int(k[b, j, t, w])).count("1") for h in range(g) for w in range(W))
+                if d > best:
+                    best, arg = d, t
+            assert victim[b, j] == arg and vdist[b, j] == best
+
+
+def test_evict_complemented_query_is_top1_retrieval():
+    """With every query bit flipped D becomes g * bits - D, so the eviction
+    victim is the top-1 retrieved token (both take the lowest index on ties)."""
+    rng = np.random.default_rng(5)
+    B, Hq, Hkv, W, N, s, l = 1, 4, 2, 4, 300, 4, 16
+    pool = rng.integers(0, 2**32, size=(16, W), dtype=np.uint64).astype(np.uint32)
+    k = pool[rng.integers(0, 16, size=(B, Hkv, N))]
+    q = rng.integers(0, 2**32, size=(B, Hq, W), dtype=np.uint64).astype(np.uint32)
+    victim, _ = oracle.evict_victim(~q, k, N, s, l)
+    idx, _ = oracle.retrieve(q, k, N, s, l, 1)
+    np.testing.assert_array_equal(victim, idx[..., 0])
+
+
+def test_evict_without_candidates():
+    q = np.zeros((1, 2, 4), dtype=np.uint32)
+    k = np.zeros((1, 1, 10, 4), dtype=np.uint32)
+    victim, vdist = oracle.evict_victim(q, k, 10, 6, 6)
+    assert victim[0, 0] == -1 and vdist[0, 0] == -1
