@@ -28,7 +28,7 @@ __all__ = [
     "HKV_HASH_SIGN", "HKV_HASH_NONE", "HkvError", "HashParams", "lib", "lib_path", "workspace", "status_word",
     "hkv_version", "hkv_last_error", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
     "hkv_encode_keys", "hkv_mlp_pack_bytes", "hkv_mlp_pack", "hkv_append", "hkv_retrieve_topk",
-    "hkv_retrieve_topk_static", "hkv_sparse_attend",
+    "hkv_retrieve_topk_static", "hkv_sparse_attend", "hkv_evict_select", "hkv_write_slots",
     "hkv_lse_merge", "hkv_decode_step", "hkv_debug_set", "EXPORTS",
 ]
 
@@ -41,7 +41,7 @@ HKV_HASH_LSH, HKV_HASH_MLP, HKV_HASH_SIGN, HKV_HASH_NONE = 0, 1, 2, 3
 EXPORTS = (
     "hkv_last_error", "hkv_version", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
     "hkv_encode_keys", "hkv_mlp_pack_bytes", "hkv_mlp_pack", "hkv_append", "hkv_retrieve_topk",
-    "hkv_retrieve_topk_static", "hkv_sparse_attend",
+    "hkv_retrieve_topk_static", "hkv_sparse_attend", "hkv_evict_select", "hkv_write_slots",
     "hkv_lse_merge", "hkv_decode_step", "hkv_debug_set",
 )
 
@@ -82,6 +82,8 @@ _SIGS = {
     "hkv_decode_step": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _F,
                              _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "hkv_debug_set": (_I, [_I, _I64]),
+    "hkv_evict_select": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _P, _P, _P, _SZ, _P]),
+    "hkv_write_slots": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P]),
 }
 _lib = None
 
@@ -330,6 +332,42 @@ def hkv_lse_merge(o1, lse1, o2, lse2, out, lse_out=None, stream=None) -> None:
         _need(lse_out, "lse_out", torch.float32, shape=(rows,))
     _ok(lib().hkv_lse_merge(rows, d, _ptr(o1), _ptr(lse1), _ptr(o2), _ptr(lse2), _ptr(out), _ptr(lse_out),
                             _stream(stream)))
+
+
+def hkv_evict_select(q_codes, k_codes, n_tokens: int, n_sink: int, n_local: int, victim, vdist=None, ws=None,
+                     stream=None) -> None:
+    """victim [B, Hkv] int32: the most dissimilar non-resident token per KV head."""
+    B, Hq, W = q_codes.shape
+    _, Hkv, cap, W2 = k_codes.shape
+    _need(q_codes, "q_codes", _U32)
+    _need(k_codes, "k_codes", _U32)
+    _need(victim, "victim", torch.int32, shape=(B, Hkv))
+    if vdist is not None:
+        _need(vdist, "vdist", torch.int32, shape=(B, Hkv))
+    if W2 != W:
+        raise ValueError("q_codes and k_codes differ in code width")
+    if ws is None:
+        ws = torch.zeros(8 * B * Hkv, dtype=torch.uint8, device=q_codes.device)
+    _ok(lib().hkv_evict_select(B, Hq, Hkv, W * 32, _ptr(q_codes), _ptr(k_codes), cap, n_tokens, n_sink, n_local,
+                               _ptr(victim), _ptr(vdist), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def hkv_write_slots(k_new, v_new, codes_new, K, V, codes, slot, norms_new=None, norms=None, status=None,
+                    stream=None) -> None:
+    """k_new, v_new [B, Hkv, 128]; codes_new [B, Hkv, W]; slot [B, Hkv] int32 (-1 skips)."""
+    B, Hkv, d = k_new.shape
+    cap = K.shape[2]
+    _need(k_new, "k_new", (torch.bfloat16, torch.float32))
+    _need(v_new, "v_new", k_new.dtype, shape=(B, Hkv, d))
+    _need(K, "K", k_new.dtype, shape=(B, Hkv, cap, d))
+    _need(V, "V", k_new.dtype, shape=(B, Hkv, cap, d))
+    _need(codes_new, "codes_new", _U32)
+    W = codes_new.shape[-1]
+    _need(codes, "codes", _U32, shape=(B, Hkv, cap, W))
+    _need(slot, "slot", torch.int32, shape=(B, Hkv))
+    _ok(lib().hkv_write_slots(B, Hkv, _dtype_code(k_new), W * 32, _ptr(k_new), _ptr(v_new), _ptr(codes_new),
+                              _ptr(norms_new), _ptr(K), _ptr(V), _ptr(codes), _ptr(norms), cap, _ptr(slot),
+                              _ptr(status), _stream(stream)))
 
 
 def hkv_decode_step(h: HashParams, q, k_codes, K, V, n_tokens: int, n_sink: int, n_local: int, top_k: int, out,

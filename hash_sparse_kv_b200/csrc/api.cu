@@ -250,6 +250,36 @@ int hkv_retrieve_topk_static(int B, int Hq, int Hkv, int code_bits, const uint32
   return launch_retrieve_static(s, q_codes, k_codes, idx, dist, status, static_cast<cudaStream_t>(stream));
 }
 
+int hkv_evict_select(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                     const uint32_t* k_codes, int64_t cap, int64_t n_tokens, int n_sink, int n_local,
+                     int32_t* victim, int32_t* vdist, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_heads(B, Hq, Hkv);
+  if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, 1);
+  if (rc != HKV_OK) return rc;
+  if (code_bits != 64 && code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "code_bits %d (64 or 128)", code_bits);
+  if (B == 0) return HKV_OK;
+  if (!q_codes || !k_codes || !victim) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_codes, code_bits / 8)) return fail(HKV_ERR_INVALID_ARG, "k_codes must be aligned to one code");
+  RetrieveShape s{B, Hq, Hkv, code_bits / 32, cap, n_tokens, n_sink, n_local, 1};
+  return launch_evict(s, q_codes, k_codes, victim, vdist, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int hkv_write_slots(int B, int Hkv, int dtype, int code_bits, const void* k_new, const void* v_new,
+                    const uint32_t* codes_new, const uint16_t* norms_new, void* K, void* V,
+                    uint32_t* codes, uint16_t* norms, int64_t capacity, const int32_t* slot,
+                    int32_t* status, void* stream) {
+  if (B < 0 || Hkv < 1) return fail(HKV_ERR_INVALID_ARG, "B %d Hkv %d", B, Hkv);
+  if (dtype != HKV_F32 && dtype != HKV_BF16) return fail(HKV_ERR_INVALID_ARG, "dtype %d", dtype);
+  if (code_bits != 64 && code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "code_bits %d (64 or 128)", code_bits);
+  if (capacity < 1) return fail(HKV_ERR_INVALID_ARG, "capacity %lld", (long long)capacity);
+  if (B == 0) return HKV_OK;
+  if (!k_new || !v_new || !codes_new || !K || !V || !codes || !slot) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(K, 16) || !aligned(V, 16))
+    return fail(HKV_ERR_INVALID_ARG, "K/V rows must be 16-byte aligned");
+  return launch_write_slots(dtype, B * Hkv, code_bits / 32, k_new, v_new, codes_new, norms_new, K, V, codes, norms,
+                            capacity, slot, status, static_cast<cudaStream_t>(stream));
+}
+
 int hkv_sparse_attend(int B, int Hq, int Hkv, int dtype, const void* q, const void* K,
                       const void* V, int64_t cap, int64_t n_tokens, const int32_t* idx,
                       int top_k, int n_sink, int n_local, float scale, float* out, float* lse,

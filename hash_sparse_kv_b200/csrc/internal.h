@@ -64,6 +64,15 @@ int launch_decode(const RetrieveShape& s, int dtype, int q_kind, const void* R, 
                   const void* V, float scale, float* out, float* lse, void* ws, size_t ws_bytes,
                   int32_t* status, cudaStream_t st);
 
+// ---- eviction (retrieve.cu) ----
+// victim[p] = the candidate with the largest group distance (lowest t on
+// ties), -1 without candidates; ws: 8 bytes per pair, zero, returned to zero.
+int launch_evict(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes, int32_t* victim,
+                 int32_t* vdist, void* ws, size_t ws_bytes, cudaStream_t st);
+int launch_write_slots(int dtype, int P, int W, const void* k_new, const void* v_new, const uint32_t* codes_new,
+                       const uint16_t* norms_new, void* K, void* V, uint32_t* codes, uint16_t* norms, int64_t cap,
+                       const int32_t* slot, int32_t* status, cudaStream_t st);
+
 // ---- attention (attend.cu) ----
 struct AttendShape {
   int B, Hq, Hkv, dtype;

@@ -212,6 +212,35 @@ int hkv_retrieve_topk_static(int B, int Hq, int Hkv, int code_bits, const uint32
                              int n_local, int top_k, int32_t* idx, int32_t* dist, int32_t* status,
                              void* stream);
 
+/* HashEvict eviction (HashEvict "Abstract": at every decoding step the new
+ * token's key and value replace the cached token expected to receive the
+ * lowest attention, found as the key whose binarized projection is farthest
+ * in Hamming distance from the query's).  For KV head j of batch b:
+ *   victim[b, j] = the t in [sink_end, local_start) with the largest
+ *                  D(t) = sum over the g query heads h of
+ *                         popcount(q_code[b, h] XOR k_code[b, j, t]),
+ *                  lowest t on ties; -1 when there is no candidate
+ *   vdist        nullable [B, Hkv] int32: D(victim), -1 without candidates
+ * Sink and local tokens are never evicted.  q_codes, k_codes, cap, n_tokens,
+ * n_sink, n_local as for hkv_retrieve_topk.  ws: 8 * B * Hkv bytes, zero
+ * before the first call; each call returns it to zero (the first bytes of a
+ * hkv_workspace_bytes workspace of the same shape qualify).  Two launches. */
+int hkv_evict_select(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                     const uint32_t* k_codes, int64_t cap, int64_t n_tokens, int n_sink, int n_local,
+                     int32_t* victim, int32_t* vdist, void* ws, size_t ws_bytes, void* stream);
+
+/* Writes one new token per (batch, KV head) into the cache at position
+ * slot[b, j] (e.g. the victim of hkv_evict_select): K and V rows, its code,
+ * and its fp16 norm when both norm pointers are given.  slot -1 skips the
+ * pair; slot >= capacity skips it and reports HKV_ERR_DEVICE_RANGE.
+ *   k_new, v_new  [B, Hkv, head_dim] in dtype;  codes_new [B, Hkv, code_bits/32]
+ *   norms_new     nullable [B, Hkv] fp16 bits;  K, V, codes, norms: the cache
+ * The new codes come from hkv_encode_keys on k_new. */
+int hkv_write_slots(int B, int Hkv, int dtype, int code_bits, const void* k_new, const void* v_new,
+                    const uint32_t* codes_new, const uint16_t* norms_new, void* K, void* V,
+                    uint32_t* codes, uint16_t* norms, int64_t capacity, const int32_t* slot,
+                    int32_t* status, void* stream);
+
 /* Sparse attention over sink + selected + local rows, with the log-sum-exp
  * merge of the partials (S6, S7, S8).  Spotlight Attention "Approach" (exact
  * attention over the retrieved tokens); RetrievalAttention "Approach" (exact

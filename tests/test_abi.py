@@ -76,3 +76,14 @@ def test_mlp_pack_sizes(lib):
     assert lib.hkv_mlp_pack_bytes(0, 128) == 0
     assert lib.hkv_mlp_pack_bytes(2048, 128) == 0
     assert lib.hkv_mlp_pack_bytes(512, 96) == 0
+
+
+def test_eviction_argument_errors(lib):
+    rc = lib.hkv_evict_select(1, 4, 2, 96, None, None, 10, 10, 0, 0, None, None, None, 0, None)
+    assert rc == hkv.HKV_ERR_UNSUPPORTED
+    rc = lib.hkv_evict_select(1, 4, 3, 128, None, None, 10, 10, 0, 0, None, None, None, 0, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG  # 4 query heads do not split over 3 KV heads
+    rc = lib.hkv_write_slots(1, 2, 7, 128, None, None, None, None, None, None, None, None, 10, None, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG
+    assert lib.hkv_write_slots(0, 2, hkv.HKV_BF16, 128, None, None, None, None, None, None, None, None, 10, None,
+                               None, None) == hkv.HKV_OK
