@@ -286,3 +286,47 @@ def decode_step(q, K, V, k_codes, N: int, n_sink: int, n_local: int, top_k: int,
             out[b, kh * g:(kh + 1) * g] = o
             lse[b, kh * g:(kh + 1) * g] = l
     return {"q_codes": qc, "idx": idx, "dist": dist, "out": out, "lse": lse}
+
+
+def retrieve_heads(q_codes, k_codes, N: int, n_sink: int, n_local: int, top_k: int):
+    """[RA] one index set per query head: head h of batch b scores the keys of
+    its KV head j = h // g by its own Hamming distance
+    D_h(t) = popcount(cq_h XOR ck_t) and keeps its k smallest (ties to the
+    lowest index).  q_codes [B, Hq, W]; k_codes [B, Hkv, cap, W].
+    Returns idx, dist [B, Hq, top_k] (ascending, -1 past k_eff)."""
+    q_codes = np.asarray(q_codes, dtype=np.uint32)
+    k_codes = np.asarray(k_codes, dtype=np.uint32)
+    B, Hq, _ = q_codes.shape
+    g = Hq // k_codes.shape[1]
+    lo, hi = candidate_range(N, n_sink, n_local)
+    idx = np.full((B, Hq, top_k), -1, dtype=np.int64)
+    dist = np.full((B, Hq, top_k), -1, dtype=np.int64)
+    for b in range(B):
+        for h in range(Hq):
+            D = hamming(q_codes[b, h:h + 1], k_codes[b, h // g, :N])
+            sel = select_topk(D, lo, hi, top_k)
+            idx[b, h, : sel.size] = sel
+            dist[b, h, : sel.size] = D[sel]
+    return idx, dist
+
+
+def decode_step_heads(q, K, V, k_codes, N: int, n_sink: int, n_local: int, top_k: int,
+                      kind: str, q_params=None, scale: float | None = None):
+    """decode_step with one index set per query head ([RA]): head h attends
+    over sink + its own selected rows + local rows of its KV head."""
+    qa = as_f64(q)
+    B, Hq, d = qa.shape
+    g = Hq // K.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    qc = encode(kind, qa, q_params)
+    if kind == "sign":
+        qc = qc[0]
+    idx, dist = retrieve_heads(qc, k_codes, N, n_sink, n_local, top_k)
+    out = np.zeros((B, Hq, d))
+    lse = np.zeros((B, Hq))
+    for b in range(B):
+        for h in range(Hq):
+            rows = attention_rows(N, n_sink, n_local, idx[b, h])
+            o, l = attend(qa[b, h:h + 1], K[b, h // g], V[b, h // g], rows, scale)
+            out[b, h], lse[b, h] = o[0], l[0]
+    return {"q_codes": qc, "idx": idx, "dist": dist, "out": out, "lse": lse}

@@ -382,3 +382,56 @@ def test_evict_without_candidates():
     k = np.zeros((1, 1, 10, 4), dtype=np.uint32)
     victim, vdist = oracle.evict_victim(q, k, 10, 6, 6)
     assert victim[0, 0] == -1 and vdist[0, 0] == -1
+
+
+# ------------------------------------------------- one index set per query head
+
+def test_heads_equal_group_selection_when_groups_are_single_heads():
+    """With g = 1 every query head has its own KV head: both readings agree."""
+    rng = np.random.default_rng(8)
+    q = rng.integers(0, 2**32, size=(2, 3, 4), dtype=np.uint64).astype(np.uint32)
+    k = rng.integers(0, 2**32, size=(2, 3, 50, 4), dtype=np.uint64).astype(np.uint32)
+    a = oracle.retrieve_heads(q, k, 50, 2, 5, 7)
+    b = oracle.retrieve(q, k, 50, 2, 5, 7)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_heads_with_identical_queries_match_the_group():
+    """If all g heads of a group share one code, the group distance is g times
+    the head distance: the same order, so the same index sets."""
+    rng = np.random.default_rng(9)
+    one = rng.integers(0, 2**32, size=(1, 2, 1, 4), dtype=np.uint64).astype(np.uint32)
+    q = np.repeat(one, 3, axis=2).reshape(1, 6, 4)  # heads 0-2 share a code, heads 3-5 another
+    pool = rng.integers(0, 2**32, size=(5, 4), dtype=np.uint64).astype(np.uint32)
+    k = pool[rng.integers(0, 5, size=(1, 2, 80))]
+    ih, dh = oracle.retrieve_heads(q, k, 80, 3, 4, 9)
+    ig, dg = oracle.retrieve(q, k, 80, 3, 4, 9)
+    for h in range(6):
+        np.testing.assert_array_equal(ih[0, h], ig[0, h // 3])
+        np.testing.assert_array_equal(dh[0, h] * 3, np.where(dg[0, h // 3] >= 0, dg[0, h // 3], -3))
+
+
+def test_heads_brute_force():
+    rng = np.random.default_rng(10)
+    B, Hq, Hkv, W, N, s, l, kk = 1, 4, 2, 2, 30, 2, 3, 5
+    q = rng.integers(0, 2**32, size=(B, Hq, W), dtype=np.uint64).astype(np.uint32)
+    k = rng.integers(0, 2**32, size=(B, Hkv, N, W), dtype=np.uint64).astype(np.uint32)
+    idx, _ = oracle.retrieve_heads(q, k, N, s, l, kk)
+    for h in range(Hq):
+        d = [sum(bin(int(q[0, h, w]) ^ int(k[0, h // 2, t, w])).count("1") for w in range(W)) for t in range(N)]
+        order = sorted(range(s, N - l), key=lambda t: (d[t], t))[:kk]
+        assert list(idx[0, h]) == sorted(order)
+
+
+def test_decode_step_heads_single_head_groups_equal_decode_step():
+    rng = np.random.default_rng(11)
+    B, H, N, d = 1, 2, 40, 128
+    q = rng.normal(size=(B, H, d))
+    K = rng.normal(size=(B, H, N, d))
+    V = rng.normal(size=(B, H, N, d))
+    kc = oracle.encode("sign", K)[0]
+    a = oracle.decode_step_heads(q, K, V, kc, N, 2, 3, 6, "sign")
+    b = oracle.decode_step(q, K, V, kc, N, 2, 3, 6, "sign")
+    np.testing.assert_array_equal(a["idx"], b["idx"])
+    np.testing.assert_allclose(a["out"], b["out"], rtol=0, atol=1e-14)
