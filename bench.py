@@ -356,6 +356,17 @@ def run_gpu(args, rank, world, local):
     qenc_ms = max_over_ranks(time_graph(g_qenc, args.steps, args.warmup, world), world, dev)
     g_att = graph_of(attend_only)
     att_ms = max_over_ranks(time_graph(g_att, args.steps, args.warmup, world), world, dev)
+    # HashEvict eviction choice for every layer (one scan of the codes each)
+    victims = [torch.zeros(w.B, w.Hkv, dtype=torch.int32, device=dev) for _ in layers]
+    ws_e = torch.zeros(8 * w.B * w.Hkv, dtype=torch.uint8, device=dev)
+
+    def evict_only():
+        for L, vic in zip(layers, victims):
+            hkv.hkv_evict_select(L.q_codes, L.codes, w.N, w.n_sink, w.n_local, vic, ws=ws_e)
+
+    g_ev = graph_of(evict_only)
+    ev_ms = max_over_ranks(time_graph(g_ev, args.steps, args.warmup, world), world, dev)
+    del g_ev
     del g_qenc, g_att
     # end to end: host q in, host out back, every step
     q_host = [torch.empty_like(L.q, device="cpu").pin_memory() for L in layers]
@@ -423,7 +434,11 @@ def run_gpu(args, rank, world, local):
         "kernels_us_per_launch": {"encode_q": qenc_ms * 1e3 / len(layers),
                                   "fused_decode": fused_launch_ms * 1e3,
                                   "retrieve_only": scan_ms * 1e3 / len(layers),
-                                  "sparse_attend_only": att_ms * 1e3 / len(layers)},
+                                  "sparse_attend_only": att_ms * 1e3 / len(layers),
+                                  "evict_select": ev_ms * 1e3 / len(layers)},
+        "evict": {"bound": "hbm", "achieved": code_bytes / (ev_ms * 1e-3 / len(layers)) / 1e9, "peak": peak,
+                  "unit": "GB/s", "frac": code_bytes / (ev_ms * 1e-3 / len(layers)) / 1e9 / peak,
+                  "bytes_per_launch": code_bytes, "launches_per_layer": 2},
         # decode with an LSH or sign query hash (query heads per KV head <= 32) is one
         # fused launch a layer; an MLP query hash adds the separate query encode launch
         "gpu_launches": (1 if w.hash in ("lsh", "sign") and w.g <= 32 else 2) * len(layers) * args.steps,

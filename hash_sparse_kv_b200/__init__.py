@@ -28,8 +28,8 @@ __all__ = [
     "HKV_HASH_SIGN", "HKV_HASH_NONE", "HkvError", "HashParams", "lib", "lib_path", "workspace", "status_word",
     "hkv_version", "hkv_last_error", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
     "hkv_encode_keys", "hkv_mlp_pack_bytes", "hkv_mlp_pack", "hkv_append", "hkv_retrieve_topk",
-    "hkv_retrieve_topk_static", "hkv_sparse_attend", "hkv_evict_select", "hkv_write_slots",
-    "hkv_lse_merge", "hkv_decode_step", "hkv_debug_set", "EXPORTS",
+    "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_sparse_attend", "hkv_evict_select",
+    "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads", "hkv_debug_set", "EXPORTS",
 ]
 
 HKV_OK, HKV_ERR_INVALID_ARG, HKV_ERR_UNSUPPORTED, HKV_ERR_CAPACITY = 0, -1, -2, -3
@@ -41,8 +41,8 @@ HKV_HASH_LSH, HKV_HASH_MLP, HKV_HASH_SIGN, HKV_HASH_NONE = 0, 1, 2, 3
 EXPORTS = (
     "hkv_last_error", "hkv_version", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
     "hkv_encode_keys", "hkv_mlp_pack_bytes", "hkv_mlp_pack", "hkv_append", "hkv_retrieve_topk",
-    "hkv_retrieve_topk_static", "hkv_sparse_attend", "hkv_evict_select", "hkv_write_slots",
-    "hkv_lse_merge", "hkv_decode_step", "hkv_debug_set",
+    "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_sparse_attend", "hkv_evict_select",
+    "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads", "hkv_debug_set",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -82,6 +82,9 @@ _SIGS = {
     "hkv_decode_step": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _F,
                              _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "hkv_debug_set": (_I, [_I, _I64]),
+    "hkv_retrieve_topk_heads": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _SZ, _P, _P]),
+    "hkv_decode_step_heads": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _F,
+                                   _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "hkv_evict_select": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _P, _P, _P, _SZ, _P]),
     "hkv_write_slots": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P]),
 }
@@ -332,6 +335,47 @@ def hkv_lse_merge(o1, lse1, o2, lse2, out, lse_out=None, stream=None) -> None:
         _need(lse_out, "lse_out", torch.float32, shape=(rows,))
     _ok(lib().hkv_lse_merge(rows, d, _ptr(o1), _ptr(lse1), _ptr(o2), _ptr(lse2), _ptr(out), _ptr(lse_out),
                             _stream(stream)))
+
+
+def hkv_retrieve_topk_heads(q_codes, k_codes, n_tokens: int, n_sink: int, n_local: int, top_k: int, idx,
+                            dist=None, ws=None, status=None, stream=None) -> None:
+    """One index set per query head: idx [B, Hq, top_k] (and dist).  Size ws
+    with workspace(B, Hq, Hq, ...)."""
+    B, Hq, W = q_codes.shape
+    _, Hkv, cap, W2 = k_codes.shape
+    _need(q_codes, "q_codes", _U32)
+    _need(k_codes, "k_codes", _U32, shape=(B, Hkv, cap, W))
+    _need(idx, "idx", torch.int32, shape=(B, Hq, top_k))
+    if dist is not None:
+        _need(dist, "dist", torch.int32, shape=(B, Hq, top_k))
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _ok(lib().hkv_retrieve_topk_heads(B, Hq, Hkv, W * 32, _ptr(q_codes), _ptr(k_codes), cap, n_tokens, n_sink,
+                                      n_local, top_k, _ptr(idx), _ptr(dist), _ptr(ws), nbytes, _ptr(status),
+                                      _stream(stream)))
+
+
+def hkv_decode_step_heads(h: HashParams, q, k_codes, K, V, n_tokens: int, n_sink: int, n_local: int, top_k: int,
+                          out, lse=None, q_codes=None, idx=None, scale: Optional[float] = None, ws=None,
+                          status=None, stream=None) -> None:
+    """hkv_decode_step with one index set per query head (idx [B, Hq, top_k])."""
+    B, Hq, d = q.shape
+    _, Hkv, cap, W = k_codes.shape
+    _need(q, "q", (torch.bfloat16, torch.float32))
+    _need(k_codes, "k_codes", _U32)
+    _need(K, "K", q.dtype, shape=(B, Hkv, cap, d))
+    _need(V, "V", q.dtype, shape=(B, Hkv, cap, d))
+    _need(out, "out", torch.float32, shape=(B, Hq, d))
+    if q_codes is not None:
+        _need(q_codes, "q_codes", _U32, shape=(B, Hq, W))
+    if idx is not None:
+        _need(idx, "idx", torch.int32, shape=(B, Hq, top_k))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, shape=(B, Hq))
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _ok(lib().hkv_decode_step_heads(ctypes.byref(h.c), B, Hq, Hkv, _ptr(q), _ptr(k_codes), _ptr(K), _ptr(V), cap,
+                                    n_tokens, n_sink, n_local, top_k, scale, _ptr(q_codes), _ptr(idx), _ptr(out),
+                                    _ptr(lse), _ptr(ws), nbytes, _ptr(status), _stream(stream)))
 
 
 def hkv_evict_select(q_codes, k_codes, n_tokens: int, n_sink: int, n_local: int, victim, vdist=None, ws=None,

@@ -305,7 +305,7 @@ int hkv_lse_merge(int rows, int d, const float* o1, const float* lse1, const flo
   return launch_lse_merge(rows, d, o1, lse1, o2, lse2, out, lse_out, static_cast<cudaStream_t>(stream));
 }
 
-int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
+static int decode_impl(bool per_head, const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
                     const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
                     int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
                     uint32_t* q_codes, int32_t* idx, float* out, float* lse,
@@ -323,8 +323,10 @@ int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* 
   if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) ||
       !aligned(k_codes, q_hash->code_bits / 8) || !aligned(next_k_codes, q_hash->code_bits / 8))
     return fail(HKV_ERR_INVALID_ARG, "q, K, V, out and k_codes must be aligned");
+  // selection units: KV heads, or query heads (one index set each)
+  const int units = per_head ? Hq : Hkv;
   DecodeLayout L;
-  rc = decode_layout(B, Hq, Hkv, n_tokens, q_hash->code_bits, top_k, n_sink, n_local, L);
+  rc = decode_layout(B, Hq, units, n_tokens, q_hash->code_bits, top_k, n_sink, n_local, L);
   if (rc != HKV_OK) return fail(rc, "unsupported decode shape");
   if (ws == nullptr || ws_bytes < L.total) return fail(HKV_ERR_CAPACITY, "workspace of %zu bytes, %zu needed", ws_bytes, L.total);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -335,7 +337,7 @@ int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* 
   int32_t* ix = idx ? idx : reinterpret_cast<int32_t*>(base + L.fused + L.attend + L.qcodes);
   const int W = q_hash->code_bits / 32;
   const Window w = window(n_tokens, n_sink, n_local);
-  RetrieveShape rs{B, Hq, Hkv, W, cap, n_tokens, n_sink, n_local, top_k};
+  RetrieveShape rs{B, Hq, units, W, cap, n_tokens, n_sink, n_local, top_k, per_head ? Hkv : 0};
   const bool fused_encode = !given_codes && w.C > 0 && top_k > 0 &&
                             decode_encodes_queries(rs, q_hash->kind, q_hash->dtype);
   if (!given_codes && !fused_encode) {
@@ -346,7 +348,7 @@ int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* 
   if (w.C == 0 || top_k == 0) {
     // nothing to retrieve: attend the resident rows only
     if (top_k > 0) {
-      rc = cuda_check(cudaMemsetAsync(ix, 0xff, sizeof(int32_t) * (size_t)B * Hkv * top_k, st), "idx fill");
+      rc = cuda_check(cudaMemsetAsync(ix, 0xff, sizeof(int32_t) * (size_t)B * units * top_k, st), "idx fill");
       if (rc != HKV_OK) return rc;
     }
     AttendShape as{B, Hq, Hkv, q_hash->dtype, cap, n_tokens, top_k, n_sink, n_local};
@@ -357,6 +359,40 @@ int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* 
                          scale, out, lse, ws_f, L.fused, status, st);
   return launch_decode(rs, q_hash->dtype, HKV_HASH_NONE, nullptr, qc, nullptr, k_codes, next_k_codes, ix, q, K, V,
                        scale, out, lse, ws_f, L.fused, status, st);
+}
+
+int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
+                    const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
+                    int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
+                    uint32_t* q_codes, int32_t* idx, float* out, float* lse,
+                    const uint32_t* next_k_codes, void* ws, size_t ws_bytes, int32_t* status,
+                    void* stream) {
+  return decode_impl(false, q_hash, B, Hq, Hkv, q, k_codes, K, V, cap, n_tokens, n_sink, n_local, top_k, scale,
+                     q_codes, idx, out, lse, next_k_codes, ws, ws_bytes, status, stream);
+}
+
+int hkv_decode_step_heads(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
+                          const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
+                          int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
+                          uint32_t* q_codes, int32_t* idx, float* out, float* lse, void* ws,
+                          size_t ws_bytes, int32_t* status, void* stream) {
+  return decode_impl(true, q_hash, B, Hq, Hkv, q, k_codes, K, V, cap, n_tokens, n_sink, n_local, top_k, scale,
+                     q_codes, idx, out, lse, nullptr, ws, ws_bytes, status, stream);
+}
+
+int hkv_retrieve_topk_heads(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                            const uint32_t* k_codes, int64_t cap, int64_t n_tokens, int n_sink,
+                            int n_local, int top_k, int32_t* idx, int32_t* dist, void* ws,
+                            size_t ws_bytes, int32_t* status, void* stream) {
+  int rc = check_heads(B, Hq, Hkv);
+  if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
+  if (rc != HKV_OK) return rc;
+  if (code_bits != 64 && code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "code_bits %d (64 or 128)", code_bits);
+  if (B == 0 || top_k == 0) return HKV_OK;
+  if (!q_codes || !k_codes || !idx) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_codes, code_bits / 8)) return fail(HKV_ERR_INVALID_ARG, "k_codes must be %d-byte aligned", code_bits / 8);
+  RetrieveShape s{B, Hq, Hq, code_bits / 32, cap, n_tokens, n_sink, n_local, top_k, Hkv};
+  return launch_retrieve(s, q_codes, k_codes, idx, dist, ws, ws_bytes, status, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -39,10 +39,14 @@ int launch_copy_rows(int dtype, int64_t groups, int64_t T, const void* src, void
                      int64_t dst_group_rows, int64_t dst_row0, cudaStream_t st);
 
 // ---- retrieval (retrieve.cu) ----
+// Hkv is the number of selection units per batch: KV heads (one index set
+// per KV head, scored by the sum over its g query heads), or the query heads
+// themselves (one index set per query head, kv_heads = the KV heads).
 struct RetrieveShape {
   int B, Hq, Hkv, words;
   int64_t cap, N;
   int n_sink, n_local, top_k;
+  int kv_heads = 0;  // KV heads of the cache when they differ from Hkv
 };
 size_t retrieve_ws_bytes(const RetrieveShape& s);
 int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,

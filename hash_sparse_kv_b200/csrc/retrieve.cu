@@ -100,12 +100,20 @@ struct FusedArgs {
   uint32_t* sync;  // [pairs][kSync]
   uint32_t* gh;    // [pairs][nbins]: histogram of the pair (returns to zero)
   const uint32_t* next_codes;  // nullable: codes of the next call, prefetched to L2 after the scan
+  int Hkv_real, unit_div;      // KV heads of the cache; selection units per KV head
   uint32_t* cum;   // [pairs][nseg][nbins]: cumulative counts, window only
   float* part;     // [pairs][nseg][g][kPart]
   int32_t* status;
   uint64_t wait_ns;
   int skip_arrive;
 };
+
+// Cache row of (batch, KV head) for selection unit p (units = KV heads, or
+// query heads with unit_div = g of them per KV head).
+__device__ __forceinline__ int64_t kv_row(const FusedArgs& a, int p) {
+  return (int64_t)(p / a.Hkv) * a.Hkv_real + (p % a.Hkv) / a.unit_div;
+}
+
 
 template <int W, int NP>
 struct Planes {
@@ -364,11 +372,11 @@ __device__ __forceinline__ void chunk_to_f32(const uint4& raw, float* dst, float
 // 64 rows per tile.  The K/V rows of tile i + 1 are loaded into registers
 // while tile i is computed, so the gather latency overlaps the arithmetic.
 template <typename T, typename RowAt>
-__device__ void attn_rows(const FusedArgs& a, int p, int nrows, RowAt row_at, const AttnSmem& sm,
+__device__ void attn_rows(const FusedArgs& a, int64_t kvc, int nrows, RowAt row_at, const AttnSmem& sm,
                           float (&acc)[kOut]) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
-  const T* Kp = tptr<T>(a.K) + (int64_t)p * a.cap * kHeadDim;
-  const T* Vp = tptr<T>(a.V) + (int64_t)p * a.cap * kHeadDim;
+  const T* Kp = tptr<T>(a.K) + kvc * kHeadDim;
+  const T* Vp = tptr<T>(a.V) + kvc * kHeadDim;
   constexpr int EPC = 16 / sizeof(T);           // elements per 16-byte chunk
   constexpr int CPR = kHeadDim / EPC;           // chunks per row
   constexpr int kPer = kRows * CPR / kThreads;  // chunks of each matrix per thread and tile
@@ -520,12 +528,12 @@ __device__ __forceinline__ void split2(float2 x, uint32_t& hi, uint32_t& lo) {
 // (token row_at(i), or -1 to skip); writes the partial (m, l, acc) of every
 // head to dst[h * kPart ...].  Uses smem_attn (kAttnMmaBytes) and tok[2 * kRows].
 template <typename RowAt>
-__device__ void attn_mma(const FusedArgs& a, int p, const float* aq_s, int nrows, RowAt row_at,
+__device__ void attn_mma(const FusedArgs& a, int64_t kvc, const float* aq_s, int nrows, RowAt row_at,
                          unsigned char* smem_attn, int* tok, float* m_s, float* l_s, float* alpha_s, float* dst) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
   const int gid = lane >> 2, tq = lane & 3;
-  const __nv_bfloat16* Kp = tptr<__nv_bfloat16>(a.K) + (int64_t)p * a.cap * kHeadDim;
-  const __nv_bfloat16* Vp = tptr<__nv_bfloat16>(a.V) + (int64_t)p * a.cap * kHeadDim;
+  const __nv_bfloat16* Kp = tptr<__nv_bfloat16>(a.K) + kvc * kHeadDim;
+  const __nv_bfloat16* Vp = tptr<__nv_bfloat16>(a.V) + kvc * kHeadDim;
   float* z = reinterpret_cast<float*>(smem_attn + 4 * kKVTile);  // [kMaxGroup][kZP] scratch
   float* pmax = z;                                  // [8 warps][kMaxGroup] tile maxima
   float* psum = z + (kRows / 8) * kMaxGroup;        // [8 warps][kMaxGroup] tile sums
@@ -905,6 +913,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   const int tid = threadIdx.x;
   const int C = a.C, nseg = a.nseg;
   const int p = a.p0 + (int)blockIdx.x / nseg, seg = (int)blockIdx.x % nseg;
+  const int64_t kvc = kv_row(a, p) * a.cap;  // first cache row of this unit's (batch, KV head)
   const int s0 = seg * a.per_block, s1 = min(s0 + a.per_block, C);
   const int len = s1 - s0;
   const int nt = tid < len ? (len - tid + kThreads - 1) / kThreads : 0;
@@ -927,7 +936,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   float4 aq = make_float4(0.f, 0.f, 0.f, 0.f);
   if (ATTEND && tid < a.g * (kHeadDim / 4))
     aq = load4_f32(tptr<T>(a.q) + qrow0 * kHeadDim + (tid / (kHeadDim / 4)) * kHeadDim + (tid % (kHeadDim / 4)) * 4);
-  const uint32_t* pf_ptr = a.k_codes + ((int64_t)p * a.cap + a.lo + s0 + tid) * W;
+  const uint32_t* pf_ptr = a.k_codes + (kvc + a.lo + s0 + tid) * W;
   constexpr int64_t kStep = (int64_t)kThreads * W;
   auto slot = [&](int k) { return ring + ((size_t)(k % kSlots) * kThreads + tid) * 4; };
 #pragma unroll
@@ -941,7 +950,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     // the block's resident rows go to L2 now; they are attended after the scan
     const int v = seg + tid * nseg;
     const int t = v < a.sink_n ? v : a.local_start + (v - a.sink_n);
-    prefetch_row_l2<T>(a.K, a.V, (int64_t)p * a.cap + t);
+    prefetch_row_l2<T>(a.K, a.V, kvc + t);
   }
   // ---------------- phase A: query codes, histogram reset -------------------
   if (ATTEND && tid < a.g * (kHeadDim / 4)) *reinterpret_cast<float4*>(&aq_s[tid * 4]) = aq;
@@ -995,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   if (a.next_codes != nullptr && tid < 32) {
     // the next call's codes for this block's range go to L2 while this call
     // selects and attends (16-byte aligned pieces; the hint skips ragged ends)
-    const uintptr_t beg = reinterpret_cast<uintptr_t>(a.next_codes + ((int64_t)p * a.cap + a.lo + s0) * W);
+    const uintptr_t beg = reinterpret_cast<uintptr_t>(a.next_codes + (kvc + a.lo + s0) * W);
     const uintptr_t end = (beg + (uintptr_t)len * W * 4) & ~(uintptr_t)15;
     constexpr uintptr_t kPiece = 16384;
     for (uintptr_t o = ((beg + 15) & ~(uintptr_t)15) + (uintptr_t)tid * kPiece; o < end; o += 32 * kPiece) {
@@ -1126,7 +1135,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
               if (dist_out) dist_out[pos] = Dv;
               if constexpr (ATTEND) {
                 if (pos < (uint32_t)kSelCap) sel_s[pos] = tok;
-                prefetch_row_l2<T>(a.K, a.V, (int64_t)p * a.cap + tok);
+                prefetch_row_l2<T>(a.K, a.V, kvc + tok);
               }
             } else {
               report(a.status, HKV_ERR_DEVICE_RANGE);  // unreachable when the counts agree
@@ -1153,13 +1162,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     };
     float* dst = a.part + ((int64_t)p * nseg + seg) * a.g * kPart;
     if constexpr (sizeof(T) == 2) {
-      attn_mma(a, p, aq_s, ns + n_res, row_at, smem, tok_s, m_s, l_s, alpha_s, dst);
+      attn_mma(a, kvc, aq_s, ns + n_res, row_at, smem, tok_s, m_s, l_s, alpha_s, dst);
     } else {
       float* attn = reinterpret_cast<float*>(smem);
       const AttnSmem sm{aq_s, attn, attn + kRows * kKP, attn + kRows * kKP + kRows * kHeadDim, tok_s, m_s, l_s, alpha_s};
       float acc[kOut];
       attn_begin(a.g, sm, acc);
-      attn_rows<T>(a, p, ns + n_res, row_at, sm, acc);
+      attn_rows<T>(a, kvc, ns + n_res, row_at, sm, acc);
       attn_end(a.g, sm, acc, dst);
     }
     __syncthreads();
@@ -1395,6 +1404,8 @@ int launch_fused(const RetrieveShape& s, bool attend, int dtype, int qenc, const
   a.qenc = qenc;
   a.k_codes = k_codes;
   a.next_codes = next_codes;
+  a.Hkv_real = s.kv_heads > 0 ? s.kv_heads : s.Hkv;
+  a.unit_div = s.Hkv / a.Hkv_real;
   a.idx = idx;
   a.dist = dist;
   a.q = q;

@@ -212,6 +212,28 @@ int hkv_retrieve_topk_static(int B, int Hq, int Hkv, int code_bits, const uint32
                              int n_local, int top_k, int32_t* idx, int32_t* dist, int32_t* status,
                              void* stream);
 
+/* One index set per query head (RetrievalAttention "Key points": each query
+ * head retrieves its own keys).  As hkv_retrieve_topk, but query head h of
+ * batch b scores the keys of its KV head j = h / g by its own distance
+ *   D_h(t) = popcount(q_code[b, h] XOR k_code[b, j, t])
+ * and keeps its own k_eff smallest (ties to the lowest t).
+ *   idx, dist  [B, Hq, top_k] (dist nullable)
+ * Workspace: hkv_workspace_bytes(B, Hq, Hq, ...) (query heads as the third
+ * argument). */
+int hkv_retrieve_topk_heads(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                            const uint32_t* k_codes, int64_t cap, int64_t n_tokens, int n_sink,
+                            int n_local, int top_k, int32_t* idx, int32_t* dist, void* ws,
+                            size_t ws_bytes, int32_t* status, void* stream);
+
+/* hkv_decode_step with one index set per query head: head h attends over
+ * sink + its own selected rows + local rows of KV head h / g.  idx is
+ * [B, Hq, top_k]; the workspace as for hkv_retrieve_topk_heads. */
+int hkv_decode_step_heads(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
+                          const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
+                          int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
+                          uint32_t* q_codes, int32_t* idx, float* out, float* lse, void* ws,
+                          size_t ws_bytes, int32_t* status, void* stream);
+
 /* HashEvict eviction (HashEvict "Abstract": at every decoding step the new
  * token's key and value replace the cached token expected to receive the
  * lowest attention, found as the key whose binarized projection is farthest
