@@ -330,3 +330,13 @@ def decode_step_heads(q, K, V, k_codes, N: int, n_sink: int, n_local: int, top_k
             o, l = attend(qa[b, h:h + 1], K[b, h // g], V[b, h // g], rows, scale)
             out[b, h], lse[b, h] = o[0], l[0]
     return {"q_codes": qc, "idx": idx, "dist": dist, "out": out, "lse": lse}
+
+
+def decode_step_ragged(q, K, V, k_codes, n_tokens_b, n_sink: int, n_local: int, top_k: int,
+                       kind: str, q_params=None, scale: float | None = None):
+    """decode_step for a batch whose sequence b holds n_tokens_b[b] tokens:
+    each sequence has its own sink, local window and candidates.  Returns the
+    per-sequence results stacked along the batch."""
+    parts = [decode_step(q[b:b + 1], K[b:b + 1], V[b:b + 1], k_codes[b:b + 1], int(n_tokens_b[b]), n_sink,
+                         n_local, top_k, kind, q_params, scale) for b in range(len(n_tokens_b))]
+    return {key: np.concatenate([r[key] for r in parts], axis=0) for key in ("q_codes", "idx", "dist", "out", "lse")}

@@ -435,3 +435,38 @@ def test_decode_step_heads_single_head_groups_equal_decode_step():
     b = oracle.decode_step(q, K, V, kc, N, 2, 3, 6, "sign")
     np.testing.assert_array_equal(a["idx"], b["idx"])
     np.testing.assert_allclose(a["out"], b["out"], rtol=0, atol=1e-14)
+
+
+# ------------------------------------------------------- ragged batches
+
+def test_ragged_with_equal_lengths_is_the_uniform_step():
+    rng = np.random.default_rng(12)
+    B, H, N, d = 3, 2, 60, 128
+    q = rng.normal(size=(B, H, d))
+    K = rng.normal(size=(B, H, N, d))
+    V = rng.normal(size=(B, H, N, d))
+    kc = oracle.encode("sign", K)[0]
+    a = oracle.decode_step_ragged(q, K, V, kc, [N] * B, 2, 5, 7, "sign")
+    b = oracle.decode_step(q, K, V, kc, N, 2, 5, 7, "sign")
+    for key in ("q_codes", "idx", "dist"):
+        np.testing.assert_array_equal(a[key], b[key])
+    np.testing.assert_allclose(a["out"], b["out"], rtol=0, atol=1e-14)
+
+
+def test_ragged_ignores_tokens_past_each_length():
+    """Garbage beyond a sequence's length changes nothing for that sequence."""
+    rng = np.random.default_rng(13)
+    B, H, N, d = 2, 1, 50, 128
+    q = rng.normal(size=(B, H, d))
+    K = rng.normal(size=(B, H, N, d))
+    V = rng.normal(size=(B, H, N, d))
+    kc = oracle.encode("sign", K)[0]
+    lens = [50, 31]
+    a = oracle.decode_step_ragged(q, K, V, kc, lens, 2, 4, 6, "sign")
+    K2, V2, kc2 = K.copy(), V.copy(), kc.copy()
+    K2[1, :, 31:] = 1e6
+    V2[1, :, 31:] = -1e6
+    kc2[1, :, 31:] = 0
+    b = oracle.decode_step_ragged(q, K2, V2, kc2, lens, 2, 4, 6, "sign")
+    np.testing.assert_array_equal(a["idx"], b["idx"])
+    np.testing.assert_allclose(a["out"], b["out"], rtol=0, atol=1e-12)
