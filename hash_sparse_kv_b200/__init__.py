@@ -29,7 +29,8 @@ __all__ = [
     "hkv_version", "hkv_last_error", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
     "hkv_encode_keys", "hkv_mlp_pack_bytes", "hkv_mlp_pack", "hkv_append", "hkv_retrieve_topk",
     "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_sparse_attend", "hkv_evict_select",
-    "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads", "hkv_debug_set", "EXPORTS",
+    "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads", "hkv_decode_step_ragged", "hkv_debug_set",
+    "EXPORTS",
 ]
 
 HKV_OK, HKV_ERR_INVALID_ARG, HKV_ERR_UNSUPPORTED, HKV_ERR_CAPACITY = 0, -1, -2, -3
@@ -42,7 +43,7 @@ EXPORTS = (
     "hkv_last_error", "hkv_version", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
     "hkv_encode_keys", "hkv_mlp_pack_bytes", "hkv_mlp_pack", "hkv_append", "hkv_retrieve_topk",
     "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_sparse_attend", "hkv_evict_select",
-    "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads", "hkv_debug_set",
+    "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads", "hkv_decode_step_ragged", "hkv_debug_set",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -85,6 +86,8 @@ _SIGS = {
     "hkv_retrieve_topk_heads": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _SZ, _P, _P]),
     "hkv_decode_step_heads": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _F,
                                    _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "hkv_decode_step_ragged": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _I64, _P, _I64, _I, _I, _I,
+                                    _F, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "hkv_evict_select": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _P, _P, _P, _SZ, _P]),
     "hkv_write_slots": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P]),
 }
@@ -376,6 +379,32 @@ def hkv_decode_step_heads(h: HashParams, q, k_codes, K, V, n_tokens: int, n_sink
     _ok(lib().hkv_decode_step_heads(ctypes.byref(h.c), B, Hq, Hkv, _ptr(q), _ptr(k_codes), _ptr(K), _ptr(V), cap,
                                     n_tokens, n_sink, n_local, top_k, scale, _ptr(q_codes), _ptr(idx), _ptr(out),
                                     _ptr(lse), _ptr(ws), nbytes, _ptr(status), _stream(stream)))
+
+
+def hkv_decode_step_ragged(h: HashParams, q, k_codes, K, V, n_tokens_b, n_tokens_max: int, n_sink: int,
+                           n_local: int, top_k: int, out, lse=None, q_codes=None, idx=None,
+                           scale: Optional[float] = None, ws=None, status=None, stream=None) -> None:
+    """hkv_decode_step with per-sequence lengths n_tokens_b (int32 [B], on the device)."""
+    B, Hq, d = q.shape
+    _, Hkv, cap, W = k_codes.shape
+    _need(q, "q", (torch.bfloat16, torch.float32))
+    _need(k_codes, "k_codes", _U32)
+    _need(K, "K", q.dtype, shape=(B, Hkv, cap, d))
+    _need(V, "V", q.dtype, shape=(B, Hkv, cap, d))
+    _need(out, "out", torch.float32, shape=(B, Hq, d))
+    _need(n_tokens_b, "n_tokens_b", torch.int32, shape=(B,))
+    if q_codes is not None:
+        _need(q_codes, "q_codes", _U32, shape=(B, Hq, W))
+    if idx is not None:
+        _need(idx, "idx", torch.int32, shape=(B, Hkv, top_k))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, shape=(B, Hq))
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _ok(lib().hkv_decode_step_ragged(ctypes.byref(h.c), B, Hq, Hkv, _ptr(q), _ptr(k_codes), _ptr(K), _ptr(V), cap,
+                                     _ptr(n_tokens_b), n_tokens_max, n_sink, n_local, top_k, scale, _ptr(q_codes),
+                                     _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws), nbytes, _ptr(status),
+                                     _stream(stream)))
 
 
 def hkv_evict_select(q_codes, k_codes, n_tokens: int, n_sink: int, n_local: int, victim, vdist=None, ws=None,

@@ -305,7 +305,8 @@ int hkv_lse_merge(int rows, int d, const float* o1, const float* lse1, const flo
   return launch_lse_merge(rows, d, o1, lse1, o2, lse2, out, lse_out, static_cast<cudaStream_t>(stream));
 }
 
-static int decode_impl(bool per_head, const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
+static int decode_impl(bool per_head, const int32_t* n_tok_b, const hkv_hash* q_hash, int B, int Hq, int Hkv,
+                       const void* q,
                     const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
                     int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
                     uint32_t* q_codes, int32_t* idx, float* out, float* lse,
@@ -337,7 +338,7 @@ static int decode_impl(bool per_head, const hkv_hash* q_hash, int B, int Hq, int
   int32_t* ix = idx ? idx : reinterpret_cast<int32_t*>(base + L.fused + L.attend + L.qcodes);
   const int W = q_hash->code_bits / 32;
   const Window w = window(n_tokens, n_sink, n_local);
-  RetrieveShape rs{B, Hq, units, W, cap, n_tokens, n_sink, n_local, top_k, per_head ? Hkv : 0};
+  RetrieveShape rs{B, Hq, units, W, cap, n_tokens, n_sink, n_local, top_k, per_head ? Hkv : 0, n_tok_b};
   const bool fused_encode = !given_codes && w.C > 0 && top_k > 0 &&
                             decode_encodes_queries(rs, q_hash->kind, q_hash->dtype);
   if (!given_codes && !fused_encode) {
@@ -345,6 +346,8 @@ static int decode_impl(bool per_head, const hkv_hash* q_hash, int B, int Hq, int
     rc = launch_encode(*q_hash, q, m, qc, nullptr, st, status);
     if (rc != HKV_OK) return rc;
   }
+  if (n_tok_b != nullptr && (w.C == 0 || top_k == 0))
+    return fail(HKV_ERR_UNSUPPORTED, "ragged decode needs top_k > 0 and n_tokens_max above n_sink + n_local");
   if (w.C == 0 || top_k == 0) {
     // nothing to retrieve: attend the resident rows only
     if (top_k > 0) {
@@ -367,8 +370,8 @@ int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* 
                     uint32_t* q_codes, int32_t* idx, float* out, float* lse,
                     const uint32_t* next_k_codes, void* ws, size_t ws_bytes, int32_t* status,
                     void* stream) {
-  return decode_impl(false, q_hash, B, Hq, Hkv, q, k_codes, K, V, cap, n_tokens, n_sink, n_local, top_k, scale,
-                     q_codes, idx, out, lse, next_k_codes, ws, ws_bytes, status, stream);
+  return decode_impl(false, nullptr, q_hash, B, Hq, Hkv, q, k_codes, K, V, cap, n_tokens, n_sink, n_local, top_k,
+                     scale, q_codes, idx, out, lse, next_k_codes, ws, ws_bytes, status, stream);
 }
 
 int hkv_decode_step_heads(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
@@ -376,8 +379,18 @@ int hkv_decode_step_heads(const hkv_hash* q_hash, int B, int Hq, int Hkv, const 
                           int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
                           uint32_t* q_codes, int32_t* idx, float* out, float* lse, void* ws,
                           size_t ws_bytes, int32_t* status, void* stream) {
-  return decode_impl(true, q_hash, B, Hq, Hkv, q, k_codes, K, V, cap, n_tokens, n_sink, n_local, top_k, scale,
-                     q_codes, idx, out, lse, nullptr, ws, ws_bytes, status, stream);
+  return decode_impl(true, nullptr, q_hash, B, Hq, Hkv, q, k_codes, K, V, cap, n_tokens, n_sink, n_local, top_k,
+                     scale, q_codes, idx, out, lse, nullptr, ws, ws_bytes, status, stream);
+}
+
+int hkv_decode_step_ragged(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
+                           const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
+                           const int32_t* n_tokens_b, int64_t n_tokens_max, int n_sink, int n_local,
+                           int top_k, float scale, uint32_t* q_codes, int32_t* idx, float* out, float* lse,
+                           void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  if (n_tokens_b == nullptr) return fail(HKV_ERR_INVALID_ARG, "n_tokens_b is NULL");
+  return decode_impl(false, n_tokens_b, q_hash, B, Hq, Hkv, q, k_codes, K, V, cap, n_tokens_max, n_sink, n_local,
+                     top_k, scale, q_codes, idx, out, lse, nullptr, ws, ws_bytes, status, stream);
 }
 
 int hkv_retrieve_topk_heads(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,

@@ -47,6 +47,7 @@ struct RetrieveShape {
   int64_t cap, N;
   int n_sink, n_local, top_k;
   int kv_heads = 0;  // KV heads of the cache when they differ from Hkv
+  const int32_t* n_tok_b = nullptr;  // device [B]: ragged lengths, each <= N (N plans the launch)
 };
 size_t retrieve_ws_bytes(const RetrieveShape& s);
 int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,

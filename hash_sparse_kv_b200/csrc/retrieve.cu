@@ -101,6 +101,8 @@ struct FusedArgs {
   uint32_t* gh;    // [pairs][nbins]: histogram of the pair (returns to zero)
   const uint32_t* next_codes;  // nullable: codes of the next call, prefetched to L2 after the scan
   int Hkv_real, unit_div;      // KV heads of the cache; selection units per KV head
+  const int32_t* n_tok_b;      // nullable [B]: tokens of each sequence (ragged batch)
+  int n_sink_cfg, n_local_cfg, n_max;
   uint32_t* cum;   // [pairs][nseg][nbins]: cumulative counts, window only
   float* part;     // [pairs][nseg][g][kPart]
   int32_t* status;
@@ -911,11 +913,27 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   __shared__ int tok_s[2 * kRows];
 
   const int tid = threadIdx.x;
-  const int C = a.C, nseg = a.nseg;
+  const int nseg = a.nseg;
   const int p = a.p0 + (int)blockIdx.x / nseg, seg = (int)blockIdx.x % nseg;
   const int64_t kvc = kv_row(a, p) * a.cap;  // first cache row of this unit's (batch, KV head)
+  // this pair's window: uniform, or from its sequence's own length
+  int lo = a.lo, C = a.C, k_eff_p = a.k_eff, sink_n = a.sink_n, local_start = a.local_start,
+      local_n = a.local_n;
+  if (a.n_tok_b != nullptr) {
+    int nb = a.n_tok_b[p / a.Hkv];
+    if (nb < 0 || nb > a.n_max) {
+      if (tid == 0 && seg == 0) report(a.status, HKV_ERR_DEVICE_RANGE);
+      nb = nb < 0 ? 0 : a.n_max;
+    }
+    sink_n = min(a.n_sink_cfg, nb);
+    local_start = max(sink_n, nb - a.n_local_cfg);
+    local_n = nb - local_start;
+    lo = sink_n;
+    C = local_start - sink_n;
+    k_eff_p = min(a.top_k, C);
+  }
   const int s0 = seg * a.per_block, s1 = min(s0 + a.per_block, C);
-  const int len = s1 - s0;
+  const int len = max(s1 - s0, 0);
   const int nt = tid < len ? (len - tid + kThreads - 1) / kThreads : 0;
   uint32_t* sync = a.sync + kSync * p;
   (void)aq_s;
@@ -936,7 +954,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   float4 aq = make_float4(0.f, 0.f, 0.f, 0.f);
   if (ATTEND && tid < a.g * (kHeadDim / 4))
     aq = load4_f32(tptr<T>(a.q) + qrow0 * kHeadDim + (tid / (kHeadDim / 4)) * kHeadDim + (tid % (kHeadDim / 4)) * 4);
-  const uint32_t* pf_ptr = a.k_codes + (kvc + a.lo + s0 + tid) * W;
+  const uint32_t* pf_ptr = a.k_codes + (kvc + lo + s0 + tid) * W;
   constexpr int64_t kStep = (int64_t)kThreads * W;
   auto slot = [&](int k) { return ring + ((size_t)(k % kSlots) * kThreads + tid) * 4; };
 #pragma unroll
@@ -944,12 +962,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     if (k < nt) cp_async_code<W>(slot(k), pf_ptr + k * kStep);
     if (k & 1) cp_async_commit();
   }
-  const int R_res = a.sink_n + a.local_n;
+  const int R_res = sink_n + local_n;
   const int n_res = seg < R_res ? (R_res - seg + nseg - 1) / nseg : 0;
   if (ATTEND && tid < n_res) {
     // the block's resident rows go to L2 now; they are attended after the scan
     const int v = seg + tid * nseg;
-    const int t = v < a.sink_n ? v : a.local_start + (v - a.sink_n);
+    const int t = v < sink_n ? v : local_start + (v - sink_n);
     prefetch_row_l2<T>(a.K, a.V, kvc + t);
   }
   // ---------------- phase A: query codes, histogram reset -------------------
@@ -1004,7 +1022,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   if (a.next_codes != nullptr && tid < 32) {
     // the next call's codes for this block's range go to L2 while this call
     // selects and attends (16-byte aligned pieces; the hint skips ragged ends)
-    const uintptr_t beg = reinterpret_cast<uintptr_t>(a.next_codes + (kvc + a.lo + s0) * W);
+    const uintptr_t beg = reinterpret_cast<uintptr_t>(a.next_codes + (kvc + lo + s0) * W);
     const uintptr_t end = (beg + (uintptr_t)len * W * 4) & ~(uintptr_t)15;
     constexpr uintptr_t kPiece = 16384;
     for (uintptr_t o = ((beg + 15) & ~(uintptr_t)15) + (uintptr_t)tid * kPiece; o < end; o += 32 * kPiece) {
@@ -1022,7 +1040,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   // threshold T is at most min over segments of hi (that segment alone has
   // k_eff tokens at or below its hi), so the global histogram is complete on
   // [0, T] and every segment's cumulative counts are known at T - 1 and T.
-  const uint32_t k_eff = (uint32_t)a.k_eff;
+  const uint32_t k_eff = (uint32_t)k_eff_p;
   {
     block_inclusive_scan(hist_s, a.nbins, warp_tmp);
     const bool enough = hist_s[a.nbins - 1] >= k_eff;
@@ -1031,7 +1049,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       if (enough && hist_s[v] >= k_eff && prev < k_eff) sh[1] = v;
     }
     __syncthreads();
-    const int hi = enough ? sh[1] : a.nbins - 1;
+    // k_eff == 0 (a ragged sequence without candidates): nothing to publish
+    const int hi = k_eff == 0 ? -1 : enough ? sh[1] : a.nbins - 1;
     uint32_t* cum_out = a.cum + ((int64_t)p * nseg + seg) * a.nbins;
     uint32_t* gh = a.gh + (int64_t)p * a.nbins;
     for (int v = tid; v <= hi; v += kThreads) {
@@ -1129,7 +1148,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
           bool take = Dv < thr;
           if (Dv == thr) take = run_eq++ < quota;
           if (take) {
-            const int tok = (int)a.lo + s0 + i;
+            const int tok = lo + s0 + i;
             if (sel_base + pos < k_eff) {
               idx_out[pos] = tok;
               if (dist_out) dist_out[pos] = Dv;
@@ -1158,7 +1177,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     auto row_at = [&](int i) -> int {
       if (i < ns) return i < kSelCap ? sel_s[i] : sel_g[i];
       const int v = seg + (i - ns) * nseg;
-      return v < a.sink_n ? v : a.local_start + (v - a.sink_n);
+      return v < sink_n ? v : local_start + (v - sink_n);
     };
     float* dst = a.part + ((int64_t)p * nseg + seg) * a.g * kPart;
     if constexpr (sizeof(T) == 2) {
@@ -1198,7 +1217,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   if (tid == 0) sh[2] = atom_acq_rel_add(&sync[1], 1u) == (uint32_t)(nseg - 1);
   __syncthreads();
   if (sh[2]) {
-    for (int i = a.k_eff + tid; i < a.top_k; i += kThreads) {
+    for (int i = k_eff_p + tid; i < a.top_k; i += kThreads) {
       a.idx[(int64_t)p * a.top_k + i] = -1;
       if (a.dist) a.dist[(int64_t)p * a.top_k + i] = -1;
     }
@@ -1406,6 +1425,10 @@ int launch_fused(const RetrieveShape& s, bool attend, int dtype, int qenc, const
   a.next_codes = next_codes;
   a.Hkv_real = s.kv_heads > 0 ? s.kv_heads : s.Hkv;
   a.unit_div = s.Hkv / a.Hkv_real;
+  a.n_tok_b = s.n_tok_b;
+  a.n_sink_cfg = s.n_sink;
+  a.n_local_cfg = s.n_local;
+  a.n_max = (int)s.N;
   a.idx = idx;
   a.dist = dist;
   a.q = q;

@@ -212,6 +212,20 @@ int hkv_retrieve_topk_static(int B, int Hq, int Hkv, int code_bits, const uint32
                              int n_local, int top_k, int32_t* idx, int32_t* dist, int32_t* status,
                              void* stream);
 
+/* hkv_decode_step for a batch of sequences of different lengths: sequence b
+ * holds n_tokens_b[b] tokens (device int32 [B], each in [0, n_tokens_max]);
+ * its sink, local window and candidates follow from its own length, as for a
+ * call with n_tokens = n_tokens_b[b].  n_tokens_max (<= cap) plans the launch
+ * and sizes the workspace (hkv_workspace_bytes with n_tokens_max).  A length
+ * outside [0, n_tokens_max] is clamped and reported as HKV_ERR_DEVICE_RANGE.
+ * top_k must be positive and n_tokens_max > n_sink + n_local (at least one
+ * sequence with candidates); HKV_ERR_UNSUPPORTED otherwise. */
+int hkv_decode_step_ragged(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
+                           const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
+                           const int32_t* n_tokens_b, int64_t n_tokens_max, int n_sink, int n_local,
+                           int top_k, float scale, uint32_t* q_codes, int32_t* idx, float* out, float* lse,
+                           void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
 /* One index set per query head (RetrievalAttention "Key points": each query
  * head retrieves its own keys).  As hkv_retrieve_topk, but query head h of
  * batch b scores the keys of its KV head j = h / g by its own distance
