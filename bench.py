@@ -438,7 +438,8 @@ def run_gpu(args, rank, world, local):
                                   "evict_select": ev_ms * 1e3 / len(layers)},
         "evict": {"bound": "hbm", "achieved": code_bytes / (ev_ms * 1e-3 / len(layers)) / 1e9, "peak": peak,
                   "unit": "GB/s", "frac": code_bytes / (ev_ms * 1e-3 / len(layers)) / 1e9 / peak,
-                  "bytes_per_launch": code_bytes, "launches_per_layer": 2},
+                  "bytes_per_launch": code_bytes, "launches_per_layer": 2,
+                  "traffic": traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "evict.cu"), w.name)},
         # decode with an LSH or sign query hash (query heads per KV head <= 32) is one
         # fused launch a layer; an MLP query hash adds the separate query encode launch
         "gpu_launches": (1 if w.hash in ("lsh", "sign") and w.g <= 32 else 2) * len(layers) * args.steps,

@@ -51,6 +51,7 @@
 #include <algorithm>
 #include <mutex>
 
+#include "hamming.cuh"
 #include "internal.h"
 
 namespace hkv {
@@ -116,83 +117,6 @@ __device__ __forceinline__ int64_t kv_row(const FusedArgs& a, int p) {
   return (int64_t)(p / a.Hkv) * a.Hkv_real + (p % a.Hkv) / a.unit_div;
 }
 
-
-template <int W, int NP>
-struct Planes {
-  uint32_t C[NP][W];
-  uint32_t U[NP][W];
-};
-
-// Bit-sliced counters: C planes count the query codes' ones, U planes their zeros.
-template <int W, int NP>
-__device__ __forceinline__ void build_planes(const uint32_t* qc, int g, Planes<W, NP>& p) {
-#pragma unroll
-  for (int b = 0; b < NP; ++b)
-#pragma unroll
-    for (int w = 0; w < W; ++w) p.C[b][w] = p.U[b][w] = 0u;
-  for (int h = 0; h < g; ++h) {
-#pragma unroll
-    for (int w = 0; w < W; ++w) {
-      const uint32_t q = qc[h * W + w];
-      uint32_t carry = q;
-#pragma unroll
-      for (int b = 0; b < NP; ++b) {
-        const uint32_t t = p.C[b][w] & carry;
-        p.C[b][w] ^= carry;
-        carry = t;
-      }
-      carry = ~q;
-#pragma unroll
-      for (int b = 0; b < NP; ++b) {
-        const uint32_t t = p.U[b][w] & carry;
-        p.U[b][w] ^= carry;
-        carry = t;
-      }
-    }
-  }
-}
-
-// s = a + b on bit-sliced numbers of NB planes (ripple of full adders).
-template <int NB>
-__device__ __forceinline__ void add_planes(const uint32_t (&a)[NB], const uint32_t (&b)[NB], uint32_t (&s)[NB + 1]) {
-  uint32_t c = 0u;
-#pragma unroll
-  for (int i = 0; i < NB; ++i) {
-    const uint32_t x = a[i], y = b[i];
-    s[i] = x ^ y ^ c;
-    c = (x & y) | (c & (x ^ y));
-  }
-  s[NB] = c;
-}
-
-template <int L>
-__device__ __forceinline__ int weighted_popc(const uint32_t (&s)[L]) {
-  int r = 0;
-#pragma unroll
-  for (int b = 0; b < L; ++b) r += __popc(s[b]) << b;
-  return r;
-}
-
-template <int W, int NP>
-__device__ __forceinline__ int token_distance(const uint32_t (&ck)[W], const Planes<W, NP>& p) {
-  uint32_t v[W][NP];
-#pragma unroll
-  for (int w = 0; w < W; ++w)
-#pragma unroll
-    for (int b = 0; b < NP; ++b) v[w][b] = (ck[w] & p.U[b][w]) | (~ck[w] & p.C[b][w]);
-  if constexpr (W == 2) {
-    uint32_t s[NP + 1];
-    add_planes<NP>(v[0], v[1], s);
-    return weighted_popc<NP + 1>(s);
-  } else {
-    static_assert(W == 4, "codes of 64 or 128 bits");
-    uint32_t s01[NP + 1], s23[NP + 1], s[NP + 2];
-    add_planes<NP>(v[0], v[1], s01);
-    add_planes<NP>(v[2], v[3], s23);
-    add_planes<NP + 1>(s01, s23, s);
-    return weighted_popc<NP + 2>(s);
-  }
-}
 
 // ---- cp.async helpers (per-thread ring; each thread reads only its own slots)
 template <int W>
@@ -1229,87 +1153,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   }
 }
 
-// ---------------------------------------------------------------- eviction
-// HashEvict ("Abstract"): the cached token least similar to the current
-// query -- the largest group distance D(t) -- is the one the new token
-// replaces.  Candidates [sink_end, local_start); ties to the lowest t.  Each
-// block reduces its range to one 64-bit key (D << 32 | ~t) and folds it into
-// the pair's slot with atomicMax; the largest key is the largest D with the
-// smallest t.  A second launch turns the keys into indices and clears them.
-template <int W, int NP>
-__global__ void __launch_bounds__(kThreads)
-evict_scan_kernel(const uint32_t* __restrict__ q_codes, const uint32_t* __restrict__ k_codes, int Hq, int Hkv, int g,
-                  int64_t cap, int lo, int C, int per_block, int nseg, unsigned long long* best) {
-  __shared__ uint32_t qc_s[kMaxGroup * W];
-  __shared__ unsigned long long warp_best[kWarps];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int p = blockIdx.x / nseg, seg = blockIdx.x % nseg;
-  const int64_t qrow0 = (int64_t)(p / Hkv) * Hq + (int64_t)(p % Hkv) * g;
-  for (int i = tid; i < g * W; i += kThreads) qc_s[i] = q_codes[qrow0 * W + i];
-  __syncthreads();
-  Planes<W, NP> planes;
-  build_planes<W, NP>(qc_s, g, planes);
-  const int s0 = seg * per_block, s1 = min(s0 + per_block, C);
-  unsigned long long mx = 0ull;
-  const uint32_t* base = k_codes + ((int64_t)p * cap + lo) * W;
-  for (int t = s0 + tid; t < s1; t += kThreads) {
-    uint32_t ck[W];
-    ld_stream(base + (int64_t)t * W, ck);
-    const unsigned long long key =
-        ((unsigned long long)token_distance<W, NP>(ck, planes) << 32) | (0xFFFFFFFFu - (uint32_t)(lo + t));
-    mx = key > mx ? key : mx;
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const unsigned long long o = __shfl_xor_sync(0xffffffffu, mx, off);
-    mx = o > mx ? o : mx;
-  }
-  if (lane == 0) warp_best[warp] = mx;
-  __syncthreads();
-  if (tid == 0) {
-    unsigned long long bm = 0ull;
-    for (int w = 0; w < kWarps; ++w) bm = warp_best[w] > bm ? warp_best[w] : bm;
-    if (bm != 0ull) atomicMax(best + p, bm);
-  }
-}
-
-__global__ void evict_finish_kernel(unsigned long long* best, int P, int32_t* victim, int32_t* vdist) {
-  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < P; p += gridDim.x * blockDim.x) {
-    const unsigned long long v = best[p];
-    victim[p] = v ? (int32_t)(0xFFFFFFFFu - (uint32_t)v) : -1;
-    if (vdist != nullptr) vdist[p] = v ? (int32_t)(v >> 32) : -1;
-    best[p] = 0ull;
-  }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kThreads)
-write_slots_kernel(int P, int W, const T* __restrict__ k_new, const T* __restrict__ v_new,
-                   const uint32_t* __restrict__ codes_new, const uint16_t* __restrict__ norms_new, T* K, T* V,
-                   uint32_t* codes, uint16_t* norms, int64_t cap, const int32_t* __restrict__ slot, int32_t* status) {
-  constexpr int EPC = 16 / sizeof(T), CPR = kHeadDim / EPC;  // 16-byte chunks per row
-  const int per_pair = 2 * CPR + 1;                          // K chunks, V chunks, code + norm
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < P * per_pair; i += gridDim.x * blockDim.x) {
-    const int p = i / per_pair, j = i % per_pair;
-    const int s = slot[p];
-    if (s < 0) continue;
-    if (s >= cap) {
-      if (j == 0) report(status, HKV_ERR_DEVICE_RANGE);
-      continue;
-    }
-    const int64_t row = (int64_t)p * cap + s;
-    if (j < CPR) {
-      reinterpret_cast<uint4*>(K + row * kHeadDim)[j] = reinterpret_cast<const uint4*>(k_new + (int64_t)p * kHeadDim)[j];
-    } else if (j < 2 * CPR) {
-      reinterpret_cast<uint4*>(V + row * kHeadDim)[j - CPR] =
-          reinterpret_cast<const uint4*>(v_new + (int64_t)p * kHeadDim)[j - CPR];
-    } else {
-      for (int w = 0; w < W; ++w) codes[row * W + w] = codes_new[(int64_t)p * W + w];
-      if (norms != nullptr && norms_new != nullptr) norms[row] = norms_new[p];
-    }
-  }
-}
-
 using KernelFn = void (*)(FusedArgs);
 
 template <bool ATTEND, typename T>
@@ -1589,55 +1432,5 @@ int launch_decode(const RetrieveShape& s, int dtype, int q_kind, const void* R, 
 }
 
 
-int launch_evict(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes, int32_t* victim,
-                 int32_t* vdist, void* ws, size_t ws_bytes, cudaStream_t st) {
-  const int P = s.B * s.Hkv;
-  if (P == 0) return HKV_OK;
-  if (ws == nullptr || ws_bytes < sizeof(unsigned long long) * (size_t)P)
-    return fail(HKV_ERR_CAPACITY, "workspace of %zu bytes, %zu needed", ws_bytes, sizeof(unsigned long long) * (size_t)P);
-  const Window w = window(s.N, s.n_sink, s.n_local);
-  const int g = s.Hq / s.Hkv, np = bit_length(g);
-  auto* best = static_cast<unsigned long long*>(ws);
-  if (w.C > 0) {
-    using EvictFn = void (*)(const uint32_t*, const uint32_t*, int, int, int, int64_t, int, int, int, int,
-                             unsigned long long*);
-    EvictFn fn = nullptr;
-#define HKV_EV(WV, NPV) \
-  if (s.words == WV && np == NPV) fn = evict_scan_kernel<WV, NPV>;
-    HKV_EV(2, 1) HKV_EV(2, 2) HKV_EV(2, 3) HKV_EV(2, 4) HKV_EV(2, 5)
-    HKV_EV(4, 1) HKV_EV(4, 2) HKV_EV(4, 3) HKV_EV(4, 4) HKV_EV(4, 5)
-#undef HKV_EV
-    if (fn == nullptr) return fail(HKV_ERR_UNSUPPORTED, "no eviction kernel for %d-bit codes and group %d", s.words * 32, g);
-    const int64_t target = 4LL * sm_count();
-    int64_t nseg = std::max<int64_t>(1, std::min<int64_t>(ceil_div(w.C, 1024), ceil_div(target, P)));
-    const int per_block = (int)ceil_div(w.C, nseg);
-    nseg = ceil_div(w.C, per_block);
-    fn<<<(unsigned)(P * nseg), kThreads, 0, st>>>(q_codes, k_codes, s.Hq, s.Hkv, g, s.cap, (int)w.sink_end,
-                                                   (int)w.C, per_block, (int)nseg, best);
-    int rc = cuda_check(cudaGetLastError(), "evict scan launch");
-    if (rc != HKV_OK) return rc;
-  }
-  evict_finish_kernel<<<(unsigned)std::min<int64_t>(ceil_div(P, 256), 1024), 256, 0, st>>>(best, P, victim, vdist);
-  return cuda_check(cudaGetLastError(), "evict finish launch");
-}
-
-int launch_write_slots(int dtype, int P, int W, const void* k_new, const void* v_new, const uint32_t* codes_new,
-                       const uint16_t* norms_new, void* K, void* V, uint32_t* codes, uint16_t* norms, int64_t cap,
-                       const int32_t* slot, int32_t* status, cudaStream_t st) {
-  if (P == 0) return HKV_OK;
-  const int per_pair = 2 * (dtype == HKV_BF16 ? 16 : 32) + 1;
-  const int64_t total = (int64_t)P * per_pair;
-  const unsigned grid = (unsigned)std::min<int64_t>(ceil_div(total, kThreads), 4LL * sm_count());
-  if (dtype == HKV_BF16)
-    write_slots_kernel<__nv_bfloat16><<<grid, kThreads, 0, st>>>(
-        P, W, static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), codes_new, norms_new,
-        static_cast<__nv_bfloat16*>(K), static_cast<__nv_bfloat16*>(V), codes, norms, cap, slot, status);
-  else
-    write_slots_kernel<float><<<grid, kThreads, 0, st>>>(P, W, static_cast<const float*>(k_new),
-                                                         static_cast<const float*>(v_new), codes_new, norms_new,
-                                                         static_cast<float*>(K), static_cast<float*>(V), codes, norms,
-                                                         cap, slot, status);
-  return cuda_check(cudaGetLastError(), "write slots launch");
-}
 
 }  // namespace hkv
