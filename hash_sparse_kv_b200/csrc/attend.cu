@@ -91,19 +91,32 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(AttendArgs a) {
     *reinterpret_cast<float4*>(&q_s[h * kHeadDim + c]) = v;
   }
   __syncthreads();
-  for (int i = tid; i < nrows * (kHeadDim / 4); i += kThreads) {
-    const int r = i / (kHeadDim / 4), c = (i % (kHeadDim / 4)) * 4;
-    const int t = tok_s[r];
-    float4 kv = make_float4(0.f, 0.f, 0.f, 0.f), vv = kv;
-    if (t >= 0) {
-      kv = load4_f32(Kp + (int64_t)t * kHeadDim + c);
-      vv = load4_f32(Vp + (int64_t)t * kHeadDim + c);
+  {
+    // every K/V load of this thread is in flight before the first shared store
+    constexpr int EPC = 16 / sizeof(T), CPR = kHeadDim / EPC, kPer = kMaxRows * CPR / kThreads;
+    uint4 kr[kPer], vr[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kThreads, r = i / CPR, c = i % CPR;
+      const int t = r < nrows ? tok_s[r] : -1;
+      kr[u] = vr[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (t >= 0) {
+        kr[u] = __ldg(reinterpret_cast<const uint4*>(Kp + (int64_t)t * kHeadDim) + c);
+        vr[u] = __ldg(reinterpret_cast<const uint4*>(Vp + (int64_t)t * kHeadDim) + c);
+      }
     }
-    K_s[r * kKP + c + 0] = kv.x;
-    K_s[r * kKP + c + 1] = kv.y;
-    K_s[r * kKP + c + 2] = kv.z;
-    K_s[r * kKP + c + 3] = kv.w;
-    *reinterpret_cast<float4*>(&V_s[r * kHeadDim + c]) = vv;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kThreads, r = i / CPR, c = i % CPR;
+      if (r >= nrows) continue;
+      const T* ke = reinterpret_cast<const T*>(&kr[u]);
+      const T* ve = reinterpret_cast<const T*>(&vr[u]);
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) {
+        K_s[r * kKP + c * EPC + e] = to_f32(ke[e]);
+        V_s[r * kHeadDim + c * EPC + e] = to_f32(ve[e]);
+      }
+    }
   }
   __syncthreads();
   // logits z[h][r] = scale * q_h . K_r  (-inf for empty slots)
@@ -113,10 +126,15 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(AttendArgs a) {
     if (tok_s[r] >= 0) {
       const float* qh = q_s + h * kHeadDim;
       const float* kr = K_s + r * kKP;
-      float acc = 0.f;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll 8
-      for (int c = 0; c < kHeadDim; ++c) acc = fmaf(qh[c], kr[c], acc);
-      z = acc * a.scale;
+      for (int c = 0; c < kHeadDim; c += 4) {
+        a0 = fmaf(qh[c], kr[c], a0);
+        a1 = fmaf(qh[c + 1], kr[c + 1], a1);
+        a2 = fmaf(qh[c + 2], kr[c + 2], a2);
+        a3 = fmaf(qh[c + 3], kr[c + 3], a3);
+      }
+      z = ((a0 + a1) + (a2 + a3)) * a.scale;
     }
     z_s[h * kMaxRows + r] = z;
   }
@@ -145,8 +163,17 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(AttendArgs a) {
   float* part = a.part + ((int64_t)p * a.splits + sp) * g * kPartStride;
   for (int o = tid; o < g * kHeadDim; o += kThreads) {
     const int h = o / kHeadDim, c = o % kHeadDim;
-    float acc = 0.f;
-    for (int r = 0; r < nrows; ++r) acc = fmaf(z_s[h * kMaxRows + r], V_s[r * kHeadDim + c], acc);
+    const float* zh = z_s + h * kMaxRows;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int r = 0;
+    for (; r + 4 <= nrows; r += 4) {
+      a0 = fmaf(zh[r], V_s[r * kHeadDim + c], a0);
+      a1 = fmaf(zh[r + 1], V_s[(r + 1) * kHeadDim + c], a1);
+      a2 = fmaf(zh[r + 2], V_s[(r + 2) * kHeadDim + c], a2);
+      a3 = fmaf(zh[r + 3], V_s[(r + 3) * kHeadDim + c], a3);
+    }
+    for (; r < nrows; ++r) a0 = fmaf(zh[r], V_s[r * kHeadDim + c], a0);
+    const float acc = (a0 + a1) + (a2 + a3);
     part[h * kPartStride + 2 + c] = acc;
     if (c == 0) {
       part[h * kPartStride + 0] = m_s[h];

@@ -11,41 +11,38 @@
 // token t is the sum over its g query heads:
 //     D(t) = sum_h popcount(cq_h XOR ck_t)  in [0, g * bits].
 //
-// One cooperative launch, one block of 512 threads per SM:
-//  * The candidate tokens of all (batch, KV head) pairs are laid end to end
-//    and cut into equal contiguous ranges, one per block, so every SM streams
-//    the same number of code bytes.  A block's range covers one or more
-//    "segments" (its part of one pair).
+// One launch, one block of 512 threads per SM (cooperative when a pair spans
+// several blocks):
+//  * The candidates of each selection unit -- a (batch, KV head) pair, or a
+//    (batch, query head) pair for per-head index sets -- are cut into equal
+//    contiguous segments, one per block, so no block straddles two units.
+//    With a ragged batch each unit takes its window from its own length.
 //  * Phase A.  Each thread streams its tokens through a private ring of
-//    cp.async slots (no block-wide synchronisation) while the block encodes
-//    the query heads it needs.  Per token it computes D, keeps it in shared
-//    memory (uint16) and counts it in its segment's histogram.
-//  * Publication.  A segment publishes its cumulative histogram only up to
-//    hi = its own k-th smallest D (all bins if it holds fewer than k_eff
-//    tokens).  The global threshold T (smallest D whose global cumulative
-//    count reaches k_eff) is at most min over segments of hi, because that
-//    segment alone already has k_eff tokens at or below its hi; so the
-//    published windows hold every count needed to find T.
-//  * Phase B, per segment.  Wait (bounded) for all segments of the pair, read
-//    the windows of all segments in one parallel pass, find T and the counts
-//    of the lower segments, then write this segment's selected tokens
-//    straight to their final, ascending positions in idx: tokens with D < T,
-//    and tokens with D == T in ascending order until k_eff is reached.
-//  * Attention.  While waiting, a block attends its share of the pair's
-//    resident sink/local rows; afterwards it adds its own selected rows
-//    (online softmax over tiles of 64 gathered K/V rows, all g query heads at
-//    once) and writes one partial (m, l, acc).  The last g blocks of the pair
-//    to finish merge one head each: M = max m_s, L = sum l_s e^{m_s - M},
+//    cp.async slots while the block encodes the query heads it needs (bf16
+//    LSH on mma.sync, sign by ballots).  Per token it computes D, keeps it in
+//    shared memory (uint16) and counts it in the block's histogram.
+//  * Publication.  A block adds its counts up to hi = its own k-th smallest D
+//    (all bins if it holds fewer than k_eff tokens) into the unit's global
+//    histogram and stores its cumulative counts over [0, hi].  The threshold
+//    T (smallest D whose cumulative count reaches k_eff) is at most min over
+//    blocks of hi, because that block alone already has k_eff tokens at or
+//    below its hi; so the global histogram is complete on [0, T].
+//  * Phase B.  Wait (bounded) for all blocks of the unit, read the global
+//    histogram, find T, read the lower blocks' cumulative counts at T - 1 and
+//    T, then write this block's selected tokens straight to their final,
+//    ascending positions in idx: tokens with D < T, and tokens with D == T in
+//    ascending order until k_eff is reached.
+//  * Attention.  The block attends its selected rows plus its share of the
+//    unit's resident sink/local rows for all of the unit's query heads (bf16:
+//    tensor-core logits and P V over 64-row tiles fetched by cp.async) and
+//    writes one partial (m, l, acc).  The last g blocks of the unit to finish
+//    merge one head each: M = max m_s, L = sum l_s e^{m_s - M},
 //    out = sum acc_s e^{m_s - M} / L, lse = M + log L.
-//  * The last block out of a pair returns the pair's counters to zero, so the
-//    workspace is ready for the next call.
+//  * The last block out of a unit returns its counters and histogram to zero,
+//    so the workspace is ready for the next call.
 //
-// The group-summed distance uses bit-sliced arithmetic instead of g * W
-// popcounts.  For bit position j let c_j = #{h : bit j of cq_h is 1}; the
-// contribution of j is (ck_j ? g - c_j : c_j).  The NP bit planes of c_j (C
-// planes) and of g - c_j (U planes) are built once per segment; per token each
-// word gives NP planes V_b = (ck & U_b) | (~ck & C_b), words are added with
-// carry-save adders, and D = sum_b 2^b popcount(S_b).
+// The group-summed distance is computed by bit-sliced arithmetic
+// (hamming.cuh) instead of g * W popcounts.
 #include <math.h>
 
 #include <algorithm>
