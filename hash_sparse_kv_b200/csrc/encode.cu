@@ -173,6 +173,9 @@ mlp_rows_kernel(const T* __restrict__ x, const float* __restrict__ W1, const flo
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   constexpr int D = kHeadDim, R = kMlpClusterRows, NB = BITS / kMlpCluster, DP = D + 4;
+  // a decode step launched next on the stream may be scheduled onto free SMs
+  // now; it waits for this grid to finish before it reads the codes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int rank = (int)cluster.block_rank(), tid = threadIdx.x;
   const int64_t row0 = (int64_t)(blockIdx.x / kMlpCluster) * R;
   const int hs = mlp_rows_slice(hidden), hid_pad = hs * kMlpCluster, HP = ((hidden + 3) & ~3) + 4;
@@ -515,6 +518,9 @@ mlp_rows_tc_kernel(const __nv_bfloat16* __restrict__ x, const void* __restrict__
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   constexpr int D = kHeadDim, R = kMlpClusterRows, NB = BITS / kMlpCluster, XP = D + 8;
+  // a decode step launched next on the stream may be scheduled onto free SMs
+  // now; it waits for this grid to finish before it reads the codes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int rank = (int)cluster.block_rank(), tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tq = lane & 3;
   const int64_t row0 = (int64_t)(blockIdx.x / kMlpCluster) * R;

@@ -837,6 +837,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   const int nseg = a.nseg;
   const int p = a.p0 + (int)blockIdx.x / nseg, seg = (int)blockIdx.x % nseg;
   const int64_t kvc = kv_row(a, p) * a.cap;  // first cache row of this unit's (batch, KV head)
+  // Programmatic dependent launch.  The next kernel on this stream may be
+  // launched now, so its blocks are ready to take each SM this grid leaves;
+  // they wait below until this grid has finished.  Before this block touches
+  // global memory, the previous kernel on the stream must have finished with
+  // its writes visible (without a programmatic predecessor the wait returns
+  // at once).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // this pair's window: uniform, or from its sequence's own length
   int lo = a.lo, C = a.C, k_eff_p = a.k_eff, sink_n = a.sink_n, local_start = a.local_start,
       local_n = a.local_n;
@@ -1315,11 +1323,18 @@ int launch_fused(const RetrieveShape& s, bool attend, int dtype, int qenc, const
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    cudaLaunchAttribute attr[2];
+    unsigned n_attr = 0;
+    // may start while the previous kernel on the stream drains (the kernel
+    // waits for it before its first global access)
+    attr[n_attr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n_attr++].val.programmaticStreamSerializationAllowed = 1;
+    if (pl.cooperative) {
+      attr[n_attr].id = cudaLaunchAttributeCooperative;
+      attr[n_attr++].val.cooperative = 1;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pl.cooperative ? 1 : 0;
+    cfg.numAttrs = n_attr;
     rc = cuda_check(cudaLaunchKernelEx(&cfg, k, a), "scan/select launch");
     if (rc != HKV_OK) return rc;
   }
