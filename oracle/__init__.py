@@ -35,7 +35,7 @@ import numpy as np
 __all__ = [
     "as_f64", "presign_lsh", "presign_mlp", "presign_sign", "pack_bits", "encode",
     "sign_norms", "hamming", "candidate_range", "select_topk", "attention_rows",
-    "attend", "lse_merge", "retrieve", "decode_step", "ROW_CHUNK",
+    "attend", "lse_merge", "retrieve", "retrieve_normw", "decode_step", "ROW_CHUNK",
 ]
 
 ROW_CHUNK = 1 << 15
@@ -234,6 +234,37 @@ def retrieve(q_codes, k_codes, N: int, n_sink: int, n_local: int, top_k: int):
             idx[b, kh, : sel.size] = sel
             dist[b, kh, : sel.size] = D[sel]
     return idx, dist
+
+
+def retrieve_normw(q_codes, k_codes, norms, N: int, n_sink: int, n_local: int, top_k: int):
+    """[SIK] "Abstract": a key's sign code together with its norm is its 1-bit
+    vector quantisation.  Reading (the page gives no scoring formula): the pair
+    stands for the key |k| sign(k) / sqrt(b), query head h for sign(q_h) / sqrt(b);
+    their inner product is |k| (b - 2 popcount(cq_h XOR ck)) / b.  Summed over
+    the g query heads of a KV head, with the constant 1/b dropped:
+        S(t) = norm_t * (g * b - 2 * D(t)).
+    The top_k candidates with the LARGEST S are kept, ties to the lowest index,
+    in ascending token order.  q_codes [B, Hq, W]; k_codes [B, Hkv, cap, W];
+    norms [B, Hkv, cap] fp16.  Returns idx [B, Hkv, top_k] (-1 past k_eff) and
+    S of the selected tokens (-inf past k_eff)."""
+    q_codes = np.asarray(q_codes, dtype=np.uint32)
+    k_codes = np.asarray(k_codes, dtype=np.uint32)
+    norms = np.asarray(norms, dtype=np.float16)
+    B, Hq, W = q_codes.shape
+    Hkv = k_codes.shape[1]
+    g = Hq // Hkv
+    bits = 32 * W
+    lo, hi = candidate_range(N, n_sink, n_local)
+    idx = np.full((B, Hkv, top_k), -1, dtype=np.int64)
+    score = np.full((B, Hkv, top_k), -np.inf)
+    for b in range(B):
+        for kh in range(Hkv):
+            D = hamming(q_codes[b, kh * g:(kh + 1) * g], k_codes[b, kh, :N])
+            S = as_f64(norms[b, kh, :N]) * (g * bits - 2 * D)
+            sel = select_topk(-S, lo, hi, top_k)
+            idx[b, kh, : sel.size] = sel
+            score[b, kh, : sel.size] = S[sel]
+    return idx, score
 
 
 def evict_victim(q_codes, k_codes, N: int, n_sink: int, n_local: int):

@@ -470,3 +470,103 @@ def test_ragged_ignores_tokens_past_each_length():
     b = oracle.decode_step_ragged(q, K2, V2, kc2, lens, 2, 4, 6, "sign")
     np.testing.assert_array_equal(a["idx"], b["idx"])
     np.testing.assert_allclose(a["out"], b["out"], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------- norm-weighted sign-VQ retrieval
+
+def _normw_golden():
+    gl = golden("normw_worked.txt")
+    q = _hex(gl["q"]).reshape(1, 1, 1)
+    keys = _hex(gl["keys"]).reshape(1, 1, -1, 1)
+    norms = np.array([float(v) for v in gl["norms"]], dtype=np.float16).reshape(1, 1, -1)
+    return gl, q, keys, norms
+
+
+@pytest.mark.parametrize("case", "abcd")
+def test_normw_fixture(case):
+    gl, q, keys, norms = _normw_golden()
+    s, l, k = (int(v) for v in gl[f"case_{case}"])
+    idx, score = oracle.retrieve_normw(q, keys, norms, keys.shape[2], s, l, k)
+    np.testing.assert_array_equal(idx[0, 0], [int(v) for v in gl[f"idx_{case}"]])
+    np.testing.assert_array_equal(score[0, 0], [float(v) for v in gl[f"score_{case}"]])
+
+
+def _pm1_codes(signs):
+    """Codes of +-1 vectors (any leading shape): bit i set where the entry is +1."""
+    signs = np.asarray(signs, dtype=np.float64)
+    return oracle.pack_bits(signs.reshape(-1, signs.shape[-1])).reshape(*signs.shape[:-1], -1)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_normw_score_is_norm_times_sign_inner_product(seed):
+    """S(t) equals norm_t * sum_h sign(q_h) . sign(k_t), the inner product of
+    the +-1 vectors themselves (no popcount), for every candidate."""
+    rng = np.random.default_rng(seed)
+    B, Hq, Hkv, bits, N = 2, 6, 2, 64, 37
+    g = Hq // Hkv
+    qs = rng.choice([-1.0, 1.0], size=(B, Hq, bits))
+    ks = rng.choice([-1.0, 1.0], size=(B, Hkv, N, bits))
+    norms = rng.uniform(0.5, 4.0, size=(B, Hkv, N)).astype(np.float16)
+    idx, score = oracle.retrieve_normw(_pm1_codes(qs), _pm1_codes(ks), norms, N, 0, 0, N)
+    for b in range(B):
+        for j in range(Hkv):
+            np.testing.assert_array_equal(idx[b, j], np.arange(N))
+            dots = (qs[b, j * g:(j + 1) * g] @ ks[b, j].T).sum(axis=0)
+            np.testing.assert_array_equal(score[b, j], norms[b, j].astype(np.float64) * dots)
+
+
+@pytest.mark.parametrize("seed", [3, 4])
+def test_normw_brute_force(seed):
+    """Few distinct codes and norms (many exact ties); the ranking is a plain
+    sort of (-S, t) with S from the +-1 inner products."""
+    rng = np.random.default_rng(seed)
+    B, Hq, Hkv, bits, N, s, l, k = 2, 4, 2, 32, 41, 3, 5, 9
+    g = Hq // Hkv
+    pool = rng.choice([-1.0, 1.0], size=(5, bits))
+    ks = pool[rng.integers(0, 5, size=(B, Hkv, N))]
+    qs = rng.choice([-1.0, 1.0], size=(B, Hq, bits))
+    norms = np.array([0.0, 1.0, 2.5], dtype=np.float16)[rng.integers(0, 3, size=(B, Hkv, N))]
+    idx, _ = oracle.retrieve_normw(_pm1_codes(qs), _pm1_codes(ks), norms, N, s, l, k)
+    for b in range(B):
+        for j in range(Hkv):
+            S = {t: float(norms[b, j, t]) * sum(float(qs[b, j * g + h] @ ks[b, j, t]) for h in range(g))
+                 for t in range(s, N - l)}
+            want = sorted(sorted(S, key=lambda t: (-S[t], t))[:k])
+            np.testing.assert_array_equal(idx[b, j], want)
+
+
+def test_normw_equal_norms_is_hamming_retrieval():
+    """With one norm for every key S decreases with D, so the selection is the
+    pinned smallest-distance retrieval."""
+    rng = np.random.default_rng(6)
+    B, Hq, Hkv, W, N = 2, 8, 2, 4, 500
+    pool = rng.integers(0, 2**32, size=(12, W), dtype=np.uint64).astype(np.uint32)
+    k = pool[rng.integers(0, 12, size=(B, Hkv, N))]
+    q = rng.integers(0, 2**32, size=(B, Hq, W), dtype=np.uint64).astype(np.uint32)
+    norms = np.full((B, Hkv, N), 3.25, dtype=np.float16)
+    for top_k in (1, 17, 300):
+        idx, _ = oracle.retrieve_normw(q, k, norms, N, 4, 16, top_k)
+        want, _ = oracle.retrieve(q, k, N, 4, 16, top_k)
+        np.testing.assert_array_equal(idx, want)
+
+
+def test_normw_norm_scaling_and_zero_norms():
+    """Doubling every norm (exact in fp16) doubles S and keeps the selection;
+    a zero norm scores 0, between every positive and every negative score."""
+    rng = np.random.default_rng(7)
+    B, Hq, Hkv, W, N = 1, 2, 1, 2, 200
+    k = rng.integers(0, 2**32, size=(B, Hkv, N, W), dtype=np.uint64).astype(np.uint32)
+    q = rng.integers(0, 2**32, size=(B, Hq, W), dtype=np.uint64).astype(np.uint32)
+    norms = rng.uniform(0.5, 3.0, size=(B, Hkv, N)).astype(np.float16)
+    i1, s1 = oracle.retrieve_normw(q, k, norms, N, 0, 0, 50)
+    i2, s2 = oracle.retrieve_normw(q, k, (norms * 2).astype(np.float16), N, 0, 0, 50)
+    np.testing.assert_array_equal(i1, i2)
+    np.testing.assert_array_equal(s2, 2 * s1)
+    z = norms.copy()
+    z[0, 0, 10] = 0.0
+    _, S = oracle.retrieve_normw(q, k, z, N, 0, 0, N)
+    D = oracle.hamming(q[0], k[0, 0])
+    m = 2 * 64 - 2 * D
+    assert S[0, 0, 10] == 0.0
+    other = np.arange(N) != 10
+    assert (S[0, 0][(m > 0) & other] > 0).all() and (S[0, 0][(m < 0) & other] < 0).all()
