@@ -227,6 +227,18 @@ class Layer:
                             None if self.norms is None else self.norms.view(-1))
 
 
+def normw_roofline(w: synth.Workload, n_layers: int, ms: float, step_ms: float, peak: float, peak_kind: str) -> dict:
+    """Norm-weighted sign-VQ retrieval: codes and fp16 norms of every candidate
+    are the algorithmic bytes of one launch."""
+    nbytes = w.B * w.Hkv * w.candidates() * (w.bits // 8 + 2)
+    launch_s = ms * 1e-3 / n_layers
+    return {"kernel": "normw_kernel (scan + radix select + ordered compaction)", "bound": "hbm",
+            "achieved": nbytes / launch_s / 1e9, "peak": peak, "unit": "GB/s",
+            "frac": nbytes / launch_s / 1e9 / peak, "bytes_per_launch": nbytes, "launch_us": launch_s * 1e6,
+            "step_us_per_layer": step_ms * 1e3 / n_layers, "launches_per_layer": 3, "peak_kind": peak_kind,
+            "traffic": traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "normw.cu"), w.name)}
+
+
 def graph_of(fn, warm=1):
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -368,6 +380,26 @@ def run_gpu(args, rank, world, local):
     ev_ms = max_over_ranks(time_graph(g_ev, args.steps, args.warmup, world), world, dev)
     del g_ev
     del g_qenc, g_att
+    # sign-VQ only: retrieval by the norm-weighted sign score (its own kernel),
+    # then the standalone sparse attention
+    normw_ms = normw_step_ms = None
+    if w.hash == "sign" and w.candidates() <= 65536:
+        def normw_only():
+            for L in layers:
+                hkv.hkv_retrieve_topk_normw(L.q_codes, L.codes, L.norms, w.N, w.n_sink, w.n_local, w.top_k, L.idx)
+
+        def normw_step():
+            for L in layers:
+                hkv.hkv_encode_keys(L.qh, L.q.view(-1, w.d), L.q_codes.view(-1, w.words))
+                hkv.hkv_retrieve_topk_normw(L.q_codes, L.codes, L.norms, w.N, w.n_sink, w.n_local, w.top_k, L.idx)
+                hkv.hkv_sparse_attend(L.q, L.K, L.V, w.N, L.idx, w.n_sink, w.n_local, L.out, ws=ws_a, status=status)
+
+        g_nw = graph_of(normw_only)
+        normw_ms = max_over_ranks(time_graph(g_nw, args.steps, args.warmup, world), world, dev)
+        del g_nw
+        g_nw = graph_of(normw_step)
+        normw_step_ms = max_over_ranks(time_graph(g_nw, args.steps, args.warmup, world), world, dev)
+        del g_nw
     # end to end: host q in, host out back, every step
     q_host = [torch.empty_like(L.q, device="cpu").pin_memory() for L in layers]
     o_host = [torch.empty_like(L.out, device="cpu").pin_memory() for L in layers]
@@ -440,6 +472,7 @@ def run_gpu(args, rank, world, local):
                   "unit": "GB/s", "frac": code_bytes / (ev_ms * 1e-3 / len(layers)) / 1e9 / peak,
                   "bytes_per_launch": code_bytes, "launches_per_layer": 2,
                   "traffic": traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "evict.cu"), w.name)},
+        "normw": None if normw_ms is None else normw_roofline(w, len(layers), normw_ms, normw_step_ms, peak, peak_kind),
         # decode with an LSH or sign query hash (query heads per KV head <= 32) is one
         # fused launch a layer; an MLP query hash adds the separate query encode launch
         "gpu_launches": (1 if w.hash in ("lsh", "sign") and w.g <= 32 else 2) * len(layers) * args.steps,

@@ -28,9 +28,9 @@ __all__ = [
     "HKV_HASH_SIGN", "HKV_HASH_NONE", "HkvError", "HashParams", "lib", "lib_path", "workspace", "status_word",
     "hkv_version", "hkv_last_error", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
     "hkv_encode_keys", "hkv_mlp_pack_bytes", "hkv_mlp_pack", "hkv_append", "hkv_retrieve_topk",
-    "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_sparse_attend", "hkv_evict_select",
-    "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads", "hkv_decode_step_ragged", "hkv_debug_set",
-    "EXPORTS",
+    "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_retrieve_topk_normw", "hkv_sparse_attend",
+    "hkv_evict_select", "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads",
+    "hkv_decode_step_ragged", "hkv_split_select", "hkv_lse_merge_n", "hkv_debug_set", "EXPORTS",
 ]
 
 HKV_OK, HKV_ERR_INVALID_ARG, HKV_ERR_UNSUPPORTED, HKV_ERR_CAPACITY = 0, -1, -2, -3
@@ -42,8 +42,9 @@ HKV_HASH_LSH, HKV_HASH_MLP, HKV_HASH_SIGN, HKV_HASH_NONE = 0, 1, 2, 3
 EXPORTS = (
     "hkv_last_error", "hkv_version", "hkv_check", "hkv_workspace_bytes", "hkv_workspace_reset",
     "hkv_encode_keys", "hkv_mlp_pack_bytes", "hkv_mlp_pack", "hkv_append", "hkv_retrieve_topk",
-    "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_sparse_attend", "hkv_evict_select",
-    "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads", "hkv_decode_step_ragged", "hkv_debug_set",
+    "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_retrieve_topk_normw", "hkv_sparse_attend",
+    "hkv_evict_select", "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads",
+    "hkv_decode_step_ragged", "hkv_split_select", "hkv_lse_merge_n", "hkv_debug_set",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -88,7 +89,10 @@ _SIGS = {
                                    _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "hkv_decode_step_ragged": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _I64, _P, _I64, _I, _I, _I,
                                     _F, _P, _P, _P, _P, _P, _SZ, _P, _P]),
+    "hkv_retrieve_topk_normw": (_I, [_I, _I, _I, _I, _P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P]),
     "hkv_evict_select": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _P, _P, _P, _SZ, _P]),
+    "hkv_split_select": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "hkv_lse_merge_n": (_I, [_I, _I64, _P, _P, _P, _P, _P]),
     "hkv_write_slots": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P]),
 }
 _lib = None
@@ -405,6 +409,46 @@ def hkv_decode_step_ragged(h: HashParams, q, k_codes, K, V, n_tokens_b, n_tokens
                                      _ptr(n_tokens_b), n_tokens_max, n_sink, n_local, top_k, scale, _ptr(q_codes),
                                      _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws), nbytes, _ptr(status),
                                      _stream(stream)))
+
+
+def hkv_retrieve_topk_normw(q_codes, k_codes, norms, n_tokens: int, n_sink: int, n_local: int, top_k: int, idx,
+                            score=None, stream=None) -> None:
+    """Top-k per KV head by the norm-weighted sign score norm * (g * bits - 2 D).
+    norms [B, Hkv, cap] fp16 (or its int16 bits); idx [B, Hkv, top_k] int32; score nullable fp32."""
+    B, Hq, W = q_codes.shape
+    _, Hkv, cap, W2 = k_codes.shape
+    _need(q_codes, "q_codes", _U32)
+    _need(k_codes, "k_codes", _U32)
+    _need(norms, "norms", (torch.float16, torch.int16), shape=(B, Hkv, cap))
+    _need(idx, "idx", torch.int32, shape=(B, Hkv, top_k))
+    if score is not None:
+        _need(score, "score", torch.float32, shape=(B, Hkv, top_k))
+    if W2 != W:
+        raise ValueError("q_codes and k_codes differ in code width")
+    _ok(lib().hkv_retrieve_topk_normw(B, Hq, Hkv, W * 32, _ptr(q_codes), _ptr(k_codes), _ptr(norms), cap, n_tokens,
+                                      n_sink, n_local, top_k, _ptr(idx), _ptr(score), _stream(stream)))
+
+
+def hkv_split_select(rank: int, Hq: int, code_bits: int, cand_idx, cand_dist, idx, status=None, stream=None) -> None:
+    """cand_idx, cand_dist [G, B, Hkv, top_k] int32 (every rank's own top-k, rank-major);
+    idx [B, Hkv, top_k] int32 out: rank `rank`'s share of the whole sequence's top-k."""
+    G, B, Hkv, k = cand_idx.shape
+    _need(cand_idx, "cand_idx", torch.int32)
+    _need(cand_dist, "cand_dist", torch.int32, shape=(G, B, Hkv, k))
+    _need(idx, "idx", torch.int32, shape=(B, Hkv, k))
+    _ok(lib().hkv_split_select(G, rank, B, Hq, Hkv, code_bits, k, _ptr(cand_idx), _ptr(cand_dist), _ptr(idx),
+                               _ptr(status), _stream(stream)))
+
+
+def hkv_lse_merge_n(o, lse, out, lse_out=None, stream=None) -> None:
+    """o [G, rows, 128], lse [G, rows] fp32 -> out [rows, 128], lse_out [rows]."""
+    G, rows, d = o.shape
+    _need(o, "o", torch.float32)
+    _need(lse, "lse", torch.float32, shape=(G, rows))
+    _need(out, "out", torch.float32, shape=(rows, d))
+    if lse_out is not None:
+        _need(lse_out, "lse_out", torch.float32, shape=(rows,))
+    _ok(lib().hkv_lse_merge_n(G, rows, _ptr(o), _ptr(lse), _ptr(out), _ptr(lse_out), _stream(stream)))
 
 
 def hkv_evict_select(q_codes, k_codes, n_tokens: int, n_sink: int, n_local: int, victim, vdist=None, ws=None,

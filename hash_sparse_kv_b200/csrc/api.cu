@@ -250,6 +250,42 @@ int hkv_retrieve_topk_static(int B, int Hq, int Hkv, int code_bits, const uint32
   return launch_retrieve_static(s, q_codes, k_codes, idx, dist, status, static_cast<cudaStream_t>(stream));
 }
 
+int hkv_retrieve_topk_normw(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                            const uint32_t* k_codes, const uint16_t* norms, int64_t cap, int64_t n_tokens,
+                            int n_sink, int n_local, int top_k, int32_t* idx, float* score, void* stream) {
+  int rc = check_heads(B, Hq, Hkv);
+  if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
+  if (rc != HKV_OK) return rc;
+  if (code_bits != 64 && code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "code_bits %d (64 or 128)", code_bits);
+  if (B == 0 || top_k == 0) return HKV_OK;
+  if (!q_codes || !k_codes || !norms || !idx) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_codes, code_bits / 8)) return fail(HKV_ERR_INVALID_ARG, "k_codes must be %d-byte aligned", code_bits / 8);
+  RetrieveShape s{B, Hq, Hkv, code_bits / 32, cap, n_tokens, n_sink, n_local, top_k};
+  return launch_retrieve_normw(s, q_codes, k_codes, norms, idx, score, static_cast<cudaStream_t>(stream));
+}
+
+int hkv_split_select(int G, int rank, int B, int Hq, int Hkv, int code_bits, int top_k, const int32_t* cand_idx,
+                     const int32_t* cand_dist, int32_t* idx, int32_t* status, void* stream) {
+  int rc = check_heads(B, Hq, Hkv);
+  if (rc != HKV_OK) return rc;
+  if (G < 1 || rank < 0 || rank >= G || top_k < 0) return fail(HKV_ERR_INVALID_ARG, "G %d rank %d top_k %d", G, rank, top_k);
+  if (code_bits != 64 && code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "code_bits %d (64 or 128)", code_bits);
+  if (B == 0 || top_k == 0) return HKV_OK;
+  if (!cand_idx || !cand_dist || !idx) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if ((int64_t)G * top_k > INT32_MAX) return fail(HKV_ERR_UNSUPPORTED, "G * top_k too large");
+  return launch_split_select(G, rank, B * Hkv, top_k, (Hq / Hkv) * code_bits + 1, cand_idx, cand_dist, idx, status,
+                             static_cast<cudaStream_t>(stream));
+}
+
+int hkv_lse_merge_n(int G, int64_t rows, const float* o, const float* lse, float* out, float* lse_out,
+                    void* stream) {
+  if (G < 1 || rows < 0) return fail(HKV_ERR_INVALID_ARG, "G %d rows %lld", G, (long long)rows);
+  if (rows == 0) return HKV_OK;
+  if (!o || !lse || !out) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(o, 16) || !aligned(out, 16)) return fail(HKV_ERR_INVALID_ARG, "o and out must be 16-byte aligned");
+  return launch_lse_merge_n(G, rows, o, lse, out, lse_out, static_cast<cudaStream_t>(stream));
+}
+
 int hkv_evict_select(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
                      const uint32_t* k_codes, int64_t cap, int64_t n_tokens, int n_sink, int n_local,
                      int32_t* victim, int32_t* vdist, void* ws, size_t ws_bytes, void* stream) {

@@ -69,7 +69,7 @@ int launch_decode(const RetrieveShape& s, int dtype, int q_kind, const void* R, 
                   const void* V, float scale, float* out, float* lse, void* ws, size_t ws_bytes,
                   int32_t* status, cudaStream_t st);
 
-// ---- eviction (retrieve.cu) ----
+// ---- eviction (evict.cu) ----
 // victim[p] = the candidate with the largest group distance (lowest t on
 // ties), -1 without candidates; ws: 8 bytes per pair, zero, returned to zero.
 int launch_evict(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes, int32_t* victim,
@@ -77,6 +77,18 @@ int launch_evict(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t
 int launch_write_slots(int dtype, int P, int W, const void* k_new, const void* v_new, const uint32_t* codes_new,
                        const uint16_t* norms_new, void* K, void* V, uint32_t* codes, uint16_t* norms, int64_t cap,
                        const int32_t* slot, int32_t* status, cudaStream_t st);
+
+// ---- norm-weighted sign-VQ retrieval (normw.cu) ----
+// idx/score [B, Hkv, top_k]; at most 65536 candidates per pair.
+int launch_retrieve_normw(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,
+                          const uint16_t* norms, int32_t* idx, float* score, cudaStream_t st);
+
+// ---- token split (split.cu) ----
+// cand_idx/cand_dist [G, P, k]; idx_out [P, k]; distances in [0, nbins).
+int launch_split_select(int G, int me, int P, int k, int nbins, const int32_t* cand_idx, const int32_t* cand_dist,
+                        int32_t* idx_out, int32_t* status, cudaStream_t st);
+int launch_lse_merge_n(int G, int64_t rows, const float* o, const float* lse, float* out, float* lse_out,
+                       cudaStream_t st);
 
 // ---- attention (attend.cu) ----
 struct AttendShape {

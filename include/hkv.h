@@ -277,6 +277,57 @@ int hkv_write_slots(int B, int Hkv, int dtype, int code_bits, const void* k_new,
                     uint32_t* codes, uint16_t* norms, int64_t capacity, const int32_t* slot,
                     int32_t* status, void* stream);
 
+/* Top-k per (batch, KV head) by the norm-weighted sign score.  Self-Indexing
+ * KVCache "Abstract": a key's sign code with its norm is its 1-bit vector
+ * quantisation.  Reading that pair as the reconstruction |k| sign(k) / sqrt(b)
+ * and each query head as sign(q_h) / sqrt(b), the inner products summed over
+ * the g query heads of KV head j give the score
+ *   S(t) = norm[b, j, t] * (g * code_bits - 2 * D(t)),
+ *   D(t) = sum_h popcount(q_codes[b, h] XOR k_codes[b, j, t]),
+ * and the top_k candidates t in [sink_end, local_start) with the LARGEST S
+ * are kept, ties to the lowest t, in ascending t order (-1 past
+ * k_eff = min(top_k, candidates)).  S is exact in fp32 (fp16 norm times an
+ * integer of at most 12 bits); -0 and +0 are one score.
+ *   q_codes [B, Hq, code_bits/32];  k_codes [B, Hkv, cap, code_bits/32]
+ *   norms   [B, Hkv, cap] fp16 bits (finite), e.g. from hkv_encode_keys
+ *           with the sign hash
+ *   idx     [B, Hkv, top_k] int32 out;  score  nullable [B, Hkv, top_k]
+ *           fp32 out (S of each selected token, -inf past k_eff)
+ * One launch, one block per (batch, KV head); no workspace.  At most 65536
+ * candidates per KV head (HKV_ERR_UNSUPPORTED beyond).  The selected rows
+ * go to hkv_sparse_attend like those of hkv_retrieve_topk. */
+int hkv_retrieve_topk_normw(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                            const uint32_t* k_codes, const uint16_t* norms, int64_t cap, int64_t n_tokens,
+                            int n_sink, int n_local, int top_k, int32_t* idx, float* score, void* stream);
+
+/* Token-split selection.  One sequence's cache is cut into G contiguous
+ * token ranges, one per rank, in token order.  Every rank first takes its
+ * own top_k with hkv_retrieve_topk over its range (local indices and
+ * distances, -1 past its own k_eff); every token of the whole sequence's
+ * top_k is among them.  Given all ranks' candidates, gathered rank-major,
+ *   cand_idx, cand_dist  [G, B, Hkv, top_k] int32,
+ * this call finds the whole sequence's top_k (smallest group distance, ties
+ * to the lowest token index: rank order, then ascending local index) and
+ * writes the selected tokens of rank `rank` as its local indices:
+ *   idx  [B, Hkv, top_k] int32 out, ascending, -1 padded.
+ * These are exactly the tokens of that range which hkv_retrieve_topk over
+ * the whole sequence would select.  RetrievalAttention "Approach" (retrieval
+ * spread over several index partitions, results merged).  A distance
+ * outside [0, g * code_bits] is skipped and reported as
+ * HKV_ERR_DEVICE_RANGE.  One launch; no workspace. */
+int hkv_split_select(int G, int rank, int B, int Hq, int Hkv, int code_bits, int top_k, const int32_t* cand_idx,
+                     const int32_t* cand_dist, int32_t* idx, int32_t* status, void* stream);
+
+/* G-way log-sum-exp merge of partial attention results (RetrievalAttention
+ * "Approach"), e.g. one partial per rank of a token split.  Per row:
+ *   M = max_g lse[g], w_g = exp(lse[g] - M)
+ *   out = sum_g w_g o[g] / sum_g w_g,  lse_out = M + log sum_g w_g
+ * Rows whose partials are all empty (lse -inf) give out 0, lse_out -inf.
+ *   o [G, rows, 128] fp32 (16-byte aligned);  lse [G, rows] fp32
+ *   out [rows, 128] fp32;  lse_out nullable [rows] fp32 */
+int hkv_lse_merge_n(int G, int64_t rows, const float* o, const float* lse, float* out, float* lse_out,
+                    void* stream);
+
 /* Sparse attention over sink + selected + local rows, with the log-sum-exp
  * merge of the partials (S6, S7, S8).  Spotlight Attention "Approach" (exact
  * attention over the retrieved tokens); RetrievalAttention "Approach" (exact

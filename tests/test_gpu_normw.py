@@ -1,0 +1,105 @@
+"""Norm-weighted sign-VQ retrieval on the GPU against the fp64 oracle
+(Self-Indexing KVCache, "Abstract": the sign code with the key's norm is a
+1-bit vector quantisation; the score is norm * (g * bits - 2 D), largest
+first, ties to the lowest index).  Index sets and scores are compared
+exactly: the fp32 score of an fp16 norm times a small integer is exact."""
+import numpy as np
+import pytest
+import torch
+
+import hash_sparse_kv_b200 as hkv
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _norms(seed, B, Hkv, cap, pool=None):
+    rng = np.random.default_rng(seed)
+    if pool is None:
+        n = rng.uniform(2.0, 5.0, size=(B, Hkv, cap))
+    else:
+        n = np.asarray(pool)[rng.integers(0, len(pool), size=(B, Hkv, cap))]
+    return n.astype(np.float16)
+
+
+def _run(qc, kc, norms, N, s, l, k):
+    B, Hq, W = qc.shape
+    Hkv = kc.shape[1]
+    idx = torch.full((B, Hkv, k), -7, dtype=torch.int32, device=DEV)
+    score = torch.full((B, Hkv, k), 7.0, dtype=torch.float32, device=DEV)
+    hkv.hkv_retrieve_topk_normw(qc.to(DEV), kc.to(DEV), torch.from_numpy(norms).to(DEV), N, s, l, k, idx, score)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), score.cpu().numpy()
+
+
+def _check(qc, kc, norms, N, s, l, k):
+    got_i, got_s = _run(qc, kc, norms, N, s, l, k)
+    want_i, want_s = oracle.retrieve_normw(qc.numpy().view(np.uint32), kc.numpy().view(np.uint32), norms, N, s, l, k)
+    np.testing.assert_array_equal(got_i, want_i)
+    np.testing.assert_array_equal(got_s, want_s.astype(np.float32))
+
+
+CASES = [
+    # B, Hq, Hkv, bits, N, cap, sink, local, top_k
+    (2, 8, 2, 128, 5000, 5000, 4, 64, 100),      # g 4, ragged tail, unaligned sink (scalar norm loads)
+    (1, 28, 4, 128, 20001, 20008, 8, 128, 1024),  # g 7, aligned window (vector norm loads)
+    (3, 32, 8, 64, 3001, 3100, 0, 0, 77),
+    (1, 16, 1, 64, 777, 800, 4, 64, 1),           # g 16, top-1
+    (2, 4, 2, 128, 300, 304, 8, 8, 400),          # top_k above the candidates
+    (2, 4, 2, 128, 50, 64, 40, 30, 8),            # no candidates
+    (4, 8, 8, 128, 65536, 65536, 0, 0, 512),      # g 1, 65536 candidates
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_normw_parity(case):
+    B, Hq, Hkv, bits, N, cap, s, l, k = case
+    W = bits // 32
+    kc = synth.random_codes(51 + N, B * Hkv * cap, W).view(B, Hkv, cap, W)
+    qc = synth.random_codes(52 + N, B * Hq, W).view(B, Hq, W)
+    _check(qc, kc, _norms(53 + N, B, Hkv, cap), N, s, l, k)
+
+
+@pytest.mark.parametrize("pool", [[1.5], [0.0, 1.0, 2.5], [0.0]])
+def test_normw_ties(pool):
+    """Few distinct codes and norms: long runs of equal scores spread over
+    every warp's range, so the tie quota crosses warps and chunks."""
+    B, Hq, Hkv, W, N = 2, 8, 2, 4, 9000
+    codes = synth.random_codes(60, 6, W)
+    rng = np.random.default_rng(61)
+    kc = codes[torch.from_numpy(rng.integers(0, 6, size=B * Hkv * N))].view(B, Hkv, N, W)
+    qc = synth.random_codes(62, B * Hq, W).view(B, Hq, W)
+    norms = _norms(63, B, Hkv, N, pool)
+    for k in (1, 333, 4000, 8990):
+        _check(qc, kc, norms, N, 4, 4, k)
+
+
+def test_normw_signvq_workload():
+    """Two KV heads of the sign-VQ workload (groups of 4 query heads, 65536
+    tokens, top 512; its other (batch, KV head) pairs are independent pairs
+    of the same shape) with the sign codes and fp16 norms of two-cone keys."""
+    w = synth.WORKLOADS["signvq"]
+    g = w.Hq // w.Hkv
+    B, Hq, Hkv, N, k = 1, 2 * g, 2, w.N, w.top_k
+    W = w.bits // 32
+    seed = synth.layer_seed(w, 0)
+    mu_k, mu_q, _ = synth.cone_means(seed, 0, w.d)
+    keys = synth.cone_rows(seed, 0, 1, mu_k, B * Hkv * N, "bf16")
+    qs = synth.cone_rows(seed, 0, 0, mu_q, B * Hq, "bf16")
+    kcodes, norms = oracle.encode("sign", keys)
+    qcodes, _ = oracle.encode("sign", qs)
+    kc = torch.from_numpy(kcodes.view(np.int32)).view(B, Hkv, N, W)
+    qc = torch.from_numpy(qcodes.view(np.int32)).view(B, Hq, W)
+    _check(qc, kc, norms.reshape(B, Hkv, N), N, w.n_sink, w.n_local, k)
+
+
+def test_normw_too_many_candidates():
+    qc = torch.zeros(1, 2, 4, dtype=torch.int32, device=DEV)
+    kc = torch.zeros(1, 1, 70000, 4, dtype=torch.int32, device=DEV)
+    norms = torch.zeros(1, 1, 70000, dtype=torch.float16, device=DEV)
+    idx = torch.empty(1, 1, 8, dtype=torch.int32, device=DEV)
+    with pytest.raises(hkv.HkvError) as e:
+        hkv.hkv_retrieve_topk_normw(qc, kc, norms, 70000, 0, 0, 8, idx)
+    assert e.value.code == hkv.HKV_ERR_UNSUPPORTED
