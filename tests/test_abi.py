@@ -87,3 +87,29 @@ def test_eviction_argument_errors(lib):
     assert rc == hkv.HKV_ERR_INVALID_ARG
     assert lib.hkv_write_slots(0, 2, hkv.HKV_BF16, 128, None, None, None, None, None, None, None, None, 10, None,
                                None, None) == hkv.HKV_OK
+
+
+def test_norm_weighted_and_split_argument_errors(lib):
+    # norm-weighted retrieval: bad code width, NULL norms, too many candidates
+    rc = lib.hkv_retrieve_topk_normw(1, 4, 2, 96, None, None, None, 10, 10, 0, 0, 4, None, None, None)
+    assert rc == hkv.HKV_ERR_UNSUPPORTED
+    rc = lib.hkv_retrieve_topk_normw(1, 4, 2, 128, 1, 16, None, 10, 10, 0, 0, 4, 1, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG  # norms is NULL
+    rc = lib.hkv_retrieve_topk_normw(1, 4, 2, 128, 16, 16, 16, 70000, 70000, 0, 0, 4, 16, None, None)
+    assert rc == hkv.HKV_ERR_UNSUPPORTED and "65536" in hkv.hkv_last_error()
+    rc = lib.hkv_retrieve_topk_normw(0, 4, 2, 128, None, None, None, 10, 10, 0, 0, 4, None, None, None)
+    assert rc == hkv.HKV_OK  # empty batch
+    # token split: rank outside [0, G), NULL candidates
+    rc = lib.hkv_split_select(2, 2, 1, 4, 2, 128, 8, None, None, None, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG
+    rc = lib.hkv_split_select(2, 1, 1, 4, 2, 128, 8, None, None, None, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG
+    rc = lib.hkv_split_select(2, 1, 1, 4, 2, 128, 0, None, None, None, None, None)
+    assert rc == hkv.HKV_OK  # top_k 0
+    # G-way merge: G 0, misaligned buffers
+    rc = lib.hkv_lse_merge_n(0, 4, None, None, None, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG
+    rc = lib.hkv_lse_merge_n(2, 4, 8, 16, 16, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG and "aligned" in hkv.hkv_last_error()
+    rc = lib.hkv_lse_merge_n(2, 0, None, None, None, None, None)
+    assert rc == hkv.HKV_OK
