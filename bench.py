@@ -453,6 +453,7 @@ def run_gpu(args, rank, world, local):
                   f"{per_layer_bytes * len(layers) / 1e9:.2f} GB algorithmic per step",
         },
         "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
+                     "frac_of_nominal_8tbs": step_gbs / 8000.0,
                      "bytes_per_layer": per_layer_bytes, "peak_kind": peak_kind},
         "roofline": {"bound": "hbm", "kernel": "fused_kernel (scan + select + attend + merge, one layer)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
