@@ -34,10 +34,15 @@
  *   - Layouts are dense row-major with the strides stated.  Codes are uint32
  *     words; bit j of a code is 1 iff the j-th pre-sign value is > 0, stored
  *     in word j / 32 at bit position j % 32.
- *   - Sequences in a batch share n_tokens (N).  Candidates for retrieval are
- *     the tokens [sink_end, local_start) with sink_end = min(n_sink, N) and
- *     local_start = max(sink_end, N - n_local); sink tokens [0, sink_end) and
- *     local tokens [local_start, N) are always attended.
+ *   - The retrieval and decode-step kernels are launched with programmatic
+ *     dependent launch: such a launch may be scheduled while the previous
+ *     kernel on the stream drains, but it reads and writes nothing in device
+ *     memory before that kernel has finished, so stream order holds as usual.
+ *   - Sequences in a batch share n_tokens (N), except in the ragged decode
+ *     step.  Candidates for retrieval are the tokens [sink_end, local_start)
+ *     with sink_end = min(n_sink, N) and local_start = max(sink_end,
+ *     N - n_local); sink tokens [0, sink_end) and local tokens
+ *     [local_start, N) are always attended.
  */
 #ifndef HKV_H
 #define HKV_H
