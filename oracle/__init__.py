@@ -35,7 +35,7 @@ import numpy as np
 __all__ = [
     "as_f64", "presign_lsh", "presign_mlp", "presign_sign", "pack_bits", "encode",
     "sign_norms", "hamming", "candidate_range", "select_topk", "attention_rows",
-    "attend", "lse_merge", "retrieve", "retrieve_normw", "decode_step", "ROW_CHUNK",
+    "attend", "lse_merge", "retrieve", "retrieve_normw", "decode_step", "gather_pages", "ROW_CHUNK",
 ]
 
 ROW_CHUNK = 1 << 15
@@ -371,3 +371,25 @@ def decode_step_ragged(q, K, V, k_codes, n_tokens_b, n_sink: int, n_local: int, 
     parts = [decode_step(q[b:b + 1], K[b:b + 1], V[b:b + 1], k_codes[b:b + 1], int(n_tokens_b[b]), n_sink,
                          n_local, top_k, kind, q_params, scale) for b in range(len(n_tokens_b))]
     return {key: np.concatenate([r[key] for r in parts], axis=0) for key in ("q_codes", "idx", "dist", "out", "lse")}
+
+
+def gather_pages(pool, page_table, page_size: int, N: int):
+    """A paged cache read back in token order (the paged layout is this
+    library's storage choice; the pages say nothing about it).  pool
+    [num_pages, Hkv, page_size, ...] holds page j of sequence b at
+    pool[page_table[b, j]]; token t of sequence b is slot t % page_size of
+    page t // page_size.  Returns [B, Hkv, N, ...], one explicit copy per
+    token, so that every other oracle function applies unchanged."""
+    table = np.asarray(page_table, dtype=np.int64)
+    B = table.shape[0]
+    is_torch = hasattr(pool, "detach")
+    if is_torch:
+        import torch
+        out = torch.empty((B, pool.shape[1], N) + tuple(pool.shape[3:]), dtype=pool.dtype)
+    else:
+        pool = np.asarray(pool)
+        out = np.empty((B, pool.shape[1], N) + pool.shape[3:], dtype=pool.dtype)
+    for b in range(B):
+        for t in range(N):
+            out[b, :, t] = pool[int(table[b, t // page_size]), :, t % page_size]
+    return out

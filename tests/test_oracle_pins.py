@@ -570,3 +570,52 @@ def test_normw_norm_scaling_and_zero_norms():
     assert S[0, 0, 10] == 0.0
     other = np.arange(N) != 10
     assert (S[0, 0][(m > 0) & other] > 0).all() and (S[0, 0][(m < 0) & other] < 0).all()
+
+
+# ------------------------------------------------------------ paged layout
+
+def test_gather_pages_identity_table_is_a_reshape():
+    """Pages laid out in order, one sequence per run of pages: gathering is
+    the plain reshape of the pool (numpy), for every N up to the capacity."""
+    rng = np.random.default_rng(8)
+    B, Hkv, P, pages, W = 2, 3, 4, 5, 2
+    pool = rng.integers(0, 2**31, size=(B * pages, Hkv, P, W))
+    table = np.arange(B * pages).reshape(B, pages)
+    whole = pool.reshape(B, pages, Hkv, P, W).transpose(0, 2, 1, 3, 4).reshape(B, Hkv, pages * P, W)
+    for N in (1, 7, 20):
+        np.testing.assert_array_equal(oracle.gather_pages(pool, table, P, N), whole[:, :, :N])
+
+
+def test_gather_pages_permuted_table():
+    """Hand-built: page size 2, two sequences sharing a pool of four pages in
+    scrambled order; every token's value names its (sequence, token)."""
+    P, Hkv = 2, 1
+    table = np.array([[3, 0], [1, 2]])
+    pool = np.zeros((4, Hkv, P), dtype=np.int64)
+    for b in range(2):
+        for t in range(4):
+            pool[table[b, t // P], 0, t % P] = 100 * b + t
+    got = oracle.gather_pages(pool, table, P, 3)
+    np.testing.assert_array_equal(got[:, 0], [[0, 1, 2], [100, 101, 102]])
+
+
+def test_paged_retrieval_equals_contiguous_retrieval():
+    """Retrieval over a gathered paged cache is the retrieval of the same
+    tokens stored contiguously (pages scattered at random in the pool)."""
+    rng = np.random.default_rng(9)
+    B, Hq, Hkv, W, P, N = 2, 4, 2, 4, 16, 100
+    pages = -(-N // P)
+    k = rng.integers(0, 2**32, size=(B, Hkv, pages * P, W), dtype=np.uint64).astype(np.uint32)
+    q = rng.integers(0, 2**32, size=(B, Hq, W), dtype=np.uint64).astype(np.uint32)
+    perm = rng.permutation(B * pages + 3)[: B * pages]
+    table = perm.reshape(B, pages)
+    pool = np.zeros((B * pages + 3, Hkv, P, W), dtype=np.uint32)
+    for b in range(B):
+        for j in range(pages):
+            pool[table[b, j]] = k[b, :, j * P:(j + 1) * P]
+    gathered = oracle.gather_pages(pool, table, P, N)
+    np.testing.assert_array_equal(gathered, k[:, :, :N])
+    i1, d1 = oracle.retrieve(q, gathered, N, 4, 16, 20)
+    i2, d2 = oracle.retrieve(q, k, N, 4, 16, 20)
+    np.testing.assert_array_equal(i1, i2)
+    np.testing.assert_array_equal(d1, d2)
