@@ -333,6 +333,61 @@ int hkv_sparse_attend(int B, int Hq, int Hkv, int dtype, const void* q, const vo
   return launch_attend(s, q, K, V, idx, scale, out, lse, ws, ws_bytes, status, static_cast<cudaStream_t>(stream));
 }
 
+static int check_pages(const int32_t* page_table, int64_t max_pages, int64_t num_pages, int page_size,
+                       int64_t n_tokens, PageMap& pm) {
+  if (page_size < 1 || max_pages < 0 || num_pages < 1)
+    return fail(HKV_ERR_INVALID_ARG, "page_size %d max_pages %lld num_pages %lld", page_size, (long long)max_pages,
+                (long long)num_pages);
+  if (max_pages * (int64_t)page_size < n_tokens)
+    return fail(HKV_ERR_INVALID_ARG, "max_pages * page_size < n_tokens");
+  if (n_tokens > 0 && page_table == nullptr) return fail(HKV_ERR_INVALID_ARG, "page_table is NULL");
+  pm.table = page_table;
+  pm.max_pages = max_pages;
+  pm.num_pages = num_pages;
+  pm.page_size = page_size;
+  return HKV_OK;
+}
+
+int hkv_retrieve_topk_paged(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                            const uint32_t* codes_pool, const int32_t* page_table, int64_t max_pages,
+                            int64_t num_pages, int page_size, int64_t n_tokens, int n_sink, int n_local, int top_k,
+                            int32_t* idx, int32_t* dist, int32_t* status, void* stream) {
+  int rc = check_heads(B, Hq, Hkv);
+  if (rc == HKV_OK) rc = check_window(n_tokens, n_tokens, n_sink, n_local, top_k);
+  if (rc != HKV_OK) return rc;
+  if (code_bits != 64 && code_bits != 128) return fail(HKV_ERR_UNSUPPORTED, "code_bits %d (64 or 128)", code_bits);
+  PageMap pm;
+  rc = check_pages(page_table, max_pages, num_pages, page_size, n_tokens, pm);
+  if (rc != HKV_OK) return rc;
+  if (B == 0 || top_k == 0) return HKV_OK;
+  if (!q_codes || !codes_pool || !idx) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(codes_pool, code_bits / 8))
+    return fail(HKV_ERR_INVALID_ARG, "codes_pool must be %d-byte aligned", code_bits / 8);
+  RetrieveShape s{B, Hq, Hkv, code_bits / 32, n_tokens, n_tokens, n_sink, n_local, top_k};
+  return launch_retrieve_paged(s, pm, q_codes, codes_pool, idx, dist, status, static_cast<cudaStream_t>(stream));
+}
+
+int hkv_sparse_attend_paged(int B, int Hq, int Hkv, int dtype, const void* q, const void* K_pool, const void* V_pool,
+                            const int32_t* page_table, int64_t max_pages, int64_t num_pages, int page_size,
+                            int64_t n_tokens, const int32_t* idx, int top_k, int n_sink, int n_local, float scale,
+                            float* out, float* lse, void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  int rc = check_heads(B, Hq, Hkv);
+  if (rc == HKV_OK) rc = check_window(n_tokens, n_tokens, n_sink, n_local, top_k);
+  if (rc != HKV_OK) return rc;
+  if (dtype != HKV_F32 && dtype != HKV_BF16) return fail(HKV_ERR_INVALID_ARG, "dtype %d", dtype);
+  if (!std::isfinite(scale)) return fail(HKV_ERR_INVALID_ARG, "scale is not finite");
+  PageMap pm;
+  rc = check_pages(page_table, max_pages, num_pages, page_size, n_tokens, pm);
+  if (rc != HKV_OK) return rc;
+  if (B == 0) return HKV_OK;
+  if (!q || !K_pool || !V_pool || !out || (top_k > 0 && !idx)) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(q, 16) || !aligned(K_pool, 16) || !aligned(V_pool, 16) || !aligned(out, 16))
+    return fail(HKV_ERR_INVALID_ARG, "q, K_pool, V_pool and out must be 16-byte aligned");
+  AttendShape s{B, Hq, Hkv, dtype, n_tokens, n_tokens, top_k, n_sink, n_local};
+  return launch_attend(s, q, K_pool, V_pool, idx, scale, out, lse, ws, ws_bytes, status,
+                       static_cast<cudaStream_t>(stream), &pm);
+}
+
 int hkv_lse_merge(int rows, int d, const float* o1, const float* lse1, const float* o2,
                   const float* lse2, float* out, float* lse_out, void* stream) {
   if (rows < 0 || d < 1) return fail(HKV_ERR_INVALID_ARG, "rows %d d %d", rows, d);

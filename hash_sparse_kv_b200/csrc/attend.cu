@@ -45,9 +45,24 @@ struct AttendArgs {
   float scale;
   int rows_per_split, splits;
   int32_t* status;
+  PageMap pm;  // paged K/V pools when PAGED
 };
 
-template <typename T>
+// K and V rows of token t of pair (b, kvh): contiguous [B, Hkv, cap, 128], or
+// slot t % page_size of pool page table[b, t / page_size] ([num_pages, Hkv,
+// page_size, 128]); -1 when that page id is outside the pool.
+template <bool PAGED>
+__device__ __forceinline__ int64_t kv_row_of(const AttendArgs& a, int b, int kvh, int p, int64_t t) {
+  if constexpr (PAGED) {
+    const int pg = a.pm.table[(int64_t)b * a.pm.max_pages + t / a.pm.page_size];
+    if (pg < 0 || pg >= a.pm.num_pages) return -1;
+    return ((int64_t)pg * a.Hkv + kvh) * a.pm.page_size + t % a.pm.page_size;
+  } else {
+    return (int64_t)p * a.cap + t;
+  }
+}
+
+template <typename T, bool PAGED>
 __global__ void __launch_bounds__(kThreads) attend_kernel(AttendArgs a) {
   extern __shared__ __align__(16) float smem[];
   float* q_s = smem;                          // [g][128]
@@ -66,8 +81,8 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(AttendArgs a) {
   const int nrows = (int)max((int64_t)0, min((int64_t)a.rows_per_split, Rv - v0));
 
   const T* qp = static_cast<const T*>(a.q) + ((int64_t)b * a.Hq + (int64_t)kvh * g) * kHeadDim;
-  const T* Kp = static_cast<const T*>(a.K) + (int64_t)p * a.cap * kHeadDim;
-  const T* Vp = static_cast<const T*>(a.V) + (int64_t)p * a.cap * kHeadDim;
+  const T* Kb = static_cast<const T*>(a.K);
+  const T* Vb = static_cast<const T*>(a.V);
 
   for (int i = tid; i < nrows; i += kThreads) {
     const int64_t v = v0 + i;
@@ -82,6 +97,10 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(AttendArgs a) {
       }
     } else {
       t = a.local_start + (v - a.sink_n - a.top_k);
+    }
+    if (PAGED && t >= 0 && kv_row_of<PAGED>(a, b, kvh, p, t) < 0) {
+      report(a.status, HKV_ERR_DEVICE_RANGE);
+      t = -1;
     }
     tok_s[i] = t < 0 ? -1 : (int)t;
   }
@@ -101,8 +120,9 @@ __global__ void __launch_bounds__(kThreads) attend_kernel(AttendArgs a) {
       const int t = r < nrows ? tok_s[r] : -1;
       kr[u] = vr[u] = make_uint4(0u, 0u, 0u, 0u);
       if (t >= 0) {
-        kr[u] = __ldg(reinterpret_cast<const uint4*>(Kp + (int64_t)t * kHeadDim) + c);
-        vr[u] = __ldg(reinterpret_cast<const uint4*>(Vp + (int64_t)t * kHeadDim) + c);
+        const int64_t row = kv_row_of<PAGED>(a, b, kvh, p, t);
+        kr[u] = __ldg(reinterpret_cast<const uint4*>(Kb + row * kHeadDim) + c);
+        vr[u] = __ldg(reinterpret_cast<const uint4*>(Vb + row * kHeadDim) + c);
       }
     }
 #pragma unroll
@@ -295,7 +315,7 @@ size_t attend_ws_bytes(const AttendShape& s) { return make_plan(s).ws_total; }
 
 int launch_attend(const AttendShape& s, const void* q, const void* K, const void* V,
                   const int32_t* idx, float scale, float* out, float* lse, void* ws,
-                  size_t ws_bytes, int32_t* status, cudaStream_t st) {
+                  size_t ws_bytes, int32_t* status, cudaStream_t st, const PageMap* pm) {
   const int P = s.B * s.Hkv;
   if (P == 0) return HKV_OK;
   const AttendPlan pl = make_plan(s);
@@ -326,16 +346,13 @@ int launch_attend(const AttendShape& s, const void* q, const void* K, const void
   a.rows_per_split = pl.rows_per_split;
   a.splits = pl.splits;
   a.status = status;
+  a.pm = pm != nullptr ? *pm : PageMap{};
   const int grid = P * pl.splits;
-  if (s.dtype == HKV_BF16) {
-    auto k = attend_kernel<__nv_bfloat16>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
-    k<<<grid, kThreads, pl.smem, st>>>(a);
-  } else {
-    auto k = attend_kernel<float>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
-    k<<<grid, kThreads, pl.smem, st>>>(a);
-  }
+  using Fn = void (*)(AttendArgs);
+  Fn k = s.dtype == HKV_BF16 ? (pm != nullptr ? attend_kernel<__nv_bfloat16, true> : attend_kernel<__nv_bfloat16, false>)
+                             : (pm != nullptr ? attend_kernel<float, true> : attend_kernel<float, false>);
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
+  k<<<grid, kThreads, pl.smem, st>>>(a);
   return cuda_check(cudaGetLastError(), "attend launch");
 }
 

@@ -90,6 +90,18 @@ int launch_split_select(int G, int me, int P, int k, int nbins, const int32_t* c
 int launch_lse_merge_n(int G, int64_t rows, const float* o, const float* lse, float* out, float* lse_out,
                        cudaStream_t st);
 
+// ---- paged caches (paged.cu, attend.cu) ----
+// Pool page table[b * max_pages + j] holds tokens [j * page_size,
+// (j + 1) * page_size) of sequence b; a page stores [Hkv, page_size, ...].
+struct PageMap {
+  const int32_t* table = nullptr;
+  int64_t max_pages = 0, num_pages = 0;
+  int page_size = 0;
+};
+// Group-Hamming top-k over a paged code pool; up to 65536 candidates per pair.
+int launch_retrieve_paged(const RetrieveShape& s, const PageMap& pm, const uint32_t* q_codes,
+                          const uint32_t* codes_pool, int32_t* idx, int32_t* dist, int32_t* status, cudaStream_t st);
+
 // ---- attention (attend.cu) ----
 struct AttendShape {
   int B, Hq, Hkv, dtype;
@@ -99,7 +111,7 @@ struct AttendShape {
 size_t attend_ws_bytes(const AttendShape& s);
 int launch_attend(const AttendShape& s, const void* q, const void* K, const void* V,
                   const int32_t* idx, float scale, float* out, float* lse, void* ws,
-                  size_t ws_bytes, int32_t* status, cudaStream_t st);
+                  size_t ws_bytes, int32_t* status, cudaStream_t st, const PageMap* pm = nullptr);
 int launch_lse_merge(int rows, int d, const float* o1, const float* lse1, const float* o2,
                      const float* lse2, float* out, float* lse_out, cudaStream_t st);
 

@@ -351,6 +351,38 @@ int hkv_sparse_attend(int B, int Hq, int Hkv, int dtype, const void* q, const vo
                       int top_k, int n_sink, int n_local, float scale, float* out, float* lse,
                       void* ws, size_t ws_bytes, int32_t* status, void* stream);
 
+/* Paged cache.  Each sequence's cache is cut into pages of page_size tokens
+ * held anywhere in one pool; page_table[b, j] (device int32 [B, max_pages])
+ * names the pool page holding tokens [j * page_size, (j + 1) * page_size) of
+ * sequence b, and a page stores all KV heads of its tokens:
+ *   codes_pool [num_pages, Hkv, page_size, code_bits/32] uint32
+ *   K_pool, V_pool [num_pages, Hkv, page_size, 128] in dtype
+ * (hkv_encode_keys on the pool viewed as [num_pages * Hkv * page_size, 128]
+ * rows fills codes_pool).  The two calls below compute exactly what
+ * hkv_retrieve_topk and hkv_sparse_attend compute on the same tokens stored
+ * contiguously; only the addressing differs.  The paged layout is this
+ * library's storage choice, not the pages' method.  Requirements:
+ * page_size >= 1, max_pages * page_size >= n_tokens, num_pages >= 1.  A
+ * page id outside [0, num_pages) met on the device is reported as
+ * HKV_ERR_DEVICE_RANGE: retrieval gives its tokens the largest distance and
+ * attention skips them.
+ *
+ * Retrieval: idx [B, Hkv, top_k] int32 and nullable dist, as
+ * hkv_retrieve_topk.  One block per (batch, KV head), no workspace; at most
+ * 65536 candidates per KV head (HKV_ERR_UNSUPPORTED beyond). */
+int hkv_retrieve_topk_paged(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
+                            const uint32_t* codes_pool, const int32_t* page_table, int64_t max_pages,
+                            int64_t num_pages, int page_size, int64_t n_tokens, int n_sink, int n_local, int top_k,
+                            int32_t* idx, int32_t* dist, int32_t* status, void* stream);
+
+/* Attention over a paged cache: hkv_sparse_attend with K and V read through
+ * the page table (q, idx, out, lse, scale, ws as there; the workspace size
+ * is the same). */
+int hkv_sparse_attend_paged(int B, int Hq, int Hkv, int dtype, const void* q, const void* K_pool, const void* V_pool,
+                            const int32_t* page_table, int64_t max_pages, int64_t num_pages, int page_size,
+                            int64_t n_tokens, const int32_t* idx, int top_k, int n_sink, int n_local, float scale,
+                            float* out, float* lse, void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
 /* Elementwise log-sum-exp merge of two partial attention results (S8 alone).
  * RetrievalAttention "Approach".  For each of `rows` rows:
  *   m = max(lse1, lse2), w_i = exp(lse_i - m)
