@@ -227,6 +227,19 @@ class Layer:
                             None if self.norms is None else self.norms.view(-1))
 
 
+def paged_roofline(w: synth.Workload, n_layers: int, ms: float, step_ms: float, page: int, peak: float,
+                   peak_kind: str) -> dict:
+    """Retrieval over a paged code pool: the candidates' codes are the
+    algorithmic bytes of one launch (the page table is negligible)."""
+    nbytes = w.B * w.Hkv * w.candidates() * w.bits // 8
+    launch_s = ms * 1e-3 / n_layers
+    return {"kernel": "paged_topk_kernel (scan through the page table + select + ordered compaction)",
+            "page_size": page, "bound": "hbm", "achieved": nbytes / launch_s / 1e9, "peak": peak, "unit": "GB/s",
+            "frac": nbytes / launch_s / 1e9 / peak, "bytes_per_launch": nbytes, "launch_us": launch_s * 1e6,
+            "step_us_per_layer": step_ms * 1e3 / n_layers, "launches_per_layer": 3, "peak_kind": peak_kind,
+            "traffic": None}
+
+
 def normw_roofline(w: synth.Workload, n_layers: int, ms: float, step_ms: float, peak: float, peak_kind: str) -> dict:
     """Norm-weighted sign-VQ retrieval: codes and fp16 norms of every candidate
     are the algorithmic bytes of one launch."""
@@ -380,6 +393,50 @@ def run_gpu(args, rank, world, local):
     ev_ms = max_over_ranks(time_graph(g_ev, args.steps, args.warmup, world), world, dev)
     del g_ev
     del g_qenc, g_att
+    # paged cache (pages of 256 tokens scattered through a pool): retrieval
+    # and attention read through the page table, after the query encode
+    paged_ms = paged_step_ms = None
+    PAGE = 256
+    if w.candidates() <= 65536 and w.N % PAGE == 0:
+        pages = w.N // PAGE
+        gen = torch.Generator(device=dev).manual_seed(1234)
+        paged_layers = []
+        for L in layers:
+            perm = torch.randperm(w.B * pages, generator=gen, device=dev)
+            table = perm.view(w.B, pages).to(torch.int32)
+
+            def to_pool(x):
+                # [B, Hkv, N, ...] -> pool page perm[b * pages + j] = tokens [j * PAGE, (j + 1) * PAGE) of b
+                tail = tuple(x.shape[3:])
+                src = x.view((w.B, w.Hkv, pages, PAGE) + tail).transpose(1, 2).reshape((w.B * pages, w.Hkv, PAGE) + tail)
+                pool = torch.empty_like(src)
+                pool[perm.long()] = src
+                return pool
+
+            paged_layers.append((L, table, to_pool(L.codes), to_pool(L.K), to_pool(L.V)))
+
+        def paged_only():
+            for L, table, cpool, _, _ in paged_layers:
+                hkv.hkv_retrieve_topk_paged(L.q_codes, cpool, table, w.N, w.n_sink, w.n_local, w.top_k, L.idx,
+                                            status=status)
+
+        def paged_step():
+            for L, table, cpool, kpool, vpool in paged_layers:
+                hkv.hkv_encode_keys(L.qh, L.q.view(-1, w.d), L.q_codes.view(-1, w.words))
+                hkv.hkv_retrieve_topk_paged(L.q_codes, cpool, table, w.N, w.n_sink, w.n_local, w.top_k, L.idx,
+                                            status=status)
+                hkv.hkv_sparse_attend_paged(L.q, kpool, vpool, table, w.N, L.idx, w.n_sink, w.n_local, L.out,
+                                            ws=ws_a, status=status)
+
+        g_pg = graph_of(paged_only)
+        paged_ms = max_over_ranks(time_graph(g_pg, args.steps, args.warmup, world), world, dev)
+        del g_pg
+        g_pg = graph_of(paged_step)
+        paged_step_ms = max_over_ranks(time_graph(g_pg, args.steps, args.warmup, world), world, dev)
+        del g_pg, paged_layers
+        rc = hkv.hkv_check(status)
+        if rc != hkv.HKV_OK:
+            raise RuntimeError(f"paged calls reported status {rc}")
     # sign-VQ only: retrieval by the norm-weighted sign score (its own kernel),
     # then the standalone sparse attention
     normw_ms = normw_step_ms = None
@@ -473,6 +530,8 @@ def run_gpu(args, rank, world, local):
                   "unit": "GB/s", "frac": code_bytes / (ev_ms * 1e-3 / len(layers)) / 1e9 / peak,
                   "bytes_per_launch": code_bytes, "launches_per_layer": 2,
                   "traffic": traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "evict.cu"), w.name)},
+        "paged": None if paged_ms is None else paged_roofline(w, len(layers), paged_ms, paged_step_ms, PAGE, peak,
+                                                              peak_kind),
         "normw": None if normw_ms is None else normw_roofline(w, len(layers), normw_ms, normw_step_ms, peak, peak_kind),
         # decode with an LSH or sign query hash (query heads per KV head <= 32) is one
         # fused launch a layer; an MLP query hash adds the separate query encode launch
