@@ -37,3 +37,29 @@ def test_gpu_arm_without_a_gpu_fails_loudly():
     r = _bench("--workload", "tiny_lsh", "--steps", "1", "--warmup", "1", "--no-cpu-baseline")
     assert r.returncode != 0
     assert r.stdout.strip() == "" or "value" not in r.stdout
+
+
+def test_roofline_arithmetic():
+    """The byte counts behind the reported fractions: the 512K layer's
+    algorithmic bytes, the norm-weighted and paged retrieval bytes, and the
+    encode roofline of each hash family."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    w = synth.WORKLOADS["qwen7b_512k"]
+    C = w.N - w.n_sink - w.n_local
+    assert w.candidates() == C
+    kv = w.B * w.Hkv * (w.top_k + w.n_sink + w.n_local) * 128 * 2 * 2
+    assert w.algorithmic_bytes() >= w.B * w.Hkv * C * 16 + kv
+    sv = synth.WORKLOADS["signvq"]
+    r = bench.normw_roofline(sv, 1, 0.1, 0.2, 6548.8, "measured")
+    assert r["bytes_per_launch"] == 16 * 8 * 65536 * (16 + 2)
+    assert r["frac"] == pytest.approx(r["bytes_per_launch"] / 1e-4 / 1e9 / 6548.8)
+    he = synth.WORKLOADS["hashevict_lsh"]
+    r = bench.paged_roofline(he, 2, 0.1, 0.3, 256, 6548.8, "measured")
+    assert r["bytes_per_launch"] == 8 * 8 * (32768 - 4 - 64) * 8
+    assert r["launch_us"] == pytest.approx(50.0) and r["step_us_per_layer"] == pytest.approx(150.0)
+    e = bench.encode_roofline(he, 1, 1.0)
+    assert e["bound"] == "hbm" and e["gbs"] == pytest.approx(8 * 8 * 32768 * (256 + 8) / 1e-3 / 1e9)
+    e = bench.encode_roofline(synth.WORKLOADS["spotlight_mlp"], 1, 1.0)
+    assert e["bound"] == "tensor" and e["unit"] == "TFLOP/s"
