@@ -111,12 +111,15 @@ class _OracleOps:
 
 
 # B, Hq, Hkv, bits, N, sink, local, top_k
-_SPLIT = (1, 4, 2, 64, 97, 3, 10, 20)
+_SPLITS = {
+    "short_window": (1, 4, 2, 64, 97, 3, 10, 20),
+    "window_covers_ranks": (2, 4, 1, 64, 90, 30, 40, 8),  # the first and last ranges hold no candidates
+}
 
 
-def _split_inputs():
+def _split_inputs(shape):
     g = torch.Generator().manual_seed(11)
-    B, Hq, Hkv, bits, N, _, _, _ = _SPLIT
+    B, Hq, Hkv, bits, N, _, _, _ = shape
     q = torch.randn(B, Hq, 128, generator=g, dtype=torch.float64)
     K = torch.randn(B, Hkv, N, 128, generator=g, dtype=torch.float64)
     V = torch.randn(B, Hkv, N, 128, generator=g, dtype=torch.float64)
@@ -124,15 +127,15 @@ def _split_inputs():
     return q, K, V, R
 
 
-def _split_worker(rank, world, port, q_out):
+def _split_worker(rank, world, port, q_out, shape):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         import numpy as np
         import oracle
         from hash_sparse_kv_b200 import split
-        B, Hq, Hkv, bits, N, s, l, k = _SPLIT
-        q, K, V, R = _split_inputs()
+        B, Hq, Hkv, bits, N, s, l, k = shape
+        q, K, V, R = _split_inputs(shape)
         kc = torch.from_numpy(oracle.encode("lsh", K, R).view(np.int32))
         r0, r1 = split.token_range(N, world, rank)
         st = split.SplitState.make(world, rank, B, Hq, Hkv, bits, k, N, s, l, "cpu", workspaces=False)
@@ -146,22 +149,24 @@ def _split_worker(rank, world, port, q_out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_token_split_protocol_equals_the_whole_sequence_step(world):
+@pytest.mark.parametrize("world,shape", [(2, "short_window"), (3, "short_window"), (3, "window_covers_ranks"),
+                                         (4, "window_covers_ranks")])
+def test_token_split_protocol_equals_the_whole_sequence_step(world, shape):
+    shape = _SPLITS[shape]
     import numpy as np
     import oracle
     ctx = mp.get_context("spawn")
     q_out = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_split_worker, args=(r, world, port, q_out)) for r in range(world)]
+    procs = [ctx.Process(target=_split_worker, args=(r, world, port, q_out, shape)) for r in range(world)]
     for p in procs:
         p.start()
     results = sorted(q_out.get(timeout=300) for _ in procs)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    B, Hq, Hkv, bits, N, s, l, k = _SPLIT
-    q, K, V, R = _split_inputs()
+    B, Hq, Hkv, bits, N, s, l, k = shape
+    q, K, V, R = _split_inputs(shape)
     ref = oracle.decode_step(q, K, V, oracle.encode("lsh", K, R), N, s, l, k, "lsh", R)
     for b in range(B):
         for j in range(Hkv):
