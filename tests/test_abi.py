@@ -131,3 +131,23 @@ def test_paged_argument_errors(lib):
     rc = lib.hkv_sparse_attend_paged(1, 4, 2, hkv.HKV_BF16, 16, 16, 16, 16, 4, 0, 4, 10, 16, 4, 0, 0, 0.088,
                                      16, None, None, 0, None, None)
     assert rc == hkv.HKV_ERR_INVALID_ARG  # num_pages 0
+
+
+def test_binding_rejects_host_tensors_and_bad_shapes(lib):
+    """The Python binding checks devices, dtypes and shapes before any call."""
+    import torch
+    q = torch.zeros(1, 4, 4, dtype=torch.int32)
+    k = torch.zeros(1, 2, 64, 4, dtype=torch.int32)
+    idx = torch.zeros(1, 2, 8, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        hkv.hkv_retrieve_topk(q, k, 64, 0, 0, 8, idx)
+    with pytest.raises(ValueError, match="CUDA"):
+        hkv.hkv_retrieve_topk_normw(q, k, torch.zeros(1, 2, 64, dtype=torch.float16), 64, 0, 0, 8, idx)
+    with pytest.raises(ValueError, match="CUDA"):
+        hkv.hkv_retrieve_topk_paged(q, torch.zeros(4, 2, 16, 4, dtype=torch.int32),
+                                    torch.zeros(1, 4, dtype=torch.int32), 64, 0, 0, 8, idx)
+    with pytest.raises(ValueError, match="CUDA"):
+        hkv.hkv_split_select(0, 4, 128, torch.zeros(2, 1, 2, 8, dtype=torch.int32),
+                             torch.zeros(2, 1, 2, 8, dtype=torch.int32), idx)
+    with pytest.raises(ValueError, match="CUDA"):
+        hkv.hkv_lse_merge_n(torch.zeros(2, 3, 128), torch.zeros(2, 3), torch.zeros(3, 128))
