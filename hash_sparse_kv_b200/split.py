@@ -139,6 +139,13 @@ def decode_step_split(st: SplitState, q_hash, q, k_codes, K, V, N: int, n_sink: 
     """One decode step of this rank (see the module docstring).  k_codes, K,
     V hold the rank's token range token_range(N, world, rank) from row 0."""
     import torch.distributed as dist
+    r0, r1 = token_range(N, st.world, st.rank)
+    for name, t in (("k_codes", k_codes), ("K", K), ("V", V)):
+        if t.shape[2] < r1 - r0:
+            raise ValueError(f"{name} holds {t.shape[2]} tokens; rank {st.rank} of {st.world} owns {r1 - r0} "
+                             f"(tokens [{r0}, {r1}) of {N})")
+    if st.cand_idx.shape[0] != st.world or tuple(st.own_idx.shape) != tuple(st.cand_idx.shape[1:]):
+        raise ValueError("split state was made for another world size or shape")
     ops = ops or LibraryOps()
     scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
     # flat views: every backend takes a 1-D concatenation of the ranks' parts

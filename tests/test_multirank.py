@@ -200,3 +200,13 @@ def test_local_windows_partition_the_sequence():
                 assert got["sink"] == list(range(0, se))
                 assert got["cand"] == list(range(se, ls))
                 assert got["local"] == list(range(ls, N))
+
+
+def test_split_step_rejects_a_short_range():
+    """A rank handed fewer tokens than its range fails before any exchange."""
+    from hash_sparse_kv_b200 import split
+    st = split.SplitState.make(2, 1, 1, 4, 2, 64, 8, 100, 0, 0, "cpu", workspaces=False)
+    kc = torch.zeros(1, 2, 49, 2, dtype=torch.int32)  # rank 1 of 2 owns tokens [50, 100)
+    K = torch.zeros(1, 2, 50, 128)
+    with pytest.raises(ValueError, match="k_codes holds 49 tokens"):
+        split.decode_step_split(st, None, torch.zeros(1, 4, 128), kc, K, K, 100, 0, 0, 64, torch.zeros(1, 4, 128))
