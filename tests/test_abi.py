@@ -151,3 +151,20 @@ def test_binding_rejects_host_tensors_and_bad_shapes(lib):
                              torch.zeros(2, 1, 2, 8, dtype=torch.int32), idx)
     with pytest.raises(ValueError, match="CUDA"):
         hkv.hkv_lse_merge_n(torch.zeros(2, 3, 128), torch.zeros(2, 3), torch.zeros(3, 128))
+
+
+def test_plain_c_program_links_and_calls_the_library(lib, tmp_path):
+    """include/hkv.h is valid C99 and libhkv.so links from C: a C program
+    checks the host-side paths (no GPU needed)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "c_abi_check"
+    libdir = os.path.dirname(hkv.lib_path)
+    cmd = ["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+           os.path.join(ROOT, "tests", "c_abi_check.c"), "-L", libdir, "-lhkv", f"-Wl,-rpath,{libdir}", "-o", str(exe)]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert "c abi ok" in r.stdout
