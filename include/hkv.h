@@ -116,8 +116,9 @@ const char* hkv_version(void);
 int hkv_check(int32_t* status, void* stream);
 
 /* Bytes of workspace that hkv_retrieve_topk, hkv_sparse_attend and
- * hkv_decode_step need for this shape on the current device (0 if the shape
- * is invalid or unsupported).  The workspace must be zero-filled once before
+ * hkv_decode_step (and their variants) need for this shape on the current
+ * device (0 if the shape is invalid or unsupported, or no CUDA device is
+ * visible: the plan depends on the device's SM count and shared memory).  The workspace must be zero-filled once before
  * first use (hkv_workspace_reset).  Each call returns the counters and
  * histograms that must start at zero to zero before it ends, including calls
  * that end in a device error, so one workspace serves any number of calls in
