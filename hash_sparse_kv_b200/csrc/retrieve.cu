@@ -1384,7 +1384,9 @@ int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint3
 // file-scope device array: every GPU that loads the library holds it until
 // the process exits.  Host code must not pass the array's name to a kernel
 // (on the host it is only a stand-in); its device address is looked up once
-// per device with cudaGetSymbolAddress and cached.
+// per device with cudaGetSymbolAddress and cached for the life of the process
+// (a cudaDeviceReset would invalidate the cached address, so the entry point
+// must not be used after one).
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 namespace {
@@ -1392,8 +1394,10 @@ constexpr int kMaxDevices = 64;
 std::mutex g_static_mu;
 void* g_static_ptr[kMaxDevices] = {};
 
-// Device address of the static scratch on the current device.  The first
-// call on a device looks it up and zero-fills it (synchronously).
+// Device address of the static scratch on the current device.  Nothing is
+// written here: each call clears, on its own stream, the part of the area
+// that must start at zero, and every other part is written by the kernel
+// before it is read.
 int static_scratch(void** out) {
   int dev = 0;
   int rc = cuda_check(cudaGetDevice(&dev), "current device");
@@ -1403,8 +1407,6 @@ int static_scratch(void** out) {
   if (g_static_ptr[dev] == nullptr) {
     void* p = nullptr;
     rc = cuda_check(cudaGetSymbolAddress(&p, g_static_scratch), "static scratch address");
-    if (rc != HKV_OK) return rc;
-    rc = cuda_check(cudaMemset(p, 0, kStaticScratchBytes), "static scratch zero fill");
     if (rc != HKV_OK) return rc;
     g_static_ptr[dev] = p;
   }
@@ -1428,7 +1430,9 @@ int launch_retrieve_static(const RetrieveShape& s, const uint32_t* q_codes, cons
   if (rc != HKV_OK) return rc;
   // The counters and the pair histograms must start at zero.  A call of the
   // same shape leaves them so, but the previous call may have had another
-  // shape (and so another layout of the area), so clear them every time.
+  // shape (and so another layout of the area), or may never have run on this
+  // device, so clear them every time, ordered on this call's stream.  The
+  // per-block cumulative counts are written before they are read.
   rc = cuda_check(cudaMemsetAsync(ws, 0, pl.ws_sync + pl.ws_gh, st), "static scratch counters");
   if (rc != HKV_OK) return rc;
   return launch_retrieve(s, q_codes, k_codes, idx, dist, ws, kStaticScratchBytes, status, st);

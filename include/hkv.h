@@ -202,14 +202,20 @@ int hkv_retrieve_topk(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_c
  *     that loads the library until the process exits.  Shapes whose
  *     hkv_workspace_bytes-style scratch need exceeds 8 MiB are rejected with
  *     HKV_ERR_CAPACITY (the message states the bytes needed).  The retrieval
- *     scratch is about nbins * 4 bytes per block plus nbins * 4 + 16 bytes
- *     per (batch, KV head), nbins = g * code_bits + 1: e.g. 0.2 MiB for
- *     4 KV heads x 512K tokens with g = 7.
- *   - The first call on a device looks up the array's device address and
- *     zero-fills it, synchronously; make that first call before any stream
- *     capture.  Later calls only enqueue work on `stream`.
- *   - Every call uses the same array and clears the counters and
- *     histograms that must start at zero before it runs.  Calls that overlap on the GPU (other
+ *     scratch is nbins * 4 bytes per block plus nbins * 4 + 16 bytes per
+ *     (batch, KV head), nbins = g * code_bits + 1, rounded up to 256-byte
+ *     pieces.  The number of blocks per (batch, KV head) follows the SM
+ *     count, so the need grows with it: on a 148-SM B200, 4 KV heads x 512K
+ *     tokens with g = 7 take 37 blocks per KV head, 4 * 37 * 897 * 4 bytes of
+ *     per-block counts plus 4 * (897 * 4 + 16) bytes, about 0.52 MiB.
+ *   - The first call on a device looks up the array's device address (a
+ *     host-side query, cached for the process; do not use this entry point
+ *     after a cudaDeviceReset).  Make that first call before any stream
+ *     capture.  Every call, the first included, only enqueues work on
+ *     `stream`.
+ *   - Every call uses the same array and first clears, on `stream`, the
+ *     counters and histograms that must start at zero; the rest of the area
+ *     is written before it is read.  Calls that overlap on the GPU (other
  *     streams, other host threads) race on the array and must not be issued.
  *   - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
  * Arguments are those of hkv_retrieve_topk, without ws and ws_bytes. */
