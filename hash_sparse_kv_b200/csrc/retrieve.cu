@@ -26,20 +26,29 @@
 //    histogram and stores its cumulative counts over [0, hi].  The threshold
 //    T (smallest D whose cumulative count reaches k_eff) is at most min over
 //    blocks of hi, because that block alone already has k_eff tokens at or
-//    below its hi; so the global histogram is complete on [0, T].
+//    below its hi; so the global histogram is complete on [0, T].  A unit
+//    served by one block needs no exchange: T is its own hi.
+//  * Speculative tile.  When a block's expected share of the selection is
+//    small (many blocks per unit), it gathers, while the other blocks
+//    publish, the K/V rows of its tokens with D <= tb (tb: the largest bin
+//    whose cumulative count fits one tile beside its resident rows) and of
+//    its share of the resident sink/local rows.  If T <= tb every selected
+//    token of the block is in that tile.
 //  * Phase B.  Wait (bounded) for all blocks of the unit, read the global
 //    histogram, find T, read the lower blocks' cumulative counts at T - 1 and
 //    T, then write this block's selected tokens straight to their final,
 //    ascending positions in idx: tokens with D < T, and tokens with D == T in
-//    ascending order until k_eff is reached.
-//  * Attention.  The block attends its selected rows plus its share of the
-//    unit's resident sink/local rows for all of the unit's query heads (bf16:
-//    tensor-core logits and P V over 64-row tiles fetched by cp.async) and
-//    writes one partial (m, l, acc).  The last g blocks of the unit to finish
-//    merge one head each: M = max m_s, L = sum l_s e^{m_s - M},
-//    out = sum acc_s e^{m_s - M} / L, lse = M + log L.
-//  * The last block out of a unit returns its counters and histogram to zero,
-//    so the workspace is ready for the next call.
+//    ascending order until k_eff is reached (a mask over the speculative
+//    tile, or an ordered compaction over 8-token octets of the distances).
+//  * Attention.  Eight warps take 16-row steps of the block's selected and
+//    resident rows, each with its own online softmax for the unit's query
+//    heads on the tensor cores (logits and P V by mma.sync, P kept in
+//    registers, two cp.async slots per warp), and the warps' partials are
+//    merged into one block partial (m, l, acc).  The last g blocks of the
+//    unit to finish merge one head each: M = max m_s, L = sum l_s e^{m_s - M},
+//    out = sum acc_s e^{m_s - M} / L, lse = M + log L; the last of them
+//    returns the unit's counters and histogram to zero, so the workspace is
+//    ready for the next call.
 //
 // The group-summed distance is computed by bit-sliced arithmetic
 // (hamming.cuh) instead of g * W popcounts.
@@ -50,6 +59,7 @@
 
 #include "hamming.cuh"
 #include "internal.h"
+#include "tc.cuh"
 
 namespace hkv {
 namespace {
@@ -57,7 +67,7 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kGroups = 4;                  // cp.async groups in flight per thread
-constexpr int kSlots = 2 * kGroups;         // two tokens per group
+constexpr int kSlots = 2 * kGroups;         // two codes per group
 constexpr int kMaxTokensPerBlock = 65536;   // uint16 distances in shared memory (when it fits)
 constexpr int kTokensPerBlockSmall = 32768; // the cap when the larger one does not fit
 constexpr size_t kStaticSmem = 2048;        // bound on the kernel's static shared memory
@@ -67,7 +77,7 @@ constexpr int kMaxGroup = 16;
 constexpr int kQRows = 32;                  // query rows one block may encode
 constexpr int kRows = 64;                   // attention tile
 constexpr int kKP = kHeadDim + 4;     // K tile pitch: float4-aligned rows
-constexpr int kPart = kHeadDim + 2;         // m, l, acc[128]
+constexpr int kPart = kHeadDim + 4;         // m, l, (2 unused), acc[128]: acc 16-byte aligned
 constexpr int kSync = 4;                    // per pair: arrivals, departures, merge ticket, merges done
 constexpr int kSelCap = 2048;               // selected rows kept in shared memory
 constexpr int kOut = (kMaxGroup * kHeadDim + kThreads - 1) / kThreads;
@@ -94,14 +104,16 @@ struct FusedArgs {
   int sink_n, local_start, local_n;
   int p0, nseg, per_block;
   int nbins, nbins_pad;
-  uint32_t off_q, off_aq, off_sel, off_hist, off_dist;  // shared memory carve-up (bytes)
+  uint32_t off_q, off_aq, off_sel, off_hist, off_dist, off_part, off_qs, off_tokw;  // shared memory (bytes)
+  int sel_cap;     // selected rows kept in shared memory
+  int spec;        // load one speculative K/V tile during the threshold exchange
   uint32_t* sync;  // [pairs][kSync]
-  uint32_t* gh;    // [pairs][nbins]: histogram of the pair (returns to zero)
+  uint32_t* gh;    // [pairs][nbins_pad]: histogram of the pair (returns to zero)
   const uint32_t* next_codes;  // nullable: codes of the next call, prefetched to L2 after the scan
   int Hkv_real, unit_div;      // KV heads of the cache; selection units per KV head
   const int32_t* n_tok_b;      // nullable [B]: tokens of each sequence (ragged batch)
   int n_sink_cfg, n_local_cfg, n_max;
-  uint32_t* cum;   // [pairs][nseg][nbins]: cumulative counts, window only
+  uint32_t* cum;   // [pairs][nseg][nbins_pad]: cumulative counts, window only
   float* part;     // [pairs][nseg][g][kPart]
   int32_t* status;
   uint64_t wait_ns;
@@ -115,19 +127,31 @@ __device__ __forceinline__ int64_t kv_row(const FusedArgs& a, int p) {
 }
 
 
-// ---- cp.async helpers (per-thread ring; each thread reads only its own slots)
-template <int W>
-__device__ __forceinline__ void cp_async_code(uint32_t* dst, const uint32_t* src) {
-  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
-  if constexpr (W == 4)
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
-  else
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(d), "l"(src) : "memory");
-}
+#ifdef HKV_TIMELINE
+// Diagnostic build only (-DHKV_TIMELINE): thread 0 of every block of the last
+// fused launch records the global timer and its SM clock at each phase
+// boundary, read back with hkv_debug_timeline.
+constexpr int kTLBlocks = 1024, kTLStamps = 24;
+__device__ unsigned long long g_hkv_tl[kTLBlocks * kTLStamps * 2];
+#define HKV_TL(i)                                                                  \
+  do {                                                                             \
+    if (threadIdx.x == 0 && blockIdx.x < kTLBlocks) {                              \
+      g_hkv_tl[(blockIdx.x * kTLStamps + (i)) * 2] = globaltimer_ns();            \
+      g_hkv_tl[(blockIdx.x * kTLStamps + (i)) * 2 + 1] = (unsigned long long)clock64(); \
+    }                                                                              \
+  } while (0)
+#else
+#define HKV_TL(i) \
+  do {            \
+  } while (0)
+#endif
+
+// ---- cp.async helpers (attention tiles) and code loads from shared memory ---
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// One code from a stage in shared memory (16- or 8-byte aligned).
 template <int W>
 __device__ __forceinline__ void load_slot(const uint32_t* sl, uint32_t (&ck)[W]) {
   if constexpr (W == 4) {
@@ -143,55 +167,53 @@ __device__ __forceinline__ void load_slot(const uint32_t* sl, uint32_t (&ck)[W])
   }
 }
 
-// In-place inclusive prefix sum over a[0, n) in shared memory.
-__device__ void block_inclusive_scan(uint32_t* a, int n, uint32_t* warp_tmp) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (n + kThreads - 1) / kThreads;
-  const int beg = min(tid * per, n), end = min(beg + per, n);
-  uint32_t s = 0;
-  for (int i = beg; i < end; ++i) s += a[i];
-  uint32_t x = s;
+__host__ __device__ constexpr int align_up_dev(int v, int a) { return (v + a - 1) / a * a; }
+
+__device__ __forceinline__ uint32_t warp_incl_u32(uint32_t x) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const uint32_t y = __shfl_up_sync(0xffffffffu, x, off);
     if (lane >= off) x += y;
   }
-  if (lane == 31) warp_tmp[warp] = x;
-  __syncthreads();
-  // totals of the warps before this one: one load per lane and a warp sum
-  uint32_t pre = lane < warp ? warp_tmp[lane] : 0u;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, off);
-  uint32_t run = x - s + pre;
-  for (int i = beg; i < end; ++i) {
-    run += a[i];
-    a[i] = run;
-  }
-  __syncthreads();
+  return x;
 }
 
-// Exclusive prefix of v over the block's threads; *total receives the sum.
-// warp_tmp: kWarps 8-byte words.
-__device__ __forceinline__ uint64_t block_exclusive(uint64_t v, uint64_t* warp_tmp, uint64_t* total) {
+// Exclusive prefix of v over the block's threads (thread order); *total
+// receives the sum.  warp_tmp: kWarps words.  Contains two barriers.
+__device__ __forceinline__ uint32_t block_excl_u32(uint32_t v, uint32_t* warp_tmp, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint64_t x = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const uint64_t y = __shfl_up_sync(0xffffffffu, x, off);
-    if (lane >= off) x += y;
-  }
+  const uint32_t x = warp_incl_u32(v);
   __syncthreads();
   if (lane == 31) warp_tmp[warp] = x;
   __syncthreads();
-  uint64_t base = 0, tot = 0;
+  uint32_t base = 0, tot = 0;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
-    const uint64_t t = warp_tmp[w];
-    base += w < warp ? t : 0ull;
+    const uint32_t t = warp_tmp[w];
+    base += w < warp ? t : 0u;
     tot += t;
   }
   *total = tot;
   return base + x - v;
+}
+
+// Cumulative counts of the histogram h[0, nbins_pad) held four bins per
+// thread: thread t owns bins [4t, 4t + 4) (h 16-byte aligned, zero past
+// nbins).  cnt receives the thread's four counts, cum the cumulative count
+// at each of its bins; returns the total.
+__device__ __forceinline__ uint32_t hist_cum4(uint4 hv, uint32_t (&cnt)[4], uint32_t (&cum)[4], uint32_t* warp_tmp) {
+  cnt[0] = hv.x;
+  cnt[1] = hv.y;
+  cnt[2] = hv.z;
+  cnt[3] = hv.w;
+  uint32_t total;
+  const uint32_t ex = block_excl_u32(hv.x + hv.y + hv.z + hv.w, warp_tmp, &total);
+  cum[0] = ex + cnt[0];
+  cum[1] = cum[0] + cnt[1];
+  cum[2] = cum[1] + cnt[2];
+  cum[3] = cum[2] + cnt[3];
+  return total;
 }
 
 // Block-wide sums of x and y; every thread receives both totals.
@@ -400,20 +422,29 @@ __device__ void attn_rows(const FusedArgs& a, int64_t kvc, int nrows, RowAt row_
   }
 }
 
-// ---- bf16 attention on the tensor cores (mma.sync m16n8k16) ------------------
-// Heads are the M dimension (g <= 16, rows >= g are zero), a 64-row tile of
-// selected tokens is N for the logits and K for P V.  K/V tiles stay bf16 in
-// shared memory (row pitch 272 bytes: conflict-free fragment loads) and are
-// fetched with cp.async, two tiles in flight.  Logits: bf16 q and K, exact
-// products, fp32 accumulation.  P V: the fp32 probabilities are split into
-// bf16 hi + lo parts (two MMAs), so P keeps 16 significant bits.
-constexpr int kKVPitch = kHeadDim + 8;           // bf16 elements per shared row
-constexpr int kKVTile = kRows * kKVPitch * 2;    // bytes per K or V tile
-constexpr int kZP = kRows + 8;                   // logit row pitch (floats)
-constexpr int kPP = kRows / 2 + 4;               // probability row pitch (bf16 pairs)
-constexpr int kQP = kHeadDim + 8;                // bf16 query row pitch (conflict-free fragment loads)
-constexpr size_t kAttnMmaBytes = 4 * (size_t)kKVTile + sizeof(float) * kMaxGroup * kZP +
-                                 2 * sizeof(uint32_t) * kMaxGroup * kPP + 2 * kMaxGroup * kQP;
+// ---- bf16 attention on the tensor cores (mma.sync m16n8k16), split by warps --
+// Each of kAW warps takes 16-row steps of the block's row list (step st =
+// warp, warp + kAW, ...), with the next step's loads in flight in its second
+// slot while it computes, and runs its own online softmax for the group's g heads
+// (heads = M, rows >= g zero): logits S = Q K^T from ldmatrix fragments
+// (bf16 q and K, exact products, fp32 sums), the running max and sum per
+// head, and P V with P taken straight from the logits' accumulator layout as
+// the A operand (split into bf16 hi + lo parts: 16 significant bits) and V
+// fragments by ldmatrix.trans.  A step's K and V rows reach the warp's own
+// shared-memory slot by cp.async; no block barrier inside the loop.  The
+// warps' partials (m, l, acc) are merged once at the end (log-sum-exp
+// rescaling, RetrievalAttention "Approach").
+constexpr int kWR = 16;                          // rows per warp step
+constexpr int kAW = 8;                           // attention warps, two slots each
+constexpr int kVP = kHeadDim + 8;                // bf16 pitch of a slot row (272 bytes: conflict-free ldmatrix)
+constexpr int kSlotBytes = 2 * kWR * kVP * 2;    // K rows then V rows of one step
+constexpr size_t kAttnWarpBytes = (size_t)2 * kAW * kSlotBytes;
+constexpr int kQP = kHeadDim + 8;                // bf16 query row pitch
+// Slot k of warp w is at (k * kAW + w) * kSlotBytes, so the first slots of
+// warps 0-3 (a speculative tile of kRows rows) come first; the compaction's
+// octet list (at most 8192 octets: 16 KB) sits in the code ring past them.
+constexpr int kCompactScratch = (kRows / kWR) * kSlotBytes;
+static_assert(kCompactScratch + 2 * 8192 <= kSlots * kThreads * 16, "compaction list inside the code ring");
 
 __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
   const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
@@ -447,192 +478,226 @@ __device__ __forceinline__ void split2(float2 x, uint32_t& hi, uint32_t& lo) {
   lo = pack_bf16(__float2bfloat16_rn(x.x - __bfloat162float(h0)), __float2bfloat16_rn(x.y - __bfloat162float(h1)));
 }
 
-// Online-softmax attention of the pair's query heads over `nrows` rows
-// (token row_at(i), or -1 to skip); writes the partial (m, l, acc) of every
-// head to dst[h * kPart ...].  Uses smem_attn (kAttnMmaBytes) and tok[2 * kRows].
-template <typename RowAt>
-__device__ void attn_mma(const FusedArgs& a, int64_t kvc, const float* aq_s, int nrows, RowAt row_at,
-                         unsigned char* smem_attn, int* tok, float* m_s, float* l_s, float* alpha_s, float* dst) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
-  const int gid = lane >> 2, tq = lane & 3;
-  const __nv_bfloat16* Kp = tptr<__nv_bfloat16>(a.K) + kvc * kHeadDim;
-  const __nv_bfloat16* Vp = tptr<__nv_bfloat16>(a.V) + kvc * kHeadDim;
-  float* z = reinterpret_cast<float*>(smem_attn + 4 * kKVTile);  // [kMaxGroup][kZP] scratch
-  float* pmax = z;                                  // [8 warps][kMaxGroup] tile maxima
-  float* psum = z + (kRows / 8) * kMaxGroup;        // [8 warps][kMaxGroup] tile sums
-  float* m_next = z + 2 * (kRows / 8) * kMaxGroup;  // [kMaxGroup]
-  // probabilities as bf16 hi and lo parts, rows of the tile in pairs: [kMaxGroup][kPP]
-  uint32_t* ph = reinterpret_cast<uint32_t*>(z + kMaxGroup * kZP);
-  uint32_t* pl = ph + kMaxGroup * kPP;
-  for (int i = tid; i < 2 * kMaxGroup * kPP; i += kThreads) ph[i] = 0u;  // heads >= g stay zero
-  // the queries as bf16 (exact: they are bf16 inputs), rows >= g zero
-  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(pl + kMaxGroup * kPP);  // [kMaxGroup][kQP]
-  for (int i = tid; i < kMaxGroup * kHeadDim; i += kThreads) {
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// The group's queries as bf16 (exact: they are bf16 inputs), rows >= g zero.
+__device__ __forceinline__ void fill_qs(int g, const float* aq_s, __nv_bfloat16* qs) {
+  for (int i = threadIdx.x; i < kMaxGroup * kHeadDim; i += kThreads) {
     const int h = i / kHeadDim, k = i % kHeadDim;
     qs[h * kQP + k] = __float2bfloat16_rn(h < g ? aq_s[h * kHeadDim + k] : 0.f);
   }
-  auto kbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem_attn + (2 * b) * kKVTile); };
-  auto vbuf = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem_attn + (2 * b + 1) * kKVTile); };
-  constexpr int CPR = kHeadDim / 8;                 // 16-byte chunks per row
-  constexpr int kPer = kRows * CPR / kThreads;      // chunks per thread per matrix
-  auto issue = [&](int r0, int b) {
+}
+
+// Rows [kWR st, kWR st + kWR) of the row list (token row_at(i), or -1) into
+// the calling warp's slot: lane l takes row l % 16 and half of its 16-byte
+// chunks of K and V (cp.async, zero-filled for skipped rows); the tokens go
+// to tokw[0, kWR).  One commit group.
+template <typename RowAt>
+__device__ __forceinline__ void warp_issue(const FusedArgs& a, int64_t kvc, int nrows, RowAt row_at, int st,
+                                           unsigned char* slot, int* tokw) {
+  const int lane = threadIdx.x & 31, r = lane & 15, hf = lane >> 4;
+  const int i = st * kWR + r;
+  const int t = i < nrows ? row_at(i) : -1;
+  if (hf == 0) tokw[r] = t;
+  const int64_t row = kvc + (t >= 0 ? t : 0);
+  const __nv_bfloat16* Kp = tptr<__nv_bfloat16>(a.K) + row * kHeadDim;
+  const __nv_bfloat16* Vp = tptr<__nv_bfloat16>(a.V) + row * kHeadDim;
+  __nv_bfloat16* ks = reinterpret_cast<__nv_bfloat16*>(slot) + r * kVP;
+  __nv_bfloat16* vs = ks + kWR * kVP;
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = tid + u * kThreads, r = i / CPR, c = i % CPR;
-      const int t = r0 + r < nrows ? row_at(r0 + r) : -1;
-      if (c == 0) tok[b * kRows + r] = t;
-      const int64_t off = (int64_t)(t >= 0 ? t : 0) * kHeadDim + c * 8;
-      cp_async16_zfill(kbuf(b) + r * kKVPitch + c * 8, Kp + off, t >= 0);
-      cp_async16_zfill(vbuf(b) + r * kKVPitch + c * 8, Vp + off, t >= 0);
-    }
-    cp_async_commit();
-  };
-  if (tid < g) {
-    m_s[tid] = -INFINITY;
-    l_s[tid] = 0.f;
+  for (int c = 0; c < 8; ++c) {
+    const int col = (hf * 8 + c) * 8;
+    cp_async16_zfill(ks + col, Kp + col, t >= 0);
+    cp_async16_zfill(vs + col, Vp + col, t >= 0);
   }
-  float o[4] = {0.f, 0.f, 0.f, 0.f};  // P V accumulator: heads gid, gid + 8; dims 8 warp + 2 tq (+1)
-  if (nrows > 0) issue(0, 0);
-  for (int r0 = 0, it = 0; r0 < nrows; r0 += kRows, ++it) {
-    const int b = it & 1, nr = min(kRows, nrows - r0);
-    if (r0 + kRows < nrows) {
-      issue(r0 + kRows, b ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const __nv_bfloat16* Ks = kbuf(b);
-    const __nv_bfloat16* Vs = vbuf(b);
-    const int* tk = tok + b * kRows;
-    // logits of rows 8 w + 2 tq (+1) for heads gid and gid + 8 (warps 0..7),
-    // then the tile maximum of each head through shared memory, and the
-    // probabilities straight from the registers: no separate softmax pass
-    float s00 = -INFINITY, s01 = -INFINITY, s10 = -INFINITY, s11 = -INFINITY;
-    if (warp < kRows / 8) {
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-      const __nv_bfloat16* kr = Ks + (warp * 8 + gid) * kKVPitch + 2 * tq;
-      const __nv_bfloat16* q0 = qs + gid * kQP + 2 * tq;
-      const __nv_bfloat16* q1 = qs + (gid + 8) * kQP + 2 * tq;
+  cp_async_commit();
+}
+
+// One 16-row step of the calling warp's online softmax.  m, l: running max
+// and (this lane's part of the) sum of heads gid and gid + 8; o[n]: P V
+// accumulator fragments of output columns [8 n, 8 n + 8).
+__device__ __forceinline__ void warp_step(const unsigned char* slot, const int* tokw, const __nv_bfloat16* qs,
+                                          float scale, float (&m)[2], float (&l)[2], float (&o)[16][4]) {
+  const int lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
+  const __nv_bfloat16* ks = reinterpret_cast<const __nv_bfloat16*>(slot);
+  const __nv_bfloat16* vs = ks + kWR * kVP;
+  const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: this lane addresses row mr of matrix mi
+  // logits of rows [0, 8) (n-block 0) and [8, 16) (n-block 1)
+  float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  const uint32_t qa = smem_addr(qs + ((mi & 1) * 8 + mr) * kQP + (mi >> 1) * 8);
+  const uint32_t ka0 = smem_addr(ks + mr * kVP + mi * 8);
+  const uint32_t ka1 = smem_addr(ks + (8 + mr) * kVP + mi * 8);
 #pragma unroll
-      for (int ks = 0; ks < kHeadDim / 16; ++ks) {
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr + ks * 16);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + ks * 16 + 8);
-        const uint32_t a0 = *reinterpret_cast<const uint32_t*>(q0 + ks * 16);
-        const uint32_t a1 = *reinterpret_cast<const uint32_t*>(q1 + ks * 16);
-        const uint32_t a2 = *reinterpret_cast<const uint32_t*>(q0 + ks * 16 + 8);
-        const uint32_t a3 = *reinterpret_cast<const uint32_t*>(q1 + ks * 16 + 8);
-        mma16816(c, a0, a1, a2, a3, b0, b1);
+  for (int k0 = 0; k0 < kHeadDim; k0 += 32) {
+    uint32_t a0[4], a1[4], b0[4], b1[4];
+    ldsm_x4(qa + 2 * k0, a0);
+    ldsm_x4(qa + 2 * (k0 + 16), a1);
+    ldsm_x4(ka0 + 2 * k0, b0);  // rows 0-7: k-step k0 (b0[0], b0[1]) and k0 + 16 (b0[2], b0[3])
+    ldsm_x4(ka1 + 2 * k0, b1);
+    mma16816(s[0], a0[0], a0[1], a0[2], a0[3], b0[0], b0[1]);
+    mma16816(s[1], a0[0], a0[1], a0[2], a0[3], b1[0], b1[1]);
+    mma16816(s[0], a1[0], a1[1], a1[2], a1[3], b0[2], b0[3]);
+    mma16816(s[1], a1[0], a1[1], a1[2], a1[3], b1[2], b1[3]);
+  }
+  // rows of this lane: 2 tq, 2 tq + 1 (n-block 0), 8 + 2 tq, 9 + 2 tq (n-block 1)
+  const bool v00 = tokw[2 * tq] >= 0, v01 = tokw[2 * tq + 1] >= 0;
+  const bool v10 = tokw[8 + 2 * tq] >= 0, v11 = tokw[9 + 2 * tq] >= 0;
+  s[0][0] = v00 ? s[0][0] * scale : -INFINITY;
+  s[0][1] = v01 ? s[0][1] * scale : -INFINITY;
+  s[0][2] = v00 ? s[0][2] * scale : -INFINITY;
+  s[0][3] = v01 ? s[0][3] * scale : -INFINITY;
+  s[1][0] = v10 ? s[1][0] * scale : -INFINITY;
+  s[1][1] = v11 ? s[1][1] * scale : -INFINITY;
+  s[1][2] = v10 ? s[1][2] * scale : -INFINITY;
+  s[1][3] = v11 ? s[1][3] * scale : -INFINITY;
+  float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+  float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+  const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+  const float al0 = mn0 == -INFINITY ? 1.f : expf(m[0] - mn0);
+  const float al1 = mn1 == -INFINITY ? 1.f : expf(m[1] - mn1);
+  auto ex = [](float z, float mx) { return z == -INFINITY ? 0.f : expf(z - mx); };
+  float p[2][4];
+#pragma unroll
+  for (int nb = 0; nb < 2; ++nb) {
+    p[nb][0] = ex(s[nb][0], mn0);
+    p[nb][1] = ex(s[nb][1], mn0);
+    p[nb][2] = ex(s[nb][2], mn1);
+    p[nb][3] = ex(s[nb][3], mn1);
+  }
+  l[0] = fmaf(l[0], al0, (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]));
+  l[1] = fmaf(l[1], al1, (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]));
+  m[0] = mn0;
+  m[1] = mn1;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) {
+    o[n][0] *= al0;
+    o[n][1] *= al0;
+    o[n][2] *= al1;
+    o[n][3] *= al1;
+  }
+  // P as the A operand over the step's 16 rows: (head gid, rows 2 tq..), (gid + 8, ..),
+  // (gid, 8 + 2 tq..), (gid + 8, 8 + 2 tq..)
+  uint32_t ph[4], pl[4];
+  split2(make_float2(p[0][0], p[0][1]), ph[0], pl[0]);
+  split2(make_float2(p[0][2], p[0][3]), ph[1], pl[1]);
+  split2(make_float2(p[1][0], p[1][1]), ph[2], pl[2]);
+  split2(make_float2(p[1][2], p[1][3]), ph[3], pl[3]);
+  const uint32_t va = smem_addr(vs + ((mi & 1) * 8 + mr) * kVP + (mi >> 1) * 8);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {  // output columns [16 j, 16 j + 16)
+    uint32_t bv[4];
+    ldsm_x4_trans(va + 2 * 16 * j, bv);
+    mma16816(o[2 * j], ph[0], ph[1], ph[2], ph[3], bv[0], bv[1]);
+    mma16816(o[2 * j], pl[0], pl[1], pl[2], pl[3], bv[0], bv[1]);
+    mma16816(o[2 * j + 1], ph[0], ph[1], ph[2], ph[3], bv[2], bv[3]);
+    mma16816(o[2 * j + 1], pl[0], pl[1], pl[2], pl[3], bv[2], bv[3]);
+  }
+}
+
+// Online-softmax attention of the pair's g query heads over `nrows` rows
+// (token row_at(i), or -1 to skip); writes the partial (m, l, acc) of every
+// head to dst[h * kPart ...].  slots: kAttnWarpBytes of shared memory (also
+// the merge scratch at the end); tokw: kWarps * kWR ints; qs: the bf16
+// queries (fill_qs).  pre: the first step of warps [0, pre_steps) was already
+// issued (warp_issue with this row_at) and tokw entries may since have been
+// set to -1 for rows to skip.  Starts and ends with a block barrier.
+template <typename RowAt>
+__device__ void attn_warps(const FusedArgs& a, int64_t kvc, int nrows, RowAt row_at, unsigned char* slots, int* tokw,
+                           const __nv_bfloat16* qs, float* dst, int pre_steps) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, tq = lane & 3, g = a.g;
+  auto slot = [&](int k) { return slots + (size_t)(k * kAW + warp) * kSlotBytes; };
+  auto tw = [&](int k) { return tokw + (k * kAW + warp) * kWR; };
+  __syncthreads();  // qs and any earlier use of the slots
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+  float o[16][4];
+#pragma unroll
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  const int nsteps = (nrows + kWR - 1) / kWR;
+  if (warp < kAW) {
+    // step j of this warp is st = warp + j kAW, in slot j % 2
+    if (warp >= pre_steps && warp < nsteps) warp_issue(a, kvc, nrows, row_at, warp, slot(0), tw(0));
+    for (int j = 0, st = warp; st < nsteps; ++j, st += kAW) {
+      const int nx = st + kAW;
+      if (nx < nsteps) {
+        warp_issue(a, kvc, nrows, row_at, nx, slot((j + 1) & 1), tw((j + 1) & 1));
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
       }
-      const int r = warp * 8 + 2 * tq;
-      const bool v0 = r < nr && tk[r] >= 0, v1 = r + 1 < nr && tk[r + 1] >= 0;
+      __syncwarp();
+      warp_step(slot(j & 1), tw(j & 1), qs, a.scale, m, l, o);
+      __syncwarp();  // slot j % 2 is refilled next
+    }
+  }
+  HKV_TL(19);
+  l[0] += __shfl_xor_sync(0xffffffffu, l[0], 1);
+  l[0] += __shfl_xor_sync(0xffffffffu, l[0], 2);
+  l[1] += __shfl_xor_sync(0xffffffffu, l[1], 1);
+  l[1] += __shfl_xor_sync(0xffffffffu, l[1], 2);
+  __syncthreads();  // every warp is done with its slots: they become the merge scratch
+  float* wp = reinterpret_cast<float*>(slots);   // [kAW][g][kPart]
+  float* wts = wp + (size_t)kAW * g * kPart;     // [kAW][kMaxGroup] weights
+  float* ML = wts + kAW * kMaxGroup;             // [g][2]: M, L
+  if (warp < kAW) {
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      if (gid < g) *reinterpret_cast<float2*>(wp + ((size_t)warp * g + gid) * kPart + 4 + 8 * n + 2 * tq) = make_float2(o[n][0], o[n][1]);
+      if (gid + 8 < g)
+        *reinterpret_cast<float2*>(wp + ((size_t)warp * g + gid + 8) * kPart + 4 + 8 * n + 2 * tq) = make_float2(o[n][2], o[n][3]);
+    }
+    if (tq == 0) {
       if (gid < g) {
-        s00 = v0 ? c[0] * a.scale : -INFINITY;
-        s01 = v1 ? c[1] * a.scale : -INFINITY;
+        wp[((size_t)warp * g + gid) * kPart] = m[0];
+        wp[((size_t)warp * g + gid) * kPart + 1] = l[0];
       }
       if (gid + 8 < g) {
-        s10 = v0 ? c[2] * a.scale : -INFINITY;
-        s11 = v1 ? c[3] * a.scale : -INFINITY;
-      }
-      float mx0 = fmaxf(s00, s01), mx1 = fmaxf(s10, s11);
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      if (tq == 0) {
-        pmax[warp * kMaxGroup + gid] = mx0;
-        pmax[warp * kMaxGroup + gid + 8] = mx1;
+        wp[((size_t)warp * g + gid + 8) * kPart] = m[1];
+        wp[((size_t)warp * g + gid + 8) * kPart + 1] = l[1];
       }
     }
-    __syncthreads();
-    if (warp < kRows / 8) {
-      float t0 = -INFINITY, t1 = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kRows / 8; ++w) {
-        t0 = fmaxf(t0, pmax[w * kMaxGroup + gid]);
-        t1 = fmaxf(t1, pmax[w * kMaxGroup + gid + 8]);
-      }
-      const float mo0 = m_s[gid < g ? gid : 0], mo1 = m_s[gid + 8 < g ? gid + 8 : 0];
-      const float mn0 = fmaxf(mo0, t0), mn1 = fmaxf(mo1, t1);
-      const float e00 = s00 == -INFINITY ? 0.f : expf(s00 - mn0), e01 = s01 == -INFINITY ? 0.f : expf(s01 - mn0);
-      const float e10 = s10 == -INFINITY ? 0.f : expf(s10 - mn1), e11 = s11 == -INFINITY ? 0.f : expf(s11 - mn1);
-      const int pr = warp * 4 + tq;  // pair index of rows 8 w + 2 tq, + 1
-      uint32_t hi, lo;
-      if (gid < g) {
-        split2(make_float2(e00, e01), hi, lo);
-        ph[gid * kPP + pr] = hi;
-        pl[gid * kPP + pr] = lo;
-      }
-      if (gid + 8 < g) {
-        split2(make_float2(e10, e11), hi, lo);
-        ph[(gid + 8) * kPP + pr] = hi;
-        pl[(gid + 8) * kPP + pr] = lo;
-      }
-      float ps0 = e00 + e01, ps1 = e10 + e11;
-      ps0 += __shfl_xor_sync(0xffffffffu, ps0, 1);
-      ps0 += __shfl_xor_sync(0xffffffffu, ps0, 2);
-      ps1 += __shfl_xor_sync(0xffffffffu, ps1, 1);
-      ps1 += __shfl_xor_sync(0xffffffffu, ps1, 2);
-      if (tq == 0) {
-        psum[warp * kMaxGroup + gid] = ps0;
-        psum[warp * kMaxGroup + gid + 8] = ps1;
-        if (warp == 0) {
-          m_next[gid] = mn0;
-          m_next[gid + 8] = mn1;
-          alpha_s[gid] = mn0 == -INFINITY ? 1.f : expf(mo0 - mn0);
-          alpha_s[gid + 8] = mn1 == -INFINITY ? 1.f : expf(mo1 - mn1);
-        }
-      }
-    }
-    __syncthreads();
-    if (tid < g) {
-      // running (m, l) of head tid; nothing reads them again before the next tile's second barrier
-      float ls = 0.f;
-#pragma unroll
-      for (int w = 0; w < kRows / 8; ++w) ls += psum[w * kMaxGroup + tid];
-      l_s[tid] = l_s[tid] * alpha_s[tid] + ls;
-      m_s[tid] = m_next[tid];
-    }
-    {
-      // warp w: output dims [8w, 8w + 8)
-      const float al0 = gid < g ? alpha_s[gid] : 1.f, al1 = gid + 8 < g ? alpha_s[gid + 8] : 1.f;
-      o[0] *= al0;
-      o[1] *= al0;
-      o[2] *= al1;
-      o[3] *= al1;
-      const uint32_t vrow = static_cast<uint32_t>(__cvta_generic_to_shared(Vs)) + (uint32_t)(warp * 8 * 2);
-#pragma unroll
-      for (int kp = 0; kp < kRows / 32; ++kp) {
-        uint32_t bv[4];  // B fragments of k-steps 2 kp and 2 kp + 1 (rows 32 kp + lane)
-        ldsm_x4_trans(vrow + (uint32_t)((kp * 32 + lane) * kKVPitch * 2), bv);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int c0 = (2 * kp + half) * 8 + tq;  // pair index of rows 16 ks + 2 tq
-          const uint32_t* h0 = ph + gid * kPP + c0;
-          const uint32_t* h1 = ph + (gid + 8) * kPP + c0;
-          const uint32_t* l0 = pl + gid * kPP + c0;
-          const uint32_t* l1 = pl + (gid + 8) * kPP + c0;
-          mma16816(o, h0[0], h1[0], h0[4], h1[4], bv[2 * half], bv[2 * half + 1]);
-          mma16816(o, l0[0], l1[0], l0[4], l1[4], bv[2 * half], bv[2 * half + 1]);
-        }
-      }
-    }
-    __syncthreads();  // buffer b is refilled by the next iteration's issue
   }
-  // partial of every head: m, l, acc[128]
-  const int c0 = warp * 8 + 2 * tq;
-  if (gid < g) {
-    dst[gid * kPart + 2 + c0] = o[0];
-    dst[gid * kPart + 2 + c0 + 1] = o[1];
+  __syncthreads();
+  HKV_TL(20);
+  if (tid < kAW * g) {  // weight of warp w for head h
+    const int w = tid / g, h = tid % g;
+    float M = -INFINITY;
+#pragma unroll
+    for (int v = 0; v < kAW; ++v) M = fmaxf(M, wp[((size_t)v * g + h) * kPart]);
+    const float mw = wp[((size_t)w * g + h) * kPart];
+    wts[w * kMaxGroup + h] = mw == -INFINITY ? 0.f : expf(mw - M);
+    if (w == 0) ML[2 * h] = M;
   }
-  if (gid + 8 < g) {
-    dst[(gid + 8) * kPart + 2 + c0] = o[2];
-    dst[(gid + 8) * kPart + 2 + c0 + 1] = o[3];
-  }
+  __syncthreads();
   if (tid < g) {
-    dst[tid * kPart + 0] = m_s[tid];
-    dst[tid * kPart + 1] = l_s[tid];
+    float L = 0.f;
+#pragma unroll
+    for (int v = 0; v < kAW; ++v) L = fmaf(wp[((size_t)v * g + tid) * kPart + 1], wts[v * kMaxGroup + tid], L);
+    ML[2 * tid + 1] = L;
   }
+  for (int i = tid; i < g * kHeadDim; i += kThreads) {
+    const int h = i / kHeadDim, c = i % kHeadDim;
+    float O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAW; ++w) O = fmaf(wp[((size_t)w * g + h) * kPart + 4 + c], wts[w * kMaxGroup + h], O);
+    dst[h * kPart + 4 + c] = O;
+  }
+  __syncthreads();  // ML (L of every head) is complete
+  if (tid < g) {
+    dst[tid * kPart] = ML[2 * tid];
+    dst[tid * kPart + 1] = ML[2 * tid + 1];
+  }
+  __syncthreads();
 }
 
 __device__ void attn_end(int g, const AttnSmem& sm, const float (&acc)[kOut], float* dst) {
@@ -643,7 +708,7 @@ __device__ void attn_end(int g, const AttnSmem& sm, const float (&acc)[kOut], fl
     const int o = tid + j * kThreads;
     if (o < g * kHeadDim) {
       const int h = o / kHeadDim, c = o % kHeadDim;
-      dst[h * kPart + 2 + c] = acc[j];
+      dst[h * kPart + 4 + c] = acc[j];
       if (c == 0) {
         dst[h * kPart + 0] = sm.m[h];
         dst[h * kPart + 1] = sm.l[h];
@@ -652,64 +717,237 @@ __device__ void attn_end(int g, const AttnSmem& sm, const float (&acc)[kOut], fl
   }
 }
 
-// Merge head h of pair p over its nseg partials into out / lse.  Thread t
-// takes column t % 128 of the partials s = t / 128 (mod 4) and folds them
-// into a running (M, L, O) by log-sum-exp rescaling; all loads of a batch are
-// issued before any is used.  The four column groups are then combined.
-// red_s: 3 * kThreads floats of shared scratch.
-__device__ void merge_head(const FusedArgs& a, int p, int nseg, int h, float* red_s) {
-  constexpr int kQ = kThreads / kHeadDim, kB = 16;
-  const int tid = threadIdx.x, g = a.g, c = tid % kHeadDim, q = tid / kHeadDim;
-  const float* parts = a.part + (int64_t)p * nseg * g * kPart;
-  float M = -INFINITY, L = 0.f, O = 0.f;
-  for (int s0 = q; s0 < nseg; s0 += kB * kQ) {
-    float2 ml[kB];
-    float x[kB];
+// Merge of the nseg partials of query head h of pair p into out / lse
+// (RetrievalAttention, "Approach": exact log-sum-exp rescaling):
+//   M = max_s m_s,  w_s = e^{m_s - M},  L = sum_s l_s w_s,
+//   out = sum_s acc_s w_s / L,  lse = M + log L.
+// Thread (q, c) sums w_s acc_s[c] over s = q, q + 4, ...; its first batch of
+// loads is issued before the weights are known; warp 0 computes the weights
+// once.
+// scratch: nseg + 4 * kThreads + 2 floats of shared memory.
+// (Not inlined, with scalar arguments: keeps the fused kernel's registers
+// for its main loop.)
+__device__ __noinline__ void merge_head(const float* part, float* out, float* lse, int Hq, int Hkv, int g, int p,
+                                        int nseg, int h, float* scratch) {
+  constexpr int kQ = kThreads / kHeadDim;  // segment groups
+  constexpr int kB = 12;                   // segments per thread and batch (48 segments in one batch)
+  const int tid = threadIdx.x, lane = tid & 31, c = tid % kHeadDim, q = tid / kHeadDim;
+  float* w_s = scratch;                  // [nseg]
+  float* red_s = scratch + nseg;         // [kThreads]
+  float* ML_s = red_s + kThreads;        // M, L
+  const float* parts = part + (int64_t)p * nseg * g * kPart + (int64_t)h * kPart;
+  const int64_t sstride = (int64_t)g * kPart;
+  float x[kB];
+#pragma unroll
+  for (int u = 0; u < kB; ++u) {
+    const int s = q + u * kQ;
+    x[u] = s < nseg ? __ldcg(parts + s * sstride + 4 + c) : 0.f;
+  }
+  if (tid < 32) {
+    float M = -INFINITY;
+    float2 ml[(kMaxSegsPerPair + 31) / 32];
+#pragma unroll
+    for (int u = 0; u < (kMaxSegsPerPair + 31) / 32; ++u) {
+      const int s = lane + 32 * u;
+      ml[u] = s < nseg ? __ldcg(reinterpret_cast<const float2*>(parts + s * sstride)) : make_float2(-INFINITY, 0.f);
+      M = fmaxf(M, ml[u].x);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+#pragma unroll
+    for (int u = 0; u < (kMaxSegsPerPair + 31) / 32; ++u) {
+      const int s = lane + 32 * u;
+      const float w = ml[u].x == -INFINITY ? 0.f : expf(ml[u].x - M);
+      if (s < nseg) w_s[s] = w;
+      L = fmaf(ml[u].y, w, L);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (lane == 0) {
+      ML_s[0] = M;
+      ML_s[1] = L;
+    }
+  }
+  __syncthreads();
+  float o = 0.f;
+  for (int s0 = q;; s0 += kB * kQ) {
 #pragma unroll
     for (int u = 0; u < kB; ++u) {
       const int s = s0 + u * kQ;
-      ml[u] = make_float2(-INFINITY, 0.f);
-      x[u] = 0.f;
-      if (s < nseg) {
-        const float* src = parts + ((int64_t)s * g + h) * kPart;
-        ml[u] = __ldcg(reinterpret_cast<const float2*>(src));
-        x[u] = __ldcg(src + 2 + c);
-      }
+      if (s < nseg) o = fmaf(x[u], w_s[s], o);
     }
+    if (s0 + kB * kQ >= nseg) break;
 #pragma unroll
     for (int u = 0; u < kB; ++u) {
-      if (ml[u].x == -INFINITY) continue;
-      const float mn = fmaxf(M, ml[u].x);
-      const float a1 = M == -INFINITY ? 0.f : expf(M - mn), a2 = expf(ml[u].x - mn);
-      L = fmaf(L, a1, ml[u].y * a2);
-      O = fmaf(O, a1, x[u] * a2);
-      M = mn;
+      const int s = s0 + kB * kQ + u * kQ;
+      x[u] = s < nseg ? __ldcg(parts + s * sstride + 4 + c) : 0.f;
     }
   }
-  red_s[tid] = M;
-  red_s[kThreads + tid] = L;
-  red_s[2 * kThreads + tid] = O;
+  red_s[tid] = o;
   __syncthreads();
   if (tid < kHeadDim) {
-    float Mt = -INFINITY;
+    float O = 0.f;
 #pragma unroll
-    for (int j = 0; j < kQ; ++j) Mt = fmaxf(Mt, red_s[j * kHeadDim + tid]);
-    float Lt = 0.f, Ot = 0.f;
-    if (Mt != -INFINITY) {
-#pragma unroll
-      for (int j = 0; j < kQ; ++j) {
-        const float mj = red_s[j * kHeadDim + tid];
-        const float w = mj == -INFINITY ? 0.f : expf(mj - Mt);
-        Lt = fmaf(red_s[kThreads + j * kHeadDim + tid], w, Lt);
-        Ot = fmaf(red_s[2 * kThreads + j * kHeadDim + tid], w, Ot);
-      }
-    }
-    const int b = p / a.Hkv, kvh = p % a.Hkv;
-    const int64_t orow = (int64_t)b * a.Hq + (int64_t)kvh * g + h;
-    a.out[orow * kHeadDim + tid] = Lt > 0.f ? Ot / Lt : 0.f;
-    if (tid == 0 && a.lse != nullptr) a.lse[orow] = Lt > 0.f ? Mt + logf(Lt) : -INFINITY;
+    for (int j = 0; j < kQ; ++j) O += red_s[j * kHeadDim + tid];
+    const float M = ML_s[0], L = ML_s[1];
+    const int b = p / Hkv, kvh = p % Hkv;
+    const int64_t orow = (int64_t)b * Hq + (int64_t)kvh * g + h;
+    out[orow * kHeadDim + tid] = L > 0.f ? O / L : 0.f;
+    if (tid == 0 && lse != nullptr) lse[orow] = L > 0.f ? M + logf(L) : -INFINITY;
   }
   __syncthreads();
+}
+
+// out / lse of every query head of pair p from the block's own partial (one
+// block per pair): out = acc / l, lse = m + log l.
+__device__ void finish_single(const FusedArgs& a, int p, const float* part_s) {
+  const int g = a.g;
+  const int b = p / a.Hkv, kvh = p % a.Hkv;
+  for (int o = threadIdx.x; o < g * 32; o += kThreads) {
+    const int h = o >> 5, c4 = o & 31;
+    const float* src = part_s + h * kPart;
+    const float l = src[1];
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const float4 x = reinterpret_cast<const float4*>(src + 4)[c4];
+    const int64_t orow = (int64_t)b * a.Hq + (int64_t)kvh * g + h;
+    *reinterpret_cast<float4*>(a.out + orow * kHeadDim + 4 * c4) = make_float4(x.x * inv, x.y * inv, x.z * inv, x.w * inv);
+    if (c4 == 0 && a.lse != nullptr) a.lse[orow] = l > 0.f ? src[0] + logf(l) : -INFINITY;
+  }
+}
+
+// Exclusive prefix over the warp's lanes of a per-lane count x in [0, 16),
+// and its warp total, from one ballot per bit (no shuffle chain).
+__device__ __forceinline__ void warp_prefix4(uint32_t x, uint32_t& excl, uint32_t& total) {
+  const uint32_t lt = lanemask_lt();
+  excl = total = 0u;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t m = __ballot_sync(0xffffffffu, (x >> b) & 1u);
+    excl += (uint32_t)__popc(m & lt) << b;
+    total += (uint32_t)__popc(m) << b;
+  }
+}
+
+// Ordered compaction of the block's distances dist_s[0, len): emits, in
+// ascending index order, every i with D < thr and the first `quota` with
+// D == thr, as emit(pos, i, D) with pos the rank among the emitted ones;
+// returns their number.  The unit of work is an octet: 8 consecutive
+// distances, one 16-byte load.
+//  1. thread t takes a contiguous run of octets (read in a rotated order, so
+//     a warp's loads hit distinct banks) and flags those whose smallest
+//     distance is <= thr; one block prefix lists the flagged octets in
+//     ascending order;
+//  2. warp w takes a contiguous run of listed octets, 32 at a time (one per
+//     lane), and sums the lanes' counts below and at thr;
+//  3. the warps' totals give each warp its base, and the warps emit their
+//     octets' tokens, ranked by ballot prefix sums of the per-lane counts.
+// scratch: 2 bytes per octet of shared memory; dist_s readable 8 entries past
+// len.  All threads call it (four barriers).
+template <typename Emit>
+__device__ uint32_t compact_block(const uint16_t* dist_s, int len, int thr, uint32_t quota, uint32_t* warp_tmp,
+                                  unsigned char* scratch, Emit emit) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int noct = (len + 7) >> 3;
+  uint16_t* olist = reinterpret_cast<uint16_t*>(scratch);  // [noct]
+  const uint32_t t = (uint32_t)thr;
+  auto oct_min = [](const uint4& v) {
+    const uint32_t m = __vminu2(__vminu2(v.x, v.y), __vminu2(v.z, v.w));
+    return min(m & 0xffffu, m >> 16);
+  };
+  // counts below and at thr among the octet's tokens [8 o, 8 o + 8) that are < len
+  auto count8 = [&](const uint4& v, int o, uint32_t& lt, uint32_t& eq) {
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+    lt = eq = 0u;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t D = (wd[e >> 1] >> (16 * (e & 1))) & 0xffffu;
+      const bool in = 8 * o + e < len;
+      lt += (in && D < t) ? 1u : 0u;
+      eq += (in && D == t) ? 1u : 0u;
+    }
+  };
+  // 1. listed octets
+  int R = 1;  // octets per thread: a power of two (<= 16 for 65536 tokens)
+  while (R * kThreads < noct) R <<= 1;
+  const int o0 = tid * R;
+  uint32_t fl = 0, nf = 0;
+  for (int j = 0; j < R; ++j) {
+    const int r = (j + tid) & (R - 1), o = o0 + r;
+    if (o < noct && oct_min(*reinterpret_cast<const uint4*>(dist_s + 8 * o)) <= t) {
+      fl |= 1u << r;
+      ++nf;
+    }
+  }
+  uint32_t nlist;
+  uint32_t pos = block_excl_u32(nf, warp_tmp, &nlist);
+  for (int r = 0; r < R; ++r)
+    if ((fl >> r) & 1u) olist[pos++] = (uint16_t)(o0 + r);
+  __syncthreads();
+  HKV_TL(16);
+  // 2. counts of each warp's run of listed octets
+  const int per = ((int)nlist + kWarps - 1) / kWarps;
+  const int f0 = min(warp * per, (int)nlist), f1 = min(f0 + per, (int)nlist);
+  uint32_t wl = 0, we = 0;
+  for (int f = f0 + lane; f < f1; f += 32) {
+    const int o = olist[f];
+    uint32_t lt, eq;
+    count8(*reinterpret_cast<const uint4*>(dist_s + 8 * o), o, lt, eq);
+    wl += lt;
+    we += eq;
+  }
+  wl = __reduce_add_sync(0xffffffffu, wl);
+  we = __reduce_add_sync(0xffffffffu, we);
+  if (lane == 0) {
+    warp_tmp[kWarps + warp] = wl;
+    warp_tmp[2 * kWarps + warp] = we;
+  }
+  __syncthreads();
+  HKV_TL(17);
+  uint32_t run_lt = 0, run_eq = 0, tot_lt = 0, tot_eq = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const uint32_t x = warp_tmp[kWarps + w], y = warp_tmp[2 * kWarps + w];
+    run_lt += w < warp ? x : 0u;
+    run_eq += w < warp ? y : 0u;
+    tot_lt += x;
+    tot_eq += y;
+  }
+  HKV_TL(18);
+  // 3. emit
+  for (int fb = f0; fb < f1; fb += 32) {
+    const int f = fb + lane;
+    const bool live = f < f1;
+    const int o = live ? olist[f] : 0;
+    const uint4 v = live ? *reinterpret_cast<const uint4*>(dist_s + 8 * o) : make_uint4(~0u, ~0u, ~0u, ~0u);
+    uint32_t lt, eq;
+    count8(v, o, lt, eq);
+    if (!live) lt = eq = 0u;
+    uint32_t ex_lt, ex_eq, row_lt, row_eq;
+    warp_prefix4(lt, ex_lt, row_lt);
+    warp_prefix4(eq, ex_eq, row_eq);
+    if (lt | eq) {
+      uint32_t bl = run_lt + ex_lt, be = run_eq + ex_eq;
+      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t D = (wd[e >> 1] >> (16 * (e & 1))) & 0xffffu;
+        const int i = 8 * o + e;
+        if (i >= len) continue;
+        if (D < t) {
+          emit(bl + min(be, quota), i, (int)D);
+          ++bl;
+        } else if (D == t) {
+          if (be < quota) emit(bl + be, i, (int)D);
+          ++be;
+        }
+      }
+    }
+    run_lt += row_lt;
+    run_eq += row_eq;
+  }
+  __syncthreads();  // warp_tmp and the list are free again
+  return tot_lt + min(tot_eq, quota);
 }
 
 // ------------------------------------------------- query encoding (in kernel)
@@ -817,19 +1055,30 @@ __device__ void project_f32_simt(const float* x0, int64_t x_stride, int rows, co
 }
 
 // ------------------------------------------------------------------ kernel
+template <int W>
+__device__ __forceinline__ void cp_async_code(uint32_t* dst, const uint32_t* src) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  if constexpr (W == 4)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(d), "l"(src) : "memory");
+}
+
 // Block b serves pair p0 + b / nseg and its candidate range
 // [s0, s1) = [(b % nseg) * per_block, ...): no block straddles two pairs.
 template <int W, int NP, bool ATTEND, typename T>
 __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t* ring = reinterpret_cast<uint32_t*>(smem);
+  extern __shared__ __align__(128) unsigned char smem[];
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + a.off_hist);
   uint16_t* dist_s = reinterpret_cast<uint16_t*>(smem + a.off_dist);
   int32_t* sel_s = reinterpret_cast<int32_t*>(smem + a.off_sel);
   float* aq_s = reinterpret_cast<float*>(smem + a.off_aq);  // [g][128] attention queries (fp32)
+  unsigned char* cscratch = smem + kCompactScratch;  // compaction lists (in the code ring, free by then)
+  __nv_bfloat16* qs_s = reinterpret_cast<__nv_bfloat16*>(smem + a.off_qs);  // [kMaxGroup][kQP] bf16 queries
+  int* tokw_s = reinterpret_cast<int*>(smem + a.off_tokw);                    // [2][kAW][kWR] rows of the warp steps
   __shared__ uint32_t qc_s[kMaxGroup * W];
-  __shared__ __align__(8) uint32_t warp_tmp[2 * kWarps];
-  __shared__ int sh[8];
+  __shared__ __align__(8) uint32_t warp_tmp[3 * kWarps];
+  __shared__ int sh[12];
   __shared__ float m_s[kMaxGroup], l_s[kMaxGroup], alpha_s[kMaxGroup];
   __shared__ int tok_s[2 * kRows];
 
@@ -845,6 +1094,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   // at once).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  HKV_TL(0);
   // this pair's window: uniform, or from its sequence's own length
   int lo = a.lo, C = a.C, k_eff_p = a.k_eff, sink_n = a.sink_n, local_start = a.local_start,
       local_n = a.local_n;
@@ -863,12 +1113,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   }
   const int s0 = seg * a.per_block, s1 = min(s0 + a.per_block, C);
   const int len = max(s1 - s0, 0);
-  const int nt = tid < len ? (len - tid + kThreads - 1) / kThreads : 0;
   uint32_t* sync = a.sync + kSync * p;
-  (void)aq_s;
 
   // ---------------- phase A: small loads first, then the code stream ------
-  // Loads issued before the code prefetch are ahead of it in the memory queues.
+  // Each thread streams its codes (tokens tid, tid + kThreads, ...) through a
+  // private ring of kSlots cp.async slots, two codes per commit group.
+  // Loads issued before the code stream are ahead of it in the memory queues.
+  const int nt = tid < len ? (len - tid + kThreads - 1) / kThreads : 0;
   const int gw = a.g * W;
   const int b = p / a.Hkv, kvh = p % a.Hkv;
   const int64_t qrow0 = (int64_t)b * a.Hq + (int64_t)kvh * a.g;  // first query head of the pair
@@ -883,6 +1134,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   float4 aq = make_float4(0.f, 0.f, 0.f, 0.f);
   if (ATTEND && tid < a.g * (kHeadDim / 4))
     aq = load4_f32(tptr<T>(a.q) + qrow0 * kHeadDim + (tid / (kHeadDim / 4)) * kHeadDim + (tid % (kHeadDim / 4)) * 4);
+  uint32_t* ring = reinterpret_cast<uint32_t*>(smem);
   const uint32_t* pf_ptr = a.k_codes + (kvc + lo + s0 + tid) * W;
   constexpr int64_t kStep = (int64_t)kThreads * W;
   auto slot = [&](int k) { return ring + ((size_t)(k % kSlots) * kThreads + tid) * 4; };
@@ -891,14 +1143,18 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     if (k < nt) cp_async_code<W>(slot(k), pf_ptr + k * kStep);
     if (k & 1) cp_async_commit();
   }
+  if (tid == 0) {
+    sh[1] = a.nbins - 1;  // defaults: block hi, speculative bound, count below hi
+    sh[3] = a.nbins - 1;
+    sh[4] = 0;
+  }
   const int R_res = sink_n + local_n;
   const int n_res = seg < R_res ? (R_res - seg + nseg - 1) / nseg : 0;
-  if (ATTEND && tid < n_res) {
-    // the block's resident rows go to L2 now; they are attended after the scan
-    const int v = seg + tid * nseg;
-    const int t = v < sink_n ? v : local_start + (v - sink_n);
-    prefetch_row_l2<T>(a.K, a.V, kvc + t);
-  }
+  auto res_row = [&](int i) {  // the block's i-th resident row
+    const int v = seg + i * nseg;
+    return v < sink_n ? v : local_start + (v - sink_n);
+  };
+  if (ATTEND && !a.spec && tid < n_res) prefetch_row_l2<T>(a.K, a.V, kvc + res_row(tid));
   // ---------------- phase A: query codes, histogram reset -------------------
   if (ATTEND && tid < a.g * (kHeadDim / 4)) *reinterpret_cast<float4*>(&aq_s[tid * 4]) = aq;
   if (a.qenc == kQGiven) {
@@ -920,6 +1176,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   }
   for (int i = tid; i < a.nbins_pad; i += kThreads) hist_s[i] = 0u;
   __syncthreads();
+  HKV_TL(1);
   if (a.q_codes_out != nullptr && seg == 0)
     for (int i = tid; i < gw; i += kThreads) a.q_codes_out[qrow0 * W + i] = qc_s[i];
 
@@ -948,6 +1205,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     }
     cp_async_wait<0>();
   }
+  __syncthreads();
   if (a.next_codes != nullptr && tid < 32) {
     // the next call's codes for this block's range go to L2 while this call
     // selects and attends (16-byte aligned pieces; the hint skips ragged ends)
@@ -959,8 +1217,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(o), "r"(n) : "memory");
     }
   }
-  if (tid == 0) sh[1] = a.nbins;  // hi
-  __syncthreads();
+  HKV_TL(2);
 
   // ---------------- publication -----------------------------------------------
   // The segment adds its histogram counts up to hi (its own k-th smallest D,
@@ -970,60 +1227,111 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   // k_eff tokens at or below its hi), so the global histogram is complete on
   // [0, T] and every segment's cumulative counts are known at T - 1 and T.
   const uint32_t k_eff = (uint32_t)k_eff_p;
+  const int spec_cap = kRows - n_res;  // speculative rows that fit beside the resident ones in one tile
+  int hi, tb;
   {
-    block_inclusive_scan(hist_s, a.nbins, warp_tmp);
-    const bool enough = hist_s[a.nbins - 1] >= k_eff;
-    for (int v = tid; v < a.nbins; v += kThreads) {
-      const uint32_t prev = v > 0 ? hist_s[v - 1] : 0u;
-      if (enough && hist_s[v] >= k_eff && prev < k_eff) sh[1] = v;
+    uint32_t cnt[4], cum[4];
+    const uint4 hv = 4 * tid < a.nbins_pad ? *reinterpret_cast<const uint4*>(hist_s + 4 * tid) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t total = hist_cum4(hv, cnt, cum, warp_tmp);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int v = 4 * tid + e;
+      if (v < a.nbins) {
+        if (k_eff > 0u && cum[e] >= k_eff && cum[e] - cnt[e] < k_eff) {
+          sh[1] = v;
+          sh[4] = (int)(cum[e] - cnt[e]);
+        }
+        // speculative bound: the largest bin whose cumulative count fits spec_cap
+        if (cum[e] > (uint32_t)max(spec_cap, 0) && cum[e] - cnt[e] <= (uint32_t)max(spec_cap, 0)) sh[3] = v - 1;
+      }
     }
     __syncthreads();
     // k_eff == 0 (a ragged sequence without candidates): nothing to publish
-    const int hi = k_eff == 0 ? -1 : enough ? sh[1] : a.nbins - 1;
-    uint32_t* cum_out = a.cum + ((int64_t)p * nseg + seg) * a.nbins;
-    uint32_t* gh = a.gh + (int64_t)p * a.nbins;
-    for (int v = tid; v <= hi; v += kThreads) {
-      const uint32_t c = hist_s[v], prev = v > 0 ? hist_s[v - 1] : 0u;
-      cum_out[v] = c;
-      if (c != prev) red_add_gpu(&gh[v], c - prev);
+    hi = k_eff == 0u ? -1 : total >= k_eff ? sh[1] : a.nbins - 1;
+    tb = spec_cap > 0 ? sh[3] : -1;
+    if (nseg > 1) {
+      uint32_t* cum_out = a.cum + ((int64_t)p * nseg + seg) * a.nbins_pad;
+      uint32_t* gh = a.gh + (int64_t)p * a.nbins_pad;
+      if (4 * tid + 3 <= hi) {
+        *reinterpret_cast<uint4*>(cum_out + 4 * tid) = make_uint4(cum[0], cum[1], cum[2], cum[3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (4 * tid + e <= hi) cum_out[4 * tid + e] = cum[e];
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (4 * tid + e <= hi && cnt[e] != 0u) red_add_gpu(&gh[4 * tid + e], cnt[e]);
+      __syncthreads();
+      if (tid == 0 && !(a.skip_arrive && blockIdx.x == 0)) red_release_add(&sync[0], 1u);
     }
-    __syncthreads();
-    if (tid == 0 && !(a.skip_arrive && blockIdx.x == 0)) red_release_add(&sync[0], 1u);
+    // (one block per pair: its own k-th smallest distance is the threshold,
+    // nothing is exchanged)
+    HKV_TL(3);
+  }
+
+  // ---------------- speculative tile -----------------------------------------
+  // While the other blocks publish, the block gathers the K/V rows of its
+  // tokens with D <= tb (tb: the largest bin whose cumulative count fits
+  // beside its resident rows in one tile) and of its resident rows.  When the
+  // pair's threshold turns out to be <= tb, every selected token of the block
+  // is in this tile and the attention needs no further gather.
+  int n_spec = 0;
+  auto spec_row = [&](int i) -> int { return i < n_spec ? sel_s[i] : res_row(i - n_spec); };
+  if constexpr (ATTEND && sizeof(T) == 2) {
+    if (a.spec) {
+      n_spec = (int)compact_block(dist_s, len, tb + 1, 0u, warp_tmp, cscratch, [&](uint32_t pos, int i, int) {
+        if (pos < (uint32_t)kRows) sel_s[pos] = lo + s0 + i;
+      });
+      n_spec = min(n_spec, max(spec_cap, 0));
+      __syncthreads();
+      HKV_TL(11);
+      if ((tid >> 5) < kAW && (tid >> 5) * kWR < n_spec + n_res)  // slot 0 of warps 0-3
+        warp_issue(a, kvc, n_spec + n_res, spec_row, tid >> 5, smem + (size_t)(tid >> 5) * kSlotBytes,
+                   tokw_s + (tid >> 5) * kWR);
+      fill_qs(a.g, aq_s, qs_s);
+      HKV_TL(12);
+    }
   }
 
   // ---------------- phase B: threshold and ordered compaction ---------------
   uint32_t n_sel = 0, sel_base = 0;
-  if (tid == 0) sh[2] = wait_count(&sync[0], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
-  __syncthreads();
-  if (sh[2]) {
-    {
-      // the pair's histogram, all loads in flight at once
-      constexpr int kGL = 5;  // ceil(2049 / kThreads): up to g * bits + 1 bins
-      const uint32_t* gh = a.gh + (int64_t)p * a.nbins;
-      uint32_t gv[kGL];
-#pragma unroll
-      for (int u = 0; u < kGL; ++u) {
-        const int v = tid + u * kThreads;
-        gv[u] = v < a.nbins ? __ldcg(gh + v) : 0u;
+  bool spec_ok = false;
+  if (nseg > 1) {
+    if (tid == 0) sh[2] = wait_count(&sync[0], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
+    __syncthreads();
+  }
+  HKV_TL(4);
+  const bool arrived = nseg == 1 || sh[2] != 0;
+  if (arrived) {
+    int thr = max(hi, 0);
+    uint32_t below = (uint32_t)sh[4];
+    if (nseg > 1) {
+      // the pair's histogram: four bins per thread, one load round
+      uint32_t cnt[4], cum[4];
+      const uint32_t* gh = a.gh + (int64_t)p * a.nbins_pad;
+      const uint4 gv = 4 * tid < a.nbins_pad ? __ldcg(reinterpret_cast<const uint4*>(gh) + tid) : make_uint4(0u, 0u, 0u, 0u);
+      if (tid == 0) {
+        sh[5] = a.nbins - 1;
+        sh[6] = 0;
       }
+      hist_cum4(gv, cnt, cum, warp_tmp);
 #pragma unroll
-      for (int u = 0; u < kGL; ++u) {
-        const int v = tid + u * kThreads;
-        if (v < a.nbins) hist_s[v] = gv[u];
+      for (int e = 0; e < 4; ++e) {
+        const int v = 4 * tid + e;
+        if (v < a.nbins && cum[e] >= k_eff && cum[e] - cnt[e] < k_eff) {
+          sh[5] = v;
+          sh[6] = (int)(cum[e] - cnt[e]);
+        }
       }
+      __syncthreads();
+      thr = sh[5];
+      below = (uint32_t)sh[6];
     }
-    if (tid == 0) sh[5] = a.nbins - 1;
-    __syncthreads();
-    block_inclusive_scan(hist_s, a.nbins, warp_tmp);
-    for (int v = tid; v < a.nbins; v += kThreads)
-      if (hist_s[v] >= k_eff && (v == 0 || hist_s[v - 1] < k_eff)) sh[5] = v;
-    __syncthreads();
-    const int thr = sh[5];
-    const uint32_t below = thr > 0 ? hist_s[thr - 1] : 0u;
     // tokens of the lower segments below and at the threshold
     uint32_t seg_lt = 0, seg_le = 0;
     for (int ss = tid; ss < seg; ss += kThreads) {
-      const uint32_t* c = a.cum + ((int64_t)p * nseg + ss) * a.nbins;
+      const uint32_t* c = a.cum + ((int64_t)p * nseg + ss) * a.nbins_pad;
       seg_lt += thr > 0 ? __ldcg(c + thr - 1) : 0u;
       seg_le += __ldcg(c + thr);
     }
@@ -1032,116 +1340,141 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     const uint32_t ties_needed = k_eff - below;
     const uint32_t quota = ties_needed > lower_eq ? ties_needed - lower_eq : 0u;
     sel_base = lower_lt + min(lower_eq, ties_needed);
-    // thread tid owns a contiguous run of this block's distances, read 8 at a
-    // time; a chunk whose smallest distance exceeds T (almost all of them,
-    // since k_eff is a small fraction of the tokens) is skipped after one
-    // SIMD minimum
-    const int per8 = (((len + kThreads - 1) / kThreads) + 7) & ~7;
-    const int r0 = min(tid * per8, len), r1 = min(r0 + per8, len);
-    const int nch = (r1 - r0 + 7) >> 3;
-    auto chunk_min = [](const uint4& v) {
-      const uint32_t m = __vminu2(__vminu2(v.x, v.y), __vminu2(v.z, v.w));
-      return min(m & 0xffffu, m >> 16);
-    };
-    uint32_t lt = 0, eq = 0;
-    for (int c = 0; c < nch; ++c) {
-      const uint4 v = *reinterpret_cast<const uint4*>(dist_s + r0 + 8 * c);
-      if (chunk_min(v) > (uint32_t)thr) continue;
-      const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int Dv = (int)((wd[e >> 1] >> (16 * (e & 1))) & 0xffffu);
-        if (r0 + 8 * c + e < r1) {
-          lt += Dv < thr;
-          eq += Dv == thr;
-        }
-      }
-    }
-    uint64_t tot;
-    const uint64_t ex = block_exclusive((uint64_t)lt | ((uint64_t)eq << 32), reinterpret_cast<uint64_t*>(warp_tmp), &tot);
-    const uint32_t ex_lt = (uint32_t)ex, ex_eq = (uint32_t)(ex >> 32);
-    n_sel = (uint32_t)tot + min((uint32_t)(tot >> 32), quota);
-    uint32_t run_eq = ex_eq, pos = ex_lt + min(ex_eq, quota);
+    HKV_TL(5);
     int32_t* idx_out = a.idx + (int64_t)p * a.top_k + sel_base;
     int32_t* dist_out = a.dist ? a.dist + (int64_t)p * a.top_k + sel_base : nullptr;
-    if (lt | eq) {
-      for (int c = 0; c < nch; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(dist_s + r0 + 8 * c);
-        if (chunk_min(v) > (uint32_t)thr) continue;
-        const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int Dv = (int)((wd[e >> 1] >> (16 * (e & 1))) & 0xffffu);
-          const int i = r0 + 8 * c + e;
-          if (i >= r1) continue;
-          bool take = Dv < thr;
-          if (Dv == thr) take = run_eq++ < quota;
+    if (ATTEND && a.spec && thr <= tb) {
+      // every selected token of the block has D <= thr <= tb, so it is in the
+      // speculative list (ascending); keep D < thr, and ties at thr in
+      // order up to the quota; mask the others out of the tile
+      spec_ok = true;
+      if (tid < 32) {
+        const int lane = tid;
+        uint32_t run = 0, run_eq = 0;
+        for (int i0 = 0; i0 < n_spec; i0 += 32) {
+          const int i = i0 + lane;
+          const bool valid = i < n_spec;
+          const int tok = valid ? sel_s[i] : 0;
+          const uint32_t D = valid ? dist_s[tok - lo - s0] : 0xffffu;
+          const bool is_eq = valid && D == (uint32_t)thr;
+          const uint32_t eq_rank = run_eq + __popc(__ballot_sync(0xffffffffu, is_eq) & lanemask_lt());
+          const bool take = valid && (D < (uint32_t)thr || (is_eq && eq_rank < quota));
+          const uint32_t tm = __ballot_sync(0xffffffffu, take);
+          const uint32_t pos = run + __popc(tm & lanemask_lt());
           if (take) {
-            const int tok = lo + s0 + i;
             if (sel_base + pos < k_eff) {
               idx_out[pos] = tok;
-              if (dist_out) dist_out[pos] = Dv;
-              if constexpr (ATTEND) {
-                if (pos < (uint32_t)kSelCap) sel_s[pos] = tok;
-                prefetch_row_l2<T>(a.K, a.V, kvc + tok);
-              }
+              if (dist_out) dist_out[pos] = (int32_t)D;
             } else {
               report(a.status, HKV_ERR_DEVICE_RANGE);  // unreachable when the counts agree
             }
-            ++pos;
           }
+          if (valid && !take) tokw_s[i] = -1;
+          run += __popc(tm);
+          run_eq += __popc(__ballot_sync(0xffffffffu, is_eq));
         }
+        if (lane == 0) sh[7] = (int)run;
       }
+      __syncthreads();
+      n_sel = (uint32_t)sh[7];
+    } else {
+      if constexpr (ATTEND && sizeof(T) == 2) {
+        if (a.spec) cp_async_wait<0>();  // the speculative tile is not used
+      }
+      n_sel = compact_block(dist_s, len, thr, quota, warp_tmp, cscratch, [&](uint32_t pos, int i, int D) {
+        const int tok = lo + s0 + i;
+        if (sel_base + pos < k_eff) {
+          idx_out[pos] = tok;
+          if (dist_out) dist_out[pos] = D;
+          if constexpr (ATTEND) {
+            if (pos < (uint32_t)a.sel_cap) sel_s[pos] = tok;
+          }
+        } else {
+          report(a.status, HKV_ERR_DEVICE_RANGE);  // unreachable when the counts agree
+        }
+      });
+      if (sel_base + n_sel > k_eff) n_sel = k_eff > sel_base ? k_eff - sel_base : 0u;
     }
-    if (sel_base + n_sel > k_eff) n_sel = k_eff > sel_base ? k_eff - sel_base : 0u;
-  } else if (tid == 0) {
-    report(a.status, HKV_ERR_TIMEOUT);
+  } else {
+    if (tid == 0) report(a.status, HKV_ERR_TIMEOUT);
+    if constexpr (ATTEND && sizeof(T) == 2) {
+      if (a.spec) cp_async_wait<0>();  // no copy may land after the block exits
+    }
   }
   __syncthreads();
+  HKV_TL(6);
 
   if constexpr (ATTEND) {
-    // ---------------- attention over selected + resident rows, partial -----
-    const int ns = (int)n_sel;
-    const int32_t* sel_g = a.idx + (int64_t)p * a.top_k + sel_base;
-    auto row_at = [&](int i) -> int {
-      if (i < ns) return i < kSelCap ? sel_s[i] : sel_g[i];
-      const int v = seg + (i - ns) * nseg;
-      return v < sink_n ? v : local_start + (v - sink_n);
-    };
-    float* dst = a.part + ((int64_t)p * nseg + seg) * a.g * kPart;
-    if constexpr (sizeof(T) == 2) {
-      attn_mma(a, kvc, aq_s, ns + n_res, row_at, smem, tok_s, m_s, l_s, alpha_s, dst);
-    } else {
-      float* attn = reinterpret_cast<float*>(smem);
-      const AttnSmem sm{aq_s, attn, attn + kRows * kKP, attn + kRows * kKP + kRows * kHeadDim, tok_s, m_s, l_s, alpha_s};
-      float acc[kOut];
-      attn_begin(a.g, sm, acc);
-      attn_rows<T>(a, kvc, ns + n_res, row_at, sm, acc);
-      attn_end(a.g, sm, acc, dst);
-    }
-    __syncthreads();
-    if (tid == 0) sh[6] = (int)atom_acq_rel_add(&sync[2], 1u);
-    __syncthreads();
-    // ---------------- the last g blocks of the pair merge one head each -----
-    const int nm = min(a.g, nseg);
-    const int mi = sh[6] - (nseg - nm);
-    if (mi >= 0) {
-      if (tid == 0) sh[7] = wait_count(&sync[2], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
-      __syncthreads();
-      if (sh[7]) {
-        for (int h = mi; h < a.g; h += nm) merge_head(a, p, nseg, h, reinterpret_cast<float*>(smem));
-      } else if (tid == 0) {
-        report(a.status, HKV_ERR_TIMEOUT);
+    if (arrived) {
+      // ---------------- attention over selected + resident rows, partial -----
+      const int ns = (int)n_sel;
+      const int32_t* sel_g = a.idx + (int64_t)p * a.top_k + sel_base;
+      auto row_at = [&](int i) -> int {
+        if (i < ns) return i < a.sel_cap ? sel_s[i] : sel_g[i];
+        return res_row(i - ns);
+      };
+      float* part_s = reinterpret_cast<float*>(smem + a.off_part);
+      float* dst = nseg == 1 ? part_s : a.part + ((int64_t)p * nseg + seg) * a.g * kPart;
+      if constexpr (sizeof(T) == 2) {
+        if (spec_ok) {
+          attn_warps(a, kvc, n_spec + n_res, spec_row, smem, tokw_s, qs_s, dst, (n_spec + n_res + kWR - 1) / kWR);
+        } else {
+          fill_qs(a.g, aq_s, qs_s);
+          attn_warps(a, kvc, ns + n_res, row_at, smem, tokw_s, qs_s, dst, 0);
+        }
+      } else {
+        float* attn = reinterpret_cast<float*>(smem);
+        const AttnSmem sm{aq_s, attn, attn + kRows * kKP, attn + kRows * kKP + kRows * kHeadDim, tok_s, m_s, l_s, alpha_s};
+        float acc[kOut];
+        attn_begin(a.g, sm, acc);
+        attn_rows<T>(a, kvc, ns + n_res, row_at, sm, acc);
+        attn_end(a.g, sm, acc, dst);
       }
       __syncthreads();
-      if (tid == 0 && atomicAdd(&sync[3], 1u) == (uint32_t)(nm - 1)) {
-        sync[2] = 0u;
-        sync[3] = 0u;
+      HKV_TL(7);
+      bool last = nseg == 1;
+      if (nseg == 1) {
+        finish_single(a, p, part_s);
+      } else {
+        // the last g blocks of the pair to finish merge one head each; the
+        // last of them to finish returns the pair's counters and histogram to
+        // zero (every block is past its last use of them)
+        if (tid == 0) sh[8] = (int)atom_acq_rel_add(&sync[2], 1u);
+        __syncthreads();
+        const int nm = min(a.g, nseg);
+        const int mi = sh[8] - (nseg - nm);
+        if (mi >= 0) {
+          if (tid == 0) sh[7] = wait_count(&sync[2], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
+          __syncthreads();
+          HKV_TL(8);
+          if (sh[7]) {
+            for (int h = mi; h < a.g; h += nm)
+              merge_head(a.part, a.out, a.lse, a.Hq, a.Hkv, a.g, p, nseg, h, reinterpret_cast<float*>(smem));
+          } else if (tid == 0) {
+            report(a.status, HKV_ERR_TIMEOUT);
+          }
+          HKV_TL(9);
+          if (tid == 0) sh[7] = atomicAdd(&sync[3], 1u) == (uint32_t)(nm - 1) ? 1 : 0;
+          __syncthreads();
+          last = sh[7] != 0;
+        }
       }
+      if (last) {
+        for (int i = k_eff_p + tid; i < a.top_k; i += kThreads) a.idx[(int64_t)p * a.top_k + i] = -1;
+        for (int v = tid; v < a.nbins_pad; v += kThreads) a.gh[(int64_t)p * a.nbins_pad + v] = 0u;
+        if (tid == 0) {
+          sync[0] = 0u;
+          sync[2] = 0u;
+          sync[3] = 0u;
+        }
+      }
+      HKV_TL(10);
+      return;
     }
   }
 
   // ---------------- departure; the last block out resets the counters -------
+  // (retrieval only, or after a timeout)
   __syncthreads();
   if (tid == 0) sh[2] = atom_acq_rel_add(&sync[1], 1u) == (uint32_t)(nseg - 1);
   __syncthreads();
@@ -1150,12 +1483,13 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       a.idx[(int64_t)p * a.top_k + i] = -1;
       if (a.dist) a.dist[(int64_t)p * a.top_k + i] = -1;
     }
-    for (int v = tid; v < a.nbins; v += kThreads) a.gh[(int64_t)p * a.nbins + v] = 0u;
+    for (int v = tid; v < a.nbins_pad; v += kThreads) a.gh[(int64_t)p * a.nbins_pad + v] = 0u;
     if (tid == 0) {
       sync[0] = 0u;
       sync[1] = 0u;
     }
   }
+  HKV_TL(10);
 }
 
 using KernelFn = void (*)(FusedArgs);
@@ -1188,9 +1522,9 @@ struct Plan {
   int g, nbins, nbins_pad, np;
   int64_t C, lo;
   int k_eff;
-  int nseg, per_block, pairs_per_launch;
+  int nseg, per_block, pairs_per_launch, sel_cap;
   bool cooperative;
-  uint32_t off_q, off_aq, off_sel, off_hist, off_dist;
+  uint32_t off_q, off_aq, off_sel, off_hist, off_dist, off_part, off_qs, off_tokw;
   size_t smem;
   size_t ws_sync, ws_gh, ws_cum, ws_part, ws_total;
 };
@@ -1215,36 +1549,56 @@ int make_plan(const RetrieveShape& s, bool attend, int q_elt, Plan& pl) {
   // blocks per pair: fill the SMs, keep blocks between kMinTokensPerBlock and
   // max_tok candidates; max_tok = kMaxTokensPerBlock when the shared memory
   // of such a block fits, else kTokensPerBlockSmall
+  // Shared memory: a region written during the scan and the selection and
+  // dead afterwards (code ring at 0, query-encode staging, histogram,
+  // distances, chunk minima), which the attention then reuses from offset 0;
+  // then the arrays that live to the end (attention queries, selected rows,
+  // the single-block partial, bf16 queries, warp-step rows).
+  const size_t attn = attend ? std::max(sizeof(float) * (kRows * kKP + kRows * kHeadDim + kMaxGroup * kRows),
+                                        kAttnWarpBytes)
+                              : 0;
+  const size_t budget = (size_t)max_smem_optin() - kStaticSmem;
+  bool fits = false;
   for (const int max_tok : {kMaxTokensPerBlock, kTokensPerBlockSmall}) {
-  int64_t bpp = std::max<int64_t>(1, G / std::max(P, 1));
-  bpp = std::min<int64_t>(bpp, ceil_div(C, kMinTokensPerBlock));
-  bpp = std::max<int64_t>(bpp, ceil_div(C, max_tok));
-  if (bpp > G || bpp + 1 > kMaxSegsPerPair)
-    return fail(HKV_ERR_UNSUPPORTED, "%lld candidates per sequence is too many for one launch", (long long)C);
-  pl.per_block = (int)(ceil_div(ceil_div(C, bpp), 32) * 32);
-  pl.nseg = (int)ceil_div(C, pl.per_block);
-  pl.cooperative = pl.nseg > 1;
-  pl.pairs_per_launch = pl.cooperative ? (int)std::max<int64_t>(1, G / pl.nseg) : std::max(P, 1);
-  const size_t ring = (size_t)kSlots * kThreads * 16;
-  const size_t attn = std::max(sizeof(float) * (kRows * kKP + kRows * kHeadDim + kMaxGroup * kRows), kAttnMmaBytes);
-  size_t off = attend ? std::max(ring, attn) : ring;
-  pl.off_aq = (uint32_t)off;
-  if (attend) off += sizeof(float) * pl.g * kHeadDim;
-  pl.off_q = (uint32_t)off;
-  if (q_elt == 2) off += align_up(sizeof(uint16_t) * (kQRows + bits) * (kHeadDim + 8) + kQRows * bits / 8, 16);
-  if (q_elt == 4) off += align_up(sizeof(float) * (kQRows * kHeadDim + bits * (kHeadDim + 1)), 16);
-  pl.off_sel = (uint32_t)off;
-  if (attend) off += sizeof(int32_t) * kSelCap;
-  pl.off_hist = (uint32_t)off;
-  off += sizeof(uint32_t) * 2 * (size_t)pl.nbins_pad;
-  pl.off_dist = (uint32_t)off;
-  off += sizeof(uint16_t) * ((size_t)pl.per_block + 16);  // vector reads may run 7 past the end
-  pl.smem = align_up(off, 16);
-  if (pl.smem + kStaticSmem <= (size_t)max_smem_optin() || max_tok == kTokensPerBlockSmall) break;
+    int64_t bpp = std::max<int64_t>(1, G / std::max(P, 1));
+    bpp = std::min<int64_t>(bpp, ceil_div(C, kMinTokensPerBlock));
+    bpp = std::max<int64_t>(bpp, ceil_div(C, max_tok));
+    if (bpp > G || bpp + 1 > kMaxSegsPerPair)
+      return fail(HKV_ERR_UNSUPPORTED, "%lld candidates per sequence is too many for one launch", (long long)C);
+    pl.per_block = (int)(ceil_div(ceil_div(C, bpp), 32) * 32);
+    pl.nseg = (int)ceil_div(C, pl.per_block);
+    pl.cooperative = pl.nseg > 1;
+    pl.pairs_per_launch = pl.cooperative ? (int)std::max<int64_t>(1, G / pl.nseg) : std::max(P, 1);
+    pl.sel_cap = attend ? (int)align_up((size_t)std::max(kRows, std::min(kSelCap, pl.k_eff)), 64) : 0;
+    size_t qst = 0;
+    if (q_elt == 2) qst = align_up(sizeof(uint16_t) * (kQRows + bits) * (kHeadDim + 8) + kQRows * bits / 8, 16);
+    if (q_elt == 4) qst = align_up(sizeof(float) * (kQRows * kHeadDim + bits * (kHeadDim + 1)), 16);
+    size_t off = (size_t)kSlots * kThreads * 16;  // code ring
+    pl.off_q = (uint32_t)off;
+    off += qst;
+    pl.off_hist = (uint32_t)off;
+    off += sizeof(uint32_t) * 2 * (size_t)pl.nbins_pad;
+    pl.off_dist = (uint32_t)off;
+    off += align_up(sizeof(uint16_t) * ((size_t)pl.per_block + 16), 16);  // vector reads run past the end
+    off = std::max(off, attn);
+    pl.off_aq = (uint32_t)off;
+    if (attend) off += align_up(sizeof(float) * pl.g * kHeadDim, 16);
+    pl.off_sel = (uint32_t)off;
+    off += align_up(sizeof(int32_t) * (size_t)pl.sel_cap, 16);
+    pl.off_part = (uint32_t)off;
+    if (attend && pl.nseg == 1) off += sizeof(float) * pl.g * kPart;
+    pl.off_qs = (uint32_t)off;
+    if (attend) off += align_up(sizeof(uint16_t) * kMaxGroup * kQP, 16);
+    pl.off_tokw = (uint32_t)off;
+    if (attend) off += sizeof(int) * 2 * kAW * kWR;
+    pl.smem = align_up(off, 16);
+    fits = pl.smem <= budget;
+    if (fits) break;
   }
+  if (!fits) return fail(HKV_ERR_UNSUPPORTED, "the scan kernel's shared memory does not fit for this shape");
   pl.ws_sync = align_up(sizeof(uint32_t) * kSync * P, 256);
-  pl.ws_gh = align_up(sizeof(uint32_t) * (size_t)P * pl.nbins, 256);
-  pl.ws_cum = align_up(sizeof(uint32_t) * (size_t)P * pl.nseg * pl.nbins, 256);
+  pl.ws_gh = align_up(sizeof(uint32_t) * (size_t)P * pl.nbins_pad, 256);
+  pl.ws_cum = align_up(sizeof(uint32_t) * (size_t)P * pl.nseg * pl.nbins_pad, 256);
   pl.ws_part = attend ? align_up(sizeof(float) * (size_t)P * pl.nseg * pl.g * kPart, 256) : 0;
   pl.ws_total = pl.ws_sync + pl.ws_gh + pl.ws_cum + pl.ws_part;
   return HKV_OK;
@@ -1305,6 +1659,17 @@ int launch_fused(const RetrieveShape& s, bool attend, int dtype, int qenc, const
   a.off_sel = pl.off_sel;
   a.off_hist = pl.off_hist;
   a.off_dist = pl.off_dist;
+  a.off_part = pl.off_part;
+  a.off_qs = pl.off_qs;
+  a.off_tokw = pl.off_tokw;
+  a.sel_cap = pl.sel_cap;
+  {
+    // speculative tile: when a block's expected share of the selection, with
+    // a two-fold margin, fits one tile beside its resident rows
+    const int64_t res = (int64_t)w.sink_end + (s.N - w.local_start);
+    const int64_t res_blk = ceil_div(res, pl.nseg);
+    a.spec = attend && dtype == HKV_BF16 && pl.nseg > 1 && 2 * ceil_div(pl.k_eff, pl.nseg) + res_blk <= kRows ? 1 : 0;
+  }
   a.sync = reinterpret_cast<uint32_t*>(base);
   a.gh = reinterpret_cast<uint32_t*>(base + pl.ws_sync);
   a.cum = reinterpret_cast<uint32_t*>(base + pl.ws_sync + pl.ws_gh);
@@ -1450,3 +1815,13 @@ int launch_decode(const RetrieveShape& s, int dtype, int q_kind, const void* R, 
 
 
 }  // namespace hkv
+
+#ifdef HKV_TIMELINE
+extern "C" int hkv_debug_timeline(unsigned long long* dst, int n) {
+  const size_t cap = sizeof(hkv::g_hkv_tl) / sizeof(unsigned long long);
+  return cudaMemcpyFromSymbol(dst, hkv::g_hkv_tl, sizeof(unsigned long long) * ((size_t)n < cap ? (size_t)n : cap)) ==
+                 cudaSuccess
+             ? 0
+             : -4;
+}
+#endif
