@@ -2,15 +2,19 @@
 attention + LSE merge, through the library's C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+                    [--main-only] [--no-cpu-baseline]
 
 One step = one pass of the whole decode path over every layer of the
 workload (28 sequential layers for the default Qwen2.5-7B-shaped 512K-token
 case), captured in one CUDA graph.  Inputs are synthetic, drawn on the device
 (same distributions as the parity tests), and larger than L2: every layer has
-its own codes and K/V buffers.  Timing uses CUDA events on the launching
-stream after W warm-up steps; the value is the max over ranks.  With N > 1
-(torchrun) each rank runs its own replica of the workload (independent
-sequences: weak scaling, no collective on the data path).
+its own codes and K/V buffers.  Timing: CUDA events on the launching stream
+between consecutive replays after W warm-up replays; the reported step time
+is the median replay (the mean is reported beside it), max over ranks.  After
+the main workload, every other workload's decode step and fused kernel are
+timed the same way and reported under "configs".  With N > 1 (torchrun) each
+rank runs its own replica (independent sequences: weak scaling, no
+collective on the data path).
 
 --impl reference times the oracle (CPU) on the same workload instead.
 """
@@ -50,6 +54,8 @@ def parse():
     ap.add_argument("--impl", default="hkv", choices=["hkv", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--main-only", action="store_true",
+                    help="measure only --workload (skip the other workloads' decode steps)")
     ap.add_argument("--layers", type=int, default=0,
                     help="number of layer buffers (default: the workload's layers, at least 3x L2 of data); "
                          "a small value makes a small case for profiling")
@@ -266,21 +272,31 @@ def graph_of(fn, warm=1):
 
 
 def time_graph(g, steps, warmup, world):
+    """Replays g: W untimed warm-up replays, then K timed replays bracketed by
+    a barrier and a synchronize on both sides, with CUDA events recorded on
+    the launching stream between consecutive replays.  Returns (mean ms,
+    median ms) per replay; the max over ranks is taken by the caller."""
     for _ in range(warmup):
         g.replay()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     stream = torch.cuda.current_stream()
-    start.record(stream)
-    for _ in range(steps):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
         g.replay()
-    end.record(stream)
+        ev[i + 1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    return start.elapsed_time(end) / steps  # ms per replay
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    return ev[0].elapsed_time(ev[-1]) / steps, statistics.median(per)
+
+
+def timed_ms(g, args, world, dev):
+    """Median ms per replay, max over ranks."""
+    return max_over_ranks(time_graph(g, args.steps, args.warmup, world)[1], world, dev)
 
 
 def source_digest(path):
@@ -301,16 +317,45 @@ def traffic_record(kernel_file: str, workload: str):
     return rec.get("bytes_per_launch")
 
 
-def run_gpu(args, rank, world, local):
-    import hash_sparse_kv_b200 as hkv
+def build_layers(w: synth.Workload, dev, hkv, n_layers: int):
+    """Device buffers of n_layers layers.  The layers' query rows live in one
+    contiguous tensor and their outputs in another, so the end-to-end step
+    moves them with one copy each way."""
+    layers = [Layer(w, l % w.layers if w.layers > 1 else 0, dev, hkv) for l in range(n_layers)]
+    q_all = torch.empty((n_layers,) + tuple(layers[0].q.shape), dtype=layers[0].q.dtype, device=dev)
+    out_all = torch.empty((n_layers,) + tuple(layers[0].out.shape), dtype=torch.float32, device=dev)
+    for i, L in enumerate(layers):
+        q_all[i].copy_(L.q)
+        L.q = q_all[i]
+        L.out = out_all[i]
+    return layers, q_all, out_all
 
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    hkv.lib()
-    w = synth.WORKLOADS[args.workload]
+
+def step_fn(w, layers, ws, status, hkv, hint=False):
+    """One decode step over every layer: hkv_decode_step per layer (query
+    encode + scan + select + attend + merge).  hint: each layer names the next
+    layer's codes for the library's L2 prefetch."""
+    def step():
+        for i, L in enumerate(layers):
+            nxt = layers[(i + 1) % len(layers)].codes if hint and len(layers) > 1 else None
+            hkv.hkv_decode_step(L.qh, L.q, L.codes, L.K, L.V, w.N, w.n_sink, w.n_local, w.top_k, L.out,
+                                q_codes=L.q_codes, idx=L.idx, ws=ws, status=status, next_k_codes=nxt)
+    return step
+
+
+def check(hkv, status, what):
+    rc = hkv.hkv_check(status)
+    if rc != hkv.HKV_OK:
+        raise RuntimeError(f"{what} reported status {rc}: {hkv.hkv_last_error()}")
+
+
+def measure_workload(w: synth.Workload, args, dev, world, hkv, full: bool):
+    """Times the decode step of workload w (all of its layers, one CUDA graph)
+    and the fused decode kernel alone; with full=True also the other entry
+    points, the encode and the end-to-end step.  Returns (dict, layers)."""
     per_layer_bytes = w.algorithmic_bytes()
     n_layers = args.layers or max(w.layers, math.ceil(3 * L2_BYTES / per_layer_bytes))
-    layers = [Layer(w, l % w.layers if w.layers > 1 else 0, dev, hkv) for l in range(n_layers)]
+    layers, q_all, out_all = build_layers(w, dev, hkv, n_layers)
     # prefill: encode the keys of every layer (timed separately, reported as encode)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -320,84 +365,131 @@ def run_gpu(args, rank, world, local):
     e1.record()
     torch.cuda.synchronize()
     encode_ms = e0.elapsed_time(e1)
-    ws = hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
+    new_ws = lambda: hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
+    ws = new_ws()
     status = hkv.status_word(dev)
-
-    def step(hint=args.prefetch_hint):
-        # layer i tells the library that layer i + 1 (wrapping to the next
-        # step's layer 0) scans next, so its codes stream into L2 during layer
-        # i's selection and attention
-        for i, L in enumerate(layers):
-            nxt = layers[(i + 1) % len(layers)].codes if hint and len(layers) > 1 else None
-            hkv.hkv_decode_step(L.qh, L.q, L.codes, L.K, L.V, w.N, w.n_sink, w.n_local, w.top_k, L.out,
-                                q_codes=L.q_codes, idx=L.idx, ws=ws, status=status, next_k_codes=nxt)
-
-    # standalone calls get their own workspaces (each entry point has its own layout)
-    ws_r = hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
-    ws_a = hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
-    ws_f = hkv.workspace(w.B, w.Hq, w.Hkv, w.N, w.bits, w.top_k, w.n_sink, w.n_local, device=dev)
-
+    peak, peak_kind = measured_peaks()
+    step = step_fn(w, layers, ws, status, hkv, hint=args.prefetch_hint)
+    g_step = graph_of(step)
+    check(hkv, status, "decode step")
+    with ClockSampler(dev.index) as clk:
+        mean_ms, med_ms = time_graph(g_step, args.steps, args.warmup, world)
+    ms = max_over_ranks(med_ms, world, dev)
+    mean_ms = max_over_ranks(mean_ms, world, dev)
+    check(hkv, status, "decode step")
+    del g_step
+    keys_per_layer = w.B * w.Hkv * w.candidates()
+    value, ms = job_throughput(keys_per_layer * len(layers), ms, world, dev)
+    # the fused kernel alone: query codes given, one hkv_decode_step launch per layer
     given = hkv.HashParams.given(hkv.HKV_BF16 if w.dtype == "bf16" else hkv.HKV_F32, w.bits)
+    ws_f = new_ws()
+    for L in layers:
+        hkv.hkv_encode_keys(L.qh, L.q.view(-1, w.d), L.q_codes.view(-1, w.words))
 
     def fused_only():
         for L in layers:
             hkv.hkv_decode_step(given, L.q, L.codes, L.K, L.V, w.N, w.n_sink, w.n_local, w.top_k, L.out,
                                 q_codes=L.q_codes, idx=L.idx, ws=ws_f, status=status)
 
-    def scan_only():
-        for L in layers:
-            hkv.hkv_retrieve_topk(L.q_codes, L.codes, w.N, w.n_sink, w.n_local, w.top_k, L.idx, ws=ws_r,
-                                  status=status)
-
-    g_step = graph_of(step)
-    rc = hkv.hkv_check(status)
-    if rc != hkv.HKV_OK:
-        raise RuntimeError(f"decode step reported status {rc}")
-    with ClockSampler(local) as clk:
-        ms = time_graph(g_step, args.steps, args.warmup, world)
-    rc = hkv.hkv_check(status)
-    if rc != hkv.HKV_OK:
-        raise RuntimeError(f"decode step reported status {rc}")
-    keys_per_layer = w.B * w.Hkv * w.candidates()
-    value, ms = job_throughput(keys_per_layer * len(layers), ms, world, dev)
-    g_other = graph_of(lambda: step(hint=not args.prefetch_hint))
-    other_ms = max_over_ranks(time_graph(g_other, args.steps, args.warmup, world), world, dev)
-    del g_other
-    # each kernel alone, one launch per layer
-    def qenc_only():
-        for L in layers:
-            hkv.hkv_encode_keys(L.qh, L.q.view(-1, w.d), L.q_codes.view(-1, w.words))
-
-    def attend_only():
-        for L in layers:
-            hkv.hkv_sparse_attend(L.q, L.K, L.V, w.N, L.idx, w.n_sink, w.n_local, L.out, ws=ws_a, status=status)
-
     g_fused = graph_of(fused_only)
-    fused_ms = max_over_ranks(time_graph(g_fused, args.steps, args.warmup, world), world, dev)
+    fused_ms = timed_ms(g_fused, args, world, dev)
     del g_fused
-    g_scan = graph_of(scan_only)
-    scan_ms = max_over_ranks(time_graph(g_scan, args.steps, args.warmup, world), world, dev)
-    g_qenc = graph_of(qenc_only)
-    qenc_ms = max_over_ranks(time_graph(g_qenc, args.steps, args.warmup, world), world, dev)
-    g_att = graph_of(attend_only)
-    att_ms = max_over_ranks(time_graph(g_att, args.steps, args.warmup, world), world, dev)
-    # HashEvict eviction choice for every layer (one scan of the codes each)
-    victims = [torch.zeros(w.B, w.Hkv, dtype=torch.int32, device=dev) for _ in layers]
-    ws_e = torch.zeros(8 * w.B * w.Hkv, dtype=torch.uint8, device=dev)
+    check(hkv, status, "fused decode")
+    fused_launch_ms = fused_ms / len(layers)
+    achieved = per_layer_bytes / (fused_launch_ms * 1e-3) / 1e9
+    step_gbs = per_layer_bytes * len(layers) / (ms * 1e-3) / 1e9
+    res = {
+        "workload": w.name, "layers_per_step": len(layers), "ms_per_step": ms, "ms_per_step_mean": mean_ms,
+        "us_per_layer": ms * 1e3 / len(layers), "keys_per_s": value,
+        "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
+                     "frac_of_nominal_8tbs": step_gbs / 8000.0, "bytes_per_layer": per_layer_bytes,
+                     "peak_kind": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": "fused_kernel (scan + select + attend + merge, one layer)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "retrieve.cu"),
+                                               w.name),
+                     "algorithmic_bytes_per_launch": per_layer_bytes, "launch_us": fused_launch_ms * 1e3,
+                     "peak_kind": peak_kind},
+        "encode": dict(encode_roofline(w, len(layers), encode_ms),
+                       traffic=traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "encode_tc.cu"),
+                                              w.name) if w.hash == "lsh" else None),
+        # decode with an LSH or sign query hash (query heads per KV head <= 32) is one
+        # fused launch a layer; an MLP query hash adds the separate query encode launch
+        "launches_per_step": (1 if w.hash in ("lsh", "sign") and w.g <= 32 else 2) * len(layers),
+        "clocks": clk.summary(),
+    }
 
-    def evict_only():
-        for L, vic in zip(layers, victims):
-            hkv.hkv_evict_select(L.q_codes, L.codes, w.N, w.n_sink, w.n_local, vic, ws=ws_e)
+    status_ok = lambda what: check(hkv, status, what)
+    if full:
+        g_other = graph_of(step_fn(w, layers, ws, status, hkv, hint=not args.prefetch_hint))
+        other_ms = timed_ms(g_other, args, world, dev)
+        del g_other
+        res["us_per_layer_without_prefetch_hint" if args.prefetch_hint else "us_per_layer_with_prefetch_hint"] = \
+            other_ms * 1e3 / len(layers)
+        # each entry point alone, one launch per layer (own workspaces: each has its own layout)
+        ws_r, ws_a = new_ws(), new_ws()
 
-    g_ev = graph_of(evict_only)
-    ev_ms = max_over_ranks(time_graph(g_ev, args.steps, args.warmup, world), world, dev)
-    del g_ev
-    del g_qenc, g_att
-    # paged cache (pages of 256 tokens scattered through a pool): retrieval
-    # and attention read through the page table, after the query encode
-    paged_ms = paged_step_ms = None
+        def scan_only():
+            for L in layers:
+                hkv.hkv_retrieve_topk(L.q_codes, L.codes, w.N, w.n_sink, w.n_local, w.top_k, L.idx, ws=ws_r,
+                                      status=status)
+
+        def qenc_only():
+            for L in layers:
+                hkv.hkv_encode_keys(L.qh, L.q.view(-1, w.d), L.q_codes.view(-1, w.words))
+
+        def attend_only():
+            for L in layers:
+                hkv.hkv_sparse_attend(L.q, L.K, L.V, w.N, L.idx, w.n_sink, w.n_local, L.out, ws=ws_a, status=status)
+
+        victims = [torch.zeros(w.B, w.Hkv, dtype=torch.int32, device=dev) for _ in layers]
+        ws_e = torch.zeros(8 * w.B * w.Hkv, dtype=torch.uint8, device=dev)
+
+        def evict_only():
+            for L, vic in zip(layers, victims):
+                hkv.hkv_evict_select(L.q_codes, L.codes, w.N, w.n_sink, w.n_local, vic, ws=ws_e)
+
+        times = {}
+        for name, fn in (("retrieve_only", scan_only), ("encode_q", qenc_only), ("sparse_attend_only", attend_only),
+                         ("evict_select", evict_only)):
+            g = graph_of(fn)
+            times[name] = timed_ms(g, args, world, dev) * 1e3 / len(layers)
+            del g
+        status_ok("stand-alone entry points")
+        times["fused_decode"] = fused_launch_ms * 1e3
+        res["kernels_us_per_launch"] = times
+        code_bytes = w.B * w.Hkv * w.candidates() * w.bits // 8
+        ev_gbs = code_bytes / (times["evict_select"] * 1e-6) / 1e9
+        res["evict"] = {"bound": "hbm", "achieved": ev_gbs, "peak": peak, "unit": "GB/s", "frac": ev_gbs / peak,
+                        "bytes_per_launch": code_bytes, "launches_per_layer": 2,
+                        "traffic": traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "evict.cu"),
+                                                  w.name)}
+        # end to end: every layer's queries in from pinned host memory and every
+        # output back, one copy each way per step, inside the timed region
+        q_host = torch.empty(q_all.shape, dtype=q_all.dtype, device="cpu").pin_memory()
+        o_host = torch.empty(out_all.shape, dtype=out_all.dtype, device="cpu").pin_memory()
+        q_host.copy_(q_all.cpu())
+
+        def e2e_step():
+            q_all.copy_(q_host, non_blocking=True)
+            step()
+            o_host.copy_(out_all, non_blocking=True)
+
+        g_e2e = graph_of(e2e_step)
+        e2e_ms = timed_ms(g_e2e, args, world, dev)
+        del g_e2e
+        status_ok("end-to-end step")
+        keys_step = keys_per_layer * len(layers) * world
+        res["e2e"] = {"value": keys_step / (e2e_ms * 1e-3), "unit": "keys/s",
+                      "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
+                      "d2h_bytes_per_step": o_host.numel() * o_host.element_size(), "ms_per_step": e2e_ms,
+                      "copies_per_step": 2}
+    # paged cache (pages of 256 tokens scattered through a pool): retrieval and
+    # attention read through the page table, after the query encode
+    res["paged"] = None
     PAGE = 256
     if w.candidates() <= 65536 and w.N % PAGE == 0:
+        ws_a = new_ws()
         pages = w.N // PAGE
         gen = torch.Generator(device=dev).manual_seed(1234)
         paged_layers = []
@@ -428,19 +520,20 @@ def run_gpu(args, rank, world, local):
                 hkv.hkv_sparse_attend_paged(L.q, kpool, vpool, table, w.N, L.idx, w.n_sink, w.n_local, L.out,
                                             ws=ws_a, status=status)
 
-        g_pg = graph_of(paged_only)
-        paged_ms = max_over_ranks(time_graph(g_pg, args.steps, args.warmup, world), world, dev)
-        del g_pg
-        g_pg = graph_of(paged_step)
-        paged_step_ms = max_over_ranks(time_graph(g_pg, args.steps, args.warmup, world), world, dev)
-        del g_pg, paged_layers
-        rc = hkv.hkv_check(status)
-        if rc != hkv.HKV_OK:
-            raise RuntimeError(f"paged calls reported status {rc}")
+        g = graph_of(paged_only)
+        paged_ms = timed_ms(g, args, world, dev)
+        del g
+        g = graph_of(paged_step)
+        paged_step_ms = timed_ms(g, args, world, dev)
+        del g, paged_layers
+        status_ok("paged calls")
+        res["paged"] = paged_roofline(w, len(layers), paged_ms, paged_step_ms, PAGE, peak, peak_kind)
     # sign-VQ only: retrieval by the norm-weighted sign score (its own kernel),
     # then the standalone sparse attention
-    normw_ms = normw_step_ms = None
+    res["normw"] = None
     if w.hash == "sign" and w.candidates() <= 65536:
+        ws_a = new_ws()
+
         def normw_only():
             for L in layers:
                 hkv.hkv_retrieve_topk_normw(L.q_codes, L.codes, L.norms, w.N, w.n_sink, w.n_local, w.top_k, L.idx)
@@ -451,51 +544,50 @@ def run_gpu(args, rank, world, local):
                 hkv.hkv_retrieve_topk_normw(L.q_codes, L.codes, L.norms, w.N, w.n_sink, w.n_local, w.top_k, L.idx)
                 hkv.hkv_sparse_attend(L.q, L.K, L.V, w.N, L.idx, w.n_sink, w.n_local, L.out, ws=ws_a, status=status)
 
-        g_nw = graph_of(normw_only)
-        normw_ms = max_over_ranks(time_graph(g_nw, args.steps, args.warmup, world), world, dev)
-        del g_nw
-        g_nw = graph_of(normw_step)
-        normw_step_ms = max_over_ranks(time_graph(g_nw, args.steps, args.warmup, world), world, dev)
-        del g_nw
-    # end to end: host q in, host out back, every step
-    q_host = [torch.empty_like(L.q, device="cpu").pin_memory() for L in layers]
-    o_host = [torch.empty_like(L.out, device="cpu").pin_memory() for L in layers]
-    for qh, L in zip(q_host, layers):
-        qh.copy_(L.q.cpu())
+        g = graph_of(normw_only)
+        normw_ms = timed_ms(g, args, world, dev)
+        del g
+        g = graph_of(normw_step)
+        normw_step_ms = timed_ms(g, args, world, dev)
+        del g
+        status_ok("norm-weighted calls")
+        res["normw"] = normw_roofline(w, len(layers), normw_ms, normw_step_ms, peak, peak_kind)
+    return res, layers
 
-    def e2e_step():
-        for qh, L in zip(q_host, layers):
-            L.q.copy_(qh, non_blocking=True)
-        step()
-        for oh, L in zip(o_host, layers):
-            oh.copy_(L.out, non_blocking=True)
+def run_gpu(args, rank, world, local):
+    """The main workload in full, then every other workload's decode step and
+    fused kernel (each workload's buffers freed before the next)."""
+    import hash_sparse_kv_b200 as hkv
 
-    g_e2e = graph_of(e2e_step)
-    e2e_ms = max_over_ranks(time_graph(g_e2e, args.steps, args.warmup, world), world, dev)
-    h2d = sum(t.numel() * t.element_size() for t in q_host)
-    d2h = sum(t.numel() * t.element_size() for t in o_host)
-    rc = hkv.hkv_check(status)
-    if rc != hkv.HKV_OK:
-        raise RuntimeError(f"e2e step reported status {rc}")
-
-    keys_step = keys_per_layer * len(layers) * world
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    hkv.lib()
+    w = synth.WORKLOADS[args.workload]
+    main, layers = measure_workload(w, args, dev, world, hkv, full=True)
+    cpu_layer = oracle_inputs_from_device(w, layers[0]) if rank == 0 and world == 1 and not args.no_cpu_baseline \
+        else None
+    del layers
+    torch.cuda.empty_cache()
+    others = {}
+    if not args.main_only:
+        for name in sorted(synth.WORKLOADS):
+            if name == w.name:
+                continue
+            r, lay = measure_workload(synth.WORKLOADS[name], args, dev, world, hkv, full=False)
+            del lay
+            torch.cuda.empty_cache()
+            others[name] = r
     peak, peak_kind = measured_peaks()
-    fused_launch_ms = fused_ms / len(layers)
-    achieved = per_layer_bytes / (fused_launch_ms * 1e-3) / 1e9
-    traffic = traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "retrieve.cu"), w.name)
-    code_bytes = w.B * w.Hkv * w.candidates() * w.bits // 8
-    step_gbs = per_layer_bytes * len(layers) / (ms * 1e-3) / 1e9
     out = {
         "metric": "decode retrieval+sparse-attn keys scanned/s (also us/layer and % HBM roofline)",
-        "value": value,
+        "value": main["keys_per_s"],
         "unit": "keys/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": ms,
-        "us_per_layer": ms * 1e3 / len(layers),
-        ("us_per_layer_without_prefetch_hint" if args.prefetch_hint else "us_per_layer_with_prefetch_hint"):
-            other_ms * 1e3 / len(layers),
+        "ms_per_step": main["ms_per_step"],
+        "ms_per_step_mean": main["ms_per_step_mean"],
+        "us_per_layer": main["us_per_layer"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -504,42 +596,29 @@ def run_gpu(args, rank, world, local):
         "config": {
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.d, "n_tokens": w.N,
             "hash": w.hash, "code_bits": w.bits, "top_k": w.top_k, "n_sink": w.n_sink, "n_local": w.n_local,
-            "layers_per_step": len(layers), "parallelism": f"replica x{world}",
+            "layers_per_step": main["layers_per_step"], "parallelism": f"replica x{world}",
             "next_layer_prefetch_hint": args.prefetch_hint,
-            "l2": f"inputs larger than L2: {len(layers)} distinct layer buffers, "
-                  f"{per_layer_bytes * len(layers) / 1e9:.2f} GB algorithmic per step",
+            "timing": "median of the per-replay CUDA-event times (max over ranks)",
+            "l2": f"inputs larger than L2: {main['layers_per_step']} distinct layer buffers, "
+                  f"{w.algorithmic_bytes() * main['layers_per_step'] / 1e9:.2f} GB algorithmic per step",
         },
-        "step_hbm": {"achieved_gbs": step_gbs, "peak_gbs": peak, "frac": step_gbs / peak,
-                     "frac_of_nominal_8tbs": step_gbs / 8000.0,
-                     "bytes_per_layer": per_layer_bytes, "peak_kind": peak_kind},
-        "roofline": {"bound": "hbm", "kernel": "fused_kernel (scan + select + attend + merge, one layer)",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "algorithmic_bytes_per_launch": per_layer_bytes,
-                     "launch_us": fused_launch_ms * 1e3, "peak_kind": peak_kind},
-        "e2e": {"value": keys_step / (e2e_ms * 1e-3), "unit": "keys/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "encode": dict(encode_roofline(w, len(layers), encode_ms),
-                       traffic=traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "encode_tc.cu"),
-                                              w.name) if w.hash == "lsh" else None),
-        "kernels_us_per_launch": {"encode_q": qenc_ms * 1e3 / len(layers),
-                                  "fused_decode": fused_launch_ms * 1e3,
-                                  "retrieve_only": scan_ms * 1e3 / len(layers),
-                                  "sparse_attend_only": att_ms * 1e3 / len(layers),
-                                  "evict_select": ev_ms * 1e3 / len(layers)},
-        "evict": {"bound": "hbm", "achieved": code_bytes / (ev_ms * 1e-3 / len(layers)) / 1e9, "peak": peak,
-                  "unit": "GB/s", "frac": code_bytes / (ev_ms * 1e-3 / len(layers)) / 1e9 / peak,
-                  "bytes_per_launch": code_bytes, "launches_per_layer": 2,
-                  "traffic": traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "evict.cu"), w.name)},
-        "paged": None if paged_ms is None else paged_roofline(w, len(layers), paged_ms, paged_step_ms, PAGE, peak,
-                                                              peak_kind),
-        "normw": None if normw_ms is None else normw_roofline(w, len(layers), normw_ms, normw_step_ms, peak, peak_kind),
-        # decode with an LSH or sign query hash (query heads per KV head <= 32) is one
-        # fused launch a layer; an MLP query hash adds the separate query encode launch
-        "gpu_launches": (1 if w.hash in ("lsh", "sign") and w.g <= 32 else 2) * len(layers) * args.steps,
-        "clocks": clk.summary(),
+        "step_hbm": main["step_hbm"],
+        "roofline": main["roofline"],
+        "e2e": main["e2e"],
+        "encode": main["encode"],
+        "kernels_us_per_launch": main["kernels_us_per_launch"],
+        "evict": main["evict"],
+        "paged": main["paged"],
+        "normw": main["normw"],
+        "configs": {n: {k: v for k, v in r.items() if k != "clocks"} for n, r in others.items()},
+        "gpu_launches": main["launches_per_step"] * args.steps,
+        "clocks": main["clocks"],
     }
-    del g_step, g_scan, g_e2e
-    return out, layers, w
+    for k in ("us_per_layer_with_prefetch_hint", "us_per_layer_without_prefetch_hint"):
+        if k in main:
+            out[k] = main[k]
+    out["peak_kind"] = peak_kind
+    return out, cpu_layer, w
 
 
 # ------------------------------------------------------------------ oracle arm --
@@ -563,9 +642,30 @@ def oracle_inputs_host(w: synth.Workload):
     return inp["q"], inp["K"], inp["V"], None, None
 
 
+def host_cpu():
+    """(usable cores, CPU model name) of this host."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return cores, model
+
+
 class OracleLayer:
     """The oracle's decode step on one layer of the workload.  The cache's key
-    codes are computed once by the oracle itself (setup, not timed)."""
+    codes are computed once by the oracle itself (setup, not timed).  (batch,
+    KV head) pairs are independent, so the step can also run as one oracle
+    call per pair on a pool of host threads (numpy releases the interpreter
+    lock inside its array operations; each call keeps BLAS to one thread)."""
 
     def __init__(self, w: synth.Workload, q, K, V, qparams, kparams):
         import oracle
@@ -573,50 +673,79 @@ class OracleLayer:
         kc = oracle.encode(w.hash, K, kparams)
         self.kc = kc[0] if w.hash == "sign" else kc
 
-    def run(self) -> float:
-        """Seconds for one decode step of this layer (single thread)."""
+    def _pair(self, b, h):
+        import oracle
+        w, g = self.w, self.w.g
+        oracle.decode_step(self.q[b:b + 1, h * g:(h + 1) * g], self.K[b:b + 1, h:h + 1], self.V[b:b + 1, h:h + 1],
+                           self.kc[b:b + 1, h:h + 1], w.N, w.n_sink, w.n_local, w.top_k, w.hash, self.qparams)
+
+    def run(self, threads: int = 1) -> float:
+        """Seconds for one decode step of this layer on `threads` host threads."""
         import oracle
         from threadpoolctl import threadpool_limits
         w = self.w
         with threadpool_limits(limits=1):
             t0 = time.perf_counter()
-            oracle.decode_step(self.q, self.K, self.V, self.kc, w.N, w.n_sink, w.n_local, w.top_k, w.hash,
-                               self.qparams)
+            if threads <= 1:
+                oracle.decode_step(self.q, self.K, self.V, self.kc, w.N, w.n_sink, w.n_local, w.top_k, w.hash,
+                                   self.qparams)
+            else:
+                import concurrent.futures
+                pairs = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+                with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+                    list(ex.map(lambda bh: self._pair(*bh), pairs))
             return time.perf_counter() - t0
 
 
 def oracle_sample(w: synth.Workload, budget_s: float, layer_inputs):
-    """Time the oracle's decode step on one whole layer, repeated until the
-    budget is spent (at most 64 times).  Returns (keys/s, sample, threads)."""
+    """Time the oracle's decode step on one whole layer on one thread and on a
+    thread per (batch, KV head) pair (up to the host's cores), each repeated
+    until its share of the budget is spent (at most 64 times)."""
     ol = OracleLayer(w, *layer_inputs)
-    elapsed, n = 0.0, 0
-    while n < 1 or (elapsed < budget_s and n < 64):
-        elapsed += ol.run()
-        n += 1
-    keys = n * w.B * w.Hkv * w.candidates()
-    return keys / elapsed, f"{n} decode step(s) of one {w.name} layer ({w.B * w.Hkv * w.candidates()} keys each), " \
-                           f"{elapsed:.2f} s", 1
+    cores, model = host_cpu()
+    pool = max(1, min(cores, w.B * w.Hkv))
+    keys_step = w.B * w.Hkv * w.candidates()
+    out = {}
+    for threads in (pool, 1):
+        elapsed, n = 0.0, 0
+        while n < 1 or (elapsed < budget_s / 2 and n < 64):
+            elapsed += ol.run(threads)
+            n += 1
+        out[threads] = (keys_step * n / elapsed, n, elapsed)
+    v, n, el = out[pool]
+    v1, n1, el1 = out[1]
+    return {"value": v, "unit": "keys/s", "cores": pool, "kind": "oracle",
+            "sample": f"{n} decode step(s) of one {w.name} layer ({keys_step} keys each) on {pool} host thread(s), "
+                      f"one per (batch, KV head) pair, {el:.2f} s; single thread: {n1} step(s), {el1:.2f} s",
+            "value_1_core": v1, "host_cores": cores, "cpu_model": model}
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the oracle's decode step of one layer per step, on a
+    host thread per (batch, KV head) pair (up to the host's cores)."""
     w = synth.WORKLOADS[args.workload]
     if rank != 0:
         return None
     ol = OracleLayer(w, *oracle_inputs_host(w))
+    cores, model = host_cpu()
+    pool = max(1, min(cores, w.B * w.Hkv))
     keys_per_step = w.B * w.Hkv * w.candidates()
     for _ in range(args.warmup):
-        ol.run()
-    per_step_s = [ol.run() for _ in range(args.steps)]
-    value = keys_per_step / statistics.mean(per_step_s)
-    sample = f"each step: one decode step of one {w.name} layer ({keys_per_step} keys), single thread"
+        ol.run(pool)
+    per_step_s = [ol.run(pool) for _ in range(args.steps)]
+    med = statistics.median(per_step_s)
+    value = keys_per_step / med
+    sample = (f"each step: one decode step of one {w.name} layer ({keys_per_step} keys) on {pool} host thread(s), "
+              f"one per (batch, KV head) pair; median of {args.steps}")
     return {
         "impl": "reference",
         "metric": "decode retrieval+sparse-attn keys scanned/s (also us/layer and % HBM roofline)",
         "value": value, "unit": "keys/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": statistics.mean(per_step_s) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": med * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (two-cone Gaussian, host generator)",
         "config": {"workload": w.name, "layers_per_step": 1},
-        "cpu_baseline": {"value": value, "unit": "keys/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "keys/s", "cores": pool, "kind": "oracle", "sample": sample,
+                         "host_cores": cores, "cpu_model": model},
         "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -630,15 +759,10 @@ def main():
             print(json.dumps(res), flush=True)
         return
     init_dist(world, local)
-    res, layers, w = run_gpu(args, rank, world, local)
+    res, cpu_layer, w = run_gpu(args, rank, world, local)
     if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
-            v, sample, cores = oracle_sample(w, args.cpu_budget_s, oracle_inputs_from_device(w, layers[0]))
-            res["cpu_baseline"] = {"value": v, "unit": "keys/s", "cores": cores, "kind": "oracle", "sample": sample}
-        else:
-            res["cpu_baseline"] = None
+        res["cpu_baseline"] = oracle_sample(w, args.cpu_budget_s, cpu_layer) if cpu_layer is not None else None
         print(json.dumps(res), flush=True)
-    del layers
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
