@@ -649,7 +649,8 @@ __device__ void attn_warps(const FusedArgs& a, int64_t kvc, int nrows, RowAt row
   float* wp = reinterpret_cast<float*>(slots);   // [kAW][g][kPart]
   float* wts = wp + (size_t)kAW * g * kPart;     // [kAW][kMaxGroup] weights
   float* ML = wts + kAW * kMaxGroup;             // [g][2]: M, L
-  if (warp < kAW) {
+  const int nact = min(kAW, nsteps);             // warps that took a step
+  if (warp < nact) {
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
       if (gid < g) *reinterpret_cast<float2*>(wp + ((size_t)warp * g + gid) * kPart + 4 + 8 * n + 2 * tq) = make_float2(o[n][0], o[n][1]);
@@ -669,11 +670,10 @@ __device__ void attn_warps(const FusedArgs& a, int64_t kvc, int nrows, RowAt row
   }
   __syncthreads();
   HKV_TL(20);
-  if (tid < kAW * g) {  // weight of warp w for head h
+  if (tid < nact * g) {  // weight of warp w for head h
     const int w = tid / g, h = tid % g;
     float M = -INFINITY;
-#pragma unroll
-    for (int v = 0; v < kAW; ++v) M = fmaxf(M, wp[((size_t)v * g + h) * kPart]);
+    for (int v = 0; v < nact; ++v) M = fmaxf(M, wp[((size_t)v * g + h) * kPart]);
     const float mw = wp[((size_t)w * g + h) * kPart];
     wts[w * kMaxGroup + h] = mw == -INFINITY ? 0.f : expf(mw - M);
     if (w == 0) ML[2 * h] = M;
@@ -681,15 +681,15 @@ __device__ void attn_warps(const FusedArgs& a, int64_t kvc, int nrows, RowAt row
   __syncthreads();
   if (tid < g) {
     float L = 0.f;
-#pragma unroll
-    for (int v = 0; v < kAW; ++v) L = fmaf(wp[((size_t)v * g + tid) * kPart + 1], wts[v * kMaxGroup + tid], L);
+    for (int v = 0; v < nact; ++v) L = fmaf(wp[((size_t)v * g + tid) * kPart + 1], wts[v * kMaxGroup + tid], L);
     ML[2 * tid + 1] = L;
+    if (nact == 0) ML[2 * tid] = -INFINITY;  // no rows: an empty partial
   }
   for (int i = tid; i < g * kHeadDim; i += kThreads) {
     const int h = i / kHeadDim, c = i % kHeadDim;
     float O = 0.f;
 #pragma unroll
-    for (int w = 0; w < kAW; ++w) O = fmaf(wp[((size_t)w * g + h) * kPart + 4 + c], wts[w * kMaxGroup + h], O);
+    for (int w = 0; w < nact; ++w) O = fmaf(wp[((size_t)w * g + h) * kPart + 4 + c], wts[w * kMaxGroup + h], O);
     dst[h * kPart + 4 + c] = O;
   }
   __syncthreads();  // ML (L of every head) is complete
@@ -1147,6 +1147,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     sh[1] = a.nbins - 1;  // defaults: block hi, speculative bound, count below hi
     sh[3] = a.nbins - 1;
     sh[4] = 0;
+    sh[9] = a.nbins - 1;
   }
   const int R_res = sink_n + local_n;
   const int n_res = seg < R_res ? (R_res - seg + nseg - 1) / nseg : 0;
@@ -1157,6 +1158,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   if (ATTEND && !a.spec && tid < n_res) prefetch_row_l2<T>(a.K, a.V, kvc + res_row(tid));
   // ---------------- phase A: query codes, histogram reset -------------------
   if (ATTEND && tid < a.g * (kHeadDim / 4)) *reinterpret_cast<float4*>(&aq_s[tid * 4]) = aq;
+
   if (a.qenc == kQGiven) {
     if (tid < gw) qc_s[tid] = qcode_reg;
   } else if (a.qenc == kQSign) {
@@ -1177,6 +1179,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   for (int i = tid; i < a.nbins_pad; i += kThreads) hist_s[i] = 0u;
   __syncthreads();
   HKV_TL(1);
+  if constexpr (ATTEND && sizeof(T) == 2) fill_qs(a.g, aq_s, qs_s);  // read only after later barriers
   if (a.q_codes_out != nullptr && seg == 0)
     for (int i = tid; i < gw; i += kThreads) a.q_codes_out[qrow0 * W + i] = qc_s[i];
 
@@ -1229,6 +1232,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   const uint32_t k_eff = (uint32_t)k_eff_p;
   const int spec_cap = kRows - n_res;  // speculative rows that fit beside the resident ones in one tile
   int hi, tb;
+  // this block's proportional share of the selection (for the threshold estimate)
+  const uint32_t share = C > 0 ? (uint32_t)max(1ll, ((long long)k_eff * len + C - 1) / C) : 1u;
   {
     uint32_t cnt[4], cum[4];
     const uint4 hv = 4 * tid < a.nbins_pad ? *reinterpret_cast<const uint4*>(hist_s + 4 * tid) : make_uint4(0u, 0u, 0u, 0u);
@@ -1241,6 +1246,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
           sh[1] = v;
           sh[4] = (int)(cum[e] - cnt[e]);
         }
+        // estimate of the pair's threshold: where this block holds its share of k_eff
+        if (cum[e] >= share && cum[e] - cnt[e] < share) sh[9] = v;
         // speculative bound: the largest bin whose cumulative count fits spec_cap
         if (cum[e] > (uint32_t)max(spec_cap, 0) && cum[e] - cnt[e] <= (uint32_t)max(spec_cap, 0)) sh[3] = v - 1;
       }
@@ -1289,7 +1296,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       if ((tid >> 5) < kAW && (tid >> 5) * kWR < n_spec + n_res)  // slot 0 of warps 0-3
         warp_issue(a, kvc, n_spec + n_res, spec_row, tid >> 5, smem + (size_t)(tid >> 5) * kSlotBytes,
                    tokw_s + (tid >> 5) * kWR);
-      fill_qs(a.g, aq_s, qs_s);
       HKV_TL(12);
     }
   }
@@ -1306,6 +1312,15 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   if (arrived) {
     int thr = max(hi, 0);
     uint32_t below = (uint32_t)sh[4];
+    // lower segments' cumulative counts over a window of 8 bins around this
+    // block's estimate of T, loaded in the same round as the pair histogram
+    // (pairs of at most kThreads / 8 blocks: one load per thread)
+    const int w0 = max(0, sh[9] - 5);
+    const bool win = seg <= kThreads / 8;
+    const int wss = tid >> 3, wj = tid & 7;
+    const uint32_t wv = win && wss < seg && w0 + wj < a.nbins
+                            ? __ldcg(a.cum + ((int64_t)p * nseg + wss) * a.nbins_pad + w0 + wj)
+                            : 0u;
     if (nseg > 1) {
       // the pair's histogram: four bins per thread, one load round
       uint32_t cnt[4], cum[4];
@@ -1328,12 +1343,21 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       thr = sh[5];
       below = (uint32_t)sh[6];
     }
-    // tokens of the lower segments below and at the threshold
+    // tokens of the lower segments below and at the threshold (from the
+    // window when it holds T - 1 and T; values past a segment's hi are stale
+    // but never used: T <= every segment's hi)
     uint32_t seg_lt = 0, seg_le = 0;
-    for (int ss = tid; ss < seg; ss += kThreads) {
-      const uint32_t* c = a.cum + ((int64_t)p * nseg + ss) * a.nbins_pad;
-      seg_lt += thr > 0 ? __ldcg(c + thr - 1) : 0u;
-      seg_le += __ldcg(c + thr);
+    if (win && thr >= w0 && thr <= w0 + 7 && (thr == 0 || thr - 1 >= w0)) {
+      if (wss < seg) {
+        if (wj == thr - w0) seg_le += wv;
+        if (wj == thr - 1 - w0) seg_lt += wv;
+      }
+    } else {
+      for (int ss = tid; ss < seg; ss += kThreads) {
+        const uint32_t* c = a.cum + ((int64_t)p * nseg + ss) * a.nbins_pad;
+        seg_lt += thr > 0 ? __ldcg(c + thr - 1) : 0u;
+        seg_le += __ldcg(c + thr);
+      }
     }
     block_sum2(seg_lt, seg_le, warp_tmp);
     const uint32_t lower_lt = seg_lt, lower_eq = seg_le - seg_lt;
@@ -1419,7 +1443,6 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
         if (spec_ok) {
           attn_warps(a, kvc, n_spec + n_res, spec_row, smem, tokw_s, qs_s, dst, (n_spec + n_res + kWR - 1) / kWR);
         } else {
-          fill_qs(a.g, aq_s, qs_s);
           attn_warps(a, kvc, ns + n_res, row_at, smem, tokw_s, qs_s, dst, 0);
         }
       } else {
