@@ -31,7 +31,7 @@ __all__ = [
     "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_retrieve_topk_normw", "hkv_sparse_attend",
     "hkv_evict_select", "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads",
     "hkv_decode_step_ragged", "hkv_split_select", "hkv_lse_merge_n", "hkv_retrieve_topk_paged",
-    "hkv_sparse_attend_paged", "hkv_debug_set", "EXPORTS",
+    "hkv_sparse_attend_paged", "hkv_decode_step_paged", "hkv_debug_set", "EXPORTS",
 ]
 
 HKV_OK, HKV_ERR_INVALID_ARG, HKV_ERR_UNSUPPORTED, HKV_ERR_CAPACITY = 0, -1, -2, -3
@@ -46,7 +46,7 @@ EXPORTS = (
     "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_retrieve_topk_normw", "hkv_sparse_attend",
     "hkv_evict_select", "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads",
     "hkv_decode_step_ragged", "hkv_split_select", "hkv_lse_merge_n", "hkv_retrieve_topk_paged",
-    "hkv_sparse_attend_paged", "hkv_debug_set",
+    "hkv_sparse_attend_paged", "hkv_decode_step_paged", "hkv_debug_set",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -95,7 +95,10 @@ _SIGS = {
     "hkv_evict_select": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _P, _P, _P, _SZ, _P]),
     "hkv_split_select": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "hkv_lse_merge_n": (_I, [_I, _I64, _P, _P, _P, _P, _P]),
-    "hkv_retrieve_topk_paged": (_I, [_I, _I, _I, _I, _P, _P, _P, _I64, _I64, _I, _I64, _I, _I, _I, _P, _P, _P, _P]),
+    "hkv_retrieve_topk_paged": (_I, [_I, _I, _I, _I, _P, _P, _P, _I64, _I64, _I, _I64, _I, _I, _I, _P, _P, _P, _SZ, _P,
+                                     _P]),
+    "hkv_decode_step_paged": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _P, _I64, _I64, _I, _I64, _I,
+                                   _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "hkv_sparse_attend_paged": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _I64, _I64, _I, _I64, _P, _I, _I, _I, _F, _P, _P,
                                      _P, _SZ, _P, _P]),
     "hkv_write_slots": (_I, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P]),
@@ -457,8 +460,9 @@ def hkv_lse_merge_n(o, lse, out, lse_out=None, stream=None) -> None:
 
 
 def hkv_retrieve_topk_paged(q_codes, codes_pool, page_table, n_tokens: int, n_sink: int, n_local: int, top_k: int,
-                            idx, dist=None, status=None, stream=None) -> None:
-    """codes_pool [num_pages, Hkv, page_size, W]; page_table [B, max_pages] int32 -> idx [B, Hkv, top_k]."""
+                            idx, dist=None, status=None, stream=None, ws=None) -> None:
+    """codes_pool [num_pages, Hkv, page_size, W]; page_table [B, max_pages] int32 -> idx [B, Hkv, top_k].
+    ws: optional workspace (hkv.workspace of the same shape) for the multi-block path at any length."""
     B, Hq, W = q_codes.shape
     num_pages, Hkv, page_size, W2 = codes_pool.shape
     _need(q_codes, "q_codes", _U32)
@@ -473,7 +477,9 @@ def hkv_retrieve_topk_paged(q_codes, codes_pool, page_table, n_tokens: int, n_si
         raise ValueError("q_codes and codes_pool differ in code width")
     _ok(lib().hkv_retrieve_topk_paged(B, Hq, Hkv, W * 32, _ptr(q_codes), _ptr(codes_pool), _ptr(page_table),
                                       page_table.shape[1], num_pages, page_size, n_tokens, n_sink, n_local, top_k,
-                                      _ptr(idx), _ptr(dist), _ptr(status), _stream(stream)))
+                                      _ptr(idx), _ptr(dist), _ptr(ws),
+                                      0 if ws is None else ws.numel() * ws.element_size(), _ptr(status),
+                                      _stream(stream)))
 
 
 def hkv_sparse_attend_paged(q, K_pool, V_pool, page_table, n_tokens: int, idx, n_sink: int, n_local: int, out,
@@ -561,3 +567,32 @@ def hkv_decode_step(h: HashParams, q, k_codes, K, V, n_tokens: int, n_sink: int,
     _ok(lib().hkv_decode_step(ctypes.byref(h.c), B, Hq, Hkv, _ptr(q), _ptr(k_codes), _ptr(K), _ptr(V), cap, n_tokens,
                               n_sink, n_local, top_k, scale, _ptr(q_codes), _ptr(idx), _ptr(out), _ptr(lse),
                               _ptr(next_k_codes), _ptr(ws), nbytes, _ptr(status), _stream(stream)))
+
+
+def hkv_decode_step_paged(h: HashParams, q, codes_pool, K_pool, V_pool, page_table, n_tokens: int, n_sink: int,
+                          n_local: int, top_k: int, out, lse=None, q_codes=None, idx=None, scale: Optional[float] = None,
+                          ws=None, status=None, stream=None) -> None:
+    """hkv_decode_step over a paged cache: codes_pool [num_pages, Hkv, page_size, W], K_pool and V_pool
+    [num_pages, Hkv, page_size, 128], page_table [B, max_pages] int32."""
+    B, Hq, d = q.shape
+    num_pages, Hkv, page_size, W = codes_pool.shape
+    _need(q, "q", (torch.bfloat16, torch.float32))
+    _need(codes_pool, "codes_pool", _U32)
+    _need(K_pool, "K_pool", q.dtype, shape=(num_pages, Hkv, page_size, d))
+    _need(V_pool, "V_pool", q.dtype, shape=(num_pages, Hkv, page_size, d))
+    _need(page_table, "page_table", torch.int32)
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, max_pages]")
+    _need(out, "out", torch.float32, shape=(B, Hq, d))
+    if q_codes is not None:
+        _need(q_codes, "q_codes", _U32, shape=(B, Hq, W))
+    if idx is not None:
+        _need(idx, "idx", torch.int32, shape=(B, Hkv, top_k))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, shape=(B, Hq))
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _ok(lib().hkv_decode_step_paged(ctypes.byref(h.c), B, Hq, Hkv, _ptr(q), _ptr(codes_pool), _ptr(K_pool),
+                                    _ptr(V_pool), _ptr(page_table), page_table.shape[1], num_pages, page_size, n_tokens,
+                                    n_sink, n_local, top_k, scale, _ptr(q_codes), _ptr(idx), _ptr(out), _ptr(lse),
+                                    _ptr(ws), nbytes, _ptr(status), _stream(stream)))

@@ -351,7 +351,7 @@ static int check_pages(const int32_t* page_table, int64_t max_pages, int64_t num
 int hkv_retrieve_topk_paged(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
                             const uint32_t* codes_pool, const int32_t* page_table, int64_t max_pages,
                             int64_t num_pages, int page_size, int64_t n_tokens, int n_sink, int n_local, int top_k,
-                            int32_t* idx, int32_t* dist, int32_t* status, void* stream) {
+                            int32_t* idx, int32_t* dist, void* ws, size_t ws_bytes, int32_t* status, void* stream) {
   int rc = check_heads(B, Hq, Hkv);
   if (rc == HKV_OK) rc = check_window(n_tokens, n_tokens, n_sink, n_local, top_k);
   if (rc != HKV_OK) return rc;
@@ -363,8 +363,14 @@ int hkv_retrieve_topk_paged(int B, int Hq, int Hkv, int code_bits, const uint32_
   if (!q_codes || !codes_pool || !idx) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned(codes_pool, code_bits / 8))
     return fail(HKV_ERR_INVALID_ARG, "codes_pool must be %d-byte aligned", code_bits / 8);
-  RetrieveShape s{B, Hq, Hkv, code_bits / 32, n_tokens, n_tokens, n_sink, n_local, top_k};
-  return launch_retrieve_paged(s, pm, q_codes, codes_pool, idx, dist, status, static_cast<cudaStream_t>(stream));
+  if (ws == nullptr) {
+    RetrieveShape s{B, Hq, Hkv, code_bits / 32, n_tokens, n_tokens, n_sink, n_local, top_k};
+    return launch_retrieve_paged(s, pm, q_codes, codes_pool, idx, dist, status, static_cast<cudaStream_t>(stream));
+  }
+  // with a workspace: the multi-block scan and selection of hkv_retrieve_topk,
+  // reading the codes through the page table
+  RetrieveShape s{B, Hq, Hkv, code_bits / 32, n_tokens, n_tokens, n_sink, n_local, top_k, 0, nullptr, &pm};
+  return launch_retrieve(s, q_codes, codes_pool, idx, dist, ws, ws_bytes, status, static_cast<cudaStream_t>(stream));
 }
 
 int hkv_sparse_attend_paged(int B, int Hq, int Hkv, int dtype, const void* q, const void* K_pool, const void* V_pool,
@@ -402,7 +408,7 @@ static int decode_impl(bool per_head, const int32_t* n_tok_b, const hkv_hash* q_
                     int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,
                     uint32_t* q_codes, int32_t* idx, float* out, float* lse,
                     const uint32_t* next_k_codes, void* ws, size_t ws_bytes, int32_t* status,
-                    void* stream) {
+                    void* stream, const PageMap* pm = nullptr) {
   int rc = check_hash(q_hash, true);
   if (rc == HKV_OK) rc = check_heads(B, Hq, Hkv);
   if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
@@ -429,7 +435,7 @@ static int decode_impl(bool per_head, const int32_t* n_tok_b, const hkv_hash* q_
   int32_t* ix = idx ? idx : reinterpret_cast<int32_t*>(base + L.fused + L.attend + L.qcodes);
   const int W = q_hash->code_bits / 32;
   const Window w = window(n_tokens, n_sink, n_local);
-  RetrieveShape rs{B, Hq, units, W, cap, n_tokens, n_sink, n_local, top_k, per_head ? Hkv : 0, n_tok_b};
+  RetrieveShape rs{B, Hq, units, W, cap, n_tokens, n_sink, n_local, top_k, per_head ? Hkv : 0, n_tok_b, pm};
   const bool fused_encode = !given_codes && w.C > 0 && top_k > 0 &&
                             decode_encodes_queries(rs, q_hash->kind, q_hash->dtype);
   if (!given_codes && !fused_encode) {
@@ -446,7 +452,7 @@ static int decode_impl(bool per_head, const int32_t* n_tok_b, const hkv_hash* q_
       if (rc != HKV_OK) return rc;
     }
     AttendShape as{B, Hq, Hkv, q_hash->dtype, cap, n_tokens, top_k, n_sink, n_local};
-    return launch_attend(as, q, K, V, ix, scale, out, lse, ws_a, L.attend, status, st);
+    return launch_attend(as, q, K, V, ix, scale, out, lse, ws_a, L.attend, status, st, pm);
   }
   if (fused_encode)
     return launch_decode(rs, q_hash->dtype, q_hash->kind, q_hash->R, nullptr, qc, k_codes, next_k_codes, ix, q, K, V,
@@ -463,6 +469,18 @@ int hkv_decode_step(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* 
                     void* stream) {
   return decode_impl(false, nullptr, q_hash, B, Hq, Hkv, q, k_codes, K, V, cap, n_tokens, n_sink, n_local, top_k,
                      scale, q_codes, idx, out, lse, next_k_codes, ws, ws_bytes, status, stream);
+}
+
+int hkv_decode_step_paged(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q, const uint32_t* codes_pool,
+                          const void* K_pool, const void* V_pool, const int32_t* page_table, int64_t max_pages,
+                          int64_t num_pages, int page_size, int64_t n_tokens, int n_sink, int n_local, int top_k,
+                          float scale, uint32_t* q_codes, int32_t* idx, float* out, float* lse, void* ws,
+                          size_t ws_bytes, int32_t* status, void* stream) {
+  PageMap pm;
+  const int rc = check_pages(page_table, max_pages, num_pages, page_size, n_tokens, pm);
+  if (rc != HKV_OK) return rc;
+  return decode_impl(false, nullptr, q_hash, B, Hq, Hkv, q, codes_pool, K_pool, V_pool, n_tokens, n_tokens, n_sink,
+                     n_local, top_k, scale, q_codes, idx, out, lse, nullptr, ws, ws_bytes, status, stream, &pm);
 }
 
 int hkv_decode_step_heads(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,

@@ -38,6 +38,15 @@ int launch_mlp_pack(const hkv_hash& h, void* packed, cudaStream_t st);
 int launch_copy_rows(int dtype, int64_t groups, int64_t T, const void* src, void* dst,
                      int64_t dst_group_rows, int64_t dst_row0, cudaStream_t st);
 
+// ---- paged caches ----
+// Pool page table[b * max_pages + j] holds tokens [j * page_size,
+// (j + 1) * page_size) of sequence b; a page stores [Hkv, page_size, ...].
+struct PageMap {
+  const int32_t* table = nullptr;
+  int64_t max_pages = 0, num_pages = 0;
+  int page_size = 0;
+};
+
 // ---- retrieval (retrieve.cu) ----
 // Hkv is the number of selection units per batch: KV heads (one index set
 // per KV head, scored by the sum over its g query heads), or the query heads
@@ -48,6 +57,7 @@ struct RetrieveShape {
   int n_sink, n_local, top_k;
   int kv_heads = 0;  // KV heads of the cache when they differ from Hkv
   const int32_t* n_tok_b = nullptr;  // device [B]: ragged lengths, each <= N (N plans the launch)
+  const PageMap* pm = nullptr;       // paged cache: codes, K and V are pools read through pm
 };
 size_t retrieve_ws_bytes(const RetrieveShape& s);
 int launch_retrieve(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,
@@ -91,13 +101,6 @@ int launch_lse_merge_n(int G, int64_t rows, const float* o, const float* lse, fl
                        cudaStream_t st);
 
 // ---- paged caches (paged.cu, attend.cu) ----
-// Pool page table[b * max_pages + j] holds tokens [j * page_size,
-// (j + 1) * page_size) of sequence b; a page stores [Hkv, page_size, ...].
-struct PageMap {
-  const int32_t* table = nullptr;
-  int64_t max_pages = 0, num_pages = 0;
-  int page_size = 0;
-};
 // Group-Hamming top-k over a paged code pool; up to 65536 candidates per pair.
 int launch_retrieve_paged(const RetrieveShape& s, const PageMap& pm, const uint32_t* q_codes,
                           const uint32_t* codes_pool, int32_t* idx, int32_t* dist, int32_t* status, cudaStream_t st);

@@ -118,12 +118,36 @@ struct FusedArgs {
   int32_t* status;
   uint64_t wait_ns;
   int skip_arrive;
+  // paged cache (ptab != nullptr): token t of a sequence is slot t % page_size
+  // of pool page ptab[b * max_pages + t / page_size]; codes, K and V are pools
+  // [num_pages, Hkv_real, page_size, ...]
+  const int32_t* ptab;
+  int64_t max_pages, num_pages;
+  int page_size, ps_shift;  // ps_shift: log2(page_size) for a power of two, else -1
 };
 
 // Cache row of (batch, KV head) for selection unit p (units = KV heads, or
 // query heads with unit_div = g of them per KV head).
 __device__ __forceinline__ int64_t kv_row(const FusedArgs& a, int p) {
   return (int64_t)(p / a.Hkv) * a.Hkv_real + (p % a.Hkv) / a.unit_div;
+}
+
+// Row of token t of unit p in the code, K and V arrays: kvc + t for a
+// contiguous cache (kvc = the unit's first row); for a paged cache the row of
+// its slot in its pool page, or -1 when the page id is outside the pool.
+__device__ __forceinline__ int64_t cache_row(const FusedArgs& a, int p, int64_t kvc, int t) {
+  if (a.ptab == nullptr) return kvc + t;
+  int j, slot;
+  if (a.ps_shift >= 0) {
+    j = t >> a.ps_shift;
+    slot = t & (a.page_size - 1);
+  } else {
+    j = t / a.page_size;
+    slot = t - j * a.page_size;
+  }
+  const int pg = __ldg(a.ptab + (int64_t)(p / a.Hkv) * a.max_pages + j);
+  if (pg < 0 || (int64_t)pg >= a.num_pages) return -1;
+  return ((int64_t)pg * a.Hkv_real + (p % a.Hkv) / a.unit_div) * a.page_size + slot;
 }
 
 
@@ -317,11 +341,11 @@ __device__ __forceinline__ void chunk_to_f32(const uint4& raw, float* dst, float
 // 64 rows per tile.  The K/V rows of tile i + 1 are loaded into registers
 // while tile i is computed, so the gather latency overlaps the arithmetic.
 template <typename T, typename RowAt>
-__device__ void attn_rows(const FusedArgs& a, int64_t kvc, int nrows, RowAt row_at, const AttnSmem& sm,
+__device__ void attn_rows(const FusedArgs& a, int p, int64_t kvc, int nrows, RowAt row_at, const AttnSmem& sm,
                           float (&acc)[kOut]) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
-  const T* Kp = tptr<T>(a.K) + kvc * kHeadDim;
-  const T* Vp = tptr<T>(a.V) + kvc * kHeadDim;
+  const T* Kp = tptr<T>(a.K);
+  const T* Vp = tptr<T>(a.V);
   constexpr int EPC = 16 / sizeof(T);           // elements per 16-byte chunk
   constexpr int CPR = kHeadDim / EPC;           // chunks per row
   constexpr int kPer = kRows * CPR / kThreads;  // chunks of each matrix per thread and tile
@@ -333,9 +357,14 @@ __device__ void attn_rows(const FusedArgs& a, int64_t kvc, int nrows, RowAt row_
       const int i = tid + u * kThreads, r = i / CPR, c = i % CPR;
       tk[u] = r0 + r < nrows ? row_at(r0 + r) : -1;
       kr[u] = vr[u] = make_uint4(0u, 0u, 0u, 0u);
+      const int64_t row = tk[u] >= 0 ? cache_row(a, p, kvc, tk[u]) : -1;
+      if (tk[u] >= 0 && row < 0) {  // a page outside the pool: the row is skipped
+        if (c == 0) report(a.status, HKV_ERR_DEVICE_RANGE);
+        tk[u] = -1;
+      }
       if (tk[u] >= 0) {
-        kr[u] = __ldg(reinterpret_cast<const uint4*>(Kp + (int64_t)tk[u] * kHeadDim) + c);
-        vr[u] = __ldg(reinterpret_cast<const uint4*>(Vp + (int64_t)tk[u] * kHeadDim) + c);
+        kr[u] = __ldg(reinterpret_cast<const uint4*>(Kp + row * kHeadDim) + c);
+        vr[u] = __ldg(reinterpret_cast<const uint4*>(Vp + row * kHeadDim) + c);
       }
     }
   };
@@ -500,13 +529,18 @@ __device__ __forceinline__ void fill_qs(int g, const float* aq_s, __nv_bfloat16*
 // chunks of K and V (cp.async, zero-filled for skipped rows); the tokens go
 // to tokw[0, kWR).  One commit group.
 template <typename RowAt>
-__device__ __forceinline__ void warp_issue(const FusedArgs& a, int64_t kvc, int nrows, RowAt row_at, int st,
+__device__ __forceinline__ void warp_issue(const FusedArgs& a, int p, int64_t kvc, int nrows, RowAt row_at, int st,
                                            unsigned char* slot, int* tokw) {
   const int lane = threadIdx.x & 31, r = lane & 15, hf = lane >> 4;
   const int i = st * kWR + r;
-  const int t = i < nrows ? row_at(i) : -1;
+  int t = i < nrows ? row_at(i) : -1;
+  int64_t row = t >= 0 ? cache_row(a, p, kvc, t) : 0;
+  if (row < 0) {  // a page outside the pool: the row is skipped
+    if (hf == 0) report(a.status, HKV_ERR_DEVICE_RANGE);
+    t = -1;
+    row = 0;
+  }
   if (hf == 0) tokw[r] = t;
-  const int64_t row = kvc + (t >= 0 ? t : 0);
   const __nv_bfloat16* Kp = tptr<__nv_bfloat16>(a.K) + row * kHeadDim;
   const __nv_bfloat16* Vp = tptr<__nv_bfloat16>(a.V) + row * kHeadDim;
   __nv_bfloat16* ks = reinterpret_cast<__nv_bfloat16*>(slot) + r * kVP;
@@ -613,7 +647,7 @@ __device__ __forceinline__ void warp_step(const unsigned char* slot, const int* 
 // issued (warp_issue with this row_at) and tokw entries may since have been
 // set to -1 for rows to skip.  Starts and ends with a block barrier.
 template <typename RowAt>
-__device__ void attn_warps(const FusedArgs& a, int64_t kvc, int nrows, RowAt row_at, unsigned char* slots, int* tokw,
+__device__ void attn_warps(const FusedArgs& a, int p, int64_t kvc, int nrows, RowAt row_at, unsigned char* slots, int* tokw,
                            const __nv_bfloat16* qs, float* dst, int pre_steps) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gid = lane >> 2, tq = lane & 3, g = a.g;
   auto slot = [&](int k) { return slots + (size_t)(k * kAW + warp) * kSlotBytes; };
@@ -626,11 +660,11 @@ __device__ void attn_warps(const FusedArgs& a, int64_t kvc, int nrows, RowAt row
   const int nsteps = (nrows + kWR - 1) / kWR;
   if (warp < kAW) {
     // step j of this warp is st = warp + j kAW, in slot j % 2
-    if (warp >= pre_steps && warp < nsteps) warp_issue(a, kvc, nrows, row_at, warp, slot(0), tw(0));
+    if (warp >= pre_steps && warp < nsteps) warp_issue(a, p, kvc, nrows, row_at, warp, slot(0), tw(0));
     for (int j = 0, st = warp; st < nsteps; ++j, st += kAW) {
       const int nx = st + kAW;
       if (nx < nsteps) {
-        warp_issue(a, kvc, nrows, row_at, nx, slot((j + 1) & 1), tw((j + 1) & 1));
+        warp_issue(a, p, kvc, nrows, row_at, nx, slot((j + 1) & 1), tw((j + 1) & 1));
         cp_async_wait<1>();
       } else {
         cp_async_wait<0>();
@@ -1063,6 +1097,15 @@ __device__ __forceinline__ void cp_async_code(uint32_t* dst, const uint32_t* src
   else
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(d), "l"(src) : "memory");
 }
+// Zero-filled instead when !valid (src must still be a valid address).
+template <int W>
+__device__ __forceinline__ void cp_async_code_zf(uint32_t* dst, const uint32_t* src, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  if constexpr (W == 4)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(valid ? 16 : 0) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(d), "l"(src), "r"(valid ? 8 : 0) : "memory");
+}
 
 // Block b serves pair p0 + b / nseg and its candidate range
 // [s0, s1) = [(b % nseg) * per_block, ...): no block straddles two pairs.
@@ -1138,9 +1181,23 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   const uint32_t* pf_ptr = a.k_codes + (kvc + lo + s0 + tid) * W;
   constexpr int64_t kStep = (int64_t)kThreads * W;
   auto slot = [&](int k) { return ring + ((size_t)(k % kSlots) * kThreads + tid) * 4; };
+  // paged cache: the code of token k of this thread comes through the page
+  // table; a page outside the pool zero-fills its slot and marks it in `bad`
+  const bool paged = a.ptab != nullptr;
+  uint32_t bad = 0, bad_seen = 0;
+  auto issue_code = [&](int k) {
+    if (!paged) {
+      cp_async_code<W>(slot(k), pf_ptr + k * kStep);
+      return;
+    }
+    const int64_t r = cache_row(a, p, 0, lo + s0 + tid + k * kThreads);
+    const uint32_t bit = 1u << (k % kSlots);
+    bad = r < 0 ? (bad | bit) : (bad & ~bit);
+    cp_async_code_zf<W>(slot(k), a.k_codes + (r < 0 ? 0 : r) * W, r >= 0);
+  };
 #pragma unroll
   for (int k = 0; k < kSlots; ++k) {
-    if (k < nt) cp_async_code<W>(slot(k), pf_ptr + k * kStep);
+    if (k < nt) issue_code(k);
     if (k & 1) cp_async_commit();
   }
   if (tid == 0) {
@@ -1155,7 +1212,10 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     const int v = seg + i * nseg;
     return v < sink_n ? v : local_start + (v - sink_n);
   };
-  if (ATTEND && !a.spec && tid < n_res) prefetch_row_l2<T>(a.K, a.V, kvc + res_row(tid));
+  if (ATTEND && !a.spec && tid < n_res) {
+    const int64_t r = cache_row(a, p, kvc, res_row(tid));
+    if (r >= 0) prefetch_row_l2<T>(a.K, a.V, r);
+  }
   // ---------------- phase A: query codes, histogram reset -------------------
   if (ATTEND && tid < a.g * (kHeadDim / 4)) *reinterpret_cast<float4*>(&aq_s[tid * 4]) = aq;
 
@@ -1193,8 +1253,14 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       load_slot<W>(slot(k), ck0);
       const bool two = k + 1 < nt;
       if (two) load_slot<W>(slot(k + 1), ck1);
-      const int D0 = token_distance<W, NP>(ck0, planes);
-      const int D1 = two ? token_distance<W, NP>(ck1, planes) : 0;
+      int D0 = token_distance<W, NP>(ck0, planes);
+      int D1 = two ? token_distance<W, NP>(ck1, planes) : 0;
+      if (paged) {
+        // a token on a page outside the pool gets the largest distance
+        if ((bad >> (k % kSlots)) & 1u) D0 = a.nbins - 1;
+        if (two && ((bad >> ((k + 1) % kSlots)) & 1u)) D1 = a.nbins - 1;
+        bad_seen |= bad & ((1u << (k % kSlots)) | (two ? 1u << ((k + 1) % kSlots) : 0u));
+      }
       const int j0 = tid + k * kThreads;
       dist_s[j0] = (uint16_t)D0;
       atomicAdd(&hist_s[D0], 1u);
@@ -1202,11 +1268,12 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
         dist_s[j0 + kThreads] = (uint16_t)D1;
         atomicAdd(&hist_s[D1], 1u);
       }
-      if (k + kSlots < nt) cp_async_code<W>(slot(k), pf_ptr + (k + kSlots) * kStep);
-      if (k + 1 + kSlots < nt) cp_async_code<W>(slot(k + 1), pf_ptr + (k + 1 + kSlots) * kStep);
+      if (k + kSlots < nt) issue_code(k + kSlots);
+      if (k + 1 + kSlots < nt) issue_code(k + 1 + kSlots);
       cp_async_commit();
     }
     cp_async_wait<0>();
+    if (bad_seen) report(a.status, HKV_ERR_DEVICE_RANGE);
   }
   __syncthreads();
   if (a.next_codes != nullptr && tid < 32) {
@@ -1294,7 +1361,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       __syncthreads();
       HKV_TL(11);
       if ((tid >> 5) < kAW && (tid >> 5) * kWR < n_spec + n_res)  // slot 0 of warps 0-3
-        warp_issue(a, kvc, n_spec + n_res, spec_row, tid >> 5, smem + (size_t)(tid >> 5) * kSlotBytes,
+        warp_issue(a, p, kvc, n_spec + n_res, spec_row, tid >> 5, smem + (size_t)(tid >> 5) * kSlotBytes,
                    tokw_s + (tid >> 5) * kWR);
       HKV_TL(12);
     }
@@ -1441,16 +1508,16 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       float* dst = nseg == 1 ? part_s : a.part + ((int64_t)p * nseg + seg) * a.g * kPart;
       if constexpr (sizeof(T) == 2) {
         if (spec_ok) {
-          attn_warps(a, kvc, n_spec + n_res, spec_row, smem, tokw_s, qs_s, dst, (n_spec + n_res + kWR - 1) / kWR);
+          attn_warps(a, p, kvc, n_spec + n_res, spec_row, smem, tokw_s, qs_s, dst, (n_spec + n_res + kWR - 1) / kWR);
         } else {
-          attn_warps(a, kvc, ns + n_res, row_at, smem, tokw_s, qs_s, dst, 0);
+          attn_warps(a, p, kvc, ns + n_res, row_at, smem, tokw_s, qs_s, dst, 0);
         }
       } else {
         float* attn = reinterpret_cast<float*>(smem);
         const AttnSmem sm{aq_s, attn, attn + kRows * kKP, attn + kRows * kKP + kRows * kHeadDim, tok_s, m_s, l_s, alpha_s};
         float acc[kOut];
         attn_begin(a.g, sm, acc);
-        attn_rows<T>(a, kvc, ns + n_res, row_at, sm, acc);
+        attn_rows<T>(a, p, kvc, ns + n_res, row_at, sm, acc);
         attn_end(a.g, sm, acc, dst);
       }
       __syncthreads();
@@ -1699,6 +1766,18 @@ int launch_fused(const RetrieveShape& s, bool attend, int dtype, int qenc, const
   a.part = reinterpret_cast<float*>(base + pl.ws_sync + pl.ws_gh + pl.ws_cum);
   a.status = status;
   a.wait_ns = wait_limit_ns();
+  if (s.pm != nullptr) {
+    a.ptab = s.pm->table;
+    a.max_pages = s.pm->max_pages;
+    a.num_pages = s.pm->num_pages;
+    a.page_size = s.pm->page_size;
+    a.ps_shift = -1;
+    if ((a.page_size & (a.page_size - 1)) == 0) {
+      a.ps_shift = 0;
+      while ((1 << a.ps_shift) < a.page_size) ++a.ps_shift;
+    }
+    a.next_codes = nullptr;  // the hint is for contiguous caches
+  }
   a.skip_arrive = (debug_flags() & kDebugSkipArrive) ? 1 : 0;
   KernelFn k = pick_kernel(attend, dtype, s.words, pl.np);
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);

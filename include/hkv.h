@@ -375,12 +375,28 @@ int hkv_sparse_attend(int B, int Hq, int Hkv, int dtype, const void* q, const vo
  * attention skips them.
  *
  * Retrieval: idx [B, Hkv, top_k] int32 and nullable dist, as
- * hkv_retrieve_topk.  One block per (batch, KV head), no workspace; at most
- * 65536 candidates per KV head (HKV_ERR_UNSUPPORTED beyond). */
+ * hkv_retrieve_topk.  ws nullable: without a workspace, one block per
+ * (batch, KV head) and at most 65536 candidates per KV head
+ * (HKV_ERR_UNSUPPORTED beyond); with one (hkv_workspace_bytes of the same
+ * shape, zeroed once, as hkv_retrieve_topk's), the multi-block scan and
+ * selection of hkv_retrieve_topk at any length. */
 int hkv_retrieve_topk_paged(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
                             const uint32_t* codes_pool, const int32_t* page_table, int64_t max_pages,
                             int64_t num_pages, int page_size, int64_t n_tokens, int n_sink, int n_local, int top_k,
-                            int32_t* idx, int32_t* dist, int32_t* status, void* stream);
+                            int32_t* idx, int32_t* dist, void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
+/* hkv_decode_step over a paged cache: the same computation (query encode,
+ * retrieval, attention over the selected and resident rows, merge), with the
+ * codes, K and V read through the page table from pools laid out as above
+ * (codes_pool, K_pool, V_pool), the sequence length n_tokens <= max_pages *
+ * page_size, and the workspace of hkv_workspace_bytes(B, Hq, Hkv, n_tokens,
+ * ...).  A page id outside the pool is reported as HKV_ERR_DEVICE_RANGE; its
+ * tokens get the largest distance and are not attended. */
+int hkv_decode_step_paged(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q, const uint32_t* codes_pool,
+                          const void* K_pool, const void* V_pool, const int32_t* page_table, int64_t max_pages,
+                          int64_t num_pages, int page_size, int64_t n_tokens, int n_sink, int n_local, int top_k,
+                          float scale, uint32_t* q_codes, int32_t* idx, float* out, float* lse, void* ws,
+                          size_t ws_bytes, int32_t* status, void* stream);
 
 /* Attention over a paged cache: hkv_sparse_attend with K and V read through
  * the page table (q, idx, out, lse, scale, ws as there; the workspace size

@@ -32,7 +32,7 @@ int main(void) {
   /* workspace sizing rejects a bad group before it asks the device anything */
   expect(hkv_workspace_bytes(1, 6, 4, 1024, 128, 16, 0, 0) == 0, "workspace of a bad shape is 0");
   /* paged: too few pages for the tokens */
-  expect(hkv_retrieve_topk_paged(1, 4, 2, 128, NULL, NULL, NULL, 2, 4, 4, 10, 0, 0, 4, NULL, NULL, NULL, NULL) ==
+  expect(hkv_retrieve_topk_paged(1, 4, 2, 128, NULL, NULL, NULL, 2, 4, 4, 10, 0, 0, 4, NULL, NULL, NULL, 0, NULL, NULL) ==
              HKV_ERR_INVALID_ARG,
          "short page table rejected");
   /* G-way merge with no partials */

@@ -117,13 +117,13 @@ def test_norm_weighted_and_split_argument_errors(lib):
 
 def test_paged_argument_errors(lib):
     # page_size 0, too few pages for n_tokens, NULL page table, too many candidates
-    rc = lib.hkv_retrieve_topk_paged(1, 4, 2, 128, 16, 16, 16, 4, 4, 0, 10, 0, 0, 4, 16, None, None, None)
+    rc = lib.hkv_retrieve_topk_paged(1, 4, 2, 128, 16, 16, 16, 4, 4, 0, 10, 0, 0, 4, 16, None, None, 0, None, None)
     assert rc == hkv.HKV_ERR_INVALID_ARG
-    rc = lib.hkv_retrieve_topk_paged(1, 4, 2, 128, 16, 16, 16, 2, 4, 4, 10, 0, 0, 4, 16, None, None, None)
+    rc = lib.hkv_retrieve_topk_paged(1, 4, 2, 128, 16, 16, 16, 2, 4, 4, 10, 0, 0, 4, 16, None, None, 0, None, None)
     assert rc == hkv.HKV_ERR_INVALID_ARG and "max_pages" in hkv.hkv_last_error()
-    rc = lib.hkv_retrieve_topk_paged(1, 4, 2, 128, 16, 16, None, 4, 4, 4, 10, 0, 0, 4, 16, None, None, None)
+    rc = lib.hkv_retrieve_topk_paged(1, 4, 2, 128, 16, 16, None, 4, 4, 4, 10, 0, 0, 4, 16, None, None, 0, None, None)
     assert rc == hkv.HKV_ERR_INVALID_ARG and "page_table" in hkv.hkv_last_error()
-    rc = lib.hkv_retrieve_topk_paged(1, 4, 2, 128, 16, 16, 16, 1000, 1000, 128, 70000, 0, 0, 4, 16, None, None, None)
+    rc = lib.hkv_retrieve_topk_paged(1, 4, 2, 128, 16, 16, 16, 1000, 1000, 128, 70000, 0, 0, 4, 16, None, None, 0, None, None)
     assert rc == hkv.HKV_ERR_UNSUPPORTED and "65536" in hkv.hkv_last_error()
     rc = lib.hkv_sparse_attend_paged(1, 4, 2, hkv.HKV_BF16, 16, 16, 16, 16, 2, 4, 4, 10, 16, 4, 0, 0, 0.088,
                                      16, None, None, 0, None, None)
