@@ -235,15 +235,17 @@ class Layer:
 
 def paged_roofline(w: synth.Workload, n_layers: int, ms: float, step_ms: float, page: int, peak: float,
                    peak_kind: str) -> dict:
-    """Retrieval over a paged code pool: the candidates' codes are the
-    algorithmic bytes of one launch (the page table is negligible)."""
+    """Paged cache: the retrieval launch (fused scan + select through the page
+    table; the candidates' codes are its algorithmic bytes, the page table is
+    negligible) and the paged decode step (the layer's algorithmic bytes)."""
     nbytes = w.B * w.Hkv * w.candidates() * w.bits // 8
     launch_s = ms * 1e-3 / n_layers
-    return {"kernel": "paged_topk_kernel (scan through the page table + select + ordered compaction)",
+    step_s = step_ms * 1e-3 / n_layers
+    return {"kernel": "fused_kernel, paged (retrieval only: scan + select through the page table)",
             "page_size": page, "bound": "hbm", "achieved": nbytes / launch_s / 1e9, "peak": peak, "unit": "GB/s",
             "frac": nbytes / launch_s / 1e9 / peak, "bytes_per_launch": nbytes, "launch_us": launch_s * 1e6,
-            "step_us_per_layer": step_ms * 1e3 / n_layers, "launches_per_layer": 3, "peak_kind": peak_kind,
-            "traffic": None}
+            "step_us_per_layer": step_s * 1e6, "step_frac": w.algorithmic_bytes() / step_s / 1e9 / peak,
+            "launches_per_layer": 1 if w.hash in ("lsh", "sign") else 2, "peak_kind": peak_kind, "traffic": None}
 
 
 def normw_roofline(w: synth.Workload, n_layers: int, ms: float, step_ms: float, peak: float, peak_kind: str) -> dict:
@@ -484,12 +486,12 @@ def measure_workload(w: synth.Workload, args, dev, world, hkv, full: bool):
                       "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
                       "d2h_bytes_per_step": o_host.numel() * o_host.element_size(), "ms_per_step": e2e_ms,
                       "copies_per_step": 2}
-    # paged cache (pages of 256 tokens scattered through a pool): retrieval and
-    # attention read through the page table, after the query encode
+    # paged cache (pages of 256 tokens scattered through a pool): the fused
+    # multi-block retrieval and the fused decode step read through the page table
     res["paged"] = None
     PAGE = 256
-    if w.candidates() <= 65536 and w.N % PAGE == 0:
-        ws_a = new_ws()
+    if w.N % PAGE == 0:
+        ws_p = new_ws()
         pages = w.N // PAGE
         gen = torch.Generator(device=dev).manual_seed(1234)
         paged_layers = []
@@ -510,15 +512,12 @@ def measure_workload(w: synth.Workload, args, dev, world, hkv, full: bool):
         def paged_only():
             for L, table, cpool, _, _ in paged_layers:
                 hkv.hkv_retrieve_topk_paged(L.q_codes, cpool, table, w.N, w.n_sink, w.n_local, w.top_k, L.idx,
-                                            status=status)
+                                            status=status, ws=ws_p)
 
         def paged_step():
             for L, table, cpool, kpool, vpool in paged_layers:
-                hkv.hkv_encode_keys(L.qh, L.q.view(-1, w.d), L.q_codes.view(-1, w.words))
-                hkv.hkv_retrieve_topk_paged(L.q_codes, cpool, table, w.N, w.n_sink, w.n_local, w.top_k, L.idx,
-                                            status=status)
-                hkv.hkv_sparse_attend_paged(L.q, kpool, vpool, table, w.N, L.idx, w.n_sink, w.n_local, L.out,
-                                            ws=ws_a, status=status)
+                hkv.hkv_decode_step_paged(L.qh, L.q, cpool, kpool, vpool, table, w.N, w.n_sink, w.n_local, w.top_k,
+                                          L.out, q_codes=L.q_codes, idx=L.idx, ws=ws_p, status=status)
 
         g = graph_of(paged_only)
         paged_ms = timed_ms(g, args, world, dev)
@@ -526,6 +525,7 @@ def measure_workload(w: synth.Workload, args, dev, world, hkv, full: bool):
         g = graph_of(paged_step)
         paged_step_ms = timed_ms(g, args, world, dev)
         del g, paged_layers
+        torch.cuda.empty_cache()
         status_ok("paged calls")
         res["paged"] = paged_roofline(w, len(layers), paged_ms, paged_step_ms, PAGE, peak, peak_kind)
     # sign-VQ only: retrieval by the norm-weighted sign score (its own kernel),

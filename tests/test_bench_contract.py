@@ -59,6 +59,7 @@ def test_roofline_arithmetic():
     r = bench.paged_roofline(he, 2, 0.1, 0.3, 256, 6548.8, "measured")
     assert r["bytes_per_launch"] == 8 * 8 * (32768 - 4 - 64) * 8
     assert r["launch_us"] == pytest.approx(50.0) and r["step_us_per_layer"] == pytest.approx(150.0)
+    assert r["step_frac"] == pytest.approx(he.algorithmic_bytes() / 150e-6 / 1e9 / 6548.8)
     e = bench.encode_roofline(he, 1, 1.0)
     assert e["bound"] == "hbm" and e["gbs"] == pytest.approx(8 * 8 * 32768 * (256 + 8) / 1e-3 / 1e9)
     e = bench.encode_roofline(synth.WORKLOADS["spotlight_mlp"], 1, 1.0)
