@@ -69,14 +69,15 @@ struct RowMap {
   int64_t x_group, x_row;  // element strides of the input vectors
   int64_t c_group, c_row;  // word strides of the codes
   int64_t n_group, n_row;  // element strides of the norms
+  // (one group -- every call from hkv_encode_keys -- needs no 64-bit division)
   __device__ __forceinline__ int64_t x_off(int64_t r) const {
-    return (r / per_group) * x_group + (r % per_group) * x_row;
+    return per_group >= rows ? r * x_row : (r / per_group) * x_group + (r % per_group) * x_row;
   }
   __device__ __forceinline__ int64_t c_off(int64_t r) const {
-    return (r / per_group) * c_group + (r % per_group) * c_row;
+    return per_group >= rows ? r * c_row : (r / per_group) * c_group + (r % per_group) * c_row;
   }
   __device__ __forceinline__ int64_t n_off(int64_t r) const {
-    return (r / per_group) * n_group + (r % per_group) * n_row;
+    return per_group >= rows ? r * n_row : (r / per_group) * n_group + (r % per_group) * n_row;
   }
 };
 

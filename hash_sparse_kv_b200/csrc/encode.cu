@@ -376,6 +376,15 @@ mlp_encode_kernel(const T* __restrict__ x, const float* __restrict__ W1,
 }
 
 // --------------------------------------------------------------- SIGN -----
+// Signs and fp16 L2 norm of each row.  The norm must equal the fp16 rounding
+// (to nearest even) of the fp64 norm.  It is first computed in fp32: every
+// square of a bf16 value is exact in fp32, so the sum of 128 of them carries a
+// relative error below 128 * 2^-24 and its square root below 4e-6.  Rounding
+// n (1 - 8e-6) and n (1 + 8e-6) to fp16 then gives the same value whenever the
+// exact norm is far enough from an fp16 rounding midpoint, and that value is
+// the exact norm's rounding; only rows whose interval straddles a midpoint
+// (a few in a hundred) are summed again in fp64.  fp32 inputs (up to 24
+// significant bits) always take the fp64 sum.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 sign_encode_kernel(const T* __restrict__ x, RowMap m, uint32_t* __restrict__ codes,
@@ -384,6 +393,7 @@ sign_encode_kernel(const T* __restrict__ x, RowMap m, uint32_t* __restrict__ cod
   // fp32: four); a warp covers four rows per step and keeps kU steps of loads
   // in flight
   constexpr int D = kHeadDim, EPL = 16, V = 16 / sizeof(T), NV = EPL / V, kU = 4;
+  constexpr bool kExactSquares = sizeof(T) == 2;
   const int lane = threadIdx.x & 31, sub = lane & 7, slot = lane >> 3;
   const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
   const int64_t warp_id = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
@@ -400,14 +410,25 @@ sign_encode_kernel(const T* __restrict__ x, RowMap m, uint32_t* __restrict__ cod
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
       const int64_t row = row0 + u * 4 + slot;
-      const T* e = reinterpret_cast<const T*>(raw[u]);
+      // element i of this lane's 16 (bit operations on the loaded words, so
+      // the loads stay in registers)
+      auto elem = [&](int i) -> float {
+        const uint4 r = raw[u][i / V];
+        const int k = i % V;
+        if constexpr (sizeof(T) == 2) {
+          const uint32_t wd = (k >> 1) == 0 ? r.x : (k >> 1) == 1 ? r.y : (k >> 1) == 2 ? r.z : r.w;
+          return __uint_as_float((k & 1) ? (wd & 0xffff0000u) : (wd << 16));
+        } else {
+          return __uint_as_float(k == 0 ? r.x : k == 1 ? r.y : k == 2 ? r.z : r.w);
+        }
+      };
       uint32_t bits = 0;
-      double ss = 0.0;
+      float ss = 0.f;
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
-        const float f = to_f32(e[i]);
+        const float f = elem(i);
         bits |= (uint32_t)(f > 0.f) << i;
-        ss = fma((double)f, (double)f, ss);
+        ss = fmaf(f, f, ss);
       }
       // word w = dims [32 w, 32 w + 32) = lanes 2 w (low half) and 2 w + 1
       const uint32_t hi_half = __shfl_down_sync(0xffffffffu, bits, 1);
@@ -418,6 +439,24 @@ sign_encode_kernel(const T* __restrict__ x, RowMap m, uint32_t* __restrict__ cod
       ss += __shfl_xor_sync(0xffffffffu, ss, 1);
       ss += __shfl_xor_sync(0xffffffffu, ss, 2);
       ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+      const float n = sqrtf(ss);
+      __half h = __float2half_rn(n);
+      const bool settled = kExactSquares && __half_as_ushort(__float2half_rn(n * (1.f - 8e-6f))) ==
+                                                __half_as_ushort(__float2half_rn(n * (1.f + 8e-6f)));
+      if (__any_sync(0xffffffffu, !settled && norms != nullptr)) {
+        // some row of the warp is close to an fp16 rounding midpoint: its
+        // norm from an fp64 sum (every lane of the warp takes part)
+        double sd = 0.0;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const double f = (double)elem(i);
+          sd = fma(f, f, sd);
+        }
+        sd += __shfl_xor_sync(0xffffffffu, sd, 1);
+        sd += __shfl_xor_sync(0xffffffffu, sd, 2);
+        sd += __shfl_xor_sync(0xffffffffu, sd, 4);
+        if (!settled) h = __double2half(sqrt(sd));
+      }
       if (sub == 0 && row < m.rows) {
         uint32_t* dst = codes + m.c_off(row);
         if (vec_store) {
@@ -428,7 +467,7 @@ sign_encode_kernel(const T* __restrict__ x, RowMap m, uint32_t* __restrict__ cod
           dst[2] = w2;
           dst[3] = w3;
         }
-        if (norms != nullptr) norms[m.n_off(row)] = __half_as_ushort(__double2half(sqrt(ss)));
+        if (norms != nullptr) norms[m.n_off(row)] = __half_as_ushort(h);
       }
     }
   }
