@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--impl", default="hkv", choices=["hkv", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--split", action="store_true",
+                    help="token split: one sequence per layer cut across the ranks (decode_step_split, "
+                         "NCCL all-gathers), strong scaling")
     ap.add_argument("--main-only", action="store_true",
                     help="measure only --workload (skip the other workloads' decode steps)")
     ap.add_argument("--layers", type=int, default=0,
@@ -621,6 +624,64 @@ def run_gpu(args, rank, world, local):
     return out, cpu_layer, w
 
 
+def run_split(args, rank, world, local):
+    """Token split of the workload's sequence across the ranks: rank r holds
+    tokens token_range(N, world, r) of every layer (K, V, codes) and a copy of
+    the queries; one step is decode_step_split on every layer (the ranks'
+    top-k candidates and partial outputs exchanged by NCCL all-gathers),
+    captured in one CUDA graph."""
+    import socket
+    import torch.distributed as dist
+    import hash_sparse_kv_b200 as hkv
+    from hash_sparse_kv_b200 import split as hsplit
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if not dist.is_initialized():
+        # one rank: a process group of one, for the same collective calls
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        import datetime
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120))
+    hkv.lib()
+    w = synth.WORKLOADS[args.workload]
+    r0, r1 = hsplit.token_range(w.N, world, rank)
+    wr = w.with_(N=r1 - r0)
+    n_layers = args.layers or w.layers
+    layers = [Layer(wr, l % w.layers if w.layers > 1 else 0, dev, hkv) for l in range(n_layers)]
+    for L in layers:
+        L.encode_keys(hkv)
+    st = hsplit.SplitState.make(world, rank, w.B, w.Hq, w.Hkv, w.bits, w.top_k, w.N, w.n_sink, w.n_local, dev)
+
+    def step():
+        for L in layers:
+            hsplit.decode_step_split(st, L.qh, L.q, L.codes, L.K, L.V, w.N, w.n_sink, w.n_local, w.bits, L.out)
+
+    g = graph_of(step)
+    check(hkv, st.status, "split decode step")
+    with ClockSampler(dev.index) as clk:
+        mean_ms, med_ms = time_graph(g, args.steps, args.warmup, world)
+    ms = max_over_ranks(med_ms, world, dev)
+    check(hkv, st.status, "split decode step")
+    del g
+    keys = w.B * w.Hkv * w.candidates() * n_layers  # the whole sequence, all ranks together
+    out = {
+        "metric": "decode retrieval+sparse-attn keys scanned/s (also us/layer and % HBM roofline)",
+        "value": keys / (ms * 1e-3), "unit": "keys/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "us_per_layer": ms * 1e3 / n_layers, "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "u32 codes + " + ("bf16" if w.dtype == "bf16" else "f32") + " K/V, f32 accumulate",
+        "data": "synthetic (two-cone Gaussian keys/queries, drawn on device)",
+        "config": {"workload": w.name, "n_tokens": w.N, "tokens_per_rank": r1 - r0, "layers_per_step": n_layers,
+                   "parallelism": f"token split x{world} (NCCL all-gathers of candidates and partials)",
+                   "timing": "median of the per-replay CUDA-event times (max over ranks)"},
+        "gpu_launches": None, "clocks": clk.summary(), "cpu_baseline": None,
+    }
+    dist.barrier()
+    return out
+
+
 # ------------------------------------------------------------------ oracle arm --
 
 def oracle_inputs_from_device(w: synth.Workload, L):
@@ -759,6 +820,13 @@ def main():
             print(json.dumps(res), flush=True)
         return
     init_dist(world, local)
+    if args.split:
+        res = run_split(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        import torch.distributed as dist
+        dist.destroy_process_group()
+        return
     res, cpu_layer, w = run_gpu(args, rank, world, local)
     if rank == 0:
         res["cpu_baseline"] = oracle_sample(w, args.cpu_budget_s, cpu_layer) if cpu_layer is not None else None

@@ -349,9 +349,10 @@ def test_lse_merge_matches_oracle():
 
 # -------------------------------------------------------------------- append
 
-@pytest.mark.parametrize("kind", ["lsh", "sign"])
+@pytest.mark.parametrize("kind", ["lsh", "sign", "mlp"])
 def test_append(kind):
-    w = synth.WORKLOADS["qwen7b_512k" if kind == "lsh" else "signvq"].with_(B=2, N=64, layers=1)
+    name = {"lsh": "qwen7b_512k", "sign": "signvq", "mlp": "spotlight_mlp"}[kind]
+    w = synth.WORKLOADS[name].with_(B=2, N=64, layers=1)
     inp = margin_inputs(w, cap=80)
     params, _, kbad = hash_params(w)
     B, Hkv, cap = w.B, w.Hkv, 80

@@ -18,7 +18,9 @@ import pytest
 import torch
 
 import hash_sparse_kv_b200 as hkv
+import oracle
 import synth
+from tests.helpers import u32
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -49,6 +51,10 @@ def test_static_scratch_matches_workspace_version(case):
     ref_dist = torch.full((B, Hkv, k), -9, dtype=torch.int32, device=DEV)
     hkv.hkv_retrieve_topk(qc, kc, N, s, l, k, ref_idx, ref_dist, ws=ws, status=st)
     assert hkv.hkv_check(st) == hkv.HKV_OK, hkv.hkv_last_error()
+    # the workspace version itself against the oracle
+    want_i, want_d = oracle.retrieve(u32(qc), u32(kc), N, s, l, k)
+    np.testing.assert_array_equal(ref_idx.cpu().numpy(), want_i)
+    np.testing.assert_array_equal(ref_dist.cpu().numpy(), want_d)
     for _ in range(2):
         idx = torch.full((B, Hkv, k), -9, dtype=torch.int32, device=DEV)
         dist = torch.full((B, Hkv, k), -9, dtype=torch.int32, device=DEV)
