@@ -506,7 +506,7 @@ def measure_workload(w: synth.Workload, args, dev, world, hkv, full: bool):
                 # [B, Hkv, N, ...] -> pool page perm[b * pages + j] = tokens [j * PAGE, (j + 1) * PAGE) of b
                 tail = tuple(x.shape[3:])
                 src = x.view((w.B, w.Hkv, pages, PAGE) + tail).transpose(1, 2).reshape((w.B * pages, w.Hkv, PAGE) + tail)
-                pool = torch.empty_like(src)
+                pool = torch.empty(src.shape, dtype=src.dtype, device=src.device)  # contiguous
                 pool[perm.long()] = src
                 return pool
 
