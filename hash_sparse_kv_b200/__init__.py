@@ -31,7 +31,8 @@ __all__ = [
     "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_retrieve_topk_normw", "hkv_sparse_attend",
     "hkv_evict_select", "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads",
     "hkv_decode_step_ragged", "hkv_split_select", "hkv_lse_merge_n", "hkv_retrieve_topk_paged",
-    "hkv_sparse_attend_paged", "hkv_decode_step_paged", "hkv_debug_set", "EXPORTS",
+    "hkv_sparse_attend_paged", "hkv_decode_step_paged", "hkv_normw_workspace_bytes", "normw_workspace",
+    "hkv_debug_set", "EXPORTS",
 ]
 
 HKV_OK, HKV_ERR_INVALID_ARG, HKV_ERR_UNSUPPORTED, HKV_ERR_CAPACITY = 0, -1, -2, -3
@@ -46,7 +47,7 @@ EXPORTS = (
     "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_retrieve_topk_normw", "hkv_sparse_attend",
     "hkv_evict_select", "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads",
     "hkv_decode_step_ragged", "hkv_split_select", "hkv_lse_merge_n", "hkv_retrieve_topk_paged",
-    "hkv_sparse_attend_paged", "hkv_decode_step_paged", "hkv_debug_set",
+    "hkv_sparse_attend_paged", "hkv_decode_step_paged", "hkv_normw_workspace_bytes", "hkv_debug_set",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -91,7 +92,8 @@ _SIGS = {
                                    _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "hkv_decode_step_ragged": (_I, [ctypes.POINTER(hkv_hash), _I, _I, _I, _P, _P, _P, _P, _I64, _P, _I64, _I, _I, _I,
                                     _F, _P, _P, _P, _P, _P, _SZ, _P, _P]),
-    "hkv_retrieve_topk_normw": (_I, [_I, _I, _I, _I, _P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P]),
+    "hkv_retrieve_topk_normw": (_I, [_I, _I, _I, _I, _P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _SZ, _P]),
+    "hkv_normw_workspace_bytes": (_SZ, [_I, _I, _I64, _I, _I, _I]),
     "hkv_evict_select": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _P, _P, _P, _SZ, _P]),
     "hkv_split_select": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "hkv_lse_merge_n": (_I, [_I, _I64, _P, _P, _P, _P, _P]),
@@ -419,10 +421,22 @@ def hkv_decode_step_ragged(h: HashParams, q, k_codes, K, V, n_tokens_b, n_tokens
                                      _stream(stream)))
 
 
+def hkv_normw_workspace_bytes(B: int, Hkv: int, n_tokens: int, n_sink: int, n_local: int, top_k: int) -> int:
+    return lib().hkv_normw_workspace_bytes(B, Hkv, n_tokens, n_sink, n_local, top_k)
+
+
+def normw_workspace(B, Hkv, n_tokens, n_sink, n_local, top_k, device=None) -> Optional[torch.Tensor]:
+    """The workspace of hkv_retrieve_topk_normw for this shape, or None when
+    the call runs one block per KV head without one."""
+    n = hkv_normw_workspace_bytes(B, Hkv, n_tokens, n_sink, n_local, top_k)
+    return None if n == 0 else torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
 def hkv_retrieve_topk_normw(q_codes, k_codes, norms, n_tokens: int, n_sink: int, n_local: int, top_k: int, idx,
-                            score=None, stream=None) -> None:
+                            score=None, ws=None, stream=None) -> None:
     """Top-k per KV head by the norm-weighted sign score norm * (g * bits - 2 D).
-    norms [B, Hkv, cap] fp16 (or its int16 bits); idx [B, Hkv, top_k] int32; score nullable fp32."""
+    norms [B, Hkv, cap] fp16 (or its int16 bits); idx [B, Hkv, top_k] int32; score nullable fp32;
+    ws nullable (normw_workspace): needed past 65536 candidates per KV head."""
     B, Hq, W = q_codes.shape
     _, Hkv, cap, W2 = k_codes.shape
     _need(q_codes, "q_codes", _U32)
@@ -433,8 +447,10 @@ def hkv_retrieve_topk_normw(q_codes, k_codes, norms, n_tokens: int, n_sink: int,
         _need(score, "score", torch.float32, shape=(B, Hkv, top_k))
     if W2 != W:
         raise ValueError("q_codes and k_codes differ in code width")
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _ok(lib().hkv_retrieve_topk_normw(B, Hq, Hkv, W * 32, _ptr(q_codes), _ptr(k_codes), _ptr(norms), cap, n_tokens,
-                                      n_sink, n_local, top_k, _ptr(idx), _ptr(score), _stream(stream)))
+                                      n_sink, n_local, top_k, _ptr(idx), _ptr(score), _ptr(ws), nbytes,
+                                      _stream(stream)))
 
 
 def hkv_split_select(rank: int, Hq: int, code_bits: int, cand_idx, cand_dist, idx, status=None, stream=None) -> None:

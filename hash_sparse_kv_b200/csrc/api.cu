@@ -252,7 +252,8 @@ int hkv_retrieve_topk_static(int B, int Hq, int Hkv, int code_bits, const uint32
 
 int hkv_retrieve_topk_normw(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
                             const uint32_t* k_codes, const uint16_t* norms, int64_t cap, int64_t n_tokens,
-                            int n_sink, int n_local, int top_k, int32_t* idx, float* score, void* stream) {
+                            int n_sink, int n_local, int top_k, int32_t* idx, float* score, void* ws,
+                            size_t ws_bytes, void* stream) {
   int rc = check_heads(B, Hq, Hkv);
   if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
   if (rc != HKV_OK) return rc;
@@ -261,7 +262,17 @@ int hkv_retrieve_topk_normw(int B, int Hq, int Hkv, int code_bits, const uint32_
   if (!q_codes || !k_codes || !norms || !idx) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned(k_codes, code_bits / 8)) return fail(HKV_ERR_INVALID_ARG, "k_codes must be %d-byte aligned", code_bits / 8);
   RetrieveShape s{B, Hq, Hkv, code_bits / 32, cap, n_tokens, n_sink, n_local, top_k};
-  return launch_retrieve_normw(s, q_codes, k_codes, norms, idx, score, static_cast<cudaStream_t>(stream));
+  return launch_retrieve_normw(s, q_codes, k_codes, norms, idx, score, ws, ws_bytes,
+                               static_cast<cudaStream_t>(stream));
+}
+
+size_t hkv_normw_workspace_bytes(int B, int Hkv, int64_t n_tokens, int n_sink, int n_local, int top_k) {
+  if (B < 0 || Hkv < 1 || check_window(n_tokens, n_tokens, n_sink, n_local, top_k) != HKV_OK) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) return 0;
+  const Window w = window(n_tokens, n_sink, n_local);
+  return normw_plan(B * Hkv, w.C, top_k, sms).ws_bytes;
 }
 
 int hkv_split_select(int G, int rank, int B, int Hq, int Hkv, int code_bits, int top_k, const int32_t* cand_idx,

@@ -89,9 +89,19 @@ int launch_write_slots(int dtype, int P, int W, const void* k_new, const void* v
                        const int32_t* slot, int32_t* status, cudaStream_t st);
 
 // ---- norm-weighted sign-VQ retrieval (normw.cu) ----
-// idx/score [B, Hkv, top_k]; at most 65536 candidates per pair.
+// Segments per pair of the norm-weighted retrieval; nseg 1 needs no
+// workspace (one block per pair, at most 65536 candidates).
+struct NormwPlan {
+  int nseg = 1;
+  int seg_len = 0;   // candidates per segment, a multiple of 4096
+  int stride = 0;    // workspace entries per (pair, segment), a multiple of 8
+  size_t ws_bytes = 0;
+};
+NormwPlan normw_plan(int P, int64_t C, int top_k, int sms);
+// idx/score [B, Hkv, top_k]; ws nullable (then at most 65536 candidates per pair).
 int launch_retrieve_normw(const RetrieveShape& s, const uint32_t* q_codes, const uint32_t* k_codes,
-                          const uint16_t* norms, int32_t* idx, float* score, cudaStream_t st);
+                          const uint16_t* norms, int32_t* idx, float* score, void* ws, size_t ws_bytes,
+                          cudaStream_t st);
 
 // ---- token split (split.cu) ----
 // cand_idx/cand_dist [G, P, k]; idx_out [P, k]; distances in [0, nbins).

@@ -305,12 +305,26 @@ int hkv_write_slots(int B, int Hkv, int dtype, int code_bits, const void* k_new,
  *           with the sign hash
  *   idx     [B, Hkv, top_k] int32 out;  score  nullable [B, Hkv, top_k]
  *           fp32 out (S of each selected token, -inf past k_eff)
- * One launch, one block per (batch, KV head); no workspace.  At most 65536
- * candidates per KV head (HKV_ERR_UNSUPPORTED beyond).  The selected rows
- * go to hkv_sparse_attend like those of hkv_retrieve_topk. */
+ * ws nullable.  Without a workspace: one launch, one block per (batch, KV
+ * head), at most 65536 candidates per KV head (HKV_ERR_UNSUPPORTED beyond).
+ * With one of hkv_normw_workspace_bytes bytes (16-byte aligned; no zero
+ * fill needed; HKV_ERR_CAPACITY if smaller): when that size is non-zero,
+ * each KV head's window is cut into segments of at most 65536 candidates
+ * (enough of them to fill the GPU when there are few KV heads), one block
+ * per segment keeps the segment's own top_k in the workspace, and a second
+ * launch, one block per KV head, selects the top_k among those lists.  The
+ * result is the same either way.  The selected rows go to
+ * hkv_sparse_attend like those of hkv_retrieve_topk. */
 int hkv_retrieve_topk_normw(int B, int Hq, int Hkv, int code_bits, const uint32_t* q_codes,
                             const uint32_t* k_codes, const uint16_t* norms, int64_t cap, int64_t n_tokens,
-                            int n_sink, int n_local, int top_k, int32_t* idx, float* score, void* stream);
+                            int n_sink, int n_local, int top_k, int32_t* idx, float* score, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* Workspace bytes of hkv_retrieve_topk_normw for this shape on the current
+ * device: 0 when one block per KV head is the plan (no workspace needed),
+ * and 0 if the shape is invalid or no CUDA device is visible (the plan
+ * depends on the SM count). */
+size_t hkv_normw_workspace_bytes(int B, int Hkv, int64_t n_tokens, int n_sink, int n_local, int top_k);
 
 /* Token-split selection.  One sequence's cache is cut into G contiguous
  * token ranges, one per rank, in token order.  Every rank first takes its

@@ -35,6 +35,10 @@ int main(void) {
   expect(hkv_retrieve_topk_paged(1, 4, 2, 128, NULL, NULL, NULL, 2, 4, 4, 10, 0, 0, 4, NULL, NULL, NULL, 0, NULL, NULL) ==
              HKV_ERR_INVALID_ARG,
          "short page table rejected");
+  /* norm-weighted retrieval past 65536 candidates without a workspace */
+  expect(hkv_retrieve_topk_normw(1, 4, 2, 128, (const uint32_t*)16, (const uint32_t*)16, (const uint16_t*)16, 70000,
+                                 70000, 0, 0, 4, (int32_t*)16, NULL, NULL, 0, NULL) == HKV_ERR_UNSUPPORTED,
+         "long normw window without a workspace rejected");
   /* G-way merge with no partials */
   expect(hkv_lse_merge_n(0, 4, NULL, NULL, NULL, NULL, NULL) == HKV_ERR_INVALID_ARG, "G = 0 rejected");
   if (failures == 0) printf("c abi ok\n");

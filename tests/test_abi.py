@@ -91,14 +91,16 @@ def test_eviction_argument_errors(lib):
 
 def test_norm_weighted_and_split_argument_errors(lib):
     # norm-weighted retrieval: bad code width, NULL norms, too many candidates
-    rc = lib.hkv_retrieve_topk_normw(1, 4, 2, 96, None, None, None, 10, 10, 0, 0, 4, None, None, None)
+    rc = lib.hkv_retrieve_topk_normw(1, 4, 2, 96, None, None, None, 10, 10, 0, 0, 4, None, None, None, 0, None)
     assert rc == hkv.HKV_ERR_UNSUPPORTED
-    rc = lib.hkv_retrieve_topk_normw(1, 4, 2, 128, 1, 16, None, 10, 10, 0, 0, 4, 1, None, None)
+    rc = lib.hkv_retrieve_topk_normw(1, 4, 2, 128, 1, 16, None, 10, 10, 0, 0, 4, 1, None, None, 0, None)
     assert rc == hkv.HKV_ERR_INVALID_ARG  # norms is NULL
-    rc = lib.hkv_retrieve_topk_normw(1, 4, 2, 128, 16, 16, 16, 70000, 70000, 0, 0, 4, 16, None, None)
-    assert rc == hkv.HKV_ERR_UNSUPPORTED and "65536" in hkv.hkv_last_error()
-    rc = lib.hkv_retrieve_topk_normw(0, 4, 2, 128, None, None, None, 10, 10, 0, 0, 4, None, None, None)
+    rc = lib.hkv_retrieve_topk_normw(1, 4, 2, 128, 16, 16, 16, 70000, 70000, 0, 0, 4, 16, None, None, 0, None)
+    assert rc == hkv.HKV_ERR_UNSUPPORTED and "workspace" in hkv.hkv_last_error()  # past 65536 without one
+    rc = lib.hkv_retrieve_topk_normw(0, 4, 2, 128, None, None, None, 10, 10, 0, 0, 4, None, None, None, 0, None)
     assert rc == hkv.HKV_OK  # empty batch
+    # no CUDA device here: the workspace size is 0 (the plan needs the SM count)
+    assert lib.hkv_normw_workspace_bytes(1, 2, 200000, 0, 0, 8) == 0
     # token split: rank outside [0, G), NULL candidates
     rc = lib.hkv_split_select(2, 2, 1, 4, 2, 128, 8, None, None, None, None, None)
     assert rc == hkv.HKV_ERR_INVALID_ARG

@@ -24,18 +24,24 @@ def _norms(seed, B, Hkv, cap, pool=None):
     return n.astype(np.float16)
 
 
-def _run(qc, kc, norms, N, s, l, k):
+def _run(qc, kc, norms, N, s, l, k, segmented=False):
     B, Hq, W = qc.shape
     Hkv = kc.shape[1]
     idx = torch.full((B, Hkv, k), -7, dtype=torch.int32, device=DEV)
     score = torch.full((B, Hkv, k), 7.0, dtype=torch.float32, device=DEV)
-    hkv.hkv_retrieve_topk_normw(qc.to(DEV), kc.to(DEV), torch.from_numpy(norms).to(DEV), N, s, l, k, idx, score)
+    ws = None
+    if segmented:
+        ws = hkv.normw_workspace(B, Hkv, N, s, l, k)
+        if ws is not None:
+            ws.fill_(0x5A)  # the call needs no zero fill: every entry it reads is written first
+    hkv.hkv_retrieve_topk_normw(qc.to(DEV), kc.to(DEV), torch.from_numpy(norms).to(DEV), N, s, l, k, idx, score,
+                                ws=ws)
     torch.cuda.synchronize()
     return idx.cpu().numpy(), score.cpu().numpy()
 
 
-def _check(qc, kc, norms, N, s, l, k):
-    got_i, got_s = _run(qc, kc, norms, N, s, l, k)
+def _check(qc, kc, norms, N, s, l, k, segmented=False):
+    got_i, got_s = _run(qc, kc, norms, N, s, l, k, segmented)
     want_i, want_s = oracle.retrieve_normw(qc.numpy().view(np.uint32), kc.numpy().view(np.uint32), norms, N, s, l, k)
     np.testing.assert_array_equal(got_i, want_i)
     np.testing.assert_array_equal(got_s, want_s.astype(np.float32))
@@ -103,3 +109,76 @@ def test_normw_too_many_candidates():
     with pytest.raises(hkv.HkvError) as e:
         hkv.hkv_retrieve_topk_normw(qc, kc, norms, 70000, 0, 0, 8, idx)
     assert e.value.code == hkv.HKV_ERR_UNSUPPORTED
+
+
+SEGMENTED_CASES = [
+    # B, Hq, Hkv, bits, N, cap, sink, local, top_k
+    (1, 8, 2, 128, 200003, 200008, 4, 64, 1024),  # past 65536: many segments per pair, ragged last one
+    (2, 4, 2, 64, 70001, 70001, 0, 0, 100),       # 64-bit codes, g 2
+    (1, 28, 4, 128, 20001, 20008, 8, 128, 1024),  # few pairs: segments fill the GPU
+    (1, 4, 1, 128, 30000, 30000, 0, 0, 5000),     # top_k above a segment: each keeps all of its tokens
+    (1, 16, 1, 64, 777, 800, 4, 64, 1),           # one segment: no workspace
+    (2, 8, 2, 128, 65536, 65536, 0, 0, 512),      # a full one-block window cut into segments
+]
+
+
+@pytest.mark.parametrize("case", SEGMENTED_CASES)
+def test_normw_segmented_parity(case):
+    """With a workspace: segments of at most 65536 candidates, each
+    segment's top-k kept, then the top-k of those lists."""
+    B, Hq, Hkv, bits, N, cap, s, l, k = case
+    W = bits // 32
+    kc = synth.random_codes(81 + N, B * Hkv * cap, W).view(B, Hkv, cap, W)
+    qc = synth.random_codes(82 + N, B * Hq, W).view(B, Hq, W)
+    _check(qc, kc, _norms(83 + N, B, Hkv, cap), N, s, l, k, segmented=True)
+
+
+@pytest.mark.parametrize("pool", [[1.5], [0.0, 1.0, 2.5]])
+def test_normw_segmented_ties(pool):
+    """Equal scores on both sides of every segment boundary: the merge must
+    take the tied tokens of earlier segments first."""
+    B, Hq, Hkv, W, N = 1, 8, 2, 4, 40000
+    codes = synth.random_codes(90, 5, W)
+    rng = np.random.default_rng(91)
+    kc = codes[torch.from_numpy(rng.integers(0, 5, size=B * Hkv * N))].view(B, Hkv, N, W)
+    qc = synth.random_codes(92, B * Hq, W).view(B, Hq, W)
+    norms = _norms(93, B, Hkv, N, pool)
+    assert hkv.hkv_normw_workspace_bytes(B, Hkv, N, 4, 4, 1) > 0
+    for k in (1, 777, 6000, 39990):
+        _check(qc, kc, norms, N, 4, 4, k, segmented=True)
+
+
+def test_normw_segmented_workspace_too_small():
+    qc = torch.zeros(1, 2, 4, dtype=torch.int32, device=DEV)
+    kc = torch.zeros(1, 1, 70000, 4, dtype=torch.int32, device=DEV)
+    norms = torch.zeros(1, 1, 70000, dtype=torch.float16, device=DEV)
+    idx = torch.empty(1, 1, 8, dtype=torch.int32, device=DEV)
+    need = hkv.hkv_normw_workspace_bytes(1, 1, 70000, 0, 0, 8)
+    assert need > 0
+    ws = torch.empty(need - 16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(hkv.HkvError) as e:
+        hkv.hkv_retrieve_topk_normw(qc, kc, norms, 70000, 0, 0, 8, idx, ws=ws)
+    assert e.value.code == hkv.HKV_ERR_CAPACITY
+
+
+@pytest.mark.parametrize("segmented", [False, True])
+def test_normw_best_tokens_in_one_warp_range(segmented):
+    """Every high score sits in the first 3000 tokens: the tokens at or
+    above the threshold bin crowd one warp's share of the block, so the
+    select falls back from its per-warp lists to full passes."""
+    B, Hq, Hkv, W, N, k = 2, 8, 2, 4, 65536, 1000
+    kc = synth.random_codes(95, B * Hkv * N, W).view(B, Hkv, N, W)
+    qc = synth.random_codes(96, B * Hq, W).view(B, Hq, W)
+    norms = _norms(97, B, Hkv, N)
+    norms[:, :, 3000:] = (norms[:, :, 3000:] / 8).astype(np.float16)
+    _check(qc, kc, norms, N, 0, 0, k, segmented)
+
+
+@pytest.mark.slow
+def test_normw_segmented_512k():
+    """One 524288-token layer of the Qwen2.5-7B-shaped cache (28 query and
+    4 KV heads, top 1024) scored norm-weighted through the workspace path."""
+    B, Hq, Hkv, W, N, s, l, k = 1, 28, 4, 4, 524288, 4, 128, 1024
+    kc = synth.random_codes(98, B * Hkv * N, W).view(B, Hkv, N, W)
+    qc = synth.random_codes(99, B * Hq, W).view(B, Hq, W)
+    _check(qc, kc, _norms(100, B, Hkv, N), N, s, l, k, segmented=True)
