@@ -119,6 +119,10 @@ SEGMENTED_CASES = [
     (1, 4, 1, 128, 30000, 30000, 0, 0, 5000),     # top_k above a segment: each keeps all of its tokens
     (1, 16, 1, 64, 777, 800, 4, 64, 1),           # one segment: no workspace
     (2, 8, 2, 128, 65536, 65536, 0, 0, 512),      # a full one-block window cut into segments
+    # 75..148 pairs: one block per pair even with a workspace
+    (16, 32, 8, 128, 65536, 65536, 0, 0, 512),    # the sign-VQ layer shape
+    (32, 12, 4, 64, 50001, 50008, 4, 64, 300),    # g 3, 64-bit codes
+    (20, 28, 4, 128, 40000, 40000, 4, 128, 1024),  # g 7
 ]
 
 
