@@ -984,6 +984,51 @@ __device__ uint32_t compact_block(const uint16_t* dist_s, int len, int thr, uint
   return tot_lt + min(tot_eq, quota);
 }
 
+// Ordered compaction of a small selection: every i < len with D < thr, in
+// ascending order, as emit(pos, i, D); returns their number.  Thread t
+// counts the tokens of its own contiguous run of octets (rotated reads, as
+// in compact_block), one block prefix gives its base, and it emits its
+// tokens in order: no octet list and one barrier pair, for selections of a
+// few dozen tokens (a thread emits at most its own run).  dist_s readable 8
+// entries past len.  All threads call it.
+template <typename Emit>
+__device__ uint32_t compact_few(const uint16_t* dist_s, int len, int thr, uint32_t* warp_tmp, Emit emit) {
+  const int tid = threadIdx.x;
+  const int noct = (len + 7) >> 3;
+  const uint32_t t = (uint32_t)thr;
+  int R = 1;
+  while (R * kThreads < noct) R <<= 1;
+  const int o0 = tid * R;
+  uint32_t fl = 0, cnt = 0;
+  for (int j = 0; j < R; ++j) {
+    const int r = (j + tid) & (R - 1), o = o0 + r;
+    if (o >= noct) continue;
+    const uint4 v = *reinterpret_cast<const uint4*>(dist_s + 8 * o);
+    const uint32_t m = __vminu2(__vminu2(v.x, v.y), __vminu2(v.z, v.w));
+    if (min(m & 0xffffu, m >> 16) >= t) continue;
+    fl |= 1u << r;
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      cnt += (8 * o + e < len && ((wd[e >> 1] >> (16 * (e & 1))) & 0xffffu) < t) ? 1u : 0u;
+  }
+  uint32_t total;
+  uint32_t pos = block_excl_u32(cnt, warp_tmp, &total);
+  while (fl) {
+    const int o = o0 + __ffs(fl) - 1;
+    fl &= fl - 1;
+    const uint4 v = *reinterpret_cast<const uint4*>(dist_s + 8 * o);
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t D = (wd[e >> 1] >> (16 * (e & 1))) & 0xffffu;
+      if (8 * o + e < len && D < t) emit(pos++, 8 * o + e, (int)D);
+    }
+  }
+  __syncthreads();  // warp_tmp is free again
+  return total;
+}
+
 // ------------------------------------------------- query encoding (in kernel)
 // The block's g query heads are encoded into qc_s[h * W + w] (h < g).
 // bf16 LSH: one m16n8k16 tensor-core tile per (16 rows, 8 bits, 16 dims):
@@ -1354,7 +1399,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   auto spec_row = [&](int i) -> int { return i < n_spec ? sel_s[i] : res_row(i - n_spec); };
   if constexpr (ATTEND && sizeof(T) == 2) {
     if (a.spec) {
-      n_spec = (int)compact_block(dist_s, len, tb + 1, 0u, warp_tmp, cscratch, [&](uint32_t pos, int i, int) {
+      n_spec = (int)compact_few(dist_s, len, tb + 1, warp_tmp, [&](uint32_t pos, int i, int) {
         if (pos < (uint32_t)kRows) sel_s[pos] = lo + s0 + i;
       });
       n_spec = min(n_spec, max(spec_cap, 0));
