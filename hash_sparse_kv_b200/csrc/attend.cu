@@ -15,7 +15,8 @@
 // counter in the workspace) merges the splits:
 //   M = max_s m_s,  L = sum_s l_s e^{m_s - M},  out = sum_s acc_s e^{m_s - M} / L,
 //   lse = M + log L.
-// Probabilities and accumulators stay fp32; K/V are widened from bf16.
+// Probabilities and accumulators stay fp32.  This SIMT kernel serves fp32
+// caches; bf16 caches go to the tensor-core kernel (launch_sattend).
 #include <math.h>
 
 #include "internal.h"
@@ -311,13 +312,19 @@ AttendPlan make_plan(const AttendShape& s) {
 
 }  // namespace
 
-size_t attend_ws_bytes(const AttendShape& s) { return make_plan(s).ws_total; }
+// A workspace sized here serves both element types (the bf16 plan is the
+// tensor-core kernel's).
+size_t attend_ws_bytes(const AttendShape& s) {
+  const size_t simt = make_plan(s).ws_total, tc = sattend_ws_bytes(s);
+  return simt > tc ? simt : tc;
+}
 
 int launch_attend(const AttendShape& s, const void* q, const void* K, const void* V,
                   const int32_t* idx, float scale, float* out, float* lse, void* ws,
                   size_t ws_bytes, int32_t* status, cudaStream_t st, const PageMap* pm) {
   const int P = s.B * s.Hkv;
   if (P == 0) return HKV_OK;
+  if (s.dtype == HKV_BF16) return launch_sattend(s, q, K, V, idx, scale, out, lse, ws, ws_bytes, status, st, pm);
   const AttendPlan pl = make_plan(s);
   if ((int64_t)pl.splits * (s.Hq / s.Hkv) > (int64_t)kMaxRows * kKP)
     return fail(HKV_ERR_UNSUPPORTED, "%lld attended rows per KV head is too many", (long long)pl.Rv);

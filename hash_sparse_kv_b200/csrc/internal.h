@@ -125,6 +125,12 @@ size_t attend_ws_bytes(const AttendShape& s);
 int launch_attend(const AttendShape& s, const void* q, const void* K, const void* V,
                   const int32_t* idx, float scale, float* out, float* lse, void* ws,
                   size_t ws_bytes, int32_t* status, cudaStream_t st, const PageMap* pm = nullptr);
+// bf16 sparse attention on the fused kernel's tensor-core attention stage
+// (retrieve.cu); launch_attend sends bf16 shapes here.
+size_t sattend_ws_bytes(const AttendShape& s);
+int launch_sattend(const AttendShape& s, const void* q, const void* K, const void* V, const int32_t* idx, float scale,
+                   float* out, float* lse, void* ws, size_t ws_bytes, int32_t* status, cudaStream_t st,
+                   const PageMap* pm);
 int launch_lse_merge(int rows, int d, const float* o1, const float* lse1, const float* o2,
                      const float* lse2, float* out, float* lse_out, cudaStream_t st);
 

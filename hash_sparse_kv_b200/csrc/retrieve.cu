@@ -984,36 +984,57 @@ __device__ uint32_t compact_block(const uint16_t* dist_s, int len, int thr, uint
   return tot_lt + min(tot_eq, quota);
 }
 
-// Ordered compaction of a small selection: every i < len with D < thr, in
-// ascending order, as emit(pos, i, D); returns their number.  Thread t
-// counts the tokens of its own contiguous run of octets (rotated reads, as
-// in compact_block), one block prefix gives its base, and it emits its
-// tokens in order: no octet list and one barrier pair, for selections of a
-// few dozen tokens (a thread emits at most its own run).  dist_s readable 8
-// entries past len.  All threads call it.
+// Ordered compaction of the block's distances dist_s[0, len) in one pass:
+// emits, in ascending index order, every i with D < thr and the first
+// `quota` with D == thr, as emit(pos, i, D) with pos the rank among the
+// emitted ones; returns their number (compact_block's contract).  Thread t
+// counts the tokens below and at thr in its own contiguous run of octets
+// (rotated reads, as in compact_block), one block prefix of both counts
+// gives its bases, and it emits its tokens in order: no octet list and one
+// barrier pair.  dist_s readable 8 entries past len.  All threads call it.
 template <typename Emit>
-__device__ uint32_t compact_few(const uint16_t* dist_s, int len, int thr, uint32_t* warp_tmp, Emit emit) {
-  const int tid = threadIdx.x;
+__device__ uint32_t compact_few(const uint16_t* dist_s, int len, int thr, uint32_t quota, uint32_t* warp_tmp,
+                                Emit emit) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int noct = (len + 7) >> 3;
   const uint32_t t = (uint32_t)thr;
   int R = 1;
   while (R * kThreads < noct) R <<= 1;
   const int o0 = tid * R;
-  uint32_t fl = 0, cnt = 0;
+  uint32_t fl = 0, lt = 0, eq = 0;
   for (int j = 0; j < R; ++j) {
     const int r = (j + tid) & (R - 1), o = o0 + r;
     if (o >= noct) continue;
     const uint4 v = *reinterpret_cast<const uint4*>(dist_s + 8 * o);
     const uint32_t m = __vminu2(__vminu2(v.x, v.y), __vminu2(v.z, v.w));
-    if (min(m & 0xffffu, m >> 16) >= t) continue;
+    if (min(m & 0xffffu, m >> 16) > t) continue;
     fl |= 1u << r;
     const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      cnt += (8 * o + e < len && ((wd[e >> 1] >> (16 * (e & 1))) & 0xffffu) < t) ? 1u : 0u;
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t D = (wd[e >> 1] >> (16 * (e & 1))) & 0xffffu;
+      const bool in = 8 * o + e < len;
+      lt += (in && D < t) ? 1u : 0u;
+      eq += (in && D == t) ? 1u : 0u;
+    }
   }
-  uint32_t total;
-  uint32_t pos = block_excl_u32(cnt, warp_tmp, &total);
+  // block-wide exclusive prefixes of lt and eq
+  const uint32_t il = warp_incl_u32(lt), ie = warp_incl_u32(eq);
+  __syncthreads();
+  if (lane == 31) {
+    warp_tmp[warp] = il;
+    warp_tmp[kWarps + warp] = ie;
+  }
+  __syncthreads();
+  uint32_t bl = il - lt, be = ie - eq, tot_lt = 0, tot_eq = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const uint32_t x = warp_tmp[w], y = warp_tmp[kWarps + w];
+    bl += w < warp ? x : 0u;
+    be += w < warp ? y : 0u;
+    tot_lt += x;
+    tot_eq += y;
+  }
   while (fl) {
     const int o = o0 + __ffs(fl) - 1;
     fl &= fl - 1;
@@ -1022,11 +1043,19 @@ __device__ uint32_t compact_few(const uint16_t* dist_s, int len, int thr, uint32
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const uint32_t D = (wd[e >> 1] >> (16 * (e & 1))) & 0xffffu;
-      if (8 * o + e < len && D < t) emit(pos++, 8 * o + e, (int)D);
+      const int i = 8 * o + e;
+      if (i >= len) continue;
+      if (D < t) {
+        emit(bl + min(be, quota), i, (int)D);
+        ++bl;
+      } else if (D == t) {
+        if (be < quota) emit(bl + be, i, (int)D);
+        ++be;
+      }
     }
   }
   __syncthreads();  // warp_tmp is free again
-  return total;
+  return tot_lt + min(tot_eq, quota);
 }
 
 // ------------------------------------------------- query encoding (in kernel)
@@ -1399,7 +1428,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   auto spec_row = [&](int i) -> int { return i < n_spec ? sel_s[i] : res_row(i - n_spec); };
   if constexpr (ATTEND && sizeof(T) == 2) {
     if (a.spec) {
-      n_spec = (int)compact_few(dist_s, len, tb + 1, warp_tmp, [&](uint32_t pos, int i, int) {
+      n_spec = (int)compact_few(dist_s, len, tb + 1, 0u, warp_tmp, [&](uint32_t pos, int i, int) {
         if (pos < (uint32_t)kRows) sel_s[pos] = lo + s0 + i;
       });
       n_spec = min(n_spec, max(spec_cap, 0));
@@ -1517,7 +1546,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       if constexpr (ATTEND && sizeof(T) == 2) {
         if (a.spec) cp_async_wait<0>();  // the speculative tile is not used
       }
-      n_sel = compact_block(dist_s, len, thr, quota, warp_tmp, cscratch, [&](uint32_t pos, int i, int D) {
+      auto emit = [&](uint32_t pos, int i, int D) {
         const int tok = lo + s0 + i;
         if (sel_base + pos < k_eff) {
           idx_out[pos] = tok;
@@ -1528,7 +1557,11 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
         } else {
           report(a.status, HKV_ERR_DEVICE_RANGE);  // unreachable when the counts agree
         }
-      });
+      };
+      // short runs per thread (at most two octets): one pass; longer runs
+      // balance better through the octet list
+      n_sel = len <= 16 * kThreads ? compact_few(dist_s, len, thr, quota, warp_tmp, emit)
+                                   : compact_block(dist_s, len, thr, quota, warp_tmp, cscratch, emit);
       if (sel_base + n_sel > k_eff) n_sel = k_eff > sel_base ? k_eff - sel_base : 0u;
     }
   } else {
@@ -1625,6 +1658,115 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
     }
   }
   HKV_TL(10);
+}
+
+// ---------------- standalone sparse attention (bf16) --------------------------
+// hkv_sparse_attend and hkv_sparse_attend_paged for bf16 caches on the fused
+// kernel's attention stage (Spotlight Attention "Approach": exact attention
+// over the retrieved tokens with the sink and local rows; RetrievalAttention
+// "Summary", "Approach": partial results merged by log-sum-exp rescaling).
+// Block x serves pair p = p0 + x / nseg and rows [seg * per_block, ...) of
+// the pair's row list [sink | idx slots | local]; eight warps take 16-row
+// steps with two cp.async slots each (attn_warps).  One segment per pair
+// writes out / lse itself; with several (a cooperative launch) the last g
+// blocks of the pair merge one head each, as in the fused kernel.
+constexpr int kSaTok = 4096;  // row tokens kept in shared memory per block
+
+struct SaLayout {
+  static constexpr size_t qs = kAttnWarpBytes;                                   // bf16 [16][kQP]
+  static constexpr size_t tokw = qs + (size_t)kMaxGroup * kQP * 2;              // int [2][kAW][kWR]
+  static constexpr size_t tok = tokw + (size_t)2 * kAW * kWR * 4;               // int [kSaTok]
+  static constexpr size_t part = tok + (size_t)kSaTok * 4;                      // float [g][kPart]
+  static constexpr size_t total = part + (size_t)kMaxGroup * kPart * 4;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) sattend_kernel(FusedArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __nv_bfloat16* qs_s = reinterpret_cast<__nv_bfloat16*>(smem + SaLayout::qs);
+  int* tokw_s = reinterpret_cast<int*>(smem + SaLayout::tokw);
+  int* tok_s = reinterpret_cast<int*>(smem + SaLayout::tok);
+  float* part_s = reinterpret_cast<float*>(smem + SaLayout::part);
+  __shared__ int sh[2];
+  const int tid = threadIdx.x, g = a.g;
+  const int p = a.p0 + (int)(blockIdx.x / a.nseg), seg = (int)(blockIdx.x % a.nseg);
+  const int nseg = a.nseg;
+  const int64_t Rv = (int64_t)a.sink_n + a.top_k + a.local_n;
+  const int64_t v0 = (int64_t)seg * a.per_block;
+  const int nrows = (int)max((int64_t)0, min((int64_t)a.per_block, Rv - v0));
+  // token of row v of the pair's list (-1: an empty idx slot or a token past N)
+  auto token_of = [&](int64_t v) -> int {
+    if (v < a.sink_n) return (int)v;
+    if (v < (int64_t)a.sink_n + a.top_k) {
+      const int t = __ldg(a.idx + (int64_t)p * a.top_k + (v - a.sink_n));
+      if (t >= a.C) {
+        report(a.status, HKV_ERR_DEVICE_RANGE);
+        return -1;
+      }
+      return t < 0 ? -1 : t;
+    }
+    return a.local_start + (int)(v - a.sink_n - a.top_k);
+  };
+  for (int i = tid; i < min(nrows, kSaTok); i += kThreads) tok_s[i] = token_of(v0 + i);
+  const int b = p / a.Hkv, kvh = p % a.Hkv;
+  const __nv_bfloat16* q0 = tptr<__nv_bfloat16>(a.q) + ((int64_t)b * a.Hq + (int64_t)kvh * g) * kHeadDim;
+  for (int i = tid; i < kMaxGroup * kHeadDim; i += kThreads) {
+    const int h = i / kHeadDim, k = i % kHeadDim;
+    qs_s[h * kQP + k] = h < g ? q0[(int64_t)h * kHeadDim + k] : __float2bfloat16_rn(0.f);
+  }
+  const int64_t kvc = kv_row(a, p) * a.cap;
+  float* dst = nseg == 1 ? part_s : a.part + ((int64_t)p * nseg + seg) * g * kPart;
+  // (attn_warps starts with a block barrier: tok_s and qs_s are complete)
+  attn_warps(a, p, kvc, nrows, [&](int i) -> int { return i < kSaTok ? tok_s[i] : token_of(v0 + i); }, smem,
+             tokw_s, qs_s, dst, 0);
+  if (nseg == 1) {
+    finish_single(a, p, part_s);
+    return;
+  }
+  uint32_t* sync = a.sync + kSync * p;
+  if (tid == 0) sh[0] = (int)atom_acq_rel_add(&sync[2], 1u);
+  __syncthreads();
+  const int nm = min(g, nseg);
+  const int mi = sh[0] - (nseg - nm);
+  if (mi < 0) return;
+  if (tid == 0) sh[1] = wait_count(&sync[2], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
+  __syncthreads();
+  if (sh[1]) {
+    for (int h = mi; h < g; h += nm)
+      merge_head(a.part, a.out, a.lse, a.Hq, a.Hkv, g, p, nseg, h, reinterpret_cast<float*>(smem));
+  } else if (tid == 0) {
+    report(a.status, HKV_ERR_TIMEOUT);
+  }
+  if (tid == 0 && atomicAdd(&sync[3], 1u) == (uint32_t)(nm - 1)) {
+    sync[2] = 0u;  // every block of the pair is past its last use of the counters
+    sync[3] = 0u;
+  }
+}
+
+struct SaPlan {
+  int nseg = 1, per_block = 0, pairs_per_launch = 1;
+  bool cooperative = false;
+  size_t ws_part = 0, ws_sync = 0, ws_total = 0;
+};
+
+SaPlan sattend_plan(const AttendShape& s) {
+  SaPlan pl;
+  const Window w = window(s.N, s.n_sink, s.n_local);
+  const int g = s.Hq / s.Hkv, P = s.B * s.Hkv;
+  const int64_t Rv = std::max<int64_t>(1, w.sink_end + s.top_k + (s.N - w.local_start));
+  const int G = sm_count();
+  // at least one 16-row step per warp and block; one wave of blocks when a
+  // pair is split (its blocks wait for each other)
+  int64_t nseg = 1;
+  if (P > 0 && P < G) nseg = std::max<int64_t>(1, std::min<int64_t>(G / P, ceil_div(Rv, (int64_t)kAW * kWR)));
+  nseg = std::min<int64_t>(nseg, kMaxSegsPerPair);
+  pl.per_block = (int)ceil_div(Rv, nseg);
+  pl.nseg = (int)ceil_div(Rv, pl.per_block);
+  pl.cooperative = pl.nseg > 1;
+  pl.pairs_per_launch = pl.cooperative ? std::max(1, G / pl.nseg) : std::max(P, 1);
+  pl.ws_part = pl.nseg > 1 ? align_up(sizeof(float) * (size_t)P * pl.nseg * g * kPart, 256) : 0;
+  pl.ws_sync = align_up(sizeof(uint32_t) * kSync * (size_t)std::max(P, 1), 256);
+  pl.ws_total = pl.ws_part + pl.ws_sync;
+  return pl;
 }
 
 using KernelFn = void (*)(FusedArgs);
@@ -1859,6 +2001,76 @@ size_t retrieve_ws_bytes(const RetrieveShape& s) {
   Plan pl;
   if (make_plan(s, false, 0, pl) != HKV_OK) return 0;
   return pl.ws_total;
+}
+
+size_t sattend_ws_bytes(const AttendShape& s) { return sattend_plan(s).ws_total; }
+
+int launch_sattend(const AttendShape& s, const void* q, const void* K, const void* V, const int32_t* idx, float scale,
+                   float* out, float* lse, void* ws, size_t ws_bytes, int32_t* status, cudaStream_t st,
+                   const PageMap* pm) {
+  const int P = s.B * s.Hkv;
+  if (P == 0) return HKV_OK;
+  const SaPlan pl = sattend_plan(s);
+  if (ws == nullptr || ws_bytes < pl.ws_total)
+    return fail(HKV_ERR_CAPACITY, "workspace of %zu bytes, %zu needed", ws_bytes, pl.ws_total);
+  const Window w = window(s.N, s.n_sink, s.n_local);
+  FusedArgs a = {};
+  a.q = q;
+  a.K = K;
+  a.V = V;
+  a.idx = const_cast<int32_t*>(idx);
+  a.out = out;
+  a.lse = lse;
+  a.scale = scale;
+  a.Hq = s.Hq;
+  a.Hkv = s.Hkv;
+  a.g = s.Hq / s.Hkv;
+  a.cap = s.cap;
+  a.C = (int)std::min<int64_t>(s.N, INT32_MAX);  // tokens: idx entries at or past it are reported
+  a.top_k = s.top_k;
+  a.sink_n = (int)w.sink_end;
+  a.local_start = (int)w.local_start;
+  a.local_n = (int)(s.N - w.local_start);
+  a.nseg = pl.nseg;
+  a.per_block = pl.per_block;
+  a.Hkv_real = s.Hkv;
+  a.unit_div = 1;
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  a.part = reinterpret_cast<float*>(base);
+  a.sync = reinterpret_cast<uint32_t*>(base + pl.ws_part);
+  a.status = status;
+  a.wait_ns = wait_limit_ns();
+  a.ps_shift = -1;
+  if (pm != nullptr) {
+    a.ptab = pm->table;
+    a.max_pages = pm->max_pages;
+    a.num_pages = pm->num_pages;
+    a.page_size = pm->page_size;
+    if ((a.page_size & (a.page_size - 1)) == 0) {
+      a.ps_shift = 0;
+      while ((1 << a.ps_shift) < a.page_size) ++a.ps_shift;
+    }
+  }
+  cudaError_t e = cudaFuncSetAttribute(sattend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)SaLayout::total);
+  if (e != cudaSuccess) return cuda_check(e, "sparse attention shared memory");
+  for (int p0 = 0; p0 < P; p0 += pl.pairs_per_launch) {
+    a.p0 = p0;
+    const int np = P - p0 < pl.pairs_per_launch ? P - p0 : pl.pairs_per_launch;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(np * pl.nseg));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SaLayout::total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pl.cooperative ? 1 : 0;
+    const int rc = cuda_check(cudaLaunchKernelEx(&cfg, sattend_kernel, a), "sparse attention launch");
+    if (rc != HKV_OK) return rc;
+  }
+  return HKV_OK;
 }
 
 size_t decode_ws_bytes(const RetrieveShape& s) {

@@ -270,6 +270,8 @@ ATTEND_CASES = [
     ("bf16", 1, 28, 4, 9000, 9000, 4, 128, 1024),
     ("bf16", 2, 32, 8, 6000, 6000, 0, 0, 512),
     ("bf16", 1, 16, 1, 500, 512, 4, 64, 2000),
+    ("bf16", 20, 32, 8, 2000, 2000, 4, 64, 300),   # more pairs than SMs: one block per pair, several waves
+    ("bf16", 20, 8, 8, 6000, 6000, 4, 64, 5000),   # rows past the block's shared token list
 ]
 
 
