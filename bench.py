@@ -251,15 +251,26 @@ def paged_roofline(w: synth.Workload, n_layers: int, ms: float, step_ms: float, 
             "launches_per_layer": 1 if w.hash in ("lsh", "sign") else 2, "peak_kind": peak_kind, "traffic": None}
 
 
+def normw_bytes_step(w: synth.Workload) -> int:
+    """Algorithmic bytes of one norm-weighted decode step on one layer: codes and norms of every candidate,
+    the K and V rows of the selected, sink and local tokens, the queries and the fp32 outputs."""
+    elt = 2 if w.dtype == "bf16" else 4
+    rows = w.B * w.Hkv * (min(w.top_k, w.candidates()) + w.n_sink + w.n_local)
+    return (w.B * w.Hkv * w.candidates() * (w.bits // 8 + 2) + rows * w.d * 2 * elt
+            + w.B * w.Hq * w.d * elt + w.B * w.Hq * w.d * 4)
+
+
 def normw_roofline(w: synth.Workload, n_layers: int, ms: float, step_ms: float, peak: float, peak_kind: str) -> dict:
     """Norm-weighted sign-VQ retrieval: codes and fp16 norms of every candidate
     are the algorithmic bytes of one launch."""
     nbytes = w.B * w.Hkv * w.candidates() * (w.bits // 8 + 2)
     launch_s = ms * 1e-3 / n_layers
-    return {"kernel": "normw_kernel (scan + radix select + ordered compaction)", "bound": "hbm",
+    return {"kernel": "normw_kernel (scan, lists at the threshold bin, select, ordered compaction)", "bound": "hbm",
             "achieved": nbytes / launch_s / 1e9, "peak": peak, "unit": "GB/s",
             "frac": nbytes / launch_s / 1e9 / peak, "bytes_per_launch": nbytes, "launch_us": launch_s * 1e6,
-            "step_us_per_layer": step_ms * 1e3 / n_layers, "launches_per_layer": 3, "peak_kind": peak_kind,
+            "step_us_per_layer": step_ms * 1e3 / n_layers, "launches_per_layer": 3,
+            "step": "query encode + norm-weighted retrieval + sparse attention (three launches); "
+                    "decode_step_us_per_layer: hkv_decode_step_normw (one launch)", "peak_kind": peak_kind,
             "traffic": traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "normw.cu"), w.name)}
 
 
@@ -547,14 +558,24 @@ def measure_workload(w: synth.Workload, args, dev, world, hkv, full: bool):
                 hkv.hkv_retrieve_topk_normw(L.q_codes, L.codes, L.norms, w.N, w.n_sink, w.n_local, w.top_k, L.idx)
                 hkv.hkv_sparse_attend(L.q, L.K, L.V, w.N, L.idx, w.n_sink, w.n_local, L.out, ws=ws_a, status=status)
 
+        def normw_decode():
+            for L in layers:
+                hkv.hkv_decode_step_normw(L.q, L.codes, L.norms, L.K, L.V, w.N, w.n_sink, w.n_local, w.top_k, L.idx,
+                                          L.out, q_codes=L.q_codes, status=status)
+
         g = graph_of(normw_only)
         normw_ms = timed_ms(g, args, world, dev)
         del g
         g = graph_of(normw_step)
         normw_step_ms = timed_ms(g, args, world, dev)
         del g
+        g = graph_of(normw_decode)
+        normw_decode_ms = timed_ms(g, args, world, dev)
+        del g
         status_ok("norm-weighted calls")
         res["normw"] = normw_roofline(w, len(layers), normw_ms, normw_step_ms, peak, peak_kind)
+        res["normw"]["decode_step_us_per_layer"] = normw_decode_ms * 1e3 / len(layers)
+        res["normw"]["decode_step_frac"] = normw_bytes_step(w) / (normw_decode_ms * 1e-3 / len(layers)) / 1e9 / peak
     return res, layers
 
 def run_gpu(args, rank, world, local):

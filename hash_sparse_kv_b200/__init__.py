@@ -32,7 +32,7 @@ __all__ = [
     "hkv_evict_select", "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads",
     "hkv_decode_step_ragged", "hkv_split_select", "hkv_lse_merge_n", "hkv_retrieve_topk_paged",
     "hkv_sparse_attend_paged", "hkv_decode_step_paged", "hkv_normw_workspace_bytes", "normw_workspace",
-    "hkv_debug_set", "EXPORTS",
+    "hkv_decode_step_normw", "normw_decode_workspace", "hkv_debug_set", "EXPORTS",
 ]
 
 HKV_OK, HKV_ERR_INVALID_ARG, HKV_ERR_UNSUPPORTED, HKV_ERR_CAPACITY = 0, -1, -2, -3
@@ -47,7 +47,8 @@ EXPORTS = (
     "hkv_retrieve_topk_static", "hkv_retrieve_topk_heads", "hkv_retrieve_topk_normw", "hkv_sparse_attend",
     "hkv_evict_select", "hkv_write_slots", "hkv_lse_merge", "hkv_decode_step", "hkv_decode_step_heads",
     "hkv_decode_step_ragged", "hkv_split_select", "hkv_lse_merge_n", "hkv_retrieve_topk_paged",
-    "hkv_sparse_attend_paged", "hkv_decode_step_paged", "hkv_normw_workspace_bytes", "hkv_debug_set",
+    "hkv_sparse_attend_paged", "hkv_decode_step_paged", "hkv_normw_workspace_bytes", "hkv_decode_step_normw",
+    "hkv_debug_set",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -94,6 +95,8 @@ _SIGS = {
                                     _F, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "hkv_retrieve_topk_normw": (_I, [_I, _I, _I, _I, _P, _P, _P, _I64, _I64, _I, _I, _I, _P, _P, _P, _SZ, _P]),
     "hkv_normw_workspace_bytes": (_SZ, [_I, _I, _I64, _I, _I, _I]),
+    "hkv_decode_step_normw": (_I, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I64, _I64, _I, _I, _I, _F, _P, _P, _P, _P, _P,
+                                   _P, _SZ, _P, _P]),
     "hkv_evict_select": (_I, [_I, _I, _I, _I, _P, _P, _I64, _I64, _I, _I, _P, _P, _P, _SZ, _P]),
     "hkv_split_select": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "hkv_lse_merge_n": (_I, [_I, _I64, _P, _P, _P, _P, _P]),
@@ -612,3 +615,43 @@ def hkv_decode_step_paged(h: HashParams, q, codes_pool, K_pool, V_pool, page_tab
                                     _ptr(V_pool), _ptr(page_table), page_table.shape[1], num_pages, page_size, n_tokens,
                                     n_sink, n_local, top_k, scale, _ptr(q_codes), _ptr(idx), _ptr(out), _ptr(lse),
                                     _ptr(ws), nbytes, _ptr(status), _stream(stream)))
+
+
+def normw_decode_workspace(B, Hq, Hkv, n_tokens, code_bits, top_k, n_sink=0, n_local=0, device=None) -> torch.Tensor:
+    """The workspace of hkv_decode_step_normw's multi-launch step: the segmented retrieval's bytes (rounded up to
+    256) then a zero-filled hkv_workspace_bytes workspace."""
+    a = hkv_normw_workspace_bytes(B, Hkv, n_tokens, n_sink, n_local, top_k)
+    a = (a + 255) // 256 * 256
+    n = hkv_workspace_bytes(B, Hq, Hkv, n_tokens, code_bits, top_k, n_sink, n_local)
+    if n == 0 and B * Hkv * max(top_k, 1) > 0:
+        raise HkvError(HKV_ERR_UNSUPPORTED, hkv_last_error() or "unsupported shape")
+    return torch.zeros(a + max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def hkv_decode_step_normw(q, k_codes, norms, K, V, n_tokens: int, n_sink: int, n_local: int, top_k: int, idx, out,
+                          lse=None, score=None, q_codes=None, scale: Optional[float] = None, ws=None, status=None,
+                          stream=None) -> None:
+    """Norm-weighted sign-VQ decode step: sign query codes, the top_k by norm * (g * bits - 2 D) per KV head,
+    attention over the selected, sink and local rows.  q [B, Hq, 128]; k_codes [B, Hkv, cap, W]; norms
+    [B, Hkv, cap] fp16; K, V [B, Hkv, cap, 128] in q's dtype; idx [B, Hkv, top_k] int32; out [B, Hq, 128] fp32."""
+    B, Hq, d = q.shape
+    _, Hkv, cap, W = k_codes.shape
+    _need(q, "q", (torch.bfloat16, torch.float32))
+    _need(k_codes, "k_codes", _U32)
+    _need(norms, "norms", (torch.float16, torch.int16), shape=(B, Hkv, cap))
+    _need(K, "K", q.dtype, shape=(B, Hkv, cap, d))
+    _need(V, "V", q.dtype, shape=(B, Hkv, cap, d))
+    _need(idx, "idx", torch.int32, shape=(B, Hkv, top_k))
+    _need(out, "out", torch.float32, shape=(B, Hq, d))
+    if q_codes is not None:
+        _need(q_codes, "q_codes", _U32, shape=(B, Hq, W))
+    if score is not None:
+        _need(score, "score", torch.float32, shape=(B, Hkv, top_k))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, shape=(B, Hq))
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _ok(lib().hkv_decode_step_normw(B, Hq, Hkv, _dtype_code(q), W * 32, _ptr(q), _ptr(k_codes), _ptr(norms), _ptr(K),
+                                    _ptr(V), cap, n_tokens, n_sink, n_local, top_k, scale, _ptr(q_codes), _ptr(idx),
+                                    _ptr(score), _ptr(out), _ptr(lse), _ptr(ws), nbytes, _ptr(status),
+                                    _stream(stream)))

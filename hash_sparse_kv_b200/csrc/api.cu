@@ -494,6 +494,51 @@ int hkv_decode_step_paged(const hkv_hash* q_hash, int B, int Hq, int Hkv, const 
                      n_local, top_k, scale, q_codes, idx, out, lse, nullptr, ws, ws_bytes, status, stream, &pm);
 }
 
+int hkv_decode_step_normw(int B, int Hq, int Hkv, int dtype, int code_bits, const void* q, const uint32_t* k_codes,
+                          const uint16_t* norms, const void* K, const void* V, int64_t cap, int64_t n_tokens,
+                          int n_sink, int n_local, int top_k, float scale, uint32_t* q_codes, int32_t* idx,
+                          float* score, float* out, float* lse, void* ws, size_t ws_bytes, int32_t* status,
+                          void* stream) {
+  int rc = check_heads(B, Hq, Hkv);
+  if (rc == HKV_OK) rc = check_window(cap, n_tokens, n_sink, n_local, top_k);
+  if (rc != HKV_OK) return rc;
+  if (dtype != HKV_F32 && dtype != HKV_BF16) return fail(HKV_ERR_INVALID_ARG, "dtype %d", dtype);
+  if (code_bits != kHeadDim) return fail(HKV_ERR_UNSUPPORTED, "code_bits %d (sign codes: 128)", code_bits);
+  if (B == 0) return HKV_OK;
+  if (!q || !k_codes || !norms || !K || !V || !idx || !out) return fail(HKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_codes, code_bits / 8)) return fail(HKV_ERR_INVALID_ARG, "k_codes must be %d-byte aligned", code_bits / 8);
+  if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16)) return fail(HKV_ERR_INVALID_ARG, "q, K, V must be 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const RetrieveShape s{B, Hq, Hkv, code_bits / 32, cap, n_tokens, n_sink, n_local, top_k};
+  const Window w = window(n_tokens, n_sink, n_local);
+  const int P = B * Hkv;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 1;
+  const NormwPlan pl = normw_plan(P, w.C, top_k, sms);
+  if (dtype == HKV_BF16 && w.C <= 65536 && (ws == nullptr || pl.nseg == 1))
+    return launch_normw_decode(s, q, k_codes, norms, K, V, scale, q_codes, idx, score, out, lse, status, st);
+  // query encode, norm-weighted retrieval (segmented with the workspace), attention
+  if (q_codes == nullptr) return fail(HKV_ERR_INVALID_ARG, "q_codes is NULL (needed by the multi-launch step)");
+  if (ws == nullptr) return fail(HKV_ERR_UNSUPPORTED, "this shape needs a workspace");
+  const size_t nw_bytes = align_up(pl.ws_bytes, 256);
+  if (ws_bytes < nw_bytes) return fail(HKV_ERR_CAPACITY, "workspace of %zu bytes, %zu needed", ws_bytes, nw_bytes);
+  hkv_hash h{};
+  h.kind = HKV_HASH_SIGN;
+  h.head_dim = kHeadDim;
+  h.code_bits = code_bits;
+  h.dtype = dtype;
+  const int64_t rows = (int64_t)B * Hq;
+  RowMap m{rows, rows, 0, kHeadDim, 0, code_bits / 32, 0, 1};
+  rc = launch_encode(h, q, m, q_codes, nullptr, st, status);
+  if (rc != HKV_OK) return rc;
+  rc = launch_retrieve_normw(s, q_codes, k_codes, norms, idx, score, pl.nseg > 1 ? ws : nullptr, nw_bytes, st);
+  if (rc != HKV_OK) return rc;
+  AttendShape as{B, Hq, Hkv, dtype, cap, n_tokens, top_k, n_sink, n_local};
+  return launch_attend(as, q, K, V, idx, scale, out, lse, static_cast<unsigned char*>(ws) + nw_bytes,
+                       ws_bytes - nw_bytes, status, st);
+}
+
 int hkv_decode_step_heads(const hkv_hash* q_hash, int B, int Hq, int Hkv, const void* q,
                           const uint32_t* k_codes, const void* K, const void* V, int64_t cap,
                           int64_t n_tokens, int n_sink, int n_local, int top_k, float scale,

@@ -125,6 +125,11 @@ size_t attend_ws_bytes(const AttendShape& s);
 int launch_attend(const AttendShape& s, const void* q, const void* K, const void* V,
                   const int32_t* idx, float scale, float* out, float* lse, void* ws,
                   size_t ws_bytes, int32_t* status, cudaStream_t st, const PageMap* pm = nullptr);
+// Norm-weighted sign-VQ decode step in one launch (retrieve.cu): bf16 q, K,
+// V; one block per pair, at most 65536 candidates per pair.
+int launch_normw_decode(const RetrieveShape& s, const void* q, const uint32_t* k_codes, const uint16_t* norms,
+                        const void* K, const void* V, float scale, uint32_t* q_codes, int32_t* idx, float* score,
+                        float* out, float* lse, int32_t* status, cudaStream_t st);
 // bf16 sparse attention on the fused kernel's tensor-core attention stage
 // (retrieve.cu); launch_attend sends bf16 shapes here.
 size_t sattend_ws_bytes(const AttendShape& s);

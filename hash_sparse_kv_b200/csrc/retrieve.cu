@@ -59,6 +59,7 @@
 
 #include "hamming.cuh"
 #include "internal.h"
+#include "normw_select.cuh"
 #include "tc.cuh"
 
 namespace hkv {
@@ -1742,6 +1743,80 @@ __global__ void __launch_bounds__(kThreads, 1) sattend_kernel(FusedArgs a) {
   }
 }
 
+// ---------------- norm-weighted decode step (sign-VQ, bf16) ------------------
+// One block per (batch, KV head) pair, windows of at most 65536 candidates:
+// the group's sign query codes by ballots, the norm-weighted top-k of
+// normw_select.cuh (Self-Indexing KVCache, "Abstract"), then the attention
+// over [sink | selected | local] on the tensor cores (attn_warps) and out /
+// lse from the block's own partial.  The selection's shared memory is reused
+// by the attention.
+struct NwDecodeArgs {
+  const uint16_t* norms;  // [B, Hkv, cap] fp16
+  int gb;                 // g * code bits
+  int vec_norms;          // norm rows start on 16-byte boundaries
+  float* score;           // nullable [B, Hkv, top_k]
+  uint32_t* q_codes_out;  // nullable [B, Hq, W]
+};
+
+struct NdLayout {
+  static constexpr size_t qs = kAttnWarpBytes;                       // bf16 [16][kQP]
+  static constexpr size_t tokw = qs + (size_t)kMaxGroup * kQP * 2;  // int [2][kAW][kWR]
+  static constexpr size_t part = tokw + (size_t)2 * kAW * kWR * 4;  // float [g][kPart]
+  static constexpr size_t attn = part + (size_t)kMaxGroup * kPart * 4;
+};
+
+template <int W, int NP>
+__global__ void __launch_bounds__(kThreads, 1) normw_decode_kernel(FusedArgs a, NwDecodeArgs n) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ uint32_t qc_s[kMaxGroup * W];
+  __shared__ uint32_t wsum[kWarps];
+  __shared__ uint32_t found[3];
+  __shared__ uint32_t cnt_s[2 * kWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = a.g;
+  const int p = blockIdx.x, b = p / a.Hkv, kvh = p % a.Hkv;
+  const int k_eff = a.k_eff;
+  int32_t* idx = a.idx + (int64_t)p * a.top_k;
+  float* score = n.score != nullptr ? n.score + (int64_t)p * a.top_k : nullptr;
+  for (int i = k_eff + tid; i < a.top_k; i += kThreads) {
+    idx[i] = -1;
+    if (score != nullptr) score[i] = -INFINITY;
+  }
+  const int64_t qrow0 = (int64_t)b * a.Hq + (int64_t)kvh * g;
+  const __nv_bfloat16* q0 = tptr<__nv_bfloat16>(a.q) + qrow0 * kHeadDim;
+  for (int r = warp; r < g; r += kWarps) {
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const uint32_t word = __ballot_sync(0xffffffffu, __bfloat162float(q0[(int64_t)r * kHeadDim + lane + 32 * w]) > 0.f);
+      if (lane == 0) qc_s[r * W + w] = word;
+    }
+  }
+  __syncthreads();
+  if (n.q_codes_out != nullptr)
+    for (int i = tid; i < g * W; i += kThreads) n.q_codes_out[qrow0 * W + i] = qc_s[i];
+  const int64_t kvc = kv_row(a, p) * a.cap;
+  if (k_eff > 0)
+    nw::block_select<W, NP>(a.k_codes + (kvc + a.lo) * W, n.norms + kvc + a.lo, n.vec_norms != 0, qc_s, g, n.gb,
+                            (int)a.lo, a.C, k_eff, smem, wsum, found, cnt_s, idx, score);
+  __syncthreads();  // idx is complete; the selection's shared memory is free
+  __nv_bfloat16* qs_s = reinterpret_cast<__nv_bfloat16*>(smem + NdLayout::qs);
+  int* tokw_s = reinterpret_cast<int*>(smem + NdLayout::tokw);
+  float* part_s = reinterpret_cast<float*>(smem + NdLayout::part);
+  for (int i = tid; i < kMaxGroup * kHeadDim; i += kThreads) {
+    const int h = i / kHeadDim, k = i % kHeadDim;
+    qs_s[h * kQP + k] = h < g ? q0[(int64_t)h * kHeadDim + k] : __float2bfloat16_rn(0.f);
+  }
+  const int nrows = a.sink_n + k_eff + a.local_n;
+  const int32_t* sel = idx;  // written by this block (plain loads, not the read-only path)
+  attn_warps(a, p, kvc, nrows,
+             [&](int i) -> int {
+               if (i < a.sink_n) return i;
+               if (i < a.sink_n + k_eff) return sel[i - a.sink_n];
+               return a.local_start + (i - a.sink_n - k_eff);
+             },
+             smem, tokw_s, qs_s, part_s, 0);
+  finish_single(a, p, part_s);
+}
+
 struct SaPlan {
   int nseg = 1, per_block = 0, pairs_per_launch = 1;
   bool cooperative = false;
@@ -2001,6 +2076,64 @@ size_t retrieve_ws_bytes(const RetrieveShape& s) {
   Plan pl;
   if (make_plan(s, false, 0, pl) != HKV_OK) return 0;
   return pl.ws_total;
+}
+
+int launch_normw_decode(const RetrieveShape& s, const void* q, const uint32_t* k_codes, const uint16_t* norms,
+                        const void* K, const void* V, float scale, uint32_t* q_codes, int32_t* idx, float* score,
+                        float* out, float* lse, int32_t* status, cudaStream_t st) {
+  const int P = s.B * s.Hkv;
+  if (P == 0 || s.top_k == 0) return HKV_OK;
+  const Window w = window(s.N, s.n_sink, s.n_local);
+  if (w.C > nw::kMaxTokens)
+    return fail(HKV_ERR_UNSUPPORTED, "%lld candidates per KV head for the one-launch step", (long long)w.C);
+  const int g = s.Hq / s.Hkv;
+  int np = 0;
+  while ((1 << np) <= g) ++np;
+  FusedArgs a = {};
+  a.k_codes = k_codes;
+  a.idx = idx;
+  a.q = q;
+  a.K = K;
+  a.V = V;
+  a.out = out;
+  a.lse = lse;
+  a.scale = scale;
+  a.Hq = s.Hq;
+  a.Hkv = s.Hkv;
+  a.g = g;
+  a.cap = s.cap;
+  a.lo = w.sink_end;
+  a.C = (int)w.C;
+  a.k_eff = (int)std::min<int64_t>(s.top_k, w.C);
+  a.top_k = s.top_k;
+  a.sink_n = (int)w.sink_end;
+  a.local_start = (int)w.local_start;
+  a.local_n = (int)(s.N - w.local_start);
+  a.Hkv_real = s.Hkv;
+  a.unit_div = 1;
+  a.status = status;
+  a.ps_shift = -1;
+  NwDecodeArgs n;
+  n.norms = norms;
+  n.gb = g * s.words * 32;
+  n.vec_norms = (reinterpret_cast<uintptr_t>(norms) % 16 == 0 && s.cap % 8 == 0 && w.sink_end % 8 == 0) ? 1 : 0;
+  n.score = score;
+  n.q_codes_out = q_codes;
+  using Fn = void (*)(FusedArgs, NwDecodeArgs);
+  Fn fn = nullptr;
+#define HKV_ND(WV, NPV) \
+  if (s.words == WV && np == NPV) fn = normw_decode_kernel<WV, NPV>;
+  HKV_ND(2, 1) HKV_ND(2, 2) HKV_ND(2, 3) HKV_ND(2, 4) HKV_ND(2, 5)
+  HKV_ND(4, 1) HKV_ND(4, 2) HKV_ND(4, 3) HKV_ND(4, 4) HKV_ND(4, 5)
+#undef HKV_ND
+  if (fn == nullptr) return fail(HKV_ERR_UNSUPPORTED, "no kernel for %d-bit codes and group %d", s.words * 32, g);
+  const int64_t range = ceil_div(std::max<int64_t>(w.C, 1), (int64_t)nw::kWarps * nw::kChunk) * nw::kChunk;
+  const size_t sel_smem = nw::kRegionBytes + (size_t)nw::kBins * 4 + (size_t)nw::kWarps * range * 2;
+  const size_t smem = std::max(sel_smem, NdLayout::attn);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return cuda_check(e, "norm-weighted decode shared memory");
+  fn<<<(unsigned)P, kThreads, smem, st>>>(a, n);
+  return cuda_check(cudaGetLastError(), "norm-weighted decode launch");
 }
 
 size_t sattend_ws_bytes(const AttendShape& s) { return sattend_plan(s).ws_total; }

@@ -320,6 +320,32 @@ int hkv_retrieve_topk_normw(int B, int Hq, int Hkv, int code_bits, const uint32_
                             int n_sink, int n_local, int top_k, int32_t* idx, float* score, void* ws,
                             size_t ws_bytes, void* stream);
 
+/* Norm-weighted sign-VQ decode step (Self-Indexing KVCache, "Abstract";
+ * Spotlight Attention "Approach"; RetrievalAttention "Approach"): the sign
+ * codes of the query heads, the top_k of each KV head by the norm-weighted
+ * score (exactly as hkv_retrieve_topk_normw), then the attention of its g
+ * query heads over the selected, sink and local rows, merged into out / lse.
+ *   dtype   HKV_BF16 or HKV_F32 (q, K, V)
+ *   code_bits 128 (the sign of each of the 128 dimensions)
+ *   q       [B, Hq, 128];  k_codes [B, Hkv, cap, 4] (sign codes)
+ *   norms   [B, Hkv, cap] fp16 bits;  K, V [B, Hkv, cap, 128]
+ *   q_codes [B, Hq, W] out, nullable on the one-launch path
+ *   idx     [B, Hkv, top_k] int32 out (required; ascending, -1 padded)
+ *   score   nullable fp32 out as in hkv_retrieve_topk_normw
+ *   out     [B, Hq, 128] fp32;  lse nullable [B, Hq] fp32
+ * bf16 windows of at most 65536 candidates run in one launch (one block per
+ * KV head: query codes by ballots, the selection, then the tensor-core
+ * attention) when ws is NULL or hkv_normw_workspace_bytes(...) is 0.  Any
+ * other shape runs query encode + norm-weighted retrieval + sparse
+ * attention; ws then holds hkv_normw_workspace_bytes(...) bytes rounded up to
+ * a multiple of 256, followed by hkv_workspace_bytes(...) bytes zero-filled
+ * once (hkv_workspace_reset), and q_codes is required. */
+int hkv_decode_step_normw(int B, int Hq, int Hkv, int dtype, int code_bits, const void* q, const uint32_t* k_codes,
+                          const uint16_t* norms, const void* K, const void* V, int64_t cap, int64_t n_tokens,
+                          int n_sink, int n_local, int top_k, float scale, uint32_t* q_codes, int32_t* idx,
+                          float* score, float* out, float* lse, void* ws, size_t ws_bytes, int32_t* status,
+                          void* stream);
+
 /* Workspace bytes of hkv_retrieve_topk_normw for this shape on the current
  * device: 0 when one block per KV head is the plan (no workspace needed),
  * and 0 if the shape is invalid or no CUDA device is visible (the plan

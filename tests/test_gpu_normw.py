@@ -10,6 +10,7 @@ import torch
 import hash_sparse_kv_b200 as hkv
 import oracle
 import synth
+from tests.helpers import ATOL
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -186,3 +187,75 @@ def test_normw_segmented_512k():
     kc = synth.random_codes(98, B * Hkv * N, W).view(B, Hkv, N, W)
     qc = synth.random_codes(99, B * Hq, W).view(B, Hq, W)
     _check(qc, kc, _norms(100, B, Hkv, N), N, s, l, k, segmented=True)
+
+
+# --------------------------------------------------- norm-weighted decode step
+
+def _sign_inputs(seed, B, Hq, Hkv, cap, dtype):
+    g = torch.Generator().manual_seed(seed)
+    def draw(*shape):
+        x = torch.randn(*shape, generator=g)
+        x = torch.where(x.abs() < 1e-2, torch.full_like(x, 0.5), x)  # no value at or near zero
+        return x.to(torch.bfloat16) if dtype == "bf16" else x
+    return draw(B, Hq, 128), draw(B, Hkv, cap, 128), draw(B, Hkv, cap, 128)
+
+
+def _check_decode_normw(B, Hq, Hkv, N, cap, s, l, k, dtype="bf16", workspace=False):
+    q, K, V = _sign_inputs(1000 + N + k, B, Hq, Hkv, cap, dtype)
+    kc, norms = oracle.encode("sign", K)
+    qc, _ = oracle.encode("sign", q)
+    kcodes = torch.from_numpy(kc.view(np.int32)).view(B, Hkv, cap, 4)
+    idx = torch.full((B, Hkv, k), -7, dtype=torch.int32, device=DEV)
+    score = torch.full((B, Hkv, k), 7.0, device=DEV)
+    out = torch.full((B, Hq, 128), float("nan"), device=DEV)
+    lse = torch.full((B, Hq), float("nan"), device=DEV)
+    q_codes = torch.zeros(B, Hq, 4, dtype=torch.int32, device=DEV)
+    ws = hkv.normw_decode_workspace(B, Hq, Hkv, N, 128, k, s, l) if workspace else None
+    st = hkv.status_word()
+    hkv.hkv_decode_step_normw(q.to(DEV), kcodes.to(DEV), torch.from_numpy(norms.reshape(B, Hkv, cap)).to(DEV),
+                              K.to(DEV), V.to(DEV), N, s, l, k, idx, out, lse=lse, score=score, q_codes=q_codes,
+                              ws=ws, status=st)
+    assert hkv.hkv_check(st) == hkv.HKV_OK, hkv.hkv_last_error()
+    np.testing.assert_array_equal(q_codes.cpu().numpy().view(np.uint32), qc.reshape(B, Hq, 4))
+    want_i, want_s = oracle.retrieve_normw(qc.reshape(B, Hq, 4), kc.reshape(B, Hkv, cap, 4), norms.reshape(B, Hkv, cap),
+                                           N, s, l, k)
+    np.testing.assert_array_equal(idx.cpu().numpy(), want_i)
+    np.testing.assert_array_equal(score.cpu().numpy(), want_s.astype(np.float32))
+    g = Hq // Hkv
+    o, ls = out.cpu().numpy(), lse.cpu().numpy()
+    for b in range(B):
+        for j in range(Hkv):
+            rows = oracle.attention_rows(N, s, l, want_i[b, j])
+            wo, wl = oracle.attend(q[b, j * g:(j + 1) * g], K[b, j], V[b, j], rows, 1.0 / np.sqrt(128))
+            assert np.abs(o[b, j * g:(j + 1) * g] - wo).max() < ATOL
+            assert np.abs(ls[b, j * g:(j + 1) * g] - wl).max() < ATOL
+
+
+DECODE_CASES = [
+    # B, Hq, Hkv, N, cap, sink, local, top_k
+    (2, 8, 2, 5000, 5000, 4, 64, 100),        # one launch, g 4, unaligned sink (scalar norm loads)
+    (1, 28, 4, 20001, 20008, 8, 128, 1024),   # g 7, aligned window
+    (1, 16, 1, 777, 800, 4, 64, 1),           # g 16, top-1
+    (2, 4, 2, 300, 304, 8, 8, 400),           # top_k above the candidates
+    (2, 4, 2, 50, 64, 40, 30, 8),             # no candidates: the sink and local rows only
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES)
+def test_decode_step_normw_one_launch(case):
+    _check_decode_normw(*case)
+
+
+@pytest.mark.parametrize("case,dtype", [
+    ((1, 8, 2, 70001, 70001, 4, 64, 300), "bf16"),   # past 65536: segmented retrieval, then the attention
+    ((1, 28, 4, 20001, 20008, 8, 128, 1024), "bf16"),  # few pairs with a workspace: segments
+    ((2, 8, 2, 5000, 5000, 4, 64, 100), "f32"),       # fp32: query encode + retrieval + SIMT attention
+])
+def test_decode_step_normw_multi_launch(case, dtype):
+    _check_decode_normw(*case, dtype=dtype, workspace=True)
+
+
+def test_decode_step_normw_signvq_workload():
+    """Two KV heads of the sign-VQ workload's shape (65536 tokens, top 512,
+    groups of 4) through the one-launch step."""
+    _check_decode_normw(1, 8, 2, 65536, 65536, 0, 0, 512)
