@@ -39,6 +39,10 @@ int main(void) {
   expect(hkv_retrieve_topk_normw(1, 4, 2, 128, (const uint32_t*)16, (const uint32_t*)16, (const uint16_t*)16, 70000,
                                  70000, 0, 0, 4, (int32_t*)16, NULL, NULL, 0, NULL) == HKV_ERR_UNSUPPORTED,
          "long normw window without a workspace rejected");
+  /* norm-weighted decode step: sign codes are 128 bits */
+  expect(hkv_decode_step_normw(1, 4, 2, HKV_BF16, 64, NULL, NULL, NULL, NULL, NULL, 10, 10, 0, 0, 4, 0.1f, NULL, NULL,
+                               NULL, NULL, NULL, NULL, 0, NULL, NULL) == HKV_ERR_UNSUPPORTED,
+         "64-bit codes rejected by the norm-weighted decode step");
   /* G-way merge with no partials */
   expect(hkv_lse_merge_n(0, 4, NULL, NULL, NULL, NULL, NULL) == HKV_ERR_INVALID_ARG, "G = 0 rejected");
   if (failures == 0) printf("c abi ok\n");

@@ -99,6 +99,15 @@ def test_norm_weighted_and_split_argument_errors(lib):
     assert rc == hkv.HKV_ERR_UNSUPPORTED and "workspace" in hkv.hkv_last_error()  # past 65536 without one
     rc = lib.hkv_retrieve_topk_normw(0, 4, 2, 128, None, None, None, 10, 10, 0, 0, 4, None, None, None, 0, None)
     assert rc == hkv.HKV_OK  # empty batch
+    # norm-weighted decode step: 64-bit codes (sign codes are 128), NULL idx, empty batch
+    rc = lib.hkv_decode_step_normw(1, 4, 2, hkv.HKV_BF16, 64, 16, 16, 16, 16, 16, 10, 10, 0, 0, 4, 0.1, None, 16,
+                                   None, 16, None, None, 0, None, None)
+    assert rc == hkv.HKV_ERR_UNSUPPORTED
+    rc = lib.hkv_decode_step_normw(1, 4, 2, hkv.HKV_BF16, 128, 16, 16, 16, 16, 16, 10, 10, 0, 0, 4, 0.1, None, None,
+                                   None, 16, None, None, 0, None, None)
+    assert rc == hkv.HKV_ERR_INVALID_ARG
+    assert lib.hkv_decode_step_normw(0, 4, 2, hkv.HKV_BF16, 128, None, None, None, None, None, 10, 10, 0, 0, 4, 0.1,
+                                     None, None, None, None, None, None, 0, None, None) == hkv.HKV_OK
     # no CUDA device here: the workspace size is 0 (the plan needs the SM count)
     assert lib.hkv_normw_workspace_bytes(1, 2, 200000, 0, 0, 8) == 0
     # token split: rank outside [0, G), NULL candidates
