@@ -271,7 +271,8 @@ def normw_roofline(w: synth.Workload, n_layers: int, ms: float, step_ms: float, 
             "step_us_per_layer": step_ms * 1e3 / n_layers, "launches_per_layer": 3,
             "step": "query encode + norm-weighted retrieval + sparse attention (three launches); "
                     "decode_step_us_per_layer: hkv_decode_step_normw (one launch)", "peak_kind": peak_kind,
-            "traffic": traffic_record(os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", "normw.cu"), w.name)}
+            "traffic": traffic_record([os.path.join(ROOT, "hash_sparse_kv_b200", "csrc", f)
+                                       for f in ("normw.cu", "normw_select.cuh")], w.name)}
 
 
 def graph_of(fn, warm=1):
@@ -315,20 +316,26 @@ def timed_ms(g, args, world, dev):
     return max_over_ranks(time_graph(g, args.steps, args.warmup, world)[1], world, dev)
 
 
-def source_digest(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_digest(paths):
+    """First 16 hex digits of the SHA-256 of the files' contents, concatenated in order."""
+    h = hashlib.sha256()
+    for path in [paths] if isinstance(paths, str) else paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
-def traffic_record(kernel_file: str, workload: str):
+def traffic_record(kernel_files, workload: str):
     """DRAM traffic per launch from the committed ncu summary, if it was taken
-    on the current source of the kernel; else None."""
+    on the current source of the kernel (one file, or the list of files its
+    code lives in, keyed by the first one's name); else None."""
+    files = [kernel_files] if isinstance(kernel_files, str) else list(kernel_files)
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        rec = json.load(f).get(workload, {}).get(os.path.basename(kernel_file))
-    if not rec or rec.get("source_sha256_16") != source_digest(kernel_file):
+        rec = json.load(f).get(workload, {}).get(os.path.basename(files[0]))
+    if not rec or rec.get("source_sha256_16") != source_digest(files):
         return None
     return rec.get("bytes_per_launch")
 
