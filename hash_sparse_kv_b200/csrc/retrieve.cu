@@ -44,8 +44,9 @@
 //    resident rows, each with its own online softmax for the unit's query
 //    heads on the tensor cores (logits and P V by mma.sync, P kept in
 //    registers, two cp.async slots per warp), and the warps' partials are
-//    merged into one block partial (m, l, acc).  The last g blocks of the
-//    unit to finish merge one head each: M = max m_s, L = sum l_s e^{m_s - M},
+//    merged into one block partial (m, l, acc).  The last blocks of the unit
+//    to finish (up to one per 32 output columns) merge a run of the unit's
+//    g * 128 output columns each: M = max m_s, L = sum l_s e^{m_s - M},
 //    out = sum acc_s e^{m_s - M} / L, lse = M + log L; the last of them
 //    returns the unit's counters and histogram to zero, so the workspace is
 //    ready for the next call.
@@ -752,39 +753,45 @@ __device__ void attn_end(int g, const AttnSmem& sm, const float (&acc)[kOut], fl
   }
 }
 
-// Merge of the nseg partials of query head h of pair p into out / lse
-// (RetrievalAttention, "Approach": exact log-sum-exp rescaling):
+// Merge of the pair's output columns [col0, col0 + ncols) (column c is
+// dimension c % 128 of query head c / 128 of the group; ncols <= kThreads
+// and a multiple of 32) from its nseg partials (RetrievalAttention,
+// "Approach": exact log-sum-exp rescaling):
 //   M = max_s m_s,  w_s = e^{m_s - M},  L = sum_s l_s w_s,
 //   out = sum_s acc_s w_s / L,  lse = M + log L.
-// Thread (q, c) sums w_s acc_s[c] over s = q, q + 4, ...; its first batch of
-// loads is issued before the weights are known; warp 0 computes the weights
-// once.
-// scratch: nseg + 4 * kThreads + 2 floats of shared memory.
-// (Not inlined, with scalar arguments: keeps the fused kernel's registers
-// for its main loop.)
-__device__ __noinline__ void merge_head(const float* part, float* out, float* lse, int Hq, int Hkv, int g, int p,
-                                        int nseg, int h, float* scratch) {
-  constexpr int kQ = kThreads / kHeadDim;  // segment groups
-  constexpr int kB = 12;                   // segments per thread and batch (48 segments in one batch)
-  const int tid = threadIdx.x, lane = tid & 31, c = tid % kHeadDim, q = tid / kHeadDim;
-  float* w_s = scratch;                  // [nseg]
-  float* red_s = scratch + nseg;         // [kThreads]
-  float* ML_s = red_s + kThreads;        // M, L
-  const float* parts = part + (int64_t)p * nseg * g * kPart + (int64_t)h * kPart;
+// Warp w computes M, the weights and L of the range's w-th head while every
+// thread has its first batch of accumulators in flight (thread (c, q):
+// column c, segments q, q + Q, ... with Q = kThreads / ncols); a shared
+// reduction over q finishes each column; the thread of a head's column 0
+// writes its lse.  scratch: 5 * nseg + kThreads + 10 floats.
+__device__ __noinline__ void merge_cols(const float* part, float* out, float* lse, int Hq, int Hkv, int g, int p,
+                                        int nseg, int col0, int ncols, float* scratch) {
+  constexpr int kB = 10;  // segments per thread and batch
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Q = kThreads / ncols, h0 = col0 / kHeadDim, nh = (col0 + ncols - 1) / kHeadDim - h0 + 1;
+  float* w_s = scratch;                   // [nh][nseg]
+  float* red_s = scratch + 5 * nseg;      // [Q][ncols]
+  float* ML_s = red_s + kThreads;         // [nh][2]
+  const float* base = part + (int64_t)p * nseg * g * kPart;
   const int64_t sstride = (int64_t)g * kPart;
+  const bool act = tid < Q * ncols;
+  const int cc = col0 + tid % ncols, q = tid / ncols, h = cc / kHeadDim, c = cc % kHeadDim;
+  const float* pc = base + (int64_t)h * kPart + 4 + c;
   float x[kB];
 #pragma unroll
   for (int u = 0; u < kB; ++u) {
-    const int s = q + u * kQ;
-    x[u] = s < nseg ? __ldcg(parts + s * sstride + 4 + c) : 0.f;
+    const int sg = q + u * Q;
+    x[u] = act && sg < nseg ? __ldcg(pc + sg * sstride) : 0.f;
   }
-  if (tid < 32) {
-    float M = -INFINITY;
+  if (warp < nh) {
+    // one round of loads: every (m, l) of the head in registers
+    const float* ph = base + (int64_t)(h0 + warp) * kPart;
     float2 ml[(kMaxSegsPerPair + 31) / 32];
+    float M = -INFINITY;
 #pragma unroll
     for (int u = 0; u < (kMaxSegsPerPair + 31) / 32; ++u) {
-      const int s = lane + 32 * u;
-      ml[u] = s < nseg ? __ldcg(reinterpret_cast<const float2*>(parts + s * sstride)) : make_float2(-INFINITY, 0.f);
+      const int sg = lane + 32 * u;
+      ml[u] = sg < nseg ? __ldcg(reinterpret_cast<const float2*>(ph + sg * sstride)) : make_float2(-INFINITY, 0.f);
       M = fmaxf(M, ml[u].x);
     }
 #pragma unroll
@@ -792,9 +799,85 @@ __device__ __noinline__ void merge_head(const float* part, float* out, float* ls
     float L = 0.f;
 #pragma unroll
     for (int u = 0; u < (kMaxSegsPerPair + 31) / 32; ++u) {
-      const int s = lane + 32 * u;
+      const int sg = lane + 32 * u;
       const float w = ml[u].x == -INFINITY ? 0.f : expf(ml[u].x - M);
-      if (s < nseg) w_s[s] = w;
+      if (sg < nseg) w_s[warp * nseg + sg] = w;
+      L = fmaf(ml[u].y, w, L);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (lane == 0) {
+      ML_s[2 * warp] = M;
+      ML_s[2 * warp + 1] = L;
+    }
+  }
+  __syncthreads();
+  const float* wh = w_s + (h - h0) * nseg;
+  float o = 0.f;
+  for (int s0 = q;; s0 += kB * Q) {
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int sg = s0 + u * Q;
+      if (act && sg < nseg) o = fmaf(x[u], wh[sg], o);
+    }
+    if (s0 + kB * Q >= nseg) break;
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int sg = s0 + kB * Q + u * Q;
+      x[u] = act && sg < nseg ? __ldcg(pc + sg * sstride) : 0.f;
+    }
+  }
+  if (act) red_s[q * ncols + tid % ncols] = o;
+  __syncthreads();
+  if (tid < ncols) {
+    float O = 0.f;
+    for (int k = 0; k < Q; ++k) O += red_s[k * ncols + tid];
+    const float M = ML_s[2 * (h - h0)], L = ML_s[2 * (h - h0) + 1];
+    const int b = p / Hkv, kvh = p % Hkv;
+    const int64_t orow = (int64_t)b * Hq + (int64_t)kvh * g + h;
+    out[orow * kHeadDim + c] = L > 0.f ? O / L : 0.f;
+    if (c == 0 && lse != nullptr) lse[orow] = L > 0.f ? M + logf(L) : -INFINITY;
+  }
+  __syncthreads();
+}
+
+// merge_cols for one run of 32 columns [32 j, 32 j + 32) (inside head j / 4),
+// with the segment groups fixed at compile time: thread (c, q) sums column
+// c over segments q, q + 16, ... (one round of loads for up to 160
+// segments).  scratch: nseg + 16 * 32 + 2 floats.
+__device__ __noinline__ void merge_slice(const float* part, float* out, float* lse, int Hq, int Hkv, int g, int p,
+                                         int nseg, int j, float* scratch) {
+  constexpr int kQ = kThreads / 32;                     // segment groups
+  constexpr int kB = (kMaxSegsPerPair + kQ - 1) / kQ;  // segments per thread
+  const int tid = threadIdx.x, lane = tid & 31, q = tid >> 5, h = j >> 2, c = ((j & 3) << 5) + lane;
+  float* w_s = scratch;           // [nseg]
+  float* red_s = scratch + nseg;  // [kQ][32]
+  float* ML_s = red_s + kQ * 32;  // M, L
+  const float* parts = part + (int64_t)p * nseg * g * kPart + (int64_t)h * kPart;
+  const int64_t sstride = (int64_t)g * kPart;
+  float x[kB];
+#pragma unroll
+  for (int u = 0; u < kB; ++u) {
+    const int sg = q + u * kQ;
+    x[u] = sg < nseg ? __ldcg(parts + sg * sstride + 4 + c) : 0.f;
+  }
+  if (tid < 32) {
+    float M = -INFINITY;
+    float2 ml[(kMaxSegsPerPair + 31) / 32];
+#pragma unroll
+    for (int u = 0; u < (kMaxSegsPerPair + 31) / 32; ++u) {
+      const int sg = lane + 32 * u;
+      ml[u] = sg < nseg ? __ldcg(reinterpret_cast<const float2*>(parts + sg * sstride)) : make_float2(-INFINITY, 0.f);
+      M = fmaxf(M, ml[u].x);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+#pragma unroll
+    for (int u = 0; u < (kMaxSegsPerPair + 31) / 32; ++u) {
+      const int sg = lane + 32 * u;
+      const float w = ml[u].x == -INFINITY ? 0.f : expf(ml[u].x - M);
+      if (sg < nseg) w_s[sg] = w;
       L = fmaf(ml[u].y, w, L);
     }
 #pragma unroll
@@ -806,32 +889,50 @@ __device__ __noinline__ void merge_head(const float* part, float* out, float* ls
   }
   __syncthreads();
   float o = 0.f;
-  for (int s0 = q;; s0 += kB * kQ) {
 #pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      const int s = s0 + u * kQ;
-      if (s < nseg) o = fmaf(x[u], w_s[s], o);
-    }
-    if (s0 + kB * kQ >= nseg) break;
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      const int s = s0 + kB * kQ + u * kQ;
-      x[u] = s < nseg ? __ldcg(parts + s * sstride + 4 + c) : 0.f;
-    }
+  for (int u = 0; u < kB; ++u) {
+    const int sg = q + u * kQ;
+    if (sg < nseg) o = fmaf(x[u], w_s[sg], o);
   }
-  red_s[tid] = o;
+  red_s[q * 32 + lane] = o;
   __syncthreads();
-  if (tid < kHeadDim) {
+  if (tid < 32) {
     float O = 0.f;
 #pragma unroll
-    for (int j = 0; j < kQ; ++j) O += red_s[j * kHeadDim + tid];
+    for (int k = 0; k < kQ; ++k) O += red_s[k * 32 + lane];
     const float M = ML_s[0], L = ML_s[1];
     const int b = p / Hkv, kvh = p % Hkv;
     const int64_t orow = (int64_t)b * Hq + (int64_t)kvh * g + h;
-    out[orow * kHeadDim + tid] = L > 0.f ? O / L : 0.f;
-    if (tid == 0 && lse != nullptr) lse[orow] = L > 0.f ? M + logf(L) : -INFINITY;
+    out[orow * kHeadDim + c] = L > 0.f ? O / L : 0.f;
+    if (c == 0 && lse != nullptr) lse[orow] = L > 0.f ? M + logf(L) : -INFINITY;
   }
   __syncthreads();
+}
+
+// The merging blocks of a pair and the columns each takes: the last nm of
+// its nseg blocks, each one run of ncols columns (a multiple of 32, at
+// least 32), so that every block's share is one pass of merge_cols.
+struct MergeSplit {
+  int nm, ncols;
+};
+__device__ __forceinline__ MergeSplit merge_split(int g, int nseg) {
+  const int cols = g * kHeadDim;
+  const int nm = min(nseg, cols / 32);
+  const int per = (cols + nm - 1) / nm;
+  return MergeSplit{nm, min(((per + 31) / 32) * 32, kThreads)};
+}
+
+// Block mi (of the nm merging blocks) merges columns [mi * ncols, ...) of
+// the pair, in pieces of at most kThreads.
+__device__ __forceinline__ void merge_share(const float* part, float* out, float* lse, int Hq, int Hkv, int g, int p,
+                                            int nseg, int mi, MergeSplit ms, float* scratch) {
+  const int cols = g * kHeadDim;
+  for (int c0 = mi * ms.ncols; c0 < cols; c0 += ms.nm * ms.ncols) {
+    if (ms.ncols == 32)
+      merge_slice(part, out, lse, Hq, Hkv, g, p, nseg, c0 / 32, scratch);
+    else
+      merge_cols(part, out, lse, Hq, Hkv, g, p, nseg, c0, min(ms.ncols, cols - c0), scratch);
+  }
 }
 
 // out / lse of every query head of pair p from the block's own partial (one
@@ -1605,20 +1706,21 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
       if (nseg == 1) {
         finish_single(a, p, part_s);
       } else {
-        // the last g blocks of the pair to finish merge one head each; the
+        // the last blocks of the pair to finish merge a run of its output
+        // columns each (merge_split, merge_cols); the
         // last of them to finish returns the pair's counters and histogram to
         // zero (every block is past its last use of them)
         if (tid == 0) sh[8] = (int)atom_acq_rel_add(&sync[2], 1u);
         __syncthreads();
-        const int nm = min(a.g, nseg);
+        const MergeSplit ms = merge_split(a.g, nseg);
+        const int nm = ms.nm;
         const int mi = sh[8] - (nseg - nm);
         if (mi >= 0) {
           if (tid == 0) sh[7] = wait_count(&sync[2], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
           __syncthreads();
           HKV_TL(8);
           if (sh[7]) {
-            for (int h = mi; h < a.g; h += nm)
-              merge_head(a.part, a.out, a.lse, a.Hq, a.Hkv, a.g, p, nseg, h, reinterpret_cast<float*>(smem));
+            merge_share(a.part, a.out, a.lse, a.Hq, a.Hkv, a.g, p, nseg, mi, ms, reinterpret_cast<float*>(smem));
           } else if (tid == 0) {
             report(a.status, HKV_ERR_TIMEOUT);
           }
@@ -1669,8 +1771,9 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
 // Block x serves pair p = p0 + x / nseg and rows [seg * per_block, ...) of
 // the pair's row list [sink | idx slots | local]; eight warps take 16-row
 // steps with two cp.async slots each (attn_warps).  One segment per pair
-// writes out / lse itself; with several (a cooperative launch) the last g
-// blocks of the pair merge one head each, as in the fused kernel.
+// writes out / lse itself; with several (a cooperative launch) the last
+// blocks of the pair merge a run of its output columns each, as in the
+// fused kernel.
 constexpr int kSaTok = 4096;  // row tokens kept in shared memory per block
 
 struct SaLayout {
@@ -1726,14 +1829,14 @@ __global__ void __launch_bounds__(kThreads, 1) sattend_kernel(FusedArgs a) {
   uint32_t* sync = a.sync + kSync * p;
   if (tid == 0) sh[0] = (int)atom_acq_rel_add(&sync[2], 1u);
   __syncthreads();
-  const int nm = min(g, nseg);
+  const MergeSplit ms = merge_split(g, nseg);
+  const int nm = ms.nm;
   const int mi = sh[0] - (nseg - nm);
   if (mi < 0) return;
   if (tid == 0) sh[1] = wait_count(&sync[2], (uint32_t)nseg, a.wait_ns) ? 1 : 0;
   __syncthreads();
   if (sh[1]) {
-    for (int h = mi; h < g; h += nm)
-      merge_head(a.part, a.out, a.lse, a.Hq, a.Hkv, g, p, nseg, h, reinterpret_cast<float*>(smem));
+    merge_share(a.part, a.out, a.lse, a.Hq, a.Hkv, g, p, nseg, mi, ms, reinterpret_cast<float*>(smem));
   } else if (tid == 0) {
     report(a.status, HKV_ERR_TIMEOUT);
   }
