@@ -82,6 +82,7 @@ constexpr int kKP = kHeadDim + 4;     // K tile pitch: float4-aligned rows
 constexpr int kPart = kHeadDim + 4;         // m, l, (2 unused), acc[128]: acc 16-byte aligned
 constexpr int kSync = 4;                    // per pair: arrivals, departures, merge ticket, merges done
 constexpr int kSelCap = 2048;               // selected rows kept in shared memory
+constexpr int kPtCap = 2048;                // page ids of a block's scan range kept in shared memory
 constexpr int kOut = (kMaxGroup * kHeadDim + kThreads - 1) / kThreads;
 
 enum QEnc { kQGiven = 0, kQLsh = 1, kQSign = 2 };
@@ -106,7 +107,7 @@ struct FusedArgs {
   int sink_n, local_start, local_n;
   int p0, nseg, per_block;
   int nbins, nbins_pad;
-  uint32_t off_q, off_aq, off_sel, off_hist, off_dist, off_part, off_qs, off_tokw;  // shared memory (bytes)
+  uint32_t off_q, off_aq, off_sel, off_hist, off_dist, off_part, off_qs, off_tokw, off_pt;  // shared memory (bytes)
   int sel_cap;     // selected rows kept in shared memory
   int spec;        // load one speculative K/V tile during the threshold exchange
   uint32_t* sync;  // [pairs][kSync]
@@ -134,10 +135,19 @@ __device__ __forceinline__ int64_t kv_row(const FusedArgs& a, int p) {
   return (int64_t)(p / a.Hkv) * a.Hkv_real + (p % a.Hkv) / a.unit_div;
 }
 
-// Row of token t of unit p in the code, K and V arrays: kvc + t for a
-// contiguous cache (kvc = the unit's first row); for a paged cache the row of
-// its slot in its pool page, or -1 when the page id is outside the pool.
-__device__ __forceinline__ int64_t cache_row(const FusedArgs& a, int p, int64_t kvc, int t) {
+// The unit's row key, computed once per block: for a contiguous cache its
+// first row in the code, K and V arrays; for a paged cache its batch index
+// (high 32 bits) and KV head within a pool page (low 32 bits), so that the
+// per-token row takes no division.
+__device__ __forceinline__ int64_t unit_rows(const FusedArgs& a, int p) {
+  if (a.ptab == nullptr) return kv_row(a, p) * a.cap;
+  return ((int64_t)(p / a.Hkv) << 32) | (int64_t)((p % a.Hkv) / a.unit_div);
+}
+
+// Row of token t of the unit with row key kvc (unit_rows) in the code, K and
+// V arrays: kvc + t for a contiguous cache; for a paged cache the row of its
+// slot in its pool page, or -1 when the page id is outside the pool.
+__device__ __forceinline__ int64_t cache_row(const FusedArgs& a, int /*p*/, int64_t kvc, int t) {
   if (a.ptab == nullptr) return kvc + t;
   int j, slot;
   if (a.ps_shift >= 0) {
@@ -147,9 +157,9 @@ __device__ __forceinline__ int64_t cache_row(const FusedArgs& a, int p, int64_t 
     j = t / a.page_size;
     slot = t - j * a.page_size;
   }
-  const int pg = __ldg(a.ptab + (int64_t)(p / a.Hkv) * a.max_pages + j);
+  const int pg = __ldg(a.ptab + (kvc >> 32) * a.max_pages + j);
   if (pg < 0 || (int64_t)pg >= a.num_pages) return -1;
-  return ((int64_t)pg * a.Hkv_real + (p % a.Hkv) / a.unit_div) * a.page_size + slot;
+  return ((int64_t)pg * a.Hkv_real + (kvc & 0xffffffffLL)) * a.page_size + slot;
 }
 
 
@@ -1304,7 +1314,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   const int tid = threadIdx.x;
   const int nseg = a.nseg;
   const int p = a.p0 + (int)blockIdx.x / nseg, seg = (int)blockIdx.x % nseg;
-  const int64_t kvc = kv_row(a, p) * a.cap;  // first cache row of this unit's (batch, KV head)
+  const int64_t kvc = unit_rows(a, p);  // this unit's row key (first cache row when contiguous)
   // Programmatic dependent launch.  The next kernel on this stream may be
   // launched now, so its blocks are ready to take each SM this grid leaves;
   // they wait below until this grid has finished.  Before this block touches
@@ -1354,19 +1364,48 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(FusedArgs a) {
   if (ATTEND && tid < a.g * (kHeadDim / 4))
     aq = load4_f32(tptr<T>(a.q) + qrow0 * kHeadDim + (tid / (kHeadDim / 4)) * kHeadDim + (tid % (kHeadDim / 4)) * 4);
   uint32_t* ring = reinterpret_cast<uint32_t*>(smem);
-  const uint32_t* pf_ptr = a.k_codes + (kvc + lo + s0 + tid) * W;
+  const uint32_t* pf_ptr = a.ptab != nullptr ? a.k_codes : a.k_codes + (kvc + lo + s0 + tid) * W;  // contiguous only
   constexpr int64_t kStep = (int64_t)kThreads * W;
   auto slot = [&](int k) { return ring + ((size_t)(k % kSlots) * kThreads + tid) * 4; };
   // paged cache: the code of token k of this thread comes through the page
   // table; a page outside the pool zero-fills its slot and marks it in `bad`
   const bool paged = a.ptab != nullptr;
   uint32_t bad = 0, bad_seen = 0;
+  // the page ids of the block's scan range go to shared memory (read from
+  // the ring's first refill on, after the first block barrier) when they fit
+  int* pt_s = reinterpret_cast<int*>(smem + a.off_pt);
+  int pj0 = 0;
+  bool pt_local = false;
+  if (paged && len > 0) {
+    const int t0 = lo + s0, t1 = lo + s0 + len - 1;
+    pj0 = a.ps_shift >= 0 ? t0 >> a.ps_shift : t0 / a.page_size;
+    const int npg = (a.ps_shift >= 0 ? t1 >> a.ps_shift : t1 / a.page_size) - pj0 + 1;
+    pt_local = npg <= kPtCap;
+    if (pt_local)
+      for (int i = tid; i < npg; i += kThreads) pt_s[i] = __ldg(a.ptab + (kvc >> 32) * a.max_pages + pj0 + i);
+  }
   auto issue_code = [&](int k) {
     if (!paged) {
       cp_async_code<W>(slot(k), pf_ptr + k * kStep);
       return;
     }
-    const int64_t r = cache_row(a, p, 0, lo + s0 + tid + k * kThreads);
+    const int t = lo + s0 + tid + k * kThreads;
+    int64_t r;
+    if (pt_local && k >= kSlots) {
+      int j, sl;
+      if (a.ps_shift >= 0) {
+        j = t >> a.ps_shift;
+        sl = t & (a.page_size - 1);
+      } else {
+        j = t / a.page_size;
+        sl = t - j * a.page_size;
+      }
+      const int pg = pt_s[j - pj0];
+      r = (pg < 0 || (int64_t)pg >= a.num_pages) ? -1
+                                                  : ((int64_t)pg * a.Hkv_real + (kvc & 0xffffffffLL)) * a.page_size + sl;
+    } else {
+      r = cache_row(a, p, kvc, t);
+    }
     const uint32_t bit = 1u << (k % kSlots);
     bad = r < 0 ? (bad | bit) : (bad & ~bit);
     cp_async_code_zf<W>(slot(k), a.k_codes + (r < 0 ? 0 : r) * W, r >= 0);
@@ -1817,7 +1856,7 @@ __global__ void __launch_bounds__(kThreads, 1) sattend_kernel(FusedArgs a) {
     const int h = i / kHeadDim, k = i % kHeadDim;
     qs_s[h * kQP + k] = h < g ? q0[(int64_t)h * kHeadDim + k] : __float2bfloat16_rn(0.f);
   }
-  const int64_t kvc = kv_row(a, p) * a.cap;
+  const int64_t kvc = unit_rows(a, p);
   float* dst = nseg == 1 ? part_s : a.part + ((int64_t)p * nseg + seg) * g * kPart;
   // (attn_warps starts with a block barrier: tok_s and qs_s are complete)
   attn_warps(a, p, kvc, nrows, [&](int i) -> int { return i < kSaTok ? tok_s[i] : token_of(v0 + i); }, smem,
@@ -1896,7 +1935,7 @@ __global__ void __launch_bounds__(kThreads, 1) normw_decode_kernel(FusedArgs a, 
   __syncthreads();
   if (n.q_codes_out != nullptr)
     for (int i = tid; i < g * W; i += kThreads) n.q_codes_out[qrow0 * W + i] = qc_s[i];
-  const int64_t kvc = kv_row(a, p) * a.cap;
+  const int64_t kvc = unit_rows(a, p);
   if (k_eff > 0)
     nw::block_select<W, NP>(a.k_codes + (kvc + a.lo) * W, n.norms + kvc + a.lo, n.vec_norms != 0, qc_s, g, n.gb,
                             (int)a.lo, a.C, k_eff, smem, wsum, found, cnt_s, idx, score);
@@ -1979,7 +2018,7 @@ struct Plan {
   int k_eff;
   int nseg, per_block, pairs_per_launch, sel_cap;
   bool cooperative;
-  uint32_t off_q, off_aq, off_sel, off_hist, off_dist, off_part, off_qs, off_tokw;
+  uint32_t off_q, off_aq, off_sel, off_hist, off_dist, off_part, off_qs, off_tokw, off_pt;
   size_t smem;
   size_t ws_sync, ws_gh, ws_cum, ws_part, ws_total;
 };
@@ -2046,6 +2085,8 @@ int make_plan(const RetrieveShape& s, bool attend, int q_elt, Plan& pl) {
     if (attend) off += align_up(sizeof(uint16_t) * kMaxGroup * kQP, 16);
     pl.off_tokw = (uint32_t)off;
     if (attend) off += sizeof(int) * 2 * kAW * kWR;
+    pl.off_pt = (uint32_t)off;
+    if (s.pm != nullptr) off += sizeof(int) * kPtCap;
     pl.smem = align_up(off, 16);
     fits = pl.smem <= budget;
     if (fits) break;
@@ -2117,6 +2158,7 @@ int launch_fused(const RetrieveShape& s, bool attend, int dtype, int qenc, const
   a.off_part = pl.off_part;
   a.off_qs = pl.off_qs;
   a.off_tokw = pl.off_tokw;
+  a.off_pt = pl.off_pt;
   a.sel_cap = pl.sel_cap;
   {
     // speculative tile: when a block's expected share of the selection, with
