@@ -69,6 +69,10 @@ struct NormwArgs {
 template <int W, int NP>
 __global__ void __launch_bounds__(kThreads, 1) normw_kernel(NormwArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
+  // programmatic dependent launch: the next kernel may launch now; this
+  // block reads global memory only after the previous kernel has finished
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ uint32_t qc_s[kMaxGroup * W];
   __shared__ uint32_t wsum[kWarps];
   __shared__ uint32_t found[3];
@@ -116,6 +120,10 @@ struct MergeArgs {
 // number of real entries, so no padding entry is selected.
 __global__ void __launch_bounds__(kThreads, 1) normw_merge_kernel(MergeArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
+  // programmatic dependent launch: the next kernel may launch now; this
+  // block reads global memory only after the previous kernel has finished
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   uint32_t* lists = reinterpret_cast<uint32_t*>(smem);  // [2][kWarps][kListCap]
   __shared__ __align__(16) uint32_t hist[kBins];
   __shared__ uint32_t wsum[kWarps];
@@ -230,8 +238,17 @@ int launch_retrieve_normw(const RetrieveShape& s, const uint32_t* q_codes, const
   const size_t smem = kRegionBytes + (size_t)kBins * 4 + (size_t)kWarps * range * sizeof(uint16_t);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_check(e, "norm-weighted retrieval shared memory");
-  fn<<<(unsigned)((int64_t)P * a.nseg), kThreads, smem, st>>>(a);
-  e = cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((int64_t)P * a.nseg));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, fn, a);
   if (e != cudaSuccess || pl.nseg == 1) return cuda_check(e, "norm-weighted retrieval launch");
 
   MergeArgs m;
@@ -245,8 +262,9 @@ int launch_retrieve_normw(const RetrieveShape& s, const uint32_t* q_codes, const
   m.score = score;
   e = cudaFuncSetAttribute(normw_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRegionBytes);
   if (e != cudaSuccess) return cuda_check(e, "norm-weighted merge shared memory");
-  normw_merge_kernel<<<(unsigned)P, kThreads, kRegionBytes, st>>>(m);
-  return cuda_check(cudaGetLastError(), "norm-weighted retrieval merge launch");
+  cfg.gridDim = dim3((unsigned)P);
+  cfg.dynamicSmemBytes = kRegionBytes;
+  return cuda_check(cudaLaunchKernelEx(&cfg, normw_merge_kernel, m), "norm-weighted retrieval merge launch");
 }
 
 }  // namespace hkv

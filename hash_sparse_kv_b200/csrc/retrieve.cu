@@ -1825,6 +1825,12 @@ struct SaLayout {
 
 __global__ void __launch_bounds__(kThreads, 1) sattend_kernel(FusedArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
+  // programmatic dependent launch, as in fused_kernel: the next kernel may
+  // launch now; this block reads global memory only after the previous
+  // kernel on the stream has finished
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   __nv_bfloat16* qs_s = reinterpret_cast<__nv_bfloat16*>(smem + SaLayout::qs);
   int* tokw_s = reinterpret_cast<int*>(smem + SaLayout::tokw);
   int* tok_s = reinterpret_cast<int*>(smem + SaLayout::tok);
@@ -1910,6 +1916,12 @@ struct NdLayout {
 template <int W, int NP>
 __global__ void __launch_bounds__(kThreads, 1) normw_decode_kernel(FusedArgs a, NwDecodeArgs n) {
   extern __shared__ __align__(128) unsigned char smem[];
+  // programmatic dependent launch, as in fused_kernel: the next kernel may
+  // launch now; this block reads global memory only after the previous
+  // kernel on the stream has finished
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   __shared__ uint32_t qc_s[kMaxGroup * W];
   __shared__ uint32_t wsum[kWarps];
   __shared__ uint32_t found[3];
@@ -2277,8 +2289,17 @@ int launch_normw_decode(const RetrieveShape& s, const void* q, const uint32_t* k
   const size_t smem = std::max(sel_smem, NdLayout::attn);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return cuda_check(e, "norm-weighted decode shared memory");
-  fn<<<(unsigned)P, kThreads, smem, st>>>(a, n);
-  return cuda_check(cudaGetLastError(), "norm-weighted decode launch");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)P);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, fn, a, n), "norm-weighted decode launch");
 }
 
 size_t sattend_ws_bytes(const AttendShape& s) { return sattend_plan(s).ws_total; }
@@ -2340,11 +2361,13 @@ int launch_sattend(const AttendShape& s, const void* q, const void* K, const voi
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = SaLayout::total;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pl.cooperative ? 1 : 0;
+    cfg.numAttrs = pl.cooperative ? 2 : 1;
     const int rc = cuda_check(cudaLaunchKernelEx(&cfg, sattend_kernel, a), "sparse attention launch");
     if (rc != HKV_OK) return rc;
   }
