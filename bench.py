@@ -704,7 +704,9 @@ def run_split(args, rank, world, local):
         "config": {"workload": w.name, "n_tokens": w.N, "tokens_per_rank": r1 - r0, "layers_per_step": n_layers,
                    "parallelism": f"token split x{world} (NCCL all-gathers of candidates and partials)",
                    "timing": "median of the per-replay CUDA-event times (max over ranks)"},
-        "gpu_launches": None, "clocks": clk.summary(), "cpu_baseline": None,
+        # per layer: query encode, retrieval, global selection, attention and
+        # the G-way merge, one launch each at this shape (the all-gathers are NCCL's)
+        "gpu_launches": 5 * n_layers * args.steps, "clocks": clk.summary(), "cpu_baseline": None,
     }
     dist.barrier()
     return out
