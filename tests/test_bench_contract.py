@@ -64,3 +64,29 @@ def test_roofline_arithmetic():
     assert e["bound"] == "hbm" and e["gbs"] == pytest.approx(8 * 8 * 32768 * (256 + 8) / 1e-3 / 1e9)
     e = bench.encode_roofline(synth.WORKLOADS["spotlight_mlp"], 1, 1.0)
     assert e["bound"] == "tensor" and e["unit"] == "TFLOP/s"
+
+
+def test_traffic_records_follow_their_sources(tmp_path, monkeypatch):
+    """A recorded DRAM byte count is reported only while every source file of
+    the kernel is unchanged: the committed records match the sources, and a
+    one-byte change to any listed file voids the record."""
+    sys.path.insert(0, ROOT)
+    import bench
+    csrc = os.path.join(ROOT, "hash_sparse_kv_b200", "csrc")
+    fused = os.path.join(csrc, "retrieve.cu")
+    normw = [os.path.join(csrc, f) for f in ("normw.cu", "normw_select.cuh")]
+    assert bench.traffic_record(fused, "qwen7b_512k") is not None
+    assert bench.traffic_record(normw, "signvq") is not None
+    # a copy of the sources with one byte changed in the second file
+    copies = []
+    for i, f in enumerate(normw):
+        dst = tmp_path / os.path.basename(f)
+        data = open(f, "rb").read()
+        dst.write_bytes(data + (b" " if i == 1 else b""))
+        copies.append(str(dst))
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "dram_traffic.json").write_bytes(
+        open(os.path.join(ROOT, "profiles", "dram_traffic.json"), "rb").read())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_record(copies, "signvq") is None
+    assert bench.source_digest(copies) != bench.source_digest(normw)
