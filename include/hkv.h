@@ -389,8 +389,12 @@ int hkv_lse_merge_n(int G, int64_t rows, const float* o, const float* lse, float
  *   lse[b, h] = log sum_t exp(scale * q[b, h] . K[b, j, t])
  * over t in [0, sink_end) + {idx[b, j, i] >= 0} + [local_start, n_tokens).
  *   q       [B, Hq, 128] in dtype;  K, V  [B, Hkv, cap, 128] in dtype
- *   idx     [B, Hkv, top_k] int32 (-1 entries are skipped; entries outside
- *           [0, n_tokens) are skipped and reported as HKV_ERR_DEVICE_RANGE)
+ *   idx     [B, Hkv, top_k] int32 (negative entries, e.g. the -1 padding,
+ *           are skipped; entries at or past n_tokens are skipped and reported
+ *           as HKV_ERR_DEVICE_RANGE)
+ * bf16: the fused decode kernel's tensor-core attention stage, a pair's rows
+ * split over up to one wave of blocks (cooperative launch) and merged by its
+ * last blocks; fp32: a SIMT kernel, split-K with a last-block merge.
  *   out     [B, Hq, 128] fp32;  lse  nullable [B, Hq] fp32
  * The selected indices must not repeat a sink or local token. */
 int hkv_sparse_attend(int B, int Hq, int Hkv, int dtype, const void* q, const void* K,
